@@ -1,0 +1,215 @@
+/*
+ * moe_oracle.c - plain, slow fp64 CPU oracle of one MoE decode-layer step.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call this code:
+ * only the test suite, the smoke check and the benchmark's CPU-baseline leg
+ * use it. It shares no code with the CUDA path.
+ *
+ * What it computes: one decode step of a sparse mixture-of-experts layer of
+ * the kind the Kimi K3 decode pages describe (page "vLLM 合併 Kimi K3 專用解碼：
+ * 官方稱 GB300 快 1.5 到 2 倍，423 tok/s 怎麼核對", section "Kimi K3 專用解碼路徑
+ * 改了什麼": 896 routed experts, 16 active per token; page
+ * post.smzdm.com/p/a6zppe4g, section "改了什么：每层 23 个 kernel 砍到 13 个":
+ * router scores and a shared expert that runs beside the routing). The pages
+ * give no formulas; the definition below is the plainest reading of the
+ * workload description, written out directly, row by row, in fp64:
+ *
+ *   n      = bf16( x * rsqrt(mean(x^2) + eps) * gamma )          RMSNorm
+ *   l[e]   = sum_h n[h] * W_r[e,h]  (+ bias[e])                   router logits
+ *   S      = the k largest l[e], ties to the lower e              top-k
+ *   w[j]   = exp(l[S_j]) / sum_i exp(l[S_i])                      renormalised
+ *   E_e(n) = W_d[e] * bf16( silu(W_g[e] n) (.) (W_u[e] n) )        SwiGLU expert
+ *   s      = W_sd  * bf16( silu(W_sg n)   (.) (W_su n) )           shared expert
+ *   y      = bf16( x + s + sum_j w[j] * E_{S_j}(n) )              combine + residual
+ *
+ * bf16 rounding (round to nearest even) is applied exactly at the three
+ * points the workload fixes as bf16 activations (n, the SwiGLU product h, and
+ * the output y); every other quantity stays fp64. silu(v) = v / (1 + exp(-v)).
+ * Rows are independent; parallelism (OpenMP) is over output features only.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "moe_oracle.h"
+
+/* ---- bf16 helpers (fp64 <-> bf16) ---------------------------------------- */
+
+double oracle_bf16_to_double(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* Round an fp64 value to the nearest bf16 value (ties to even), directly from
+ * fp64 (no intermediate fp32 rounding). bf16: 8 significant bits, the fp32
+ * exponent range, subnormals below 2^-126. */
+double oracle_bf16_round(double v) {
+  if (v == 0.0 || !isfinite(v)) return v;
+  int e;
+  (void)frexp(v, &e); /* |v| in [2^(e-1), 2^e) */
+  int ulp_exp = e - 8;
+  if (ulp_exp < -133) ulp_exp = -133; /* subnormal spacing 2^-133 */
+  double r = ldexp(nearbyint(ldexp(v, -ulp_exp)), ulp_exp);
+  const double max_bf16 = ldexp(255.0, 120); /* (2 - 2^-7) * 2^127 */
+  if (fabs(r) > max_bf16) return v > 0 ? INFINITY : -INFINITY;
+  return r;
+}
+
+uint16_t oracle_double_to_bf16_bits(double v) {
+  float f = (float)oracle_bf16_round(v); /* exact: the value is a bf16 value */
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  if (isnan(v)) return 0x7FC0u;
+  return (uint16_t)(u >> 16);
+}
+
+static inline double bf(uint16_t b) { return oracle_bf16_to_double(b); }
+
+static double silu(double v) { return v / (1.0 + exp(-v)); }
+
+/* Planted-mistake switch, used only by the test that proves the pins catch
+ * mistakes. 0 (the default) is the oracle; each other value swaps in one
+ * plausible error (see ORACLE_MUT_* in moe_oracle.h). */
+static int g_mutant = 0;
+void oracle_set_mutant(int m) { g_mutant = m; }
+#define MUT(m) (g_mutant == (m))
+
+/* ---- stages ---------------------------------------------------------------- */
+
+/* RMSNorm of one row: n = bf16(x * rsqrt(mean(x^2) + eps) * gamma). */
+void oracle_rmsnorm(int H, double eps, const uint16_t* x, const uint16_t* gamma, double* n_out) {
+  double ss = 0.0;
+  for (int h = 0; h < H; ++h) ss += bf(x[h]) * bf(x[h]);
+  double r = 1.0 / sqrt(ss / (double)H + eps);
+  if (MUT(ORACLE_MUT_EPS_OUTSIDE)) r = 1.0 / (sqrt(ss / (double)H) + eps);
+  for (int h = 0; h < H; ++h) {
+    const double g = MUT(ORACLE_MUT_NO_GAMMA) ? 1.0 : bf(gamma[h]);
+    const double v = bf(x[h]) * r * g;
+    n_out[h] = MUT(ORACLE_MUT_NO_N_ROUND) ? v : oracle_bf16_round(v);
+  }
+}
+
+/* y[m] = sum_k W[m,k] * v[k] for a row-major bf16 matrix W [M][K]. */
+static void matvec(int M, int K, const uint16_t* W, const double* v, double* out) {
+  int m;
+#pragma omp parallel for schedule(static)
+  for (m = 0; m < M; ++m) {
+    const uint16_t* row = W + (size_t)m * (size_t)K;
+    double acc = 0.0;
+    for (int k = 0; k < K; ++k) acc += bf(row[k]) * v[k];
+    out[m] = acc;
+  }
+}
+
+/* Router logits of one row: l[e] = n . W_r[e] (+ bias[e]). */
+void oracle_router(int H, int E, const double* n, const uint16_t* w_router, const float* bias,
+                   double* logits) {
+  matvec(E, H, w_router, n, logits);
+  if (bias && !MUT(ORACLE_MUT_NO_BIAS))
+    for (int e = 0; e < E; ++e) logits[e] += (double)bias[e];
+}
+
+/* The k largest values, ties to the lower index; idx_out in descending value
+ * order. Returns -1 on a non-finite value or bad k. Plain O(k E) selection. */
+int oracle_topk(int E, int k, const double* v, int32_t* idx_out) {
+  if (E < 1 || k < 1 || k > E) return -1;
+  for (int e = 0; e < E; ++e)
+    if (!isfinite(v[e])) return -1;
+  unsigned char* taken = (unsigned char*)calloc((size_t)E, 1);
+  for (int j = 0; j < k; ++j) {
+    int best = -1;
+    for (int e = 0; e < E; ++e) {
+      if (taken[e]) continue;
+      if (best < 0 || v[e] > v[best]) best = e; /* strict: the lower index keeps a tie */
+      else if (MUT(ORACLE_MUT_TIES_HIGH) && v[e] == v[best]) best = e;
+    }
+    taken[best] = 1;
+    idx_out[j] = best;
+  }
+  free(taken);
+  return 0;
+}
+
+/* Softmax over the selected logits (the full softmax renormalised over S). */
+void oracle_softmax_selected(int k, const double* logits, const int32_t* idx, double* w_out) {
+  double m = logits[idx[0]];
+  for (int j = 1; j < k; ++j)
+    if (logits[idx[j]] > m) m = logits[idx[j]];
+  double z = 0.0;
+  for (int j = 0; j < k; ++j) z += exp(logits[idx[j]] - m);
+  for (int j = 0; j < k; ++j) w_out[j] = exp(logits[idx[j]] - m) / z;
+  if (MUT(ORACLE_MUT_EQUAL_WEIGHTS))
+    for (int j = 0; j < k; ++j) w_out[j] = 1.0 / (double)k;
+}
+
+/* SwiGLU expert: out = W_d * bf16(silu(W_g n) (.) (W_u n)); W_g,W_u [F][H], W_d [H][F]. */
+void oracle_swiglu(int H, int F, const double* n, const uint16_t* wg, const uint16_t* wu,
+                   const uint16_t* wd, double* out) {
+  double* g = (double*)malloc(sizeof(double) * (size_t)F);
+  double* u = (double*)malloc(sizeof(double) * (size_t)F);
+  matvec(F, H, wg, n, g);
+  matvec(F, H, wu, n, u);
+  for (int i = 0; i < F; ++i) {
+    double v = MUT(ORACLE_MUT_SILU_ON_UP) ? g[i] * silu(u[i]) : silu(g[i]) * u[i];
+    g[i] = MUT(ORACLE_MUT_NO_H_ROUND) ? v : oracle_bf16_round(v);
+  }
+  if (MUT(ORACLE_MUT_DOWN_TRANSPOSED)) {
+    for (int m = 0; m < H; ++m) {
+      double acc = 0.0;
+      for (int k = 0; k < F; ++k) acc += bf(wd[(size_t)k * H + m]) * g[k];
+      out[m] = acc;
+    }
+  } else {
+    matvec(H, F, wd, g, out);
+  }
+  free(g);
+  free(u);
+}
+
+/* ---- whole layer ------------------------------------------------------------ */
+
+int oracle_layer(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
+                 double* logits, int32_t* topk_idx, double* topk_w, double* y_pre, uint16_t* y) {
+  const int H = d->H, E = d->E, k = d->k, I = d->I, Is = d->Is;
+  if (B < 0 || H < 1 || E < 1 || k < 1 || k > E || I < 1 || Is < 1) return ORACLE_EINVAL;
+  double* n = (double*)malloc(sizeof(double) * (size_t)H);
+  double* s = (double*)malloc(sizeof(double) * (size_t)H);
+  double* ex = (double*)malloc(sizeof(double) * (size_t)H);
+  double* acc = (double*)malloc(sizeof(double) * (size_t)H);
+  int rc = ORACLE_OK;
+  for (int b = 0; b < B && rc == ORACLE_OK; ++b) {
+    const uint16_t* xb = x + (size_t)b * H;
+    double* lb = logits + (size_t)b * E;
+    int32_t* ib = topk_idx + (size_t)b * k;
+    double* wb = topk_w + (size_t)b * k;
+
+    oracle_rmsnorm(H, d->eps, xb, w->gamma, n);
+    oracle_router(H, E, n, w->w_router, w->router_bias, lb);
+    if (oracle_topk(E, k, lb, ib) != 0) { rc = ORACLE_ENONFINITE; break; }
+    oracle_softmax_selected(k, lb, ib, wb);
+
+    oracle_swiglu(H, Is, n, w->ws_gate, w->ws_up, w->ws_down, s);
+    for (int h = 0; h < H; ++h) {
+      const double res = MUT(ORACLE_MUT_RESIDUAL_N) ? n[h] : bf(xb[h]);
+      acc[h] = res + (MUT(ORACLE_MUT_NO_SHARED) ? 0.0 : s[h]);
+    }
+    for (int j = 0; j < k; ++j) {
+      const int e = ib[j];
+      if (!w->w_gate[e] || !w->w_up[e] || !w->w_down[e]) { rc = ORACLE_EMISSING; break; }
+      oracle_swiglu(H, I, n, w->w_gate[e], w->w_up[e], w->w_down[e], ex);
+      for (int h = 0; h < H; ++h) acc[h] += wb[j] * ex[h];
+    }
+    for (int h = 0; h < H; ++h) {
+      if (y_pre) y_pre[(size_t)b * H + h] = acc[h];
+      if (y) y[(size_t)b * H + h] = oracle_double_to_bf16_bits(acc[h]);
+    }
+  }
+  free(n);
+  free(s);
+  free(ex);
+  free(acc);
+  return rc;
+}

@@ -1,0 +1,265 @@
+"""Seeded synthetic inputs for the MoE decode-layer workloads.
+
+This package generates inputs only; it holds none of the layer's arithmetic.
+It is the one module that both the CPU oracle side (tests, the timed CPU
+baseline) and the GPU side (tests, bench) use, so that any expert's weights
+can be regenerated on the host bit-identically to what the device holds.
+
+The element generator is defined in ``moe_synth.h`` (SplitMix64 counter
+stream, Irwin-Hall normal approximation, bf16 round-to-nearest-even).
+
+Workloads (``WORKLOADS``) follow the five layer configurations the decode path
+is measured on: a tiny CPU-sized layer, and the 7168-hidden / 896-expert /
+top-16 layer at batch 1, batch 8, batch 64 with a Zipf-skewed router, and a
+32-row two-layer speculative-verify shape.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+HOST_LIB = os.path.join(_HERE, "libmoe_synth_host.so")
+CUDA_LIB = os.path.join(_HERE, "libmoe_synth_cuda.so")
+
+KIND_GAMMA = 1
+KIND_W_ROUTER = 2
+KIND_W_GATE = 3
+KIND_W_UP = 4
+KIND_W_DOWN = 5
+KIND_WS_GATE = 6
+KIND_WS_UP = 7
+KIND_WS_DOWN = 8
+KIND_X = 9
+KIND_BIAS_PERM = 10
+KIND_ROW_NOISE = 11
+KIND_ROW_BASE = 12
+
+
+def tensor_id(layer: int, kind: int) -> int:
+    return (int(layer) << 8) | int(kind)
+
+
+def build(verbose: bool = False) -> None:
+    """Compile the host fill library (gcc) and the device fill library (nvcc, sm_100a)."""
+    cmds = [
+        ["gcc", "-O3", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+         "-o", HOST_LIB, os.path.join(_HERE, "synth_host.c"), "-lm"],
+        ["nvcc", "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+         "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+         "-o", CUDA_LIB, os.path.join(_HERE, "synth_cuda.cu")],
+    ]
+    for cmd in cmds:
+        if verbose:
+            print(" ".join(cmd))
+        subprocess.run(cmd, check=True, cwd=_HERE)
+
+
+_host = None
+_cuda = None
+
+
+def _host_lib():
+    global _host
+    if _host is None:
+        if not os.path.exists(HOST_LIB):
+            build()
+        lib = ctypes.CDLL(HOST_LIB)
+        u64, f32 = ctypes.c_uint64, ctypes.c_float
+        vp = ctypes.c_void_p
+        lib.ms_fill_host.argtypes = [u64, u64, u64, u64, f32, f32, vp]
+        lib.ms_fill_host.restype = None
+        lib.ms_z_host.argtypes = [u64, u64, u64, u64, vp]
+        lib.ms_z_host.restype = None
+        lib.ms_words_host.argtypes = [u64, u64, u64, u64, vp]
+        lib.ms_words_host.restype = None
+        lib.ms_mix64_host.argtypes = [u64]
+        lib.ms_mix64_host.restype = u64
+        lib.ms_fill_rows_correlated.argtypes = [u64, ctypes.c_uint32, ctypes.c_int, ctypes.c_int,
+                                                ctypes.c_int, vp]
+        lib.ms_fill_rows_correlated.restype = None
+        lib.ms_router_bias.argtypes = [u64, ctypes.c_uint32, ctypes.c_int, vp]
+        lib.ms_router_bias.restype = None
+        _host = lib
+    return _host
+
+
+def _cuda_lib():
+    global _cuda
+    if _cuda is None:
+        if not os.path.exists(CUDA_LIB):
+            raise RuntimeError(f"{CUDA_LIB} is missing: run synth.build() first")
+        lib = ctypes.CDLL(CUDA_LIB)
+        u64, f32, vp = ctypes.c_uint64, ctypes.c_float, ctypes.c_void_p
+        lib.ms_fill_device.argtypes = [u64, u64, u64, u64, f32, f32, vp, vp]
+        lib.ms_fill_device.restype = ctypes.c_int
+        _cuda = lib
+    return _cuda
+
+
+def _ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+def fill_host(seed: int, tid: int, start: int, n: int, sigma: float, mean: float = 0.0) -> np.ndarray:
+    out = np.empty(int(n), dtype=np.uint16)
+    _host_lib().ms_fill_host(seed, tid, start, n, np.float32(sigma), np.float32(mean), _ptr(out))
+    return out
+
+
+def z_host(seed: int, tid: int, start: int, n: int) -> np.ndarray:
+    out = np.empty(int(n), dtype=np.float32)
+    _host_lib().ms_z_host(seed, tid, start, n, _ptr(out))
+    return out
+
+
+def words_host(seed: int, tid: int, start: int, n: int) -> np.ndarray:
+    out = np.empty(int(n), dtype=np.uint64)
+    _host_lib().ms_words_host(seed, tid, start, n, _ptr(out))
+    return out
+
+
+def mix64(z: int) -> int:
+    return int(_host_lib().ms_mix64_host(z))
+
+
+def rows_correlated(seed: int, layer: int, nseq: int, rows_per_seq: int, H: int) -> np.ndarray:
+    out = np.empty((nseq * rows_per_seq, H), dtype=np.uint16)
+    _host_lib().ms_fill_rows_correlated(seed, layer, nseq, rows_per_seq, H, _ptr(out))
+    return out
+
+
+def router_bias(seed: int, layer: int, E: int) -> np.ndarray:
+    out = np.empty(E, dtype=np.float32)
+    _host_lib().ms_router_bias(seed, layer, E, _ptr(out))
+    return out
+
+
+def fill_device(ptr: int, seed: int, tid: int, start: int, n: int, sigma: float, mean: float = 0.0,
+                stream: int = 0) -> None:
+    rc = _cuda_lib().ms_fill_device(seed, tid, start, n, np.float32(sigma), np.float32(mean),
+                                    ctypes.c_void_p(ptr), ctypes.c_void_p(stream))
+    if rc != 0:
+        raise RuntimeError(f"ms_fill_device failed with cudaError {rc}")
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit patterns, round to nearest even (NaN -> quiet NaN)."""
+    u = np.ascontiguousarray(v, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    nan = ((u & 0x7F800000) == 0x7F800000) & ((u & 0x007FFFFF) != 0)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16).astype(np.uint16)
+    r[nan] = 0x7FC0
+    return r
+
+
+def sigma_for(fan_in: int) -> np.float32:
+    """Weight standard deviation 1/sqrt(fan_in), rounded once to fp32."""
+    return np.float32(1.0 / np.sqrt(float(fan_in)))
+
+
+@dataclass(frozen=True)
+class Workload:
+    """One layer configuration and its seeded inputs."""
+
+    name: str
+    B: int
+    H: int
+    E: int
+    k: int
+    I: int
+    Is: int
+    seed: int
+    layers: int = 1
+    eps: float = 1e-6
+    router: str = "uniform"        # "uniform" | "zipf"
+    rows: str = "iid"              # "iid" | "correlated"
+    nseq: int = 0
+    rows_per_seq: int = 0
+    gamma_sigma: float = 0.1
+    notes: str = field(default="", compare=False)
+
+    # ---- hidden states --------------------------------------------------
+    def x_host(self, batch: int | None = None) -> np.ndarray:
+        """Input rows, bf16 bits [B, H] (layer 0 input)."""
+        if self.rows == "correlated":
+            x = rows_correlated(self.seed, 0, self.nseq, self.rows_per_seq, self.H)
+        else:
+            x = fill_host(self.seed, tensor_id(0, KIND_X), 0, self.B * self.H, 1.0).reshape(self.B, self.H)
+        return x if batch is None else x[:batch].copy()
+
+    def x_pool_host(self, count: int) -> np.ndarray:
+        """`count` distinct input batches [count, B, H] for timing loops (variant v uses seed + 1000*v)."""
+        out = np.empty((count, self.B, self.H), dtype=np.uint16)
+        for v in range(count):
+            s = self.seed + 1000 * v
+            if self.rows == "correlated":
+                out[v] = rows_correlated(s, 0, self.nseq, self.rows_per_seq, self.H)
+            else:
+                out[v] = fill_host(s, tensor_id(0, KIND_X), 0, self.B * self.H, 1.0).reshape(self.B, self.H)
+        return out
+
+    # ---- per-layer parameters --------------------------------------------
+    def gamma_host(self, layer: int = 0) -> np.ndarray:
+        return fill_host(self.seed, tensor_id(layer, KIND_GAMMA), 0, self.H, self.gamma_sigma, 1.0)
+
+    def bias_host(self, layer: int = 0):
+        if self.router != "zipf":
+            return None
+        return router_bias(self.seed, layer, self.E)
+
+    def w_router_host(self, layer: int = 0) -> np.ndarray:
+        return fill_host(self.seed, tensor_id(layer, KIND_W_ROUTER), 0, self.E * self.H,
+                         sigma_for(self.H)).reshape(self.E, self.H)
+
+    def shared_host(self, layer: int = 0):
+        H, Is = self.H, self.Is
+        g = fill_host(self.seed, tensor_id(layer, KIND_WS_GATE), 0, Is * H, sigma_for(H)).reshape(Is, H)
+        u = fill_host(self.seed, tensor_id(layer, KIND_WS_UP), 0, Is * H, sigma_for(H)).reshape(Is, H)
+        d = fill_host(self.seed, tensor_id(layer, KIND_WS_DOWN), 0, H * Is, sigma_for(Is)).reshape(H, Is)
+        return g, u, d
+
+    def expert_host(self, layer: int, e: int):
+        """(W_gate[e] [I,H], W_up[e] [I,H], W_down[e] [H,I]) as bf16 bits."""
+        H, I = self.H, self.I
+        n = I * H
+        g = fill_host(self.seed, tensor_id(layer, KIND_W_GATE), e * n, n, sigma_for(H)).reshape(I, H)
+        u = fill_host(self.seed, tensor_id(layer, KIND_W_UP), e * n, n, sigma_for(H)).reshape(I, H)
+        d = fill_host(self.seed, tensor_id(layer, KIND_W_DOWN), e * n, n, sigma_for(I)).reshape(H, I)
+        return g, u, d
+
+    # ---- device generation (whole tensors) ----------------------------------
+    def device_specs(self, layer: int):
+        """(name, kind, numel, sigma, mean) of every bf16 tensor of one layer."""
+        H, E, I, Is = self.H, self.E, self.I, self.Is
+        return [
+            ("gamma", KIND_GAMMA, H, np.float32(self.gamma_sigma), 1.0),
+            ("w_router", KIND_W_ROUTER, E * H, sigma_for(H), 0.0),
+            ("w_gate", KIND_W_GATE, E * I * H, sigma_for(H), 0.0),
+            ("w_up", KIND_W_UP, E * I * H, sigma_for(H), 0.0),
+            ("w_down", KIND_W_DOWN, E * H * I, sigma_for(I), 0.0),
+            ("ws_gate", KIND_WS_GATE, Is * H, sigma_for(H), 0.0),
+            ("ws_up", KIND_WS_UP, Is * H, sigma_for(H), 0.0),
+            ("ws_down", KIND_WS_DOWN, H * Is, sigma_for(Is), 0.0),
+        ]
+
+    def weight_bytes_per_layer(self) -> int:
+        return 2 * sum(s[2] for s in self.device_specs(0))
+
+
+WORKLOADS = {
+    0: Workload("tiny_b1_h256_e64_k4", B=1, H=256, E=64, k=4, I=128, Is=128, seed=0),
+    1: Workload("b1_h7168_e896_k16", B=1, H=7168, E=896, k=16, I=1024, Is=2048, seed=1),
+    2: Workload("b8_h7168_e896_k16", B=8, H=7168, E=896, k=16, I=1024, Is=2048, seed=2),
+    3: Workload("b64_h7168_e896_k16_zipf", B=64, H=7168, E=896, k=16, I=1024, Is=2048, seed=3,
+                router="zipf"),
+    4: Workload("verify_4x8_h7168_e896_k16_2layer", B=32, H=7168, E=896, k=16, I=1024, Is=2048,
+                seed=4, layers=2, rows="correlated", nseq=4, rows_per_seq=8),
+}
