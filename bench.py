@@ -1,0 +1,393 @@
+#!/usr/bin/env python
+"""Benchmark of the persistent MoE decode-layer step on B200.
+
+Prints ONE JSON line (rank 0). The metric is the layer step's µs/step and the
+HBM bandwidth it sustains over the bytes the step must touch (router, shared
+expert, and each selected expert once however many rows chose it), against the
+measured B200 copy bandwidth. `value` is that bandwidth in GB/s (whole job:
+bytes of all ranks / max-over-ranks time); `ms_per_step` is the step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
+
+One step = one moe_decode_step call (one persistent launch per layer) on a
+batch from a pool of 32 seeded inputs, with L2 flushed (256 MB write) between
+timed steps. Under torchrun every rank runs an independent replica (the path
+does not shard; no data-path collective): weak scaling.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE decode-layer µs/step and HBM GB/s (% of B200 peak) at batch 1–64"
+FALLBACK_HBM_GBS = 6650.0
+POOL = 32
+FLUSH_BYTES = 256 << 20
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--config", type=int, default=1, help="workload index (synth.WORKLOADS)")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline oracle budget")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def step_bytes(wl, n_unique_per_layer, batch=None):
+    """Algorithmic bytes of one step: every weight byte the step must read once
+    (router, shared expert, each unique selected expert) plus x, y and gamma."""
+    B = wl.B if batch is None else batch
+    H, E, I, Is = wl.H, wl.E, wl.I, wl.Is
+    per_layer_fixed = 2 * (E * H + 3 * Is * H + H) + (4 * E if wl.router == "zipf" else 0)
+    total = 0
+    for U in n_unique_per_layer:
+        total += per_layer_fixed + U * 3 * I * H * 2 + 2 * B * H * 2
+    return total
+
+
+def workload_config(wl, flush):
+    return {"workload": wl.name, "batch": wl.B, "hidden": wl.H, "experts": wl.E, "top_k": wl.k,
+            "expert_inter": wl.I, "shared_inter": wl.Is, "layers": wl.layers,
+            "router": wl.router, "rows": wl.rows, "input_pool": POOL,
+            "l2": flush, "parallelism": "replicas"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------------
+# CPU oracle arm (baseline leg and --impl reference)
+# ---------------------------------------------------------------------------------------
+
+def cpu_oracle_full_steps(wl, pool, budget_s):
+    """Time the oracle on full single-row layer steps of distinct pool inputs until the
+    oracle time reaches budget_s. Weights are regenerated on the host before each timed
+    call (not timed). Returns (GB/s, seconds, steps)."""
+    import oracle
+
+    shared = [wl.shared_host(l) for l in range(wl.layers)]
+    w_router = [wl.w_router_host(l) for l in range(wl.layers)]
+    dims = dict(H=wl.H, E=wl.E, k=wl.k, I=wl.I, Is=wl.Is, eps=wl.eps)
+    t_tot, bytes_tot, steps = 0.0, 0, 0
+    v = 0
+    while t_tot < budget_s and v < len(pool):
+        x = pool[v][:1]
+        uniq = []
+        for l in range(wl.layers):
+            gamma, bias = wl.gamma_host(l), wl.bias_host(l)
+            n = oracle.rmsnorm(x[0], gamma, wl.eps)
+            sel = oracle.topk(oracle.router(n, w_router[l], bias), wl.k)
+            experts = {int(e): wl.expert_host(l, int(e)) for e in sel}
+            W = dict(gamma=gamma, w_router=w_router[l], router_bias=bias, experts=experts,
+                     ws_gate=shared[l][0], ws_up=shared[l][1], ws_down=shared[l][2])
+            t0 = time.perf_counter()
+            r = oracle.layer(dims, W, x)
+            t_tot += time.perf_counter() - t0
+            x = r["y"]
+            uniq.append(len(sel))
+        bytes_tot += step_bytes(wl, uniq, batch=1)
+        steps += 1
+        v += 1
+    return bytes_tot / t_tot / 1e9, t_tot, steps
+
+
+def run_reference(args, wl):
+    """--impl reference: the fp64 CPU oracle as it stands, timed on the host cores."""
+    import oracle
+
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    pool = wl.x_pool_host(2)
+    gamma, bias = wl.gamma_host(0), wl.bias_host(0)
+    w_router = wl.w_router_host(0)
+    sg, su, sd = wl.shared_host(0)
+    n = oracle.rmsnorm(pool[0][0], gamma, wl.eps)
+    sel = oracle.topk(oracle.router(n, w_router, bias), wl.k)
+    experts = [wl.expert_host(0, int(e)) for e in sel]
+    budget = max(0.02, min(1.0, 150.0 / max(1, args.steps + args.warmup)))
+
+    def one_step(i):
+        # a bounded sample of the layer: RMSNorm + router for one row, then SwiGLU
+        # experts (shared first, then the row's selected experts, cycling) until the
+        # per-step budget is used; bytes = weight bytes processed
+        t0 = time.perf_counter()
+        b = 0
+        x = pool[i % len(pool)][0]
+        nn = oracle.rmsnorm(x, gamma, wl.eps)
+        oracle.router(nn, w_router, bias)
+        b += 2 * (wl.E * wl.H + wl.H) + 2 * wl.H
+        j = i
+        while time.perf_counter() - t0 < budget:
+            if j % (len(experts) + 1) == 0:
+                oracle.swiglu(nn, sg, su, sd)
+                b += 2 * 3 * wl.Is * wl.H
+            else:
+                g, u, d = experts[j % (len(experts) + 1) - 1]
+                oracle.swiglu(nn, g, u, d)
+                b += 2 * 3 * wl.I * wl.H
+            j += 1
+        return b, time.perf_counter() - t0
+
+    for i in range(args.warmup):
+        one_step(i)
+    tot_b, tot_t = 0, 0.0
+    for i in range(args.steps):
+        b, t = one_step(i)
+        tot_b += b
+        tot_t += t
+    value = tot_b / tot_t / 1e9
+    cores = len(os.sched_getaffinity(0))
+    sample = (f"per step: RMSNorm + router of one row of {wl.name}, then SwiGLU experts (shared, "
+              f"then the row's 16 selected, cycling) for ~{budget:.3f} s; weights pre-generated "
+              f"on the host")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * tot_t / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(wl, "n/a (host)"),
+            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------------------
+
+def aggregate(local_bytes, local_ms, world):
+    """Whole-job totals: bytes summed over ranks, time = max over ranks."""
+    if world == 1:
+        return float(local_bytes), float(local_ms)
+    import torch
+    import torch.distributed as dist
+
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    b = torch.tensor([float(local_bytes)], dtype=torch.float64, device=dev)
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=dev)
+    dist.all_reduce(b, op=dist.ReduceOp.SUM)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(b.item()), float(t.item())
+
+
+def run_ours(args, wl):
+    import torch
+
+    import moe_decode_persistent_b200 as mdp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+
+    stream = torch.cuda.current_stream()
+    layers = [wl.device_layer(l, device=f"cuda:{local}") for l in range(wl.layers)]
+    h = mdp.MoeDecode(wl.H, wl.E, wl.k, wl.I, wl.Is, wl.B, layers, eps=wl.eps, device=local)
+    pool_host = wl.x_pool_host(POOL)
+    pool = torch.from_numpy(pool_host.view(np.int16)).view(torch.bfloat16).to(f"cuda:{local}")
+    y = torch.empty((wl.B, wl.H), dtype=torch.bfloat16, device=f"cuda:{local}")
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=f"cuda:{local}")
+    K, W = args.steps, args.warmup
+    nuniq = torch.zeros((K, wl.layers), dtype=torch.int32, device=f"cuda:{local}")
+
+    def dbg_for(i):
+        return [dict(n_unique=nuniq[i, l:l + 1]) for l in range(wl.layers)]
+
+    for i in range(W):
+        flush.zero_()
+        h.step(pool[i % POOL], y, wl.B, wl.k, stream=stream)
+    torch.cuda.synchronize()
+    if h.status() != 0:
+        raise RuntimeError("device status error during warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        h.step(pool[i % POOL], y, wl.B, wl.k, stream=stream, debug=dbg_for(i))
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    status = h.status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}: {mdp.strerror(status)}")
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    U = nuniq.cpu().numpy()
+    bytes_steps = [step_bytes(wl, list(U[i])) for i in range(K)]
+    local_ms = float(sum(step_ms))
+    tot_bytes, max_ms = aggregate(sum(bytes_steps), local_ms, world)
+    value = tot_bytes / (max_ms * 1e-3) / 1e9
+
+    # end to end through the host-buffer entry point: H2D x, step, D2H y per step
+    e2e = None
+    if not args.no_e2e:
+        xh = torch.from_numpy(pool_host.view(np.int16)).pin_memory()
+        yh = torch.empty((wl.B, wl.H), dtype=torch.int16).pin_memory()
+        for i in range(min(W, 10)):
+            h.step_host(xh[i % POOL], yh, wl.B, wl.k, stream=stream)
+        torch.cuda.synchronize()
+        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.zero_()
+            ee[i][0].record(stream)
+            h.step_host(xh[i % POOL], yh, wl.B, wl.k, stream=stream, debug=dbg_for(i))
+            ee[i][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        if h.status() != 0:
+            raise RuntimeError("device status error in the end-to-end loop")
+        e_ms = float(sum(a.elapsed_time(b) for a, b in ee))
+        U2 = nuniq.cpu().numpy()
+        e_bytes, e_max = aggregate(sum(step_bytes(wl, list(U2[i])) for i in range(K)), e_ms, world)
+        e2e = {"value": round(e_bytes / (e_max * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(xh[0].numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
+               "ms_per_step": round(e_max / K, 4)}
+
+    peak, peak_kind = measured_peaks()
+    achieved = sum(bytes_steps) / (local_ms * 1e-3) / 1e9  # per launch-stream, this rank
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        with open(tpath) as f:
+            t = json.load(f).get(wl.name)
+        traffic = None if t is None else t.get("bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": W, "ms_per_step": round(max_ms / K, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic: seeded counter-hash weights ~N(0,1/sqrt(fan_in)) and inputs, no trained weights",
+        "config": workload_config(wl, "flushed between timed steps (256 MB write)"),
+        "us_per_step": round(1e3 * max_ms / K, 2),
+        "tokens_per_s": round(world * wl.B * K / (max_ms * 1e-3), 1),
+        "unique_experts_mean": float(U.mean()),
+        "bytes_per_step_mean": float(np.mean(bytes_steps)),
+        "hbm_frac_of_peak": round(value / world / peak, 4),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
+                     "kernel": "moe_decode_layer_kernel"},
+        "e2e": e2e,
+        "gpu_launches": K * h.launches_per_step(),
+        "clocks": clocks,
+        "wall_s_timed_region": round(wall, 4),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, secs, steps = cpu_oracle_full_steps(wl, pool_host[:, :1], args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": round(gbs, 4), "unit": "GB/s", "cores": len(os.sched_getaffinity(0)),
+            "kind": "oracle",
+            "sample": f"{steps} full single-row layer steps of {wl.name} on distinct pool inputs "
+                      f"({secs:.1f} s of oracle time; host weight regeneration not timed)"}
+    h.close()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    wl = synth.WORKLOADS[args.config]
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+/*
+ * moe_decode.h - C ABI of the B200 (sm_100a) persistent MoE decode-layer step.
+ *
+ * One call of moe_decode_step runs one low-batch decode step (1..64 token rows)
+ * of a sparse mixture-of-experts transformer layer as ONE persistent kernel
+ * launch per layer: RMSNorm, router logits over all experts, top-k selection
+ * with softmax renormalisation, a unique-expert schedule, the shared expert
+ * (streamed while the routing resolves), the SwiGLU expert projections
+ * (gate/up, SiLU * up, down) over only the selected experts, and the weighted
+ * combine with the residual add.
+ *
+ * The method is the one the Kimi K3 decode pages describe: the per-layer chain
+ * of kernels replaced by fused, persistent work (page "Kimi K3推理吞吐提升1.68倍",
+ * section "为什么解码阶段适合Megakernel"); 896 experts with 16 active per token
+ * (page "vLLM 合併 Kimi K3 專用解碼：官方稱 GB300 快 1.5 到 2 倍，423 tok/s 怎麼核對",
+ * section "Kimi K3 專用解碼路徑改了什麼"); a batch-shape switch between small-matrix
+ * and split-K kernels, router scores, the shared expert beside the routing and an
+ * L2 prefetch of the next weights (page post.smzdm.com/p/a6zppe4g, section
+ * "改了什么：每层 23 个 kernel 砍到 13 个"). The layer's arithmetic is:
+ *
+ *   n    = bf16(x * rsqrt(mean(x^2) + eps) * gamma)        (fp32)
+ *   l[e] = n . W_r[e] (+ bias[e])                         (fp32 accumulate)
+ *   S    = top-k of l, ties to the lower expert index;  w = softmax(l[S])
+ *   h_e  = bf16(silu(W_g[e] n) * (W_u[e] n));  d_e = W_d[e] h_e
+ *   s    = W_sd bf16(silu(W_sg n) * (W_su n))
+ *   y    = bf16(x + s + sum_{e in S} w_e d_e)
+ *
+ * Conventions
+ *  - All tensors are row-major. bf16 = IEEE bfloat16 bit patterns.
+ *  - Device pointers are owned by the caller; the library never copies or
+ *    repacks weights and must not outlive them. The library owns only its
+ *    workspace (allocated by moe_decode_create, freed by moe_decode_destroy).
+ *  - Every function returns 0 on success or a negative MOE_ERR_* code; nothing
+ *    throws, exits or traps across this boundary.
+ *  - moe_decode_step is asynchronous on the caller's stream and allocates
+ *    nothing. Device-side failures (a bounded wait that ran out, a non-finite
+ *    router logit) are recorded in a status word read by moe_decode_get_status
+ *    after the stream has been synchronised.
+ *  - A handle is not thread-safe: use it from one host thread and one stream at
+ *    a time (steps on one handle must not overlap on the GPU).
+ */
+#ifndef MOE_DECODE_H
+#define MOE_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_OK 0
+#define MOE_ERR_INVALID_ARG (-1)        /* null pointer, bad size, batch/top_k out of range */
+#define MOE_ERR_UNSUPPORTED_ARCH (-2)   /* device is not sm_100 (B200) */
+#define MOE_ERR_UNSUPPORTED_SHAPE (-3)  /* dimensions the kernel does not tile (see create) */
+#define MOE_ERR_COOPERATIVE (-4)        /* cooperative launch unsupported or grid not co-resident */
+#define MOE_ERR_CUDA (-5)               /* a CUDA runtime/driver call failed */
+#define MOE_ERR_TIMEOUT (-6)            /* device status: a bounded wait ran out */
+#define MOE_ERR_NONFINITE (-7)          /* device status: a router logit was NaN or infinite */
+#define MOE_ERR_NO_MEMORY (-8)          /* workspace allocation failed */
+
+/* Layer dimensions, fixed at create time.
+ *  hidden        H   (multiple of 32; multiple of 256 or at most 256)
+ *  n_experts     E   (multiple of 32, at most 1024)
+ *  top_k_max     largest k a step may use (1..32, <= E)
+ *  inter         I   expert SwiGLU intermediate (multiple of 32; multiple of 256 or <= 256)
+ *  shared_inter  Is  shared-expert intermediate (same rule as inter)
+ *  max_batch     largest number of token rows per step (1..64)
+ *  n_layers      layers run back-to-back by one step (1..8); layer l+1's input is
+ *                layer l's output, and layer l prefetches layer l+1's router and
+ *                shared-expert weights into L2 while it finishes
+ *  eps           RMSNorm epsilon */
+typedef struct {
+  int hidden;
+  int n_experts;
+  int top_k_max;
+  int inter;
+  int shared_inter;
+  int max_batch;
+  int n_layers;
+  float eps;
+} moe_decode_config;
+
+/* Device pointers of one layer's parameters (bf16 unless noted). All must be
+ * 16-byte aligned. */
+typedef struct {
+  const void* gamma;        /* [H] RMSNorm gain */
+  const void* w_router;     /* [E][H] */
+  const float* router_bias; /* fp32 [E], or NULL for no bias */
+  const void* w_gate;       /* [E][I][H] */
+  const void* w_up;         /* [E][I][H] */
+  const void* w_down;       /* [E][H][I] */
+  const void* ws_gate;      /* [Is][H] */
+  const void* ws_up;        /* [Is][H] */
+  const void* ws_down;      /* [H][Is] */
+} moe_decode_layer_weights;
+
+/* Optional per-layer debug outputs of a step (device pointers; any may be NULL). */
+typedef struct {
+  float* logits;      /* fp32 [B][E]: router logits (bias included) */
+  int32_t* topk_idx;  /* int32 [B][k]: selected experts, descending logit, ties to lower index */
+  float* topk_w;      /* fp32 [B][k]: softmax weights of the selected experts */
+  int32_t* n_unique;  /* int32 [1]: number of distinct experts selected by the batch */
+} moe_decode_debug;
+
+typedef struct moe_decode_handle moe_decode_handle;
+
+/* Checks the device (sm_100, cooperative launch, one 1-CTA-per-SM persistent
+ * grid), validates the shapes, records the caller's weight pointers for
+ * cfg->n_layers layers (array `layers`), builds the TMA descriptors of every
+ * weight matrix and allocates the workspace on `device`. On success *out holds
+ * a handle owned by the caller (free it with moe_decode_destroy). */
+int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weights* layers,
+                      int device, moe_decode_handle** out);
+
+/* One decode step over all layers. x_in: device bf16 [batch][H]; y_out: device
+ * bf16 [batch][H] (may not alias x_in). 1 <= batch <= max_batch, 1 <= top_k <=
+ * top_k_max. stream: a cudaStream_t (NULL = legacy default stream). dbg: NULL or
+ * an array of n_layers debug records. Launches exactly one kernel per layer;
+ * returns MOE_ERR_* for argument errors and launch failures. */
+int moe_decode_step(moe_decode_handle* h, const void* x_in, void* y_out, int batch, int top_k,
+                    void* stream, const moe_decode_debug* dbg);
+
+/* Same step on HOST buffers: copies x_host (bf16 [batch][H], preferably pinned)
+ * to the device, runs the step and copies the result back into y_host, all
+ * asynchronous on `stream` (synchronise before reading y_host). Uses staging
+ * buffers inside the handle's workspace. */
+int moe_decode_step_host(moe_decode_handle* h, const void* x_host, void* y_host, int batch,
+                         int top_k, void* stream, const moe_decode_debug* dbg);
+
+/* Reads and clears the device status word of the last completed steps (call
+ * after synchronising the stream). *device_status receives MOE_OK or the
+ * first device-side MOE_ERR_* recorded. The return value reports whether the
+ * read itself succeeded. */
+int moe_decode_get_status(moe_decode_handle* h, int* device_status);
+
+/* Number of kernel launches one moe_decode_step makes (= n_layers). */
+int moe_decode_launches_per_step(const moe_decode_handle* h);
+
+/* Sets debug behaviour of later steps (tests only): bit 0 = per-CTA random
+ * __nanosleep jitter at unit boundaries; bit 1 = withhold the normalised-row
+ * ready signal so that every waiting CTA's bounded wait runs out. wait_ms is the
+ * bound of every device-side wait (default 2000 ms). */
+int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms);
+
+void moe_decode_destroy(moe_decode_handle* h);
+
+const char* moe_decode_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_DECODE_H */

@@ -1,0 +1,206 @@
+"""Python binding of the B200 persistent MoE decode-layer step (include/moe_decode.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels of
+``libmoe_decode.so``. There is no CPU or PyTorch fallback; constructing a
+``MoeDecode`` without the built library or without a B200 raises.
+
+PyTorch is used by callers for device memory and streams; this module accepts
+either torch tensors or raw device pointers (ints).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+import subprocess
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(_HERE)
+LIB = os.path.join(_HERE, "libmoe_decode.so")
+HEADER = os.path.join(ROOT, "include", "moe_decode.h")
+SOURCES = [os.path.join(_HERE, "csrc", f) for f in ("moe_decode_kernel.cu", "moe_decode_api.cu")]
+
+MOE_OK = 0
+MOE_ERR_INVALID_ARG = -1
+MOE_ERR_UNSUPPORTED_ARCH = -2
+MOE_ERR_UNSUPPORTED_SHAPE = -3
+MOE_ERR_COOPERATIVE = -4
+MOE_ERR_CUDA = -5
+MOE_ERR_TIMEOUT = -6
+MOE_ERR_NONFINITE = -7
+MOE_ERR_NO_MEMORY = -8
+
+DEBUG_JITTER = 1
+DEBUG_WITHHOLD_NREADY = 2
+
+
+def nvcc_command(out: str = LIB) -> list[str]:
+    return ["nvcc", "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
+            "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+            "-I" + os.path.join(ROOT, "include"), "-o", out, *SOURCES]
+
+
+def build(verbose: bool = False) -> None:
+    """Compile libmoe_decode.so in-tree for sm_100a."""
+    cmd = nvcc_command()
+    if verbose:
+        print(" ".join(cmd))
+    subprocess.run(cmd, check=True, cwd=_HERE)
+
+
+def declared_symbols() -> list[str]:
+    """Function names declared by include/moe_decode.h."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"\b(moe_decode_[a-z_]+)\s*\(", text)))
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int), ("n_experts", ctypes.c_int), ("top_k_max", ctypes.c_int),
+                ("inter", ctypes.c_int), ("shared_inter", ctypes.c_int), ("max_batch", ctypes.c_int),
+                ("n_layers", ctypes.c_int), ("eps", ctypes.c_float)]
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [("gamma", ctypes.c_void_p), ("w_router", ctypes.c_void_p),
+                ("router_bias", ctypes.c_void_p), ("w_gate", ctypes.c_void_p),
+                ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
+                ("ws_gate", ctypes.c_void_p), ("ws_up", ctypes.c_void_p),
+                ("ws_down", ctypes.c_void_p)]
+
+
+class Debug(ctypes.Structure):
+    _fields_ = [("logits", ctypes.c_void_p), ("topk_idx", ctypes.c_void_p),
+                ("topk_w", ctypes.c_void_p), ("n_unique", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded C-ABI library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise RuntimeError(f"{LIB} is missing: build it with moe_decode_persistent_b200.build()")
+        L = ctypes.CDLL(LIB)
+        vp, i, u = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
+        L.moe_decode_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerWeights), i,
+                                        ctypes.POINTER(vp)]
+        L.moe_decode_create.restype = i
+        L.moe_decode_step.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.moe_decode_step.restype = i
+        L.moe_decode_step_host.argtypes = [vp, vp, vp, i, i, vp, vp]
+        L.moe_decode_step_host.restype = i
+        L.moe_decode_get_status.argtypes = [vp, ctypes.POINTER(i)]
+        L.moe_decode_get_status.restype = i
+        L.moe_decode_launches_per_step.argtypes = [vp]
+        L.moe_decode_launches_per_step.restype = i
+        L.moe_decode_set_debug.argtypes = [vp, u, u]
+        L.moe_decode_set_debug.restype = i
+        L.moe_decode_destroy.argtypes = [vp]
+        L.moe_decode_destroy.restype = None
+        L.moe_decode_strerror.argtypes = [i]
+        L.moe_decode_strerror.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def strerror(code: int) -> str:
+    return lib().moe_decode_strerror(int(code)).decode()
+
+
+class MoeDecodeError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {strerror(code)} ({code})")
+        self.code = code
+
+
+def _check(code: int, what: str) -> None:
+    if code != MOE_OK:
+        raise MoeDecodeError(code, what)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return int(t.data_ptr())
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        return None
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+class MoeDecode:
+    """Handle of one configured decode layer stack on one device.
+
+    layers: sequence of mappings with keys gamma, w_router, router_bias (or None),
+    w_gate, w_up, w_down, ws_gate, ws_up, ws_down (torch tensors or device pointers).
+    The caller keeps those tensors alive for the handle's lifetime.
+    """
+
+    def __init__(self, hidden, n_experts, top_k_max, inter, shared_inter, max_batch, layers,
+                 eps=1e-6, device=0):
+        self.cfg = Config(hidden, n_experts, top_k_max, inter, shared_inter, max_batch,
+                          len(layers), eps)
+        arr = (LayerWeights * len(layers))()
+        for i, w in enumerate(layers):
+            arr[i] = LayerWeights(*(_ptr(w.get(name)) for name, _ in LayerWeights._fields_))
+        self._weights_keepalive = layers
+        h = ctypes.c_void_p()
+        _check(lib().moe_decode_create(ctypes.byref(self.cfg), arr, int(device), ctypes.byref(h)),
+               "moe_decode_create")
+        self.handle = h
+        self.n_layers = len(layers)
+
+    def step(self, x, y, batch, top_k, stream=None, debug=None) -> None:
+        """y <- layer stack(x); x, y device bf16 [batch, hidden]; asynchronous on `stream`."""
+        dbg = self._debug(debug)
+        _check(lib().moe_decode_step(self.handle, _ptr(x), _ptr(y), int(batch), int(top_k),
+                                     _stream_handle(stream), dbg), "moe_decode_step")
+
+    def step_host(self, x_host, y_host, batch, top_k, stream=None, debug=None) -> None:
+        """Same step on host buffers (pinned torch CPU tensors or host pointers)."""
+        dbg = self._debug(debug)
+        _check(lib().moe_decode_step_host(self.handle, _ptr(x_host), _ptr(y_host), int(batch),
+                                          int(top_k), _stream_handle(stream), dbg),
+               "moe_decode_step_host")
+
+    def _debug(self, debug):
+        if debug is None:
+            return None
+        arr = (Debug * self.n_layers)()
+        for i, d in enumerate(debug):
+            if d is not None:
+                arr[i] = Debug(_ptr(d.get("logits")), _ptr(d.get("topk_idx")),
+                               _ptr(d.get("topk_w")), _ptr(d.get("n_unique")))
+        self._dbg_keepalive = (arr, debug)
+        return ctypes.cast(arr, ctypes.c_void_p)
+
+    def status(self) -> int:
+        """Device status of the completed steps (MOE_OK or a MOE_ERR_* code); clears it."""
+        v = ctypes.c_int(0)
+        _check(lib().moe_decode_get_status(self.handle, ctypes.byref(v)), "moe_decode_get_status")
+        return v.value
+
+    def launches_per_step(self) -> int:
+        return lib().moe_decode_launches_per_step(self.handle)
+
+    def set_debug(self, flags: int, wait_ms: int = 2000) -> None:
+        _check(lib().moe_decode_set_debug(self.handle, int(flags), int(wait_ms)), "moe_decode_set_debug")
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            lib().moe_decode_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,349 @@
+// moe_decode_api.cu - the C ABI (include/moe_decode.h): handle creation, TMA
+// descriptors, workspace, per-layer cooperative launches, status.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "kernel_params.h"
+#include "moe_decode.h"
+
+namespace moe {
+size_t smem_bytes();
+int threads_per_cta();
+const void* kernel_fn();
+}  // namespace moe
+
+using moe::Params;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct moe_decode_handle {
+  moe_decode_config cfg;
+  int device;
+  int num_sms;
+  moe_decode_layer_weights* layers;
+  CUtensorMap* d_tmaps;  // [n_layers][TM_COUNT]
+  // workspace
+  void* ws;              // one allocation, carved below
+  uint16_t* n;
+  float* logits;
+  uint16_t* hs;
+  uint16_t* he;
+  float* partial;
+  uint32_t* ctr;
+  uint32_t* tickets;
+  uint32_t* pair_done;
+  int* status;
+  uint16_t* layer_io;    // [n_layers - 1][max_batch][H] intermediate outputs
+  uint16_t* x_stage;     // [max_batch][H] host-step staging
+  uint16_t* y_stage;
+  unsigned max_units, max_tiles;
+  unsigned flags;
+  unsigned long long wait_ns;
+};
+
+static int cuda_fail(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static bool tile_dim_ok(int v) { return v >= 32 && v % 32 == 0 && (v % 256 == 0 || v <= 256); }
+
+static int encode_2d(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint64_t rows,
+                     uint64_t cols) {
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return MOE_ERR_INVALID_ARG;
+  const uint32_t box_cols = cols < (uint64_t)moe::kBoxColsMax ? (uint32_t)cols : (uint32_t)moe::kBoxColsMax;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, (cuuint32_t)moe::kBoxRows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+extern "C" {
+
+const char* moe_decode_strerror(int code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_ARCH: return "device is not an sm_100 (B200) GPU";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported layer shape";
+    case MOE_ERR_COOPERATIVE: return "cooperative persistent launch not possible on this device";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_NONFINITE: return "non-finite router logit";
+    case MOE_ERR_NO_MEMORY: return "workspace allocation failed";
+    default: return "unknown error";
+  }
+}
+
+int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weights* layers,
+                      int device, moe_decode_handle** out) {
+  if (!cfg || !layers || !out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  const moe_decode_config c = *cfg;
+  if (c.n_layers < 1 || c.n_layers > 8 || c.max_batch < 1 || c.max_batch > 64 || c.top_k_max < 1 ||
+      c.top_k_max > 32 || c.top_k_max > c.n_experts || !(c.eps >= 0.0f))
+    return MOE_ERR_INVALID_ARG;
+  if (c.max_batch * c.top_k_max > moe::kMaxSlots) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!tile_dim_ok(c.hidden) || !tile_dim_ok(c.inter) || !tile_dim_ok(c.shared_inter) ||
+      c.n_experts < 32 || c.n_experts % 32 != 0 || c.n_experts > moe::kMaxE)
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  for (int l = 0; l < c.n_layers; ++l) {
+    const moe_decode_layer_weights& w = layers[l];
+    if (!w.gamma || !w.w_router || !w.w_gate || !w.w_up || !w.w_down || !w.ws_gate || !w.ws_up ||
+        !w.ws_down)
+      return MOE_ERR_INVALID_ARG;
+  }
+
+  cudaError_t e = cudaSetDevice(device);
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  int major = 0, minor = 0, coop = 0, sms = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device);
+  cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, device);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+  if (major != 10 || minor != 0) return MOE_ERR_UNSUPPORTED_ARCH;
+  if (!coop) return MOE_ERR_COOPERATIVE;
+
+  const size_t smem = moe::smem_bytes();
+  e = cudaFuncSetAttribute(moe::kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return MOE_ERR_COOPERATIVE;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe::kernel_fn(), moe::threads_per_cta(),
+                                                    smem);
+  if (e != cudaSuccess || per_sm < 1) return MOE_ERR_COOPERATIVE;
+
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return MOE_ERR_CUDA;
+  EncodeTiledFn enc = reinterpret_cast<EncodeTiledFn>(fn);
+
+  moe_decode_handle* h = (moe_decode_handle*)calloc(1, sizeof(moe_decode_handle));
+  if (!h) return MOE_ERR_NO_MEMORY;
+  h->cfg = c;
+  h->device = device;
+  h->num_sms = sms;
+  h->wait_ns = 2000ull * 1000000ull;
+  h->layers = (moe_decode_layer_weights*)malloc(sizeof(moe_decode_layer_weights) * c.n_layers);
+  memcpy(h->layers, layers, sizeof(moe_decode_layer_weights) * c.n_layers);
+
+  const int H = c.hidden, E = c.n_experts, I = c.inter, Is = c.shared_inter, L = c.n_layers;
+  // host tensor maps
+  CUtensorMap* maps = (CUtensorMap*)aligned_alloc(64, sizeof(CUtensorMap) * moe::TM_COUNT * L);
+  int rc = MOE_OK;
+  for (int l = 0; l < L && rc == MOE_OK; ++l) {
+    const moe_decode_layer_weights& w = layers[l];
+    CUtensorMap* m = maps + l * moe::TM_COUNT;
+    rc |= encode_2d(enc, &m[moe::TM_WR], w.w_router, (uint64_t)E, (uint64_t)H);
+    rc |= encode_2d(enc, &m[moe::TM_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H);
+    rc |= encode_2d(enc, &m[moe::TM_WU], w.w_up, (uint64_t)E * I, (uint64_t)H);
+    rc |= encode_2d(enc, &m[moe::TM_WD], w.w_down, (uint64_t)E * H, (uint64_t)I);
+    rc |= encode_2d(enc, &m[moe::TM_WSG], w.ws_gate, (uint64_t)Is, (uint64_t)H);
+    rc |= encode_2d(enc, &m[moe::TM_WSU], w.ws_up, (uint64_t)Is, (uint64_t)H);
+    rc |= encode_2d(enc, &m[moe::TM_WSD], w.ws_down, (uint64_t)H, (uint64_t)Is);
+  }
+  if (rc != MOE_OK) {
+    free(maps);
+    free(h->layers);
+    free(h);
+    return rc < 0 ? MOE_ERR_INVALID_ARG : rc;
+  }
+
+  // workspace bounds (see the unit enumeration in the kernel)
+  const int maxB = c.max_batch, maxSlots = c.max_batch * c.top_k_max;
+  const int GB = (maxB + moe::kActGroup - 1) / moe::kActGroup;
+  const int boxH = H < moe::kBoxColsMax ? H : moe::kBoxColsMax;
+  const int nkbH = H / boxH;
+  const int KS = nkbH < 4 ? nkbH : 4;
+  const int RT = E / 32, ST = Is / 32, IT = I / 32, DT = H / 32;
+  const int maxP = maxSlots;
+  h->max_units = (unsigned)(GB * RT * KS + GB * ST * KS + maxP * IT * KS +
+                            DT * (GB + (maxP + moe::kDownPairsPerSplit - 1) / moe::kDownPairsPerSplit));
+  h->max_tiles = (unsigned)(GB * (RT + ST) + maxP * IT + DT);
+
+  size_t off = 0;
+  auto carve = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_n = carve((size_t)maxB * H * 2);
+  const size_t o_logits = carve((size_t)maxB * E * 4);
+  const size_t o_hs = carve((size_t)maxB * Is * 2);
+  const size_t o_he = carve((size_t)moe::kMaxSlots * I * 2);
+  const size_t o_part = carve((size_t)h->max_units * moe::kPartialFloats * 4);
+  const size_t o_ctr = carve(moe::CTR_COUNT * 4);
+  const size_t o_tix = carve((size_t)h->max_tiles * 4);
+  const size_t o_pd = carve(moe::kMaxSlots * 4);
+  const size_t o_status = carve(16);
+  const size_t o_io = carve((size_t)(L > 1 ? L - 1 : 1) * maxB * H * 2);
+  const size_t o_xs = carve((size_t)maxB * H * 2);
+  const size_t o_ys = carve((size_t)maxB * H * 2);
+  const size_t o_maps = carve(sizeof(CUtensorMap) * moe::TM_COUNT * L);
+  e = cudaMalloc(&h->ws, off);
+  if (e != cudaSuccess) {
+    free(maps);
+    free(h->layers);
+    free(h);
+    return MOE_ERR_NO_MEMORY;
+  }
+  uint8_t* b = (uint8_t*)h->ws;
+  h->n = (uint16_t*)(b + o_n);
+  h->logits = (float*)(b + o_logits);
+  h->hs = (uint16_t*)(b + o_hs);
+  h->he = (uint16_t*)(b + o_he);
+  h->partial = (float*)(b + o_part);
+  h->ctr = (uint32_t*)(b + o_ctr);
+  h->tickets = (uint32_t*)(b + o_tix);
+  h->pair_done = (uint32_t*)(b + o_pd);
+  h->status = (int*)(b + o_status);
+  h->layer_io = (uint16_t*)(b + o_io);
+  h->x_stage = (uint16_t*)(b + o_xs);
+  h->y_stage = (uint16_t*)(b + o_ys);
+  h->d_tmaps = (CUtensorMap*)(b + o_maps);
+  // counters, tickets, flags and status start at zero; activations zeroed for hygiene
+  e = cudaMemset(h->ws, 0, off);
+  if (e == cudaSuccess)
+    e = cudaMemcpy(h->d_tmaps, maps, sizeof(CUtensorMap) * moe::TM_COUNT * L, cudaMemcpyHostToDevice);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  free(maps);
+  if (e != cudaSuccess) {
+    cudaFree(h->ws);
+    free(h->layers);
+    free(h);
+    return MOE_ERR_CUDA;
+  }
+  *out = h;
+  return MOE_OK;
+}
+
+static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, int batch, int top_k,
+                         cudaStream_t stream, const moe_decode_debug* dbg) {
+  const moe_decode_config& c = h->cfg;
+  const int L = c.n_layers;
+  for (int l = 0; l < L; ++l) {
+    Params p;
+    memset(&p, 0, sizeof p);
+    p.H = c.hidden;
+    p.E = c.n_experts;
+    p.I = c.inter;
+    p.Is = c.shared_inter;
+    p.B = batch;
+    p.k = top_k;
+    p.eps = c.eps;
+    p.x = l == 0 ? (const uint16_t*)x_in : h->layer_io + (size_t)(l - 1) * c.max_batch * c.hidden;
+    p.y = l == L - 1 ? (uint16_t*)y_out : h->layer_io + (size_t)l * c.max_batch * c.hidden;
+    const moe_decode_layer_weights& w = h->layers[l];
+    p.tmaps = h->d_tmaps + l * moe::TM_COUNT;
+    p.gamma = (const uint16_t*)w.gamma;
+    p.bias = w.router_bias;
+    if (l + 1 < L) {
+      const moe_decode_layer_weights& nx = h->layers[l + 1];
+      p.pf_ptr[0] = nx.w_router;
+      p.pf_bytes[0] = (unsigned long long)c.n_experts * c.hidden * 2;
+      p.pf_ptr[1] = nx.ws_gate;
+      p.pf_bytes[1] = (unsigned long long)c.shared_inter * c.hidden * 2;
+      p.pf_ptr[2] = nx.ws_up;
+      p.pf_bytes[2] = (unsigned long long)c.shared_inter * c.hidden * 2;
+      p.pf_ptr[3] = nx.ws_down;
+      p.pf_bytes[3] = (unsigned long long)c.shared_inter * c.hidden * 2;
+    }
+    p.n = h->n;
+    p.logits = h->logits;
+    p.hs = h->hs;
+    p.he = h->he;
+    p.partial = h->partial;
+    p.ctr = h->ctr;
+    p.tickets = h->tickets;
+    p.pair_done = h->pair_done;
+    p.status = h->status;
+    p.max_units = h->max_units;
+    p.max_tiles = h->max_tiles;
+    if (dbg) {
+      p.dbg_logits = dbg[l].logits;
+      p.dbg_idx = dbg[l].topk_idx;
+      p.dbg_w = dbg[l].topk_w;
+      p.dbg_nuniq = dbg[l].n_unique;
+    }
+    p.flags = h->flags;
+    p.wait_ns = h->wait_ns;
+    void* args[] = {&p};
+    cudaError_t e = cudaLaunchCooperativeKernel(moe::kernel_fn(), dim3(h->num_sms), dim3(moe::threads_per_cta()),
+                                                args, moe::smem_bytes(), stream);
+    if (e == cudaErrorCooperativeLaunchTooLarge) return MOE_ERR_COOPERATIVE;
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+static int check_step_args(moe_decode_handle* h, const void* x, void* y, int batch, int top_k) {
+  if (!h || !x || !y || x == y) return MOE_ERR_INVALID_ARG;
+  if (batch < 1 || batch > h->cfg.max_batch || top_k < 1 || top_k > h->cfg.top_k_max ||
+      top_k > h->cfg.n_experts)
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+int moe_decode_step(moe_decode_handle* h, const void* x_in, void* y_out, int batch, int top_k,
+                    void* stream, const moe_decode_debug* dbg) {
+  int rc = check_step_args(h, x_in, y_out, batch, top_k);
+  if (rc != MOE_OK) return rc;
+  if ((reinterpret_cast<uintptr_t>(x_in) & 15u) || (reinterpret_cast<uintptr_t>(y_out) & 15u))
+    return MOE_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_layers(h, x_in, y_out, batch, top_k, (cudaStream_t)stream, dbg);
+}
+
+int moe_decode_step_host(moe_decode_handle* h, const void* x_host, void* y_host, int batch,
+                         int top_k, void* stream, const moe_decode_debug* dbg) {
+  int rc = check_step_args(h, x_host, y_host, batch, top_k);
+  if (rc != MOE_OK) return rc;
+  if (cudaSetDevice(h->device) != cudaSuccess) return MOE_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t bytes = (size_t)batch * h->cfg.hidden * 2;
+  if (cudaMemcpyAsync(h->x_stage, x_host, bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  rc = launch_layers(h, h->x_stage, h->y_stage, batch, top_k, s, dbg);
+  if (rc != MOE_OK) return rc;
+  return cuda_fail(cudaMemcpyAsync(y_host, h->y_stage, bytes, cudaMemcpyDeviceToHost, s));
+}
+
+int moe_decode_get_status(moe_decode_handle* h, int* device_status) {
+  if (!h || !device_status) return MOE_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, h->status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0 && cudaMemset(h->status, 0, sizeof v) != cudaSuccess) return MOE_ERR_CUDA;
+  *device_status = v;
+  return MOE_OK;
+}
+
+int moe_decode_launches_per_step(const moe_decode_handle* h) {
+  return h ? h->cfg.n_layers : MOE_ERR_INVALID_ARG;
+}
+
+int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms) {
+  if (!h || wait_ms == 0) return MOE_ERR_INVALID_ARG;
+  h->flags = flags;
+  h->wait_ns = (unsigned long long)wait_ms * 1000000ull;
+  return MOE_OK;
+}
+
+void moe_decode_destroy(moe_decode_handle* h) {
+  if (!h) return;
+  cudaSetDevice(h->device);
+  cudaFree(h->ws);
+  free(h->layers);
+  free(h);
+}
+
+}  // extern "C"

@@ -250,6 +250,32 @@ class Workload:
             ("ws_down", KIND_WS_DOWN, H * Is, sigma_for(Is), 0.0),
         ]
 
+    def device_layer(self, layer: int, device="cuda", stream: int = 0) -> dict:
+        """All of one layer's parameters generated on the device (torch tensors).
+
+        bf16 tensors are returned as torch.bfloat16 holding exactly the bit
+        patterns of the host generator; the router bias (zipf workloads) as fp32.
+        """
+        import torch
+
+        out = {}
+        for name, kind, numel, sigma, mean in self.device_specs(layer):
+            t = torch.empty(int(numel), dtype=torch.bfloat16, device=device)
+            fill_device(t.data_ptr(), self.seed, tensor_id(layer, kind), 0, int(numel), sigma, mean,
+                        stream)
+            out[name] = t
+        H, E, I, Is = self.H, self.E, self.I, self.Is
+        out["w_router"] = out["w_router"].view(E, H)
+        out["w_gate"] = out["w_gate"].view(E, I, H)
+        out["w_up"] = out["w_up"].view(E, I, H)
+        out["w_down"] = out["w_down"].view(E, H, I)
+        out["ws_gate"] = out["ws_gate"].view(Is, H)
+        out["ws_up"] = out["ws_up"].view(Is, H)
+        out["ws_down"] = out["ws_down"].view(H, Is)
+        bias = self.bias_host(layer)
+        out["router_bias"] = None if bias is None else torch.from_numpy(bias).to(device)
+        return out
+
     def weight_bytes_per_layer(self) -> int:
         return 2 * sum(s[2] for s in self.device_specs(0))
 

@@ -1,0 +1,188 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small workloads run the oracle on every row; they span several tiles, K splits
+and ragged tails (batch not a multiple of the row group, odd k, k = E, k = 1,
+a skewed router, correlated rows, two layers). The five measured workloads run
+at full size with the oracle on sampled rows (rows are independent) plus
+properties checked on every row.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+from harness import bf, check_layer, check_y, make_handle, oracle_rows, run_gpu
+
+torch = pytest.importorskip("torch")
+
+pytestmark = pytest.mark.gpu
+
+W = synth.Workload
+SMALL = [
+    synth.WORKLOADS[0],
+    W("ragged_b5_k6", B=5, H=1024, E=96, k=6, I=256, Is=512, seed=21),
+    W("b13_k3", B=13, H=512, E=64, k=3, I=128, Is=256, seed=22),
+    W("b64_k16", B=64, H=256, E=64, k=16, I=128, Is=128, seed=23),
+    W("k_equals_E", B=2, H=256, E=32, k=32, I=64, Is=64, seed=24),
+    W("zipf_b16", B=16, H=512, E=128, k=8, I=256, Is=256, seed=25, router="zipf"),
+    W("corr_2layer", B=8, H=512, E=64, k=4, I=128, Is=256, seed=26, layers=2, rows="correlated",
+      nseq=2, rows_per_seq=4),
+    W("b1_k1", B=1, H=256, E=32, k=1, I=32, Is=32, seed=27),
+    W("b7_h2048", B=7, H=2048, E=64, k=5, I=512, Is=768 - 256, seed=28),
+]
+
+
+def _layers(wl):
+    return [wl.device_layer(l) for l in range(wl.layers)]
+
+
+def _free():
+    import gc
+
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+@pytest.fixture(autouse=True)
+def _cuda_only():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    yield
+    _free()
+
+
+def run_and_check(wl, rows=None, handle=None, layers=None):
+    layers = layers if layers is not None else _layers(wl)
+    h = handle or make_handle(wl, layers)
+    x = wl.x_host()
+    out = run_gpu(h, wl, x, n_layers=wl.layers)
+    assert out["status"] == 0, f"device status {out['status']}"
+    rows = list(range(wl.B)) if rows is None else rows
+    orc = oracle_rows(wl, x, rows, n_layers=wl.layers)
+    skip = set()
+    for l in range(wl.layers):
+        ties = check_layer(out["layers"][l], orc[l], rows, wl.k, tag=f"{wl.name} layer {l}")
+        skip |= {rows.index(b) for b in ties}
+        idx = out["layers"][l]["idx"]
+        assert out["layers"][l]["U"] == len(np.unique(idx)), "unique-expert count"
+    err = check_y(out["y"][rows], orc[-1]["y"], tag=wl.name, skip=skip)
+    if handle is None:
+        h.close()
+    return out, err
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=[w.name for w in SMALL])
+def test_small_workloads_match_oracle(wl):
+    run_and_check(wl)
+
+
+def test_device_generator_matches_host():
+    wl = W("gen", B=1, H=512, E=32, k=2, I=128, Is=256, seed=99)
+    lay = wl.device_layer(0)
+    rng = np.random.default_rng(0)
+    for name, kind, numel, sigma, mean in wl.device_specs(0):
+        t = lay[name].reshape(-1)
+        for start in rng.integers(0, max(1, numel - 300), 3):
+            got = t[int(start):int(start) + 300].view(torch.int16).cpu().numpy().view(np.uint16)
+            want = synth.fill_host(wl.seed, synth.tensor_id(0, kind), int(start), len(got), sigma, mean)
+            assert np.array_equal(got, want), name
+
+
+def test_bitwise_deterministic_and_jitter_invariant():
+    import moe_decode_persistent_b200 as mdp
+
+    wl = SMALL[1]
+    layers = _layers(wl)
+    h = make_handle(wl, layers)
+    x = wl.x_host()
+    a = run_gpu(h, wl, x)
+    b = run_gpu(h, wl, x)
+    h.set_debug(mdp.DEBUG_JITTER)
+    c = run_gpu(h, wl, x)
+    h.set_debug(0)
+    for o in (a, b, c):
+        assert o["status"] == 0
+    assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["y"], c["y"])
+    assert np.array_equal(a["layers"][0]["logits"], c["layers"][0]["logits"])
+    h.close()
+
+
+def test_timeout_is_reported_and_handle_recovers():
+    import moe_decode_persistent_b200 as mdp
+
+    wl = SMALL[2]
+    layers = _layers(wl)
+    h = make_handle(wl, layers)
+    x = wl.x_host()
+    h.set_debug(mdp.DEBUG_WITHHOLD_NREADY, wait_ms=300)
+    bad = run_gpu(h, wl, x)
+    assert bad["status"] == mdp.MOE_ERR_TIMEOUT
+    h.set_debug(0)
+    good = run_and_check(wl, handle=h, layers=layers)[0]
+    assert good["status"] == 0
+    h.close()
+
+
+def test_host_entry_point_matches_device_entry_point():
+    wl = SMALL[1]
+    layers = _layers(wl)
+    h = make_handle(wl, layers)
+    x = wl.x_host()
+    dev = run_gpu(h, wl, x)
+    xh = torch.from_numpy(x.view(np.int16)).pin_memory()
+    yh = torch.empty_like(xh).pin_memory()
+    h.step_host(xh, yh, wl.B, wl.k, stream=torch.cuda.current_stream())
+    torch.cuda.synchronize()
+    assert h.status() == 0
+    assert np.array_equal(yh.numpy().view(np.uint16), dev["y"])
+    h.close()
+
+
+def test_smaller_batch_and_k_than_configured():
+    wl = SMALL[1]
+    layers = _layers(wl)
+    h = make_handle(wl, layers)
+    sub = dataclasses.replace(wl, B=3, k=4)
+    out, _ = run_and_check(sub, handle=h, layers=layers)
+    assert h.launches_per_step() == 1
+    h.close()
+
+
+FULL = [1, 2, 3, 4]
+SAMPLE_ROWS = {1: [0], 2: [0, 5], 3: [0, 37, 63], 4: [0, 9, 31]}
+
+
+@pytest.mark.parametrize("cfg", FULL)
+def test_full_size_workload(cfg):
+    wl = synth.WORKLOADS[cfg]
+    layers = _layers(wl)
+    h = make_handle(wl, layers)
+    x = wl.x_host()
+    out = run_gpu(h, wl, x, n_layers=wl.layers)
+    assert out["status"] == 0
+    assert h.launches_per_step() == wl.layers
+    # every row: indices equal the oracle's top-k of the GPU's own logits; weights sum to 1
+    for l in range(wl.layers):
+        lay = out["layers"][l]
+        for b in range(wl.B):
+            assert np.array_equal(lay["idx"][b], oracle.topk(lay["logits"][b], wl.k))
+        np.testing.assert_allclose(lay["w"].sum(axis=1), 1.0, atol=1e-5)
+        assert lay["U"] == len(np.unique(lay["idx"]))
+    # every row of layer 0: logits against the oracle router
+    gamma, wr, bias = wl.gamma_host(0), wl.w_router_host(0), wl.bias_host(0)
+    for b in range(wl.B):
+        lo = oracle.router(oracle.rmsnorm(x[b], gamma, wl.eps), wr, bias)
+        lg = out["layers"][0]["logits"][b].astype(np.float64)
+        assert np.max(np.abs(lg - lo)) <= 1e-3 * np.max(np.abs(lo))
+    # sampled rows: the whole layer stack against the oracle
+    rows = SAMPLE_ROWS[cfg]
+    orc = oracle_rows(wl, x, rows, n_layers=wl.layers)
+    skip = set()
+    for l in range(wl.layers):
+        ties = check_layer(out["layers"][l], orc[l], rows, wl.k, tag=f"{wl.name} layer {l}")
+        skip |= {rows.index(b) for b in ties}
+    check_y(out["y"][rows], orc[-1]["y"], tag=wl.name, skip=skip)
+    h.close()
