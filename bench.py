@@ -67,7 +67,7 @@ def step_bytes(wl, n_unique_per_layer, batch=None):
     per_layer_fixed = 2 * (E * H + 3 * Is * H + H) + (4 * E if wl.router == "zipf" else 0)
     total = 0
     for U in n_unique_per_layer:
-        total += per_layer_fixed + U * 3 * I * H * 2 + 2 * B * H * 2
+        total += per_layer_fixed + int(U) * 3 * I * H * 2 + 2 * B * H * 2
     return total
 
 

@@ -815,6 +815,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
       if (u >= pre && !sched_ready) {
         ok = wait_bar(&sm.empty[slot], phase ^ 1u);
         if (!ok) break;
+        last_tx_parity[slot] = -1;  // the slot's previous stage was consumed
         if (lane == 0) {
           sm.hdr[slot].kind = HK_SCHED;
           mbar_arrive(&sm.full[slot]);
@@ -909,13 +910,16 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
     }
     // tell the consumers to stop (bounded)
     if (wait_bar(&sm.empty[slot], phase ^ 1u)) {
+      last_tx_parity[slot] = -1;
       if (lane == 0) {
         sm.hdr[slot].kind = HK_END;
         mbar_arrive(&sm.full[slot]);
       }
     }
     __syncwarp();
-    // drain: every issued bulk copy must have landed before the CTA exits
+    // drain: every issued bulk copy must have landed before the CTA exits. A slot's
+    // record is the phase of its last TMA stage that no later use of the slot has
+    // shown to be complete (only possible after an abort).
     if (lane == 0) {
       for (int s = 0; s < kStages; ++s) {
         if (last_tx_parity[s] < 0) continue;

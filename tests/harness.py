@@ -3,9 +3,15 @@ it with the fp64 oracle. Tolerances:
 
 * router logits, per row:  max_e |l_gpu - l_orc| <= 1e-3 * max_e |l_orc|
 * expert indices:          idx_gpu == oracle top-k of the GPU's own fp32 logits (exact)
-* routing weights:         |w_gpu - softmax(l_orc[idx_gpu])| <= 1e-5 + 1e-4 |w|
+* routing weights:         |w_gpu - softmax(l_orc[idx_gpu])| <= w (2.2 d + 1e-5) + 1e-6, where
+                           d = max_e |l_gpu - l_orc| of the row: a softmax weight moves by at
+                           most a factor exp(2 d) when every logit moves by at most d (a layer
+                           after the first sees inputs that may differ by one bf16 step)
 * layer output:            max |y_gpu - y_orc| <= 2e-2 * max |y_orc|       (the stated bar)
-                           and, tighter, |y_gpu - y_orc| <= ulp_bf16(y_orc) + 1e-3
+                           and, tighter, |y_gpu - y_orc| <= sum_l ulp_bf16(y_orc,l) + 1e-3 over
+                           the layers l (the residual add passes a layer's output rounding on
+                           at that layer's magnitude), plus 5e-3 per layer after the first for
+                           the MoE path's response to those flips
   The tight bound follows from the arithmetic: both sides round the same
   pre-rounding value to bf16 once, and the GPU's fp32 accumulation over at
   most 7168 products of magnitude ~1/sqrt(fan_in) errs by ~1e-5, so outputs
@@ -85,7 +91,9 @@ def check_layer(gpu_layer, orc, rows, k, tag=""):
         want = oracle.topk(gpu_layer["logits"][b], k)
         assert np.array_equal(gpu_layer["idx"][b], want), f"{tag}: row {b} idx {gpu_layer['idx'][b]} != {want}"
         wref = oracle.softmax_selected(lg_o[i], gpu_layer["idx"][b])
-        np.testing.assert_allclose(gpu_layer["w"][b], wref, rtol=1e-4, atol=1e-5, err_msg=tag)
+        dmax = float(np.max(np.abs(lg_g[i] - lg_o[i])))
+        tol = wref * (2.2 * dmax + 1e-5) + 1e-6
+        assert np.all(np.abs(gpu_layer["w"][b] - wref) <= tol), f"{tag}: row {b} routing weights"
         if not np.array_equal(np.sort(orc["idx"][i]), np.sort(gpu_layer["idx"][b])):
             diff = set(orc["idx"][i]) ^ set(gpu_layer["idx"][b])
             vals = lg_o[i][list(diff)]
@@ -94,18 +102,25 @@ def check_layer(gpu_layer, orc, rows, k, tag=""):
     return near_tie
 
 
-def check_y(y_gpu_rows, orc_y_bits, tag="", skip=()):
+def check_y(y_gpu_rows, orc_layers, tag="", skip=()):
+    """orc_layers: the oracle's per-layer results of these rows (last = output)."""
     yg = bf(y_gpu_rows)
-    yo = bf(orc_y_bits)
+    yo = bf(orc_layers[-1]["y"])
     keep = [i for i in range(yg.shape[0]) if i not in skip]
     yg, yo = yg[keep], yo[keep]
+    # each layer's bf16 output rounding can move the output by one step at that
+    # layer's magnitude; the residual add carries it into the next layer unchanged
+    steps = sum(bf16_ulp(bf(r["y"])[keep]) for r in orc_layers)
+    # a later layer also sees the earlier layers' rounding flips through its MoE
+    # path; measured worst case 1.3e-3 (two 7168-wide layers), allowance 5e-3 per layer
+    steps = steps + 5e-3 * (len(orc_layers) - 1)
     if yg.size == 0:
         return 0.0
     d = np.abs(yg - yo)
     assert np.all(np.isfinite(yg)), f"{tag}: non-finite output"
     bar = 2e-2 * np.max(np.abs(yo))
     assert d.max() <= bar, f"{tag}: max |dy| {d.max():.4e} > 2e-2*max|y| = {bar:.4e}"
-    tight = bf16_ulp(yo) + 1e-3
+    tight = steps + 1e-3
     bad = d > tight
     assert not bad.any(), f"{tag}: {bad.sum()} outputs beyond one bf16 step (worst {d.max():.3e})"
     return float(d.max())
