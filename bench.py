@@ -47,6 +47,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline oracle budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-small", action="store_true",
+                    help="the batch-1 layer with 64 experts instead of 896 (same per-expert shapes, "
+                         "~2.9 GB of weights): the small case for full ncu captures")
     return ap.parse_args(argv)
 
 
@@ -383,6 +386,8 @@ def run_ours(args, wl):
 def main(argv=None):
     args = parse_args(argv)
     wl = synth.WORKLOADS[args.config]
+    if args.profile_small:
+        wl = synth.Workload("b1_h7168_e64_k16_profile", B=1, H=7168, E=64, k=16, I=1024, Is=2048, seed=1)
     if args.impl == "reference":
         run_reference(args, wl)
     else:
