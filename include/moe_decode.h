@@ -143,6 +143,31 @@ int moe_decode_launches_per_step(const moe_decode_handle* h);
  * bound of every device-side wait (default 2000 ms). */
 int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms);
 
+/* The same decode step for callers that cannot allocate device memory: code on a
+ * path where cudaMalloc is not allowed (inside a framework or plugin that owns
+ * all device memory, an allocator callback, a process whose memory budget is
+ * fixed up front). It takes no handle and allocates nothing; its scratch is one
+ * device array of about 16.7 MB inside this library, which every GPU that loads
+ * the library holds until the process exits. The pages have no counterpart to
+ * this entry point.
+ *  - Limits: batch <= 4, top_k <= 16, hidden <= 7168, n_experts <= 1024, inter <=
+ *    1024, shared_inter <= 2048, n_layers <= 2 (cfg->max_batch and top_k_max are
+ *    not used); beyond them it returns MOE_ERR_UNSUPPORTED_SHAPE.
+ *  - cfg, layers, x_in, y_out, batch, top_k and stream mean what they mean for
+ *    moe_decode_create and moe_decode_step; the TMA descriptors are built on
+ *    every call.
+ *  - The first call on a device (the current device) sets up that device: it
+ *    looks up the scratch array's device address and the kernel's attributes.
+ *    Make that first call before any stream capture.
+ *  - All calls share the one array and each call clears its counters before it
+ *    runs: calls that overlap on the GPU (other streams, other threads) race and
+ *    must be serialised by the caller.
+ *  - device_status: NULL, or a caller-zeroed device int into which the kernel
+ *    records the first device-side MOE_ERR_* of the step (read it after a sync). */
+int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_decode_layer_weights* layers,
+                            const void* x_in, void* y_out, int batch, int top_k, void* stream,
+                            int* device_status);
+
 void moe_decode_destroy(moe_decode_handle* h);
 
 const char* moe_decode_strerror(int code);

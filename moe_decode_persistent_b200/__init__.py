@@ -18,7 +18,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(_HERE)
 LIB = os.path.join(_HERE, "libmoe_decode.so")
 HEADER = os.path.join(ROOT, "include", "moe_decode.h")
-SOURCES = [os.path.join(_HERE, "csrc", f) for f in ("moe_decode_kernel.cu", "moe_decode_api.cu")]
+SOURCES = [os.path.join(_HERE, "csrc", f)
+           for f in ("moe_decode_kernel.cu", "moe_decode_api.cu", "moe_decode_noalloc.cu")]
 
 MOE_OK = 0
 MOE_ERR_INVALID_ARG = -1
@@ -99,6 +100,9 @@ def lib():
         L.moe_decode_set_debug.restype = i
         L.moe_decode_destroy.argtypes = [vp]
         L.moe_decode_destroy.restype = None
+        L.moe_decode_step_noalloc.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerWeights),
+                                              vp, vp, i, i, vp, vp]
+        L.moe_decode_step_noalloc.restype = i
         L.moe_decode_strerror.argtypes = [i]
         L.moe_decode_strerror.restype = ctypes.c_char_p
         _lib = L
@@ -134,6 +138,24 @@ def _stream_handle(stream) -> int | None:
     if isinstance(stream, int):
         return stream
     return int(stream.cuda_stream)
+
+
+def step_noalloc(hidden, n_experts, inter, shared_inter, layers, x, y, batch, top_k, eps=1e-6,
+                 stream=None, device_status=None) -> None:
+    """The decode step without a handle and without any device allocation (the
+    library's built-in scratch; see moe_decode_step_noalloc in the header).
+
+    For callers that cannot allocate device memory. Limits: batch <= 4, top_k <=
+    16, hidden <= 7168, n_experts <= 1024, inter <= 1024, shared_inter <= 2048,
+    at most 2 layers. Calls that overlap on the GPU race on the shared scratch.
+    """
+    cfg = Config(hidden, n_experts, top_k, inter, shared_inter, batch, len(layers), eps)
+    arr = (LayerWeights * len(layers))()
+    for i, w in enumerate(layers):
+        arr[i] = LayerWeights(*(_ptr(w.get(name)) for name, _ in LayerWeights._fields_))
+    _check(lib().moe_decode_step_noalloc(ctypes.byref(cfg), arr, _ptr(x), _ptr(y), int(batch), int(top_k),
+                                         _stream_handle(stream), _ptr(device_status)),
+           "moe_decode_step_noalloc")
 
 
 class MoeDecode:
