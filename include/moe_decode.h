@@ -60,7 +60,7 @@ extern "C" {
 #define MOE_ERR_NO_MEMORY (-8)          /* workspace allocation failed */
 
 /* Layer dimensions, fixed at create time.
- *  hidden        H   (multiple of 32; multiple of 256 or at most 256)
+ *  hidden        H   (multiple of 32; multiple of 256 or at most 256; at most 16384)
  *  n_experts     E   (multiple of 32, at most 1024)
  *  top_k_max     largest k a step may use (1..32, <= E)
  *  inter         I   expert SwiGLU intermediate (multiple of 32; multiple of 256 or <= 256)
@@ -82,7 +82,7 @@ typedef struct {
 } moe_decode_config;
 
 /* Device pointers of one layer's parameters (bf16 unless noted). All must be
- * 16-byte aligned. */
+ * 16-byte aligned (router_bias: 4-byte aligned). */
 typedef struct {
   const void* gamma;        /* [H] RMSNorm gain */
   const void* w_router;     /* [E][H] */
@@ -142,6 +142,26 @@ int moe_decode_launches_per_step(const moe_decode_handle* h);
  * ready signal so that every waiting CTA's bounded wait runs out. wait_ms is the
  * bound of every device-side wait (default 2000 ms). */
 int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms);
+
+/* Per-CTA timeline of later steps (profiling aid). trace: NULL to switch it off,
+ * or a device buffer of n_layers * moe_decode_trace_slots(h) uint64 values,
+ * 8-byte aligned, owned by the caller. Per layer and CTA, 40 slots: global-timer
+ * stamps (ns) of the kernel start, normalised rows acquired, schedule seen, first
+ * expert and first down stage issued, last stage issued, last stage consumed, last
+ * epilogue, exit; then clock64 sums of the producer's waits for ring slots, for
+ * published activations and for queue tickets, MAC warp 0's waits for stages and
+ * for result buffers, the epilogue warp's busy time, the number of units, MAC
+ * warp 0's arithmetic cycles and stage count, the producer's issue cycles and
+ * stage count, MAC warp 0's schedule-building, reduction and total loop
+ * cycles, the producer's unit-setup, schedule-wait and total loop cycles, and
+ * stamps of the router tiles seen finished, of the schedule built, and of the
+ * schedule's top-k, top-k rendezvous and unique-expert steps, of a
+ * normalised row published by the CTA, and of the first top-k row's logits
+ * loaded and selection done (slots 34-39 are reserved). */
+int moe_decode_set_trace(moe_decode_handle* h, void* trace);
+
+/* uint64 trace slots of one layer (number of CTAs x 40). */
+int moe_decode_trace_slots(const moe_decode_handle* h);
 
 /* The same decode step for callers that cannot allocate device memory: code on a
  * path where cudaMalloc is not allowed (inside a framework or plugin that owns

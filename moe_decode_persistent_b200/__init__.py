@@ -96,6 +96,10 @@ def lib():
         L.moe_decode_get_status.restype = i
         L.moe_decode_launches_per_step.argtypes = [vp]
         L.moe_decode_launches_per_step.restype = i
+        L.moe_decode_set_trace.argtypes = [vp, vp]
+        L.moe_decode_set_trace.restype = i
+        L.moe_decode_trace_slots.argtypes = [vp]
+        L.moe_decode_trace_slots.restype = i
         L.moe_decode_set_debug.argtypes = [vp, u, u]
         L.moe_decode_set_debug.restype = i
         L.moe_decode_destroy.argtypes = [vp]
@@ -215,6 +219,22 @@ class MoeDecode:
 
     def set_debug(self, flags: int, wait_ms: int = 2000) -> None:
         _check(lib().moe_decode_set_debug(self.handle, int(flags), int(wait_ms)), "moe_decode_set_debug")
+
+    TRACE_FIELDS = ("start", "nready", "sched", "first_expert", "first_down", "prod_end", "mac_end",
+                    "epi_end", "exit", "prod_wait_slot_cyc", "prod_wait_dep_cyc", "prod_grab_cyc",
+                    "mac_wait_full_cyc", "mac_wait_rb_cyc", "epi_busy_cyc", "units",
+                    "mac_compute_cyc", "mac_stages", "prod_issue_cyc", "prod_stages", "mac_sched_cyc",
+                    "mac_reduce_cyc", "mac_loop_cyc", "prod_setup_cyc", "prod_sched_cyc",
+                    "prod_loop_cyc", "router_seen", "sched_built", "topk_done", "topk_synced",
+                    "unique_done", "n_published", "topk_loaded", "topk_selected", "r34", "r35",
+                    "r36", "r37", "r38", "r39")
+
+    def trace_slots(self) -> int:
+        return lib().moe_decode_trace_slots(self.handle)
+
+    def set_trace(self, buf) -> None:
+        """buf: None, or a device uint64/int64 tensor of n_layers * trace_slots() values."""
+        _check(lib().moe_decode_set_trace(self.handle, _ptr(buf)), "moe_decode_set_trace")
 
     def close(self) -> None:
         if getattr(self, "handle", None):

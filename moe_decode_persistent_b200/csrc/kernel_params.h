@@ -70,6 +70,46 @@ struct Params {
   int* dbg_nuniq;
   unsigned flags;        // bit 0: jitter, bit 1: withhold the n-ready signal
   unsigned long long wait_ns;
+  unsigned long long* trace;  // nullable: [gridDim.x][kTraceSlots] timeline (see TraceSlot)
+};
+
+// Per-CTA timeline of one launch (global-timer ns stamps; *_CYC slots are clock64 sums).
+enum TraceSlot {
+  TR_START = 0,         // kernel start
+  TR_NREADY = 1,        // producer acquired the normalised rows
+  TR_SCHED = 2,         // producer saw the routing schedule
+  TR_FIRST_EXPERT = 3,  // producer issued its first expert gate/up stage
+  TR_FIRST_DOWN = 4,    // producer issued its first down stage
+  TR_PROD_END = 5,      // producer issued its last stage
+  TR_MAC_END = 6,       // MAC warps consumed the last stage
+  TR_EPI_END = 7,       // epilogue warp finished its last unit
+  TR_EXIT = 8,          // CTA done
+  TR_PROD_WAIT_SLOT_CYC = 9,   // producer cycles waiting for a free ring slot
+  TR_PROD_WAIT_DEP_CYC = 10,   // producer cycles waiting for activations to be published
+  TR_PROD_GRAB_CYC = 11,       // producer cycles waiting for the queue's next unit
+  TR_MAC_WAIT_FULL_CYC = 12,   // MAC warp 0 cycles waiting for a stage
+  TR_MAC_WAIT_RB_CYC = 13,     // MAC warp 0 cycles waiting for a free result buffer
+  TR_EPI_BUSY_CYC = 14,        // epilogue warp cycles inside unit epilogues
+  TR_UNITS = 15,               // units this CTA processed
+  TR_MAC_COMPUTE_CYC = 16,     // MAC warp 0 cycles in the stage arithmetic
+  TR_MAC_STAGES = 17,          // stages MAC warp 0 consumed
+  TR_PROD_ISSUE_CYC = 18,      // producer cycles issuing stages (waits excluded)
+  TR_PROD_STAGES = 19,         // stages the producer issued
+  TR_MAC_SCHED_CYC = 20,       // MAC warp 0 cycles building the schedule
+  TR_MAC_REDUCE_CYC = 21,      // MAC warp 0 cycles in reductions and result hand-off
+  TR_MAC_LOOP_CYC = 22,        // MAC warp 0 cycles in the stage loop in total
+  TR_PROD_SETUP_CYC = 23,      // producer cycles decoding units and building segment contexts
+  TR_PROD_SCHED_CYC = 24,      // producer cycles waiting for the routing schedule
+  TR_PROD_LOOP_CYC = 25,       // producer cycles in its unit loop in total
+  TR_ROUTER_SEEN = 26,         // MAC warps observed all router tiles finished (stamp)
+  TR_SCHED_BUILT = 27,         // MAC warps finished the schedule (stamp)
+  TR_TOPK_DONE = 28,           // schedule: this CTA's top-k rows done (stamp)
+  TR_TOPK_SYNCED = 29,         // schedule: all MAC warps past the top-k (stamp)
+  TR_UNIQUE_DONE = 30,         // schedule: unique-expert list and pairs done (stamp)
+  TR_N_PUBLISHED = 31,         // a normalised row published by this CTA (stamp)
+  TR_TOPK_LOADED = 32,         // schedule: first top-k row's logits loaded (stamp)
+  TR_TOPK_SELECTED = 33,       // schedule: first top-k row's selection rounds done (stamp)
+  kTraceSlots = 40
 };
 
 constexpr unsigned kFlagJitter = 1u;

@@ -13,6 +13,7 @@ namespace moe {
 size_t smem_bytes();
 int threads_per_cta();
 const void* kernel_fn();
+const void* kernel_fn_trace();
 }  // namespace moe
 
 using moe::Params;
@@ -45,6 +46,7 @@ struct moe_decode_handle {
   unsigned max_units, max_tiles;
   unsigned flags;
   unsigned long long wait_ns;
+  unsigned long long* trace;  // nullable [n_layers][num_sms][kTraceSlots]
 };
 
 static int cuda_fail(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -93,13 +95,15 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
       c.top_k_max > 32 || c.top_k_max > c.n_experts || !(c.eps >= 0.0f))
     return MOE_ERR_INVALID_ARG;
   if (c.max_batch * c.top_k_max > moe::kMaxSlots) return MOE_ERR_UNSUPPORTED_SHAPE;
-  if (!tile_dim_ok(c.hidden) || !tile_dim_ok(c.inter) || !tile_dim_ok(c.shared_inter) ||
+  if (!tile_dim_ok(c.hidden) || c.hidden > 16384 || !tile_dim_ok(c.inter) || !tile_dim_ok(c.shared_inter) ||
       c.n_experts < 32 || c.n_experts % 32 != 0 || c.n_experts > moe::kMaxE)
     return MOE_ERR_UNSUPPORTED_SHAPE;
   for (int l = 0; l < c.n_layers; ++l) {
     const moe_decode_layer_weights& w = layers[l];
     if (!w.gamma || !w.w_router || !w.w_gate || !w.w_up || !w.w_down || !w.ws_gate || !w.ws_up ||
         !w.ws_down)
+      return MOE_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(w.gamma) & 15u) || (reinterpret_cast<uintptr_t>(w.router_bias) & 3u))
       return MOE_ERR_INVALID_ARG;
   }
 
@@ -115,6 +119,8 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
 
   const size_t smem = moe::smem_bytes();
   e = cudaFuncSetAttribute(moe::kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(moe::kernel_fn_trace(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return MOE_ERR_COOPERATIVE;
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe::kernel_fn(), moe::threads_per_cta(),
@@ -276,8 +282,10 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     }
     p.flags = h->flags;
     p.wait_ns = h->wait_ns;
+    p.trace = h->trace ? h->trace + (size_t)l * h->num_sms * moe::kTraceSlots : nullptr;
     void* args[] = {&p};
-    cudaError_t e = cudaLaunchCooperativeKernel(moe::kernel_fn(), dim3(h->num_sms), dim3(moe::threads_per_cta()),
+    const void* fn = h->trace ? moe::kernel_fn_trace() : moe::kernel_fn();
+    cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(h->num_sms), dim3(moe::threads_per_cta()),
                                                 args, moe::smem_bytes(), stream);
     if (e == cudaErrorCooperativeLaunchTooLarge) return MOE_ERR_COOPERATIVE;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
@@ -335,6 +343,17 @@ int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms)
   if (!h || wait_ms == 0) return MOE_ERR_INVALID_ARG;
   h->flags = flags;
   h->wait_ns = (unsigned long long)wait_ms * 1000000ull;
+  return MOE_OK;
+}
+
+int moe_decode_trace_slots(const moe_decode_handle* h) {
+  return h ? h->num_sms * (int)moe::kTraceSlots : MOE_ERR_INVALID_ARG;
+}
+
+int moe_decode_set_trace(moe_decode_handle* h, void* trace) {
+  if (!h) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(trace) & 7u) return MOE_ERR_INVALID_ARG;
+  h->trace = static_cast<unsigned long long*>(trace);
   return MOE_OK;
 }
 

@@ -6,19 +6,24 @@
 // 1.68倍", section "为什么解码阶段适合Megakernel"; page post.smzdm.com/p/a6zppe4g,
 // section "改了什么：每层 23 个 kernel 砍到 13 个": 23 -> 13 kernels per layer).
 //
-// Roles inside a CTA
-//   warp 0           producer: takes units of work from a global queue and streams
-//                    their weight tiles (2-D TMA boxes of 32 rows x up to 256 K
-//                    columns) plus the matching activation rows (1-D bulk copies)
-//                    into a kStages-deep shared-memory ring, mbarrier-completed.
-//   warps 1..8       consumers: CUDA-core GEMV over each stage (each warp owns 4
-//                    weight rows of the box, each lane 8 K columns), fp32
-//                    accumulation in registers across the stages of a unit, warp
-//                    shuffle reductions, split-K partials and last-arriver fixups.
+// Roles inside a CTA (10 warps)
+//   warp 0      producer: takes units of work from a global queue and streams their
+//               weight tiles (2-D TMA boxes of 32 rows x up to 256 K columns, two
+//               boxes per stage) plus the matching activation rows (1-D bulk copies)
+//               into a kStages-deep shared-memory ring, completed on mbarriers.
+//   warps 1..8  MAC warps: CUDA-core GEMV over each stage (each warp owns 4 weight
+//               rows of a box, each lane 8 K columns), fp32 accumulation in
+//               registers across a unit's stages, warp-shuffle reductions into a
+//               shared-memory result buffer.
+//   warp 9      epilogue warp: per finished unit, the split-K partial, the tile's
+//               ticket, the fixed-order fix-up of the tile's last split and the
+//               unit's outputs (logits, SwiGLU rows, or the combined layer output),
+//               then the release that publishes them. The MAC warps never wait on
+//               global round trips.
 //
 // Units of work (queue order)
-//   router    (act group g, tile of 32 experts, K split)      -> logits
-//   shared    (act group g, tile of 32 rows of Ws_gate/Ws_up, K split) -> h_s
+//   router    (row group g, tile of 32 experts, K split)        -> logits
+//   shared    (row group g, tile of 32 rows of Ws_gate/Ws_up, K split) -> h_s
 //   -- every CTA then builds the same routing schedule from the final logits:
 //      warp-level top-k per row, softmax over the selected logits, the
 //      expert -> rows map and the list of unique experts (each selected expert's
@@ -35,12 +40,13 @@
 // h, partials) is read only after an acquire on the counter that publishes it,
 // and never through the non-coherent path; only static weights are loaded
 // ahead of a wait (the pages' review finding: page "vLLM 合併 Kimi K3 專用解碼…",
-// section "AI 寫的 GPU 核心 vLLM 怎麼驗證正確"). Every spin-wait is bounded;
-// when one runs out the kernel records MOE_ERR_TIMEOUT, all CTAs unwind, drain
-// their bulk copies and exit.
+// section "AI 寫的 GPU 核心 vLLM 怎麼驗證正確"). Every wait, between CTAs and
+// between warps of a CTA, is bounded; when one runs out the kernel records
+// MOE_ERR_TIMEOUT, all CTAs unwind, drain their bulk copies and exit.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <stddef.h>
 #include <stdint.h>
 
 #include "kernel_params.h"
@@ -49,23 +55,31 @@
 
 namespace moe {
 
-constexpr int kConsumerWarps = 8;
-constexpr int kConsumerThreads = 32 * kConsumerWarps;
-constexpr int kThreads = 32 + kConsumerThreads;
-constexpr int kRowsPerWarp = kBoxRows / kConsumerWarps;      // 4
-constexpr int kBoxBytesMax = kBoxRows * kBoxColsMax * 2;      // 16 KB
-constexpr int kActBytesMax = kActGroup * kBoxColsMax * 2;     // 4 KB
-constexpr int kSlotBytes = 2 * kBoxBytesMax + kActBytesMax;   // 36 KB
+constexpr int kMacWarps = 8;
+constexpr int kMacThreads = 32 * kMacWarps;
+constexpr int kThreads = 32 * (kMacWarps + 2);
+constexpr int kRowsPerWarp = kBoxRows / kMacWarps;                // 4
+constexpr int kBoxBytesMax = kBoxRows * kBoxColsMax * 2;          // 16 KB
+constexpr int kActSegBytes = kActGroup * kBoxColsMax * 2;         // 2 KB: one K box of <= 4 rows
+constexpr int kSlotBytes = 2 * kBoxBytesMax + 2 * kActSegBytes;   // 36 KB
 constexpr int kStages = 5;
 constexpr int kKSplits = 4;
-constexpr uint32_t kConsumerBar = 1;
+constexpr int kRB = 4;  // MAC -> epilogue result buffers
 
 enum UnitType { UT_ROUTER = 0, UT_SHARED = 1, UT_EXPERT = 2, UT_DOWN_SHARED = 3, UT_DOWN_EXPERT = 4 };
 enum HeaderKind { HK_STAGE = 0, HK_SCHED = 1, HK_END = 2 };
 
+// Written by the producer for every ring slot; everything a MAC warp needs for the
+// stage, so the MAC warps never decode units.
 struct StageHeader {
-  int kind, unit, stage, pad;
+  int kind;  // HK_*
+  int unit;
+  int info;  // bits 0-1 boxes, 2 K-pair, 3-5 activation rows, 6 segment end, 7 unit end,
+             // 8 pair index in the unit, 9 first stage of the unit, 16-31 box columns
+  int wrow;  // down-expert stages: first slot row of the pair (routing weights); else -1
 };
+
+constexpr int kInfoKpair = 1 << 2, kInfoSegEnd = 1 << 6, kInfoUnitEnd = 1 << 7, kInfoFirst = 1 << 9;
 
 // Layout constants of one step (identical in every CTA).
 struct Shape {
@@ -74,6 +88,7 @@ struct Shape {
   int RT, ST, IT, DT;
   int RS, SS, ES;
   int NR, NS;
+  int spp;  // stages per (expert, row group) pair of a down unit
 };
 
 // Routing schedule (identical in every CTA once built).
@@ -93,22 +108,38 @@ struct Smem {
   uint8_t ring[kStages][kSlotBytes];
   uint64_t full[kStages];
   uint64_t empty[kStages];
-  uint64_t sched_bar;
+  uint64_t sched_bar;       // schedule built (MAC warps -> producer)
+  uint64_t mac_bar;         // MAC-warp rendezvous (bounded)
+  uint64_t rb_full[kRB];    // MAC warps -> epilogue warp
+  uint64_t rb_empty[kRB];   // epilogue warp -> MAC warps
   StageHeader hdr[kStages];
-  int abort_flag[2];
+  int rb_unit[kRB];         // unit id of the buffer, or -1 (stop)
   int bcast;
-  float red_ss[kConsumerWarps];
+  int bcast2;
+  int nuniq;
+  int16_t chunk_cnt[kMaxE / 32];
+  float red_ss[kMacWarps];
+  unsigned known_done[kMaxSlots / 32];  // producer: pairs known complete
   Shape sh;
   Sched sc;
-  float red[2][kBoxRows][kActGroup];
-  float fin[2][kBoxRows][kActGroup];
-  int topk_idx[kMaxSlots];
-  float topk_w[kMaxSlots];
-  unsigned long long mask[kMaxE];
+  alignas(16) float rb[kRB][2][kBoxRows][kActGroup];   // read as float4 by the epilogue warp
+  alignas(16) float fin[2][kBoxRows][kActGroup];       // written as float4
+  union alignas(16) {
+    struct {
+      int topk_idx[kMaxSlots];
+      float topk_w[kMaxSlots];
+      unsigned long long mask[kMaxE];
+    } t;                               // schedule construction
+    float yacc[kBoxRows][65];          // down-tile fix-up (epilogue warp)
+  } u;
 };
 
 static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget of one CTA");
-static_assert(kConsumerThreads / kBoxRows * 8 == 64, "down fixup covers 64 token rows");
+static_assert(offsetof(Smem, rb) % 16 == 0 && offsetof(Smem, fin) % 16 == 0, "float4 views of rb / fin");
+static_assert(offsetof(Smem, full) % 8 == 0 && offsetof(Smem, rb_full) % 8 == 0, "mbarrier alignment");
+static_assert(kSlotBytes % 1024 == 0 && kBoxBytesMax % 128 == 0 && kActSegBytes % 16 == 0,
+              "TMA / bulk-copy destinations");
+static_assert(kRowsPerWarp == 4 && kActGroup == 4, "MAC lane mapping assumes 4 rows x 4 row slots");
 
 struct UnitDesc {
   int type;
@@ -118,9 +149,8 @@ struct UnitDesc {
   int g;         // row group (router / shared / down-shared)
   int pair;      // expert: the pair; down-expert: first pair
   int npair;     // down-expert
-  int kb0;       // first K box
+  int kb0, nkb;  // K boxes of this unit (router / gate-up split)
   int nstages;
-  int nbox;
 };
 
 // ---- small helpers -------------------------------------------------------------------
@@ -159,18 +189,42 @@ __device__ __forceinline__ bool abort_seen(const Params& p) {
   return ld_relaxed_gpu(&p.ctr[CTR_ABORT]) != 0u;
 }
 
-// Bounded wait on an mbarrier phase (any thread).
+constexpr uint32_t kSuspendNs = 20000;  // longest single suspension inside a wait
+
+// Bounded wait on an mbarrier phase by one thread (suspended while waiting).
 __device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Params& p) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0u) {
-      if (abort_seen(p)) return false;
-      if (globaltimer_ns() - t0 > p.wait_ns) {
-        record_abort(p, MOE_ERR_TIMEOUT);
-        return false;
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if (abort_seen(p)) return false;
+    if (globaltimer_ns() - t0 > p.wait_ns) {
+      record_abort(p, MOE_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+// Bounded wait on an mbarrier phase by a whole warp: every lane observes the
+// completion itself, lane 0 alone decides to give up, and the result is uniform.
+__device__ bool warp_wait(uint64_t* bar, uint32_t parity, const Params& p, int lane) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  uint64_t t0 = 0;
+  if (lane == 0) t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    const bool done = mbar_try_wait_sleep(bar, parity, kSuspendNs);
+    if (__all_sync(0xffffffffu, done)) return true;
+    if ((it & 3u) == 3u) {
+      int stop = 0;
+      if (lane == 0) {
+        if (abort_seen(p)) {
+          stop = 1;
+        } else if (globaltimer_ns() - t0 > p.wait_ns) {
+          record_abort(p, MOE_ERR_TIMEOUT);
+          stop = 1;
+        }
       }
+      if (__shfl_sync(0xffffffffu, stop, 0)) return false;
     }
   }
 }
@@ -190,6 +244,15 @@ __device__ bool wait_counter(const uint32_t* c, uint32_t target, const Params& p
   }
 }
 
+// Rendezvous of the 8 MAC warps (an mbarrier with bounded waits).
+__device__ __forceinline__ bool mac_sync(Smem& sm, uint32_t& phase, const Params& p, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&sm.mac_bar);
+  const bool ok = warp_wait(&sm.mac_bar, phase, p, lane);
+  phase ^= 1u;
+  return ok;
+}
+
 __device__ __forceinline__ uint32_t hash32(uint32_t a) {
   a ^= a >> 16;
   a *= 0x7feb352dU;
@@ -197,6 +260,22 @@ __device__ __forceinline__ uint32_t hash32(uint32_t a) {
   a *= 0x846ca68bU;
   a ^= a >> 16;
   return a;
+}
+
+// Timeline instrumentation: compiled into the tracing instance of the kernel only.
+template <bool kTrace>
+__device__ __forceinline__ void trace_stamp(const Params& p, int slot) {
+  if (kTrace) p.trace[(size_t)blockIdx.x * kTraceSlots + slot] = globaltimer_ns();
+}
+
+template <bool kTrace>
+__device__ __forceinline__ void trace_put(const Params& p, int slot, unsigned long long v) {
+  if (kTrace) p.trace[(size_t)blockIdx.x * kTraceSlots + slot] = v;
+}
+
+template <bool kTrace>
+__device__ __forceinline__ long long tclock() {
+  return kTrace ? clock64() : 0;
 }
 
 // ---- shape and unit decoding ---------------------------------------------------------------
@@ -220,6 +299,7 @@ __device__ void make_shape(const Params& p, Shape& s) {
   s.ES = s.RS;
   s.NR = s.GB * s.RT * s.RS;
   s.NS = s.GB * s.ST * s.SS;
+  s.spp = (s.nkbI + 1) / 2;
 }
 
 __device__ __forceinline__ void split_range(int nkb, int nsplit, int s, int& kb0, int& nkb_s) {
@@ -232,6 +312,8 @@ __device__ UnitDesc decode_unit(const Shape& sh, const Sched& sc, int u) {
   d.npair = 0;
   d.pair = 0;
   d.g = 0;
+  d.kb0 = 0;
+  d.nkb = 0;
   if (u < sh.NR) {
     d.type = UT_ROUTER;
     d.split = u % sh.RS;
@@ -239,8 +321,8 @@ __device__ UnitDesc decode_unit(const Shape& sh, const Sched& sc, int u) {
     d.g = u / (sh.RS * sh.RT);
     d.nsplit = sh.RS;
     d.ticket = d.g * sh.RT + d.tile;
-    split_range(sh.nkbH, sh.RS, d.split, d.kb0, d.nstages);
-    d.nbox = 1;
+    split_range(sh.nkbH, sh.RS, d.split, d.kb0, d.nkb);
+    d.nstages = (d.nkb + 1) / 2;  // two K boxes per stage
   } else if (u < sh.NR + sh.NS) {
     const int v = u - sh.NR;
     d.type = UT_SHARED;
@@ -249,8 +331,8 @@ __device__ UnitDesc decode_unit(const Shape& sh, const Sched& sc, int u) {
     d.g = v / (sh.SS * sh.ST);
     d.nsplit = sh.SS;
     d.ticket = sh.GB * sh.RT + d.g * sh.ST + d.tile;
-    split_range(sh.nkbH, sh.SS, d.split, d.kb0, d.nstages);
-    d.nbox = 2;
+    split_range(sh.nkbH, sh.SS, d.split, d.kb0, d.nkb);
+    d.nstages = d.nkb;  // gate box + up box per stage
   } else if (u < sh.NR + sh.NS + sc.NE) {
     const int v = u - sh.NR - sh.NS;
     d.type = UT_EXPERT;
@@ -259,25 +341,24 @@ __device__ UnitDesc decode_unit(const Shape& sh, const Sched& sc, int u) {
     d.pair = v / (sh.ES * sh.IT);
     d.nsplit = sh.ES;
     d.ticket = sh.GB * (sh.RT + sh.ST) + d.pair * sh.IT + d.tile;
-    split_range(sh.nkbH, sh.ES, d.split, d.kb0, d.nstages);
-    d.nbox = 2;
+    split_range(sh.nkbH, sh.ES, d.split, d.kb0, d.nkb);
+    d.nstages = d.nkb;
   } else {
     const int v = u - sh.NR - sh.NS - sc.NE;
     d.tile = v % sh.DT;
     d.split = v / sh.DT;
     d.nsplit = sc.down_splits;
     d.ticket = sh.GB * (sh.RT + sh.ST) + sc.P * sh.IT + d.tile;
-    d.kb0 = 0;
-    d.nbox = 1;
     if (d.split < sh.GB) {
       d.type = UT_DOWN_SHARED;
       d.g = d.split;
-      d.nstages = sh.nkbIs;
+      d.nkb = sh.nkbIs;
+      d.nstages = (sh.nkbIs + 1) / 2;
     } else {
       d.type = UT_DOWN_EXPERT;
       d.pair = (d.split - sh.GB) * kDownPairsPerSplit;
       d.npair = sc.P - d.pair < kDownPairsPerSplit ? sc.P - d.pair : kDownPairsPerSplit;
-      d.nstages = d.npair * sh.nkbI;
+      d.nstages = d.npair * sh.spp;
     }
   }
   return d;
@@ -310,13 +391,18 @@ __device__ __forceinline__ int pair_first_slot_row(const Sched& sc, int pr) {
   return sc.slot_base[sc.pair_slot[pr]] + sc.pair_group[pr] * kActGroup;
 }
 
-// Per-stage geometry shared by producer and consumers.
+// Per-stage geometry shared by producer and MAC warps. A stage holds one or two
+// weight boxes: gate and up rows of the same K box (`kpair` 0), or two
+// consecutive K boxes of the same rows (`kpair` 1, one activation segment each).
 struct StageDesc {
-  int box_cols;  // K columns of the boxes of this stage
-  int c;         // activation rows
-  int pair;      // down-expert: the pair of this stage
-  int q;         // down-expert: index of the pair within the unit
-  int kb;        // K box index
+  int nbox;
+  int kpair;
+  int box_cols;
+  int c;     // activation rows
+  int pair;  // down-expert: the pair of this stage
+  int q;     // down-expert: index of the pair within the unit
+  int kb;    // first K box
+  int last_of_pair;
 };
 
 __device__ __forceinline__ StageDesc stage_desc(const Shape& sh, const Sched& sc, const UnitDesc& d,
@@ -324,37 +410,149 @@ __device__ __forceinline__ StageDesc stage_desc(const Shape& sh, const Sched& sc
   StageDesc s;
   s.pair = d.pair;
   s.q = 0;
+  s.last_of_pair = 0;
   switch (d.type) {
     case UT_ROUTER:
+      s.kpair = 1;
+      s.box_cols = sh.boxH;
+      s.c = group_rows(sh.B, d.g);
+      s.kb = d.kb0 + 2 * st;
+      s.nbox = d.kb0 + d.nkb - s.kb < 2 ? 1 : 2;
+      break;
     case UT_SHARED:
+      s.kpair = 0;
       s.box_cols = sh.boxH;
       s.c = group_rows(sh.B, d.g);
       s.kb = d.kb0 + st;
+      s.nbox = 2;
       break;
     case UT_EXPERT:
+      s.kpair = 0;
       s.box_cols = sh.boxH;
       s.c = pair_rows(sc, d.pair);
       s.kb = d.kb0 + st;
+      s.nbox = 2;
       break;
     case UT_DOWN_SHARED:
+      s.kpair = 1;
       s.box_cols = sh.boxIs;
       s.c = group_rows(sh.B, d.g);
-      s.kb = st;
+      s.kb = 2 * st;
+      s.nbox = sh.nkbIs - s.kb < 2 ? 1 : 2;
       break;
-    default:
-      s.q = st / sh.nkbI;
+    default: {
+      s.kpair = 1;
+      s.q = st / sh.spp;
+      const int local = st % sh.spp;
       s.pair = d.pair + s.q;
       s.box_cols = sh.boxI;
       s.c = pair_rows(sc, s.pair);
-      s.kb = st % sh.nkbI;
+      s.kb = 2 * local;
+      s.nbox = sh.nkbI - s.kb < 2 ? 1 : 2;
+      s.last_of_pair = local == sh.spp - 1;
       break;
+    }
   }
   return s;
 }
 
-// ---- consumer math -----------------------------------------------------------------------------
+// Producer-side context of one unit (or, for a down-expert unit, of one of its pairs):
+// tensor maps, box row, K-box range and the activation rows, computed once.
+struct SegCtx {
+  const CUtensorMap* tm0;
+  const CUtensorMap* tm1;
+  int y0;
+  int box_cols;
+  int kpair;
+  int kb0, kb_end;
+  int c;
+  int wrow;
+  int dep;  // 0: normalised rows, 1: shared h, 2: the pair's h
+  int pair;
+  const uint16_t* abase;     // activation matrix
+  uint32_t aoff[kActGroup];  // element offsets of the activation rows
+};
 
-template <int NBOX, int CP>
+__device__ __forceinline__ void make_seg(const Params& p, const Shape& sh, const Sched& sc, const UnitDesc& d,
+                                         int q, SegCtx& x) {
+  x.wrow = -1;
+  x.pair = d.pair;
+  switch (d.type) {
+    case UT_ROUTER:
+    case UT_SHARED: {
+      const bool r = d.type == UT_ROUTER;
+      x.tm0 = &p.tmaps[r ? TM_WR : TM_WSG];
+      x.tm1 = &p.tmaps[r ? TM_WR : TM_WSU];
+      x.y0 = d.tile * kBoxRows;
+      x.box_cols = sh.boxH;
+      x.kpair = r ? 1 : 0;
+      x.kb0 = d.kb0;
+      x.kb_end = d.kb0 + d.nkb;
+      x.c = group_rows(sh.B, d.g);
+      x.dep = 0;
+      x.abase = p.n;
+#pragma unroll
+      for (int j = 0; j < kActGroup; ++j) x.aoff[j] = (uint32_t)((d.g * kActGroup + (j < x.c ? j : 0)) * p.H);
+      break;
+    }
+    case UT_EXPERT: {
+      const int e = sc.slot_expert[sc.pair_slot[d.pair]];
+      const int r0 = pair_first_slot_row(sc, d.pair);
+      x.tm0 = &p.tmaps[TM_WG];
+      x.tm1 = &p.tmaps[TM_WU];
+      x.y0 = e * p.I + d.tile * kBoxRows;
+      x.box_cols = sh.boxH;
+      x.kpair = 0;
+      x.kb0 = d.kb0;
+      x.kb_end = d.kb0 + d.nkb;
+      x.c = pair_rows(sc, d.pair);
+      x.dep = 0;
+      x.abase = p.n;
+#pragma unroll
+      for (int j = 0; j < kActGroup; ++j) x.aoff[j] = (uint32_t)(sc.row_of[r0 + (j < x.c ? j : 0)] * p.H);
+      break;
+    }
+    case UT_DOWN_SHARED:
+      x.tm0 = x.tm1 = &p.tmaps[TM_WSD];
+      x.y0 = d.tile * kBoxRows;
+      x.box_cols = sh.boxIs;
+      x.kpair = 1;
+      x.kb0 = 0;
+      x.kb_end = sh.nkbIs;
+      x.c = group_rows(sh.B, d.g);
+      x.dep = 1;
+      x.abase = p.hs;
+#pragma unroll
+      for (int j = 0; j < kActGroup; ++j) x.aoff[j] = (uint32_t)((d.g * kActGroup + (j < x.c ? j : 0)) * p.Is);
+      break;
+    default: {
+      const int pr = d.pair + q;
+      const int e = sc.slot_expert[sc.pair_slot[pr]];
+      const int r0 = pair_first_slot_row(sc, pr);
+      x.pair = pr;
+      x.tm0 = x.tm1 = &p.tmaps[TM_WD];
+      x.y0 = e * p.H + d.tile * kBoxRows;
+      x.box_cols = sh.boxI;
+      x.kpair = 1;
+      x.kb0 = 0;
+      x.kb_end = sh.nkbI;
+      x.c = pair_rows(sc, pr);
+      x.wrow = r0;
+      x.dep = 2;
+      x.abase = p.he;
+#pragma unroll
+      for (int j = 0; j < kActGroup; ++j) x.aoff[j] = (uint32_t)((r0 + (j < x.c ? j : 0)) * p.I);
+      break;
+    }
+  }
+}
+
+// ---- MAC warps: math ---------------------------------------------------------------------------
+
+// One stage: box m's rows (warp + 8 r) times the activation rows of its segment.
+// KPAIR 0: box 0 -> acc[0] (gate), box 1 -> acc[1] (up), one activation segment.
+// KPAIR 1: both boxes -> acc[0], box m uses activation segment m.
+template <int KPAIR, int NBOX, int CP>
 __device__ __forceinline__ void mac_stage(const uint8_t* slot, int box_cols, int c,
                                           float (&acc)[2][kRowsPerWarp][kActGroup], int warp,
                                           int lane) {
@@ -364,43 +562,52 @@ __device__ __forceinline__ void mac_stage(const uint8_t* slot, int box_cols, int
   const uint8_t* act = slot + 2 * kBoxBytesMax;
   float a[CP][8];
 #pragma unroll
-  for (int j = 0; j < CP; ++j) {
-    if (j < c) {
-      const uint4 v = *reinterpret_cast<const uint4*>(act + j * row_bytes + colb);
-      unpack8(v, a[j]);
-    } else {
-#pragma unroll
-      for (int t = 0; t < 8; ++t) a[j][t] = 0.0f;
-    }
-  }
-#pragma unroll
   for (int m = 0; m < NBOX; ++m) {
+    if (m == 0 || KPAIR) {
+      const uint8_t* seg = act + (KPAIR ? m : 0) * kActSegBytes;
+#pragma unroll
+      for (int j = 0; j < CP; ++j) {
+        if (j < c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(seg + j * row_bytes + colb);
+          unpack8(v, a[j]);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 8; ++t) a[j][t] = 0.0f;
+        }
+      }
+    }
+    const int am = KPAIR ? 0 : m;
 #pragma unroll
     for (int r = 0; r < kRowsPerWarp; ++r) {
       const uint4 wv = *reinterpret_cast<const uint4*>(slot + m * kBoxBytesMax +
-                                                       (warp + kConsumerWarps * r) * row_bytes + colb);
+                                                       (warp + kMacWarps * r) * row_bytes + colb);
       float w[8];
       unpack8(wv, w);
 #pragma unroll
       for (int j = 0; j < CP; ++j) {
 #pragma unroll
-        for (int t = 0; t < 8; ++t) acc[m][r][j] = fmaf(w[t], a[j][t], acc[m][r][j]);
+        for (int t = 0; t < 8; ++t) acc[am][r][j] = fmaf(w[t], a[j][t], acc[am][r][j]);
       }
     }
   }
 }
 
-__device__ __forceinline__ void mac_dispatch(const uint8_t* slot, int nbox, int box_cols, int c,
+template <int KPAIR, int NBOX>
+__device__ __forceinline__ void mac_cp(const uint8_t* slot, int box_cols, int c,
+                                       float (&acc)[2][kRowsPerWarp][kActGroup], int warp, int lane) {
+  if (c <= 1) mac_stage<KPAIR, NBOX, 1>(slot, box_cols, c, acc, warp, lane);
+  else if (c <= 2) mac_stage<KPAIR, NBOX, 2>(slot, box_cols, c, acc, warp, lane);
+  else mac_stage<KPAIR, NBOX, kActGroup>(slot, box_cols, c, acc, warp, lane);
+}
+
+__device__ __forceinline__ void mac_dispatch(const uint8_t* slot, int kpair, int nbox, int box_cols, int c,
                                              float (&acc)[2][kRowsPerWarp][kActGroup], int warp,
                                              int lane) {
-  if (nbox == 1) {
-    if (c <= 1) mac_stage<1, 1>(slot, box_cols, c, acc, warp, lane);
-    else if (c <= 2) mac_stage<1, 2>(slot, box_cols, c, acc, warp, lane);
-    else mac_stage<1, kActGroup>(slot, box_cols, c, acc, warp, lane);
+  if (kpair) {
+    if (nbox == 2) mac_cp<1, 2>(slot, box_cols, c, acc, warp, lane);
+    else mac_cp<1, 1>(slot, box_cols, c, acc, warp, lane);
   } else {
-    if (c <= 1) mac_stage<2, 1>(slot, box_cols, c, acc, warp, lane);
-    else if (c <= 2) mac_stage<2, 2>(slot, box_cols, c, acc, warp, lane);
-    else mac_stage<2, kActGroup>(slot, box_cols, c, acc, warp, lane);
+    mac_cp<0, 2>(slot, box_cols, c, acc, warp, lane);
   }
 }
 
@@ -413,123 +620,153 @@ __device__ __forceinline__ void zero_acc(float (&acc)[2][kRowsPerWarp][kActGroup
       for (int j = 0; j < kActGroup; ++j) acc[m][r][j] = 0.0f;
 }
 
-// Warp-reduce the accumulators of boxes [0, nbox) into red[m0 + m][row][j] (lane 0 writes).
-// `wscale` (nullable) multiplies column j (routing weight of the pair's row j).
-__device__ __forceinline__ void reduce_acc(float (&acc)[2][kRowsPerWarp][kActGroup], int nbox,
-                                           int c, float (*red)[kBoxRows][kActGroup], int m0,
-                                           const float* wscale, int warp, int lane) {
+// Warp-reduce the 32 accumulators acc[m][r][j] (value v = m*16 + r*4 + j) with a
+// butterfly reduce-scatter: 31 shuffles in 5 dependent steps, after which lane L
+// holds the full sum of value L. Lanes holding values of boxes [0, nacc) store
+// (m, row = warp + 8 r, j) into dst[m0 + m][row][j]; `wscale` (nullable) scales j.
+__device__ __forceinline__ void reduce_to(float (&acc)[2][kRowsPerWarp][kActGroup], int nacc,
+                                          float (*dst)[kBoxRows][kActGroup], int m0,
+                                          const float* wscale, int c, int warp, int lane) {
+  float v[32];
 #pragma unroll
-  for (int m = 0; m < 2; ++m) {
+  for (int m = 0; m < 2; ++m)
 #pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
+    for (int r = 0; r < kRowsPerWarp; ++r)
 #pragma unroll
-      for (int j = 0; j < kActGroup; ++j) {
-        if (m >= nbox || j >= c) continue;  // warp-uniform
-        float v = acc[m][r][j];
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        if (lane == 0) red[m0 + m][warp + kConsumerWarps * r][j] = wscale ? v * wscale[j] : v;
-      }
+      for (int j = 0; j < kActGroup; ++j) v[m * 16 + r * 4 + j] = acc[m][r][j];
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    const bool upper = (lane & half) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float keep = upper ? v[half + i] : v[i];
+      const float send = upper ? v[i] : v[half + i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
     }
+  }
+  const int m = lane >> 4, r = (lane >> 2) & 3, j = lane & 3;
+  if (m < nacc) {
+    float out = v[0];
+    if (wscale) out = j < c ? out * wscale[j] : 0.0f;
+    dst[m0 + m][warp + kMacWarps * r][j] = out;
   }
 }
 
-// ---- routing schedule (consumer warps, all CTAs) ---------------------------------------------
+// ---- routing schedule (MAC warps, every CTA) ---------------------------------------------
+
+// Order-preserving 32-bit key of a finite float (larger float -> larger key; -0 and +0
+// map to the same key, so they tie like equal floats).
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t u = __float_as_uint(f == 0.0f ? 0.0f : f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
 // Top-k of one row by one warp: the k largest logits, ties to the lower expert index,
-// then softmax over the selected logits.
+// then softmax over the selected logits. Each round takes the warp-wide maximum key
+// (redux.sync) and, among lanes holding it, the lowest expert index (redux.sync).
+template <bool kTrace>
 __device__ void warp_topk_row(const Params& p, Smem& sm, int b, int lane) {
   const int E = p.E, k = p.k;
   const int nq = E / 32;
-  float v[kMaxE / 32];
-  uint32_t taken = 0;
+  uint32_t key[kMaxE / 32];
   bool bad = false;
 #pragma unroll
   for (int q = 0; q < kMaxE / 32; ++q) {
+    key[q] = 0u;  // below every finite key: never selected while a real value remains
     if (q < nq) {
-      float t = ld_cg_f32(&p.logits[(size_t)b * E + lane + 32 * q]);
-      if (!isfinite(t)) {
-        bad = true;
-        t = -INFINITY;
-      }
-      v[q] = t;
-    } else {
-      v[q] = -INFINITY;
+      const float t = ld_cg_f32(&p.logits[(size_t)b * E + lane + 32 * q]);
+      if (!isfinite(t)) bad = true;
+      else key[q] = float_key(t);
     }
   }
   if (__any_sync(0xffffffffu, bad) && lane == 0) record_error(p, MOE_ERR_NONFINITE);
+  if (b == 0 && lane == 0) trace_stamp<kTrace>(p, TR_TOPK_LOADED);
+  uint32_t taken = 0;
   int my_idx = 0;
-  float my_val = 0.0f;
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+    // lane-local best: largest key, lowest q (= lowest expert index) among equals
+    uint32_t bk = 0u;
+    int bq = -1;
 #pragma unroll
     for (int q = 0; q < kMaxE / 32; ++q) {
-      if (q < nq && !((taken >> q) & 1u)) {
-        const int e = lane + 32 * q;
-        if (bi == 0x7fffffff || v[q] > bv) {
-          bv = v[q];
-          bi = e;
-        }
+      if (q < nq && !((taken >> q) & 1u) && (bq < 0 || key[q] > bk)) {
+        bk = key[q];
+        bq = q;
       }
     }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > bv || (ov == bv && oi < bi))) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (lane == j) {
-      my_idx = bi;
-      my_val = bv;
-    }
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, bq >= 0 ? bk : 0u);
+    const uint32_t cand = (bq >= 0 && bk == kmax) ? (uint32_t)(lane + 32 * bq) : 0xffffffffu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    if ((int)(win & 31u) == lane) taken |= 1u << (win >> 5);
+    if (lane == j) my_idx = (int)win;
   }
+  if (b == 0 && lane == 0) trace_stamp<kTrace>(p, TR_TOPK_SELECTED);
+  const float my_val = lane < k ? ld_cg_f32(&p.logits[(size_t)b * E + my_idx]) : 0.0f;
   const float mx = __shfl_sync(0xffffffffu, my_val, 0);
   const float ex = lane < k ? expf(my_val - mx) : 0.0f;
   float z = ex;
 #pragma unroll
   for (int off = 16; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
   if (lane < k) {
-    sm.topk_idx[b * k + lane] = my_idx;
-    sm.topk_w[b * k + lane] = ex / z;
-    atomicOr(&sm.mask[my_idx], 1ull << b);
+    sm.u.t.topk_idx[b * k + lane] = my_idx;
+    sm.u.t.topk_w[b * k + lane] = ex / z;
+    atomicOr(&sm.u.t.mask[my_idx], 1ull << b);
   }
 }
 
-// Builds sm.sc from the final logits. Called by all consumer threads; returns false on abort.
-__device__ bool build_schedule(const Params& p, Smem& sm, int ctid, int warp, int lane) {
+// Builds sm.sc from the final logits. Called by all MAC warps; false on abort.
+template <bool kTrace>
+__device__ bool build_schedule(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
   const Shape& sh = sm.sh;
   Sched& sc = sm.sc;
-  if (ctid == 0) {
-    const bool ok = wait_counter(&p.ctr[CTR_ROUTER], (uint32_t)(sh.GB * sh.RT), p);
-    sm.bcast = ok ? 1 : 0;
+  const int mtid = mw * 32 + lane;
+  if (mw == 0) {
+    int ok = 1;
+    if (lane == 0) ok = wait_counter(&p.ctr[CTR_ROUTER], (uint32_t)(sh.GB * sh.RT), p) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (lane == 0) sm.bcast = ok;
   }
-  for (int e = ctid; e < p.E; e += kConsumerThreads) sm.mask[e] = 0ull;
-  named_bar_sync(kConsumerBar, kConsumerThreads);
+  for (int e = mtid; e < p.E; e += kMacThreads) sm.u.t.mask[e] = 0ull;
+  if (!mac_sync(sm, mphase, p, lane)) return false;
   if (!sm.bcast) return false;
-  for (int b = warp; b < p.B; b += kConsumerWarps) warp_topk_row(p, sm, b, lane);
-  named_bar_sync(kConsumerBar, kConsumerThreads);
-  if (warp == 0) {
-    // unique experts in ascending id; rows per expert
-    int base = 0;
-    for (int e0 = 0; e0 < p.E; e0 += 32) {
-      const unsigned long long m = sm.mask[e0 + lane];
+  if (mtid == 0) trace_stamp<kTrace>(p, TR_ROUTER_SEEN);
+  for (int b = mw; b < p.B; b += kMacWarps) warp_topk_row<kTrace>(p, sm, b, lane);
+  if (mtid == 0) trace_stamp<kTrace>(p, TR_TOPK_DONE);
+  if (!mac_sync(sm, mphase, p, lane)) return false;
+  if (mtid == 0) trace_stamp<kTrace>(p, TR_TOPK_SYNCED);
+  // unique experts in ascending id: per-chunk counts by all MAC warps, then placement
+  const int nchunk = p.E / 32;
+  for (int ch = mw; ch < nchunk; ch += kMacWarps) {
+    const uint32_t bal = __ballot_sync(0xffffffffu, sm.u.t.mask[ch * 32 + lane] != 0ull);
+    if (lane == 0) sm.chunk_cnt[ch] = (int16_t)__popc(bal);
+  }
+  if (!mac_sync(sm, mphase, p, lane)) return false;
+  {
+    // exclusive prefix of the chunk counts (each warp computes it; kMaxE / 32 <= 32 chunks)
+    const int cnt = lane < nchunk ? sm.chunk_cnt[lane] : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += t;
+    }
+    for (int ch = mw; ch < nchunk; ch += kMacWarps) {
+      const int chbase = __shfl_sync(0xffffffffu, incl - cnt, ch);
+      const unsigned long long m = sm.u.t.mask[ch * 32 + lane];
       const uint32_t bal = __ballot_sync(0xffffffffu, m != 0ull);
-      const int pos = base + __popc(bal & ((1u << lane) - 1u));
       if (m != 0ull) {
-        sc.slot_expert[pos] = (int16_t)(e0 + lane);
+        const int pos = chbase + __popc(bal & ((1u << lane) - 1u));
+        sc.slot_expert[pos] = (int16_t)(ch * 32 + lane);
         sc.slot_cnt[pos] = (int16_t)__popcll(m);
       }
-      base += __popc(bal);
     }
-    const int U = base;
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (mw == 0 && lane == 0) sm.nuniq = total;
+  }
+  if (!mac_sync(sm, mphase, p, lane)) return false;
+  if (mw == 0) {
+    const int U = sm.nuniq;
+    __syncwarp();
     // slot bases and (expert, row group) pairs
     int rbase = 0, pbase = 0;
     for (int i0 = 0; i0 < U; i0 += 32) {
@@ -567,42 +804,106 @@ __device__ bool build_schedule(const Params& p, Smem& sm, int ctid, int warp, in
       sc.ND = sh.DT * sc.down_splits;
       sc.total = sh.NR + sh.NS + sc.NE + sc.ND;
       const unsigned tiles = (unsigned)(sh.GB * (sh.RT + sh.ST) + pbase * sh.IT + sh.DT);
-      sm.bcast = ((unsigned)sc.total <= p.max_units && tiles <= p.max_tiles) ? 1 : 0;
-      if (!sm.bcast) record_abort(p, MOE_ERR_UNSUPPORTED_SHAPE);
+      sm.bcast2 = ((unsigned)sc.total <= p.max_units && tiles <= p.max_tiles && pbase <= kMaxSlots) ? 1 : 0;
+      if (!sm.bcast2) record_abort(p, MOE_ERR_UNSUPPORTED_SHAPE);
     }
   }
-  named_bar_sync(kConsumerBar, kConsumerThreads);
-  if (!sm.bcast) return false;
+  if (mtid == 0) trace_stamp<kTrace>(p, TR_UNIQUE_DONE);
+  if (!mac_sync(sm, mphase, p, lane)) return false;
+  if (!sm.bcast2) return false;
   // token rows and routing weights of every slot row (rows ascending within an expert)
-  for (int i = ctid; i < sc.U; i += kConsumerThreads) {
+  for (int i = mtid; i < sc.U; i += kMacThreads) {
     const int e = sc.slot_expert[i];
-    unsigned long long m = sm.mask[e];
+    unsigned long long m = sm.u.t.mask[e];
     int r = sc.slot_base[i];
     while (m) {
       const int b = __ffsll((long long)m) - 1;
       m &= m - 1ull;
       float w = 0.0f;
       for (int j = 0; j < p.k; ++j)
-        if (sm.topk_idx[b * p.k + j] == e) w = sm.topk_w[b * p.k + j];
+        if (sm.u.t.topk_idx[b * p.k + j] == e) w = sm.u.t.topk_w[b * p.k + j];
       sc.row_of[r] = (uint8_t)b;
       sc.w_of[r] = w;
       ++r;
     }
   }
   if (blockIdx.x == 0) {
-    for (int t = ctid; t < p.B * p.k; t += kConsumerThreads) {
-      if (p.dbg_idx) p.dbg_idx[t] = sm.topk_idx[t];
-      if (p.dbg_w) p.dbg_w[t] = sm.topk_w[t];
+    for (int t = mtid; t < p.B * p.k; t += kMacThreads) {
+      if (p.dbg_idx) p.dbg_idx[t] = sm.u.t.topk_idx[t];
+      if (p.dbg_w) p.dbg_w[t] = sm.u.t.topk_w[t];
     }
-    if (ctid == 0 && p.dbg_nuniq) *p.dbg_nuniq = sc.U;
+    if (mtid == 0 && p.dbg_nuniq) *p.dbg_nuniq = sc.U;
   }
-  named_bar_sync(kConsumerBar, kConsumerThreads);
+  const bool ok = mac_sync(sm, mphase, p, lane);
+  if (mtid == 0) trace_stamp<kTrace>(p, TR_SCHED_BUILT);
+  return ok;
+}
+
+// ---- RMSNorm of the rows this CTA publishes (MAC warps) ---------------------------------------
+
+template <bool kTrace>
+__device__ bool normalise_rows(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
+  // each MAC thread holds up to kNormVec 16-byte vectors of x and gamma in registers:
+  // one round of independent loads, then both passes from registers
+  constexpr int kNormVec = 8;  // hidden <= 8 * 8 * 256 = 16384
+  const int mtid = mw * 32 + lane;
+  const int nv = p.H / 8;
+  const uint4* g4 = reinterpret_cast<const uint4*>(p.gamma);
+  for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+    const uint4* x4 = reinterpret_cast<const uint4*>(p.x + (size_t)b * p.H);
+    uint4 xv[kNormVec], gv[kNormVec];
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+      const int v = mtid + i * kMacThreads;
+      if (v < nv) {
+        xv[i] = x4[v];
+        gv[i] = g4[v];
+      }
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+      if (mtid + i * kMacThreads < nv) {
+        float f[8];
+        unpack8(xv[i], f);
+#pragma unroll
+        for (int t = 0; t < 8; ++t) ss = fmaf(f[t], f[t], ss);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (lane == 0) sm.red_ss[mw] = ss;
+    if (!mac_sync(sm, mphase, p, lane)) return false;
+    float tot = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kMacWarps; ++w) tot += sm.red_ss[w];
+    const float r = 1.0f / sqrtf(tot / (float)p.H + p.eps);
+    uint4* n4 = reinterpret_cast<uint4*>(p.n + (size_t)b * p.H);
+#pragma unroll
+    for (int i = 0; i < kNormVec; ++i) {
+      const int v = mtid + i * kMacThreads;
+      if (v < nv) {
+        float f[8], g[8];
+        unpack8(xv[i], f);
+        unpack8(gv[i], g);
+        uint32_t o[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+          o[t] = (uint32_t)f2bf(f[2 * t] * r * g[2 * t]) | ((uint32_t)f2bf(f[2 * t + 1] * r * g[2 * t + 1]) << 16);
+        n4[v] = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+    fence_proxy_async_global();
+    if (!mac_sync(sm, mphase, p, lane)) return false;
+    if (mtid == 0 && !((p.flags & kFlagWithholdNReady) && b == 0)) red_release_add(&p.ctr[CTR_NREADY], 1u);
+    if (mtid == 0) trace_stamp<kTrace>(p, TR_N_PUBLISHED);
+  }
   return true;
 }
 
-// ---- consumer: end of a unit --------------------------------------------------------------------
+// ---- epilogue warp: one finished unit ------------------------------------------------------------
 
-// Completion counter a finished tile of unit type `type` releases.
+// Completion counter a finished tile of this unit's type releases.
 __device__ __forceinline__ uint32_t* done_counter(const Params& p, const UnitDesc& d) {
   switch (d.type) {
     case UT_ROUTER: return &p.ctr[CTR_ROUTER];
@@ -612,146 +913,110 @@ __device__ __forceinline__ uint32_t* done_counter(const Params& p, const UnitDes
   }
 }
 
-__device__ void finish_unit(const Params& p, Smem& sm, const UnitDesc& d, int u, int ctid) {
+// Lane = tile row everywhere. `res` holds the unit's reduced values [2][32][4].
+__device__ void epi_finish(const Params& p, Smem& sm, const UnitDesc& d, int u,
+                           float (*res)[kBoxRows][kActGroup], int lane) {
   const Shape& sh = sm.sh;
   const Sched& sc = sm.sc;
   const bool down = d.type == UT_DOWN_SHARED || d.type == UT_DOWN_EXPERT;
-  named_bar_sync(kConsumerBar, kConsumerThreads);  // sm.red complete
-  float(*fin)[kBoxRows][kActGroup] = sm.red;
+  float(*src)[kBoxRows][kActGroup] = res;
   if (d.nsplit > 1) {
-    float* part = p.partial + (size_t)u * kPartialFloats;
-    const float* red = &sm.red[0][0][0];
-    for (int t = ctid; t < kPartialFloats; t += kConsumerThreads) part[t] = red[t];
-    __threadfence();
-    named_bar_sync(kConsumerBar, kConsumerThreads);
-    if (ctid == 0) {
+    float4* part = reinterpret_cast<float4*>(p.partial + (size_t)u * kPartialFloats);
+    const float4* r4 = reinterpret_cast<const float4*>(&res[0][0][0]);
+    part[lane] = r4[lane];
+    part[32 + lane] = r4[32 + lane];
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) {
+      // acq_rel: releases this warp's partial (ordered by the warp barrier above),
+      // acquires the other splits' partials when this split is the tile's last
       const uint32_t old = atom_add_acq_rel(&p.tickets[d.ticket], 1u);
-      const bool last = old == (uint32_t)(d.nsplit - 1);
+      last = old == (uint32_t)(d.nsplit - 1);
       if (last) st_relaxed_gpu(&p.tickets[d.ticket], 0u);
-      sm.bcast = last ? 1 : 0;
     }
-    named_bar_sync(kConsumerBar, kConsumerThreads);
-    if (!sm.bcast) return;
-    __threadfence();
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
+    __syncwarp();
     if (!down) {
       // fixed split order -> deterministic sums
-      for (int t = ctid; t < kPartialFloats; t += kConsumerThreads) {
-        float s = 0.0f;
-        for (int sp = 0; sp < d.nsplit; ++sp)
-          s += ld_cg_f32(p.partial + (size_t)unit_of_split(sh, sc, d, sp) * kPartialFloats + t);
-        (&sm.fin[0][0][0])[t] = s;
+      float4 s0 = make_float4(0.f, 0.f, 0.f, 0.f), s1 = s0;
+      for (int sp = 0; sp < d.nsplit; ++sp) {
+        const float4* q = reinterpret_cast<const float4*>(
+            p.partial + (size_t)unit_of_split(sh, sc, d, sp) * kPartialFloats);
+        const float4 a = __ldcg(q + lane), b = __ldcg(q + 32 + lane);
+        s0.x += a.x; s0.y += a.y; s0.z += a.z; s0.w += a.w;
+        s1.x += b.x; s1.y += b.y; s1.z += b.z; s1.w += b.w;
       }
-      named_bar_sync(kConsumerBar, kConsumerThreads);
-      fin = sm.fin;
+      reinterpret_cast<float4*>(&sm.fin[0][0][0])[lane] = s0;
+      reinterpret_cast<float4*>(&sm.fin[0][0][0])[32 + lane] = s1;
+      __syncwarp();
+      src = sm.fin;
     }
   }
-  // ---- epilogues ----
+  const int row = lane;
   if (d.type == UT_ROUTER) {
     const int c = group_rows(sh.B, d.g);
-    for (int t = ctid; t < kBoxRows * c; t += kConsumerThreads) {
-      const int row = t / c, j = t % c;
-      const int e = d.tile * kBoxRows + row;
+    const int e = d.tile * kBoxRows + row;
+    const float bias = p.bias ? p.bias[e] : 0.0f;
+    for (int j = 0; j < c; ++j) {
       const int b = d.g * kActGroup + j;
-      float v = fin[0][row][j];
-      if (p.bias) v += p.bias[e];
+      const float v = src[0][row][j] + bias;
       p.logits[(size_t)b * p.E + e] = v;
       if (p.dbg_logits) p.dbg_logits[(size_t)b * p.E + e] = v;
     }
-  } else if (d.type == UT_SHARED || d.type == UT_EXPERT) {
-    const int c = d.type == UT_SHARED ? group_rows(sh.B, d.g) : pair_rows(sc, d.pair);
-    for (int t = ctid; t < kBoxRows * c; t += kConsumerThreads) {
-      const int row = t / c, j = t % c;
-      const float h = silu(fin[0][row][j]) * fin[1][row][j];
-      if (d.type == UT_SHARED) {
-        const int b = d.g * kActGroup + j;
-        p.hs[(size_t)b * p.Is + d.tile * kBoxRows + row] = f2bf(h);
-      } else {
-        const int r = pair_first_slot_row(sc, d.pair) + j;
-        p.he[(size_t)r * p.I + d.tile * kBoxRows + row] = f2bf(h);
-      }
+  } else if (d.type == UT_SHARED) {
+    const int c = group_rows(sh.B, d.g);
+    for (int j = 0; j < c; ++j) {
+      const int b = d.g * kActGroup + j;
+      p.hs[(size_t)b * p.Is + d.tile * kBoxRows + row] = f2bf(silu(src[0][row][j]) * src[1][row][j]);
     }
+  } else if (d.type == UT_EXPERT) {
+    const int c = pair_rows(sc, d.pair);
+    const int r0 = pair_first_slot_row(sc, d.pair);
+    for (int j = 0; j < c; ++j)
+      p.he[(size_t)(r0 + j) * p.I + d.tile * kBoxRows + row] = f2bf(silu(src[0][row][j]) * src[1][row][j]);
   } else {
-    // down tile fixup: y = bf16(x + s + sum_e w_e d_e), fixed split / pair / row order.
-    // Thread (row, bg) owns output feature `row` of the tile for token rows b = bg (mod 8).
-    constexpr int kRes = kConsumerThreads / kBoxRows;  // 8
-    const int row = ctid / kRes, bg = ctid % kRes;
-    float yacc[64 / kRes];
-#pragma unroll
-    for (int i = 0; i < 64 / kRes; ++i) yacc[i] = 0.0f;
+    // down tile fix-up: y = bf16(x + s + sum_e w_e d_e) in fixed split / pair / row order
+    float* yacc = sm.u.yacc[row];
+    for (int b = 0; b < sh.B; ++b) yacc[b] = 0.0f;
     for (int sp = 0; sp < d.nsplit; ++sp) {
       const float* part =
           p.partial + (size_t)(sh.NR + sh.NS + sc.NE + sp * sh.DT + d.tile) * kPartialFloats;
       if (sp < sh.GB) {
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(part) + row);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
         const int c = group_rows(sh.B, sp);
-        for (int j = 0; j < c; ++j) {
-          const int b = sp * kActGroup + j;
-          if (b % kRes == bg) yacc[b / kRes] += ld_cg_f32(part + row * kActGroup + j);
-        }
+        for (int j = 0; j < c; ++j) yacc[sp * kActGroup + j] += vv[j];
       } else {
         const int pr0 = (sp - sh.GB) * kDownPairsPerSplit;
         const int np = sc.P - pr0 < kDownPairsPerSplit ? sc.P - pr0 : kDownPairsPerSplit;
         for (int q = 0; q < np; ++q) {
           const int pr = pr0 + q;
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(part + q * kBoxRows * kActGroup) + row);
+          const float vv[4] = {v.x, v.y, v.z, v.w};
           const int c = pair_rows(sc, pr);
           const int r0 = pair_first_slot_row(sc, pr);
-          for (int j = 0; j < c; ++j) {
-            const int b = sc.row_of[r0 + j];
-            if (b % kRes == bg)
-              yacc[b / kRes] += ld_cg_f32(part + q * kBoxRows * kActGroup + row * kActGroup + j);
-          }
+          for (int j = 0; j < c; ++j) yacc[sc.row_of[r0 + j]] += vv[j];
         }
       }
     }
     const int h = d.tile * kBoxRows + row;
-#pragma unroll
-    for (int i = 0; i < 64 / kRes; ++i) {
-      const int b = i * kRes + bg;
-      if (b < sh.B) {
-        const float xv = bf2f(p.x[(size_t)b * p.H + h]);
-        p.y[(size_t)b * p.H + h] = f2bf(xv + yacc[i]);
-      }
+    for (int b = 0; b < sh.B; ++b) {
+      const float xv = bf2f(p.x[(size_t)b * p.H + h]);
+      p.y[(size_t)b * p.H + h] = f2bf(xv + yacc[b]);
     }
   }
   uint32_t* done = done_counter(p, d);
   if (done) {
     fence_proxy_async_global();
-    __threadfence();
-    named_bar_sync(kConsumerBar, kConsumerThreads);
-    if (ctid == 0) red_release_add(done, 1u);
-  }
-}
-
-// ---- RMSNorm of the rows this CTA publishes ---------------------------------------------------
-
-__device__ void normalise_rows(const Params& p, Smem& sm, int ctid, int warp, int lane) {
-  for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-    const uint16_t* xb = p.x + (size_t)b * p.H;
-    float ss = 0.0f;
-    for (int h = ctid; h < p.H; h += kConsumerThreads) {
-      const float v = bf2f(xb[h]);
-      ss = fmaf(v, v, ss);
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
-    if (lane == 0) sm.red_ss[warp] = ss;
-    named_bar_sync(kConsumerBar, kConsumerThreads);
-    float tot = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kConsumerWarps; ++w) tot += sm.red_ss[w];
-    const float r = 1.0f / sqrtf(tot / (float)p.H + p.eps);
-    for (int h = ctid; h < p.H; h += kConsumerThreads) {
-      const float v = bf2f(xb[h]) * r * bf2f(p.gamma[h]);
-      p.n[(size_t)b * p.H + h] = f2bf(v);
-    }
-    fence_proxy_async_global();
-    __threadfence();
-    named_bar_sync(kConsumerBar, kConsumerThreads);
-    if (ctid == 0 && !((p.flags & kFlagWithholdNReady) && b == 0)) red_release_add(&p.ctr[CTR_NREADY], 1u);
+    __syncwarp();
+    if (lane == 0) red_release_add(done, 1u);
   }
 }
 
 // ---- the kernel ----------------------------------------------------------------------------------
 
+template <bool kTrace>
 __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
@@ -762,11 +1027,20 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kConsumerWarps);
+      mbar_init(&sm.empty[s], kMacWarps);
+    }
+    for (int b = 0; b < kRB; ++b) {
+      mbar_init(&sm.rb_full[b], kMacWarps);
+      mbar_init(&sm.rb_empty[b], 1);
     }
     mbar_init(&sm.sched_bar, 1);
+    mbar_init(&sm.mac_bar, kMacWarps);
     make_shape(p, sm.sh);
-    sm.abort_flag[0] = sm.abort_flag[1] = 0;
+    for (int w = 0; w < kMaxSlots / 32; ++w) sm.known_done[w] = 0u;
+    if (kTrace) {
+      for (int t = 0; t < kTraceSlots; ++t) p.trace[(size_t)blockIdx.x * kTraceSlots + t] = 0ull;
+      trace_stamp<kTrace>(p, TR_START);
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -779,9 +1053,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
       for (int t = 0; t < TM_COUNT; ++t) prefetch_tensormap(&p.tmaps[t]);
     int slot = 0;
     uint32_t phase = 0;
-    int last_tx_parity[kStages];
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) last_tx_parity[s] = -1;
+    // slots whose last TMA stage no later use has shown complete, and that stage's parity
+    uint32_t pend_mask = 0u, pend_parity = 0u;
     bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
     const int pre = sh.NR + sh.NS;
     auto grab = [&]() -> int {
@@ -808,109 +1081,160 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
         r = wait_counter(c, target, p) ? 1 : 0;
         fence_proxy_async_global();
       }
-      return __shfl_sync(0xffffffffu, r, 0) != 0;
+      r = __shfl_sync(0xffffffffu, r, 0);
+      __syncwarp();
+      return r != 0;
+    };
+    // (expert, row group) pair pr complete? One acquire round trip polls 32 pairs.
+    auto wait_pair = [&](int pr) -> bool {
+      if ((sm.known_done[pr >> 5] >> (pr & 31)) & 1u) return true;
+      const int q = pr + lane;
+      const bool done = q < sm.sc.P && ld_acquire_gpu(&p.pair_done[q]) >= (uint32_t)sh.IT;
+      const uint32_t bal = __ballot_sync(0xffffffffu, done);
+      if (lane == 0) {
+        for (int i = 0; i < 32; ++i)
+          if ((bal >> i) & 1u) sm.known_done[(pr + i) >> 5] |= 1u << ((pr + i) & 31);
+      }
+      __syncwarp();
+      bool r = (bal & 1u) != 0u;
+      if (!r) {
+        r = wait_dep(&p.pair_done[pr], (uint32_t)sh.IT);
+        if (r && lane == 0) sm.known_done[pr >> 5] |= 1u << (pr & 31);
+        __syncwarp();
+      } else if (lane == 0) {
+        fence_proxy_async_global();
+      }
+      return r;
     };
     int u = grab();
+    bool first_expert = true, first_down = true;
+    unsigned long long c_slot = 0, c_dep = 0, c_grab = 0, c_issue = 0, c_stages = 0, c_units = 0;
+    unsigned long long c_setup = 0, c_schedw = 0;
+    const long long tploop0 = tclock<kTrace>();
     while (ok) {
       if (u >= pre && !sched_ready) {
         ok = wait_bar(&sm.empty[slot], phase ^ 1u);
         if (!ok) break;
-        last_tx_parity[slot] = -1;  // the slot's previous stage was consumed
+        pend_mask &= ~(1u << slot);  // the slot's previous stage was consumed
         if (lane == 0) {
           sm.hdr[slot].kind = HK_SCHED;
           mbar_arrive(&sm.full[slot]);
         }
         __syncwarp();
         advance();
+        const long long tw0 = tclock<kTrace>();
         ok = wait_bar(&sm.sched_bar, 0u);
+        c_schedw += (unsigned long long)(tclock<kTrace>() - tw0);
         if (!ok) break;
         sched_ready = true;
+        if (lane == 0) trace_stamp<kTrace>(p, TR_SCHED);
       }
       if (sched_ready && u >= sm.sc.total) break;
+      const long long tu0 = tclock<kTrace>();
       const UnitDesc d = decode_unit(sh, sm.sc, u);
-      const int next_u = grab();
-      if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(blockIdx.x * 7919u + (uint32_t)u) % 3000u);
-      for (int st = 0; st < d.nstages && ok; ++st) {
-        ok = wait_bar(&sm.empty[slot], phase ^ 1u);
-        if (!ok) break;
-        const StageDesc s = stage_desc(sh, sm.sc, d, st);
-        const uint32_t box_bytes = (uint32_t)(s.box_cols * kBoxRows * 2);
-        const uint32_t row_bytes = (uint32_t)(s.box_cols * 2);
-        uint8_t* dst = sm.ring[slot];
-        uint64_t* fb = &sm.full[slot];
-        if (lane == 0) {
-          sm.hdr[slot].kind = HK_STAGE;
-          sm.hdr[slot].unit = u;
-          sm.hdr[slot].stage = st;
-          mbar_arrive_expect_tx(fb, (uint32_t)d.nbox * box_bytes + (uint32_t)s.c * row_bytes);
-          last_tx_parity[slot] = (int)phase;
-          const int x = s.kb * s.box_cols;
-          switch (d.type) {
-            case UT_ROUTER:
-              tma_load_2d(dst, &p.tmaps[TM_WR], x, d.tile * kBoxRows, fb, pol);
-              break;
-            case UT_SHARED:
-              tma_load_2d(dst, &p.tmaps[TM_WSG], x, d.tile * kBoxRows, fb, pol);
-              tma_load_2d(dst + kBoxBytesMax, &p.tmaps[TM_WSU], x, d.tile * kBoxRows, fb, pol);
-              break;
-            case UT_EXPERT: {
-              const int e = sm.sc.slot_expert[sm.sc.pair_slot[d.pair]];
-              const int row = e * p.I + d.tile * kBoxRows;
-              tma_load_2d(dst, &p.tmaps[TM_WG], x, row, fb, pol);
-              tma_load_2d(dst + kBoxBytesMax, &p.tmaps[TM_WU], x, row, fb, pol);
-              break;
-            }
-            case UT_DOWN_SHARED:
-              tma_load_2d(dst, &p.tmaps[TM_WSD], x, d.tile * kBoxRows, fb, pol);
-              break;
-            default: {
-              const int e = sm.sc.slot_expert[sm.sc.pair_slot[s.pair]];
-              tma_load_2d(dst, &p.tmaps[TM_WD], x, e * p.H + d.tile * kBoxRows, fb, pol);
-              break;
-            }
-          }
-        }
-        // activations: only after the acquire that publishes them
-        bool dep_ok = true;
-        if (d.type == UT_ROUTER || d.type == UT_SHARED || d.type == UT_EXPERT) {
-          if (!n_ok) dep_ok = n_ok = wait_dep(&p.ctr[CTR_NREADY], (uint32_t)p.B);
-        } else if (d.type == UT_DOWN_SHARED) {
-          if (!hs_ok) dep_ok = hs_ok = wait_dep(&p.ctr[CTR_HS], (uint32_t)(sh.GB * sh.ST));
-        } else if (st % sh.nkbI == 0) {
-          dep_ok = wait_dep(&p.pair_done[s.pair], (uint32_t)sh.IT);
-        }
-        if (lane == 0) {
-          uint8_t* act = dst + 2 * kBoxBytesMax;
-          const int x = s.kb * s.box_cols;
-          for (int j = 0; j < s.c; ++j) {
-            const uint16_t* src;
-            switch (d.type) {
-              case UT_ROUTER:
-              case UT_SHARED:
-                src = p.n + (size_t)(d.g * kActGroup + j) * p.H + x;
-                break;
-              case UT_EXPERT:
-                src = p.n + (size_t)sm.sc.row_of[pair_first_slot_row(sm.sc, d.pair) + j] * p.H + x;
-                break;
-              case UT_DOWN_SHARED:
-                src = p.hs + (size_t)(d.g * kActGroup + j) * p.Is + x;
-                break;
-              default:
-                src = p.he + (size_t)(pair_first_slot_row(sm.sc, s.pair) + j) * p.I + x;
-                break;
-            }
-            bulk_load(act + j * row_bytes, src, row_bytes, fb);
-          }
-        }
-        __syncwarp();
-        advance();
-        if (!dep_ok) ok = false;
+      // the next unit's queue ticket is requested now and read after this unit's
+      // stages are issued, so the atomic's round trip overlaps the issue loop
+      uint32_t next_ticket = 0;
+      if (lane == 0) next_ticket = atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
+      if (lane == 0 && kTrace) {
+        if (first_expert && d.type == UT_EXPERT) { trace_stamp<kTrace>(p, TR_FIRST_EXPERT); first_expert = false; }
+        if (first_down && (d.type == UT_DOWN_SHARED || d.type == UT_DOWN_EXPERT)) { trace_stamp<kTrace>(p, TR_FIRST_DOWN); first_down = false; }
+        ++c_units;
       }
-      u = next_u;
+      if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(blockIdx.x * 7919u + (uint32_t)u) % 3000u);
+      const int nseg_units = d.type == UT_DOWN_EXPERT ? d.npair : 1;
+      c_setup += (unsigned long long)(tclock<kTrace>() - tu0);
+      for (int q = 0; q < nseg_units && ok; ++q) {
+        SegCtx x;
+        const long long tm0 = tclock<kTrace>();
+        make_seg(p, sh, sm.sc, d, q, x);
+        c_setup += (unsigned long long)(tclock<kTrace>() - tm0);
+        const uint32_t box_bytes = (uint32_t)(x.box_cols * kBoxRows * 2);
+        const uint32_t row_bytes = (uint32_t)(x.box_cols * 2);
+        const int step = x.kpair ? 2 : 1;
+        const int info0 = (x.kpair ? kInfoKpair : 0) | (x.c << 3) | (q << 8) | (x.box_cols << 16);
+        for (int kb = x.kb0; kb < x.kb_end && ok; kb += step) {
+          {
+            const long long t0 = tclock<kTrace>();
+            ok = wait_bar(&sm.empty[slot], phase ^ 1u);
+            c_slot += (unsigned long long)(tclock<kTrace>() - t0);
+          }
+          if (!ok) break;
+          const long long ti0 = tclock<kTrace>();
+          const int nbox = x.kpair ? (x.kb_end - kb < 2 ? 1 : 2) : 2;
+          const int nseg = x.kpair ? nbox : 1;
+          const bool seg_end = kb + step >= x.kb_end;
+          uint8_t* dst = sm.ring[slot];
+          uint64_t* fb = &sm.full[slot];
+          pend_mask |= 1u << slot;
+          pend_parity = (pend_parity & ~(1u << slot)) | (phase << slot);
+          if (lane == 0) {
+            StageHeader h;
+            h.kind = HK_STAGE;
+            h.unit = u;
+            h.info = info0 | nbox | (seg_end ? kInfoSegEnd : 0) | (seg_end && q == nseg_units - 1 ? kInfoUnitEnd : 0) |
+                     (kb == x.kb0 && q == 0 ? kInfoFirst : 0);
+            h.wrow = x.wrow;
+            sm.hdr[slot] = h;
+            mbar_arrive_expect_tx(fb, (uint32_t)nbox * box_bytes + (uint32_t)(nseg * x.c) * row_bytes);
+            const int col = kb * x.box_cols;
+            tma_load_2d(dst, x.tm0, col, x.y0, fb, pol);
+            if (nbox == 2) tma_load_2d(dst + kBoxBytesMax, x.tm1, x.kpair ? col + x.box_cols : col, x.y0, fb, pol);
+          }
+          // activations: only after the acquire that publishes them
+          bool dep_ok = true;
+          const long long td0 = tclock<kTrace>();
+          if (kb == x.kb0) {
+            if (x.dep == 0) {
+              if (!n_ok) {
+                dep_ok = n_ok = wait_dep(&p.ctr[CTR_NREADY], (uint32_t)p.B);
+                if (lane == 0) trace_stamp<kTrace>(p, TR_NREADY);
+              }
+            } else if (x.dep == 1) {
+              if (!hs_ok) dep_ok = hs_ok = wait_dep(&p.ctr[CTR_HS], (uint32_t)(sh.GB * sh.ST));
+            } else {
+              dep_ok = wait_pair(x.pair);
+            }
+          }
+          const long long td1 = tclock<kTrace>();
+          c_dep += (unsigned long long)(td1 - td0);
+          if (lane == 0) {
+            uint8_t* act = dst + 2 * kBoxBytesMax;
+            for (int sg = 0; sg < nseg; ++sg) {
+              const int col = (kb + sg) * x.box_cols;
+#pragma unroll
+              for (int j = 0; j < kActGroup; ++j)
+                if (j < x.c) bulk_load(act + sg * kActSegBytes + j * row_bytes, x.abase + x.aoff[j] + col, row_bytes, fb);
+            }
+          }
+          __syncwarp();
+          advance();
+          c_issue += (unsigned long long)(tclock<kTrace>() - ti0) - (unsigned long long)(td1 - td0);
+          ++c_stages;
+          if (!dep_ok) ok = false;
+        }
+      }
+      {
+        const long long t0 = tclock<kTrace>();
+        u = __shfl_sync(0xffffffffu, (int)next_ticket, 0);
+        c_grab += (unsigned long long)(tclock<kTrace>() - t0);
+      }
     }
-    // tell the consumers to stop (bounded)
+    if (lane == 0 && kTrace) {
+      trace_stamp<kTrace>(p, TR_PROD_END);
+      trace_put<kTrace>(p, TR_PROD_WAIT_SLOT_CYC, c_slot);
+      trace_put<kTrace>(p, TR_PROD_WAIT_DEP_CYC, c_dep);
+      trace_put<kTrace>(p, TR_PROD_GRAB_CYC, c_grab);
+      trace_put<kTrace>(p, TR_PROD_ISSUE_CYC, c_issue);
+      trace_put<kTrace>(p, TR_PROD_STAGES, c_stages);
+      trace_put<kTrace>(p, TR_UNITS, c_units);
+      trace_put<kTrace>(p, TR_PROD_SETUP_CYC, c_setup);
+      trace_put<kTrace>(p, TR_PROD_SCHED_CYC, c_schedw);
+      trace_put<kTrace>(p, TR_PROD_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tploop0));
+    }
+    // tell the MAC warps to stop (bounded)
     if (wait_bar(&sm.empty[slot], phase ^ 1u)) {
-      last_tx_parity[slot] = -1;
+      pend_mask &= ~(1u << slot);
       if (lane == 0) {
         sm.hdr[slot].kind = HK_END;
         mbar_arrive(&sm.full[slot]);
@@ -922,9 +1246,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
     // shown to be complete (only possible after an abort).
     if (lane == 0) {
       for (int s = 0; s < kStages; ++s) {
-        if (last_tx_parity[s] < 0) continue;
+        if (!((pend_mask >> s) & 1u)) continue;
         const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(&sm.full[s], (uint32_t)last_tx_parity[s])) {
+        while (!mbar_try_wait(&sm.full[s], (pend_parity >> s) & 1u)) {
           if (globaltimer_ns() - t0 > 50000000ull) break;
         }
       }
@@ -932,8 +1256,9 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
       for (int r = 0; r < 4; ++r) {
         if (!p.pf_ptr[r] || !p.pf_bytes[r]) continue;
         const unsigned long long tot = p.pf_bytes[r];
-        unsigned long long lo = (tot * blockIdx.x / gridDim.x) & ~15ull;
-        unsigned long long hi = blockIdx.x + 1 == gridDim.x ? tot : (tot * (blockIdx.x + 1) / gridDim.x) & ~15ull;
+        const unsigned long long lo = (tot * blockIdx.x / gridDim.x) & ~15ull;
+        const unsigned long long hi =
+            blockIdx.x + 1 == gridDim.x ? (tot & ~15ull) : (tot * (blockIdx.x + 1) / gridDim.x) & ~15ull;
         const uint8_t* base = reinterpret_cast<const uint8_t*>(p.pf_ptr[r]);
         for (unsigned long long o = lo; o < hi; o += 65536ull) {
           const unsigned long long n = hi - o < 65536ull ? hi - o : 65536ull;
@@ -942,65 +1267,142 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
       }
     }
     __syncwarp();
-  } else {
-    // =========================== consumer warps ===========================
-    const int cw = warp_id - 1;
-    const int ctid = tid - 32;
-    normalise_rows(p, sm, ctid, cw, lane);
+  } else if (warp_id <= kMacWarps) {
+    // =========================== MAC warps ===========================
+    const int mw = warp_id - 1;
+    uint32_t mphase = 0;
+    bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
     int slot = 0;
     uint32_t phase = 0;
-    int cur_u = -1;
-    UnitDesc d;
-    d.type = UT_ROUTER;
-    d.nstages = 0;
+    int ub = 0;
+    uint32_t ubphase = 0;
+    bool rb_claimed = false;
     float acc[2][kRowsPerWarp][kActGroup];
     zero_acc(acc);
-    for (uint32_t it = 0;; ++it) {
-      if (ctid == 0) sm.abort_flag[it & 1u] = wait_mbar(&sm.full[slot], phase, p) ? 0 : 1;
-      named_bar_sync(kConsumerBar, kConsumerThreads);
-      if (sm.abort_flag[it & 1u]) break;
+    const long long tloop0 = tclock<kTrace>();
+    unsigned long long c_full = 0, c_rb = 0, c_comp = 0, c_st = 0, c_sched = 0, c_red = 0;
+    while (ok) {
+      {
+        const long long t0 = tclock<kTrace>();
+        const bool got = warp_wait(&sm.full[slot], phase, p, lane);
+        c_full += (unsigned long long)(tclock<kTrace>() - t0);
+        if (!got) break;
+      }
       const StageHeader hd = sm.hdr[slot];
-      if (hd.kind == HK_END) break;
+      if (hd.kind == HK_END) {
+        if (mw == 0 && lane == 0) trace_stamp<kTrace>(p, TR_MAC_END);
+        break;
+      }
       if (hd.kind == HK_SCHED) {
-        const bool ok = build_schedule(p, sm, ctid, cw, lane);
+        const long long ts0 = tclock<kTrace>();
+        ok = build_schedule<kTrace>(p, sm, mw, lane, mphase);
+        c_sched += (unsigned long long)(tclock<kTrace>() - ts0);
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[slot]);
-        if (ctid == 0 && ok) mbar_arrive(&sm.sched_bar);
+        if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
         if (++slot == kStages) {
           slot = 0;
           phase ^= 1u;
         }
-        if (!ok) break;
         continue;
       }
-      if (hd.unit != cur_u) {
-        cur_u = hd.unit;
-        d = decode_unit(sh, sm.sc, cur_u);
+      const int info = hd.info;
+      const int kpair = (info & kInfoKpair) ? 1 : 0;
+      const int nbox = info & 3;
+      const int c = (info >> 3) & 7;
+      const int box_cols = info >> 16;
+      if (info & kInfoFirst) {
         zero_acc(acc);
+        rb_claimed = false;
+        if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(hd.unit * 131u + mw * 7u + blockIdx.x) % 1500u);
+        __syncwarp();
       }
-      const StageDesc s = stage_desc(sh, sm.sc, d, hd.stage);
-      mac_dispatch(sm.ring[slot], d.nbox, s.box_cols, s.c, acc, cw, lane);
+      const long long tc0 = tclock<kTrace>();
+      mac_dispatch(sm.ring[slot], kpair, nbox, box_cols, c, acc, mw, lane);
       __syncwarp();
+      c_comp += (unsigned long long)(tclock<kTrace>() - tc0);
+      ++c_st;
       if (lane == 0) mbar_arrive(&sm.empty[slot]);
       if (++slot == kStages) {
         slot = 0;
         phase ^= 1u;
       }
-      if (d.type == UT_DOWN_EXPERT) {
-        if (hd.stage % sh.nkbI == sh.nkbI - 1) {
-          const float* wsc = &sm.sc.w_of[pair_first_slot_row(sm.sc, s.pair)];
-          reduce_acc(acc, 1, s.c, sm.red, s.q, wsc, cw, lane);
-          zero_acc(acc);
+      const bool unit_end = (info & kInfoUnitEnd) != 0;
+      const bool seg_end = (info & kInfoSegEnd) != 0;
+      const long long tr0 = tclock<kTrace>();
+      if (seg_end) {
+        if (!rb_claimed) {
+          const long long t0 = tclock<kTrace>();
+          const bool got = warp_wait(&sm.rb_empty[ub], ubphase ^ 1u, p, lane);
+          c_rb += (unsigned long long)(tclock<kTrace>() - t0);
+          if (!got) break;
+          rb_claimed = true;
         }
-      } else if (hd.stage == d.nstages - 1) {
-        reduce_acc(acc, d.nbox, s.c, sm.red, 0, nullptr, cw, lane);
+        if (hd.wrow >= 0) {
+          reduce_to(acc, 1, sm.rb[ub], (info >> 8) & 1, &sm.sc.w_of[hd.wrow], c, mw, lane);
+          zero_acc(acc);
+        } else {
+          reduce_to(acc, kpair ? 1 : 2, sm.rb[ub], 0, nullptr, c, mw, lane);
+        }
       }
-      if (hd.stage == d.nstages - 1) finish_unit(p, sm, d, cur_u, ctid);
+      if (unit_end) {
+        if (mw == 0 && lane == 0) sm.rb_unit[ub] = hd.unit;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.rb_full[ub]);
+        if (++ub == kRB) {
+          ub = 0;
+          ubphase ^= 1u;
+        }
+        rb_claimed = false;
+      }
+      if (seg_end || unit_end) c_red += (unsigned long long)(tclock<kTrace>() - tr0);
+    }
+    if (mw == 0 && lane == 0 && kTrace) {
+      trace_put<kTrace>(p, TR_MAC_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tloop0));
+      trace_put<kTrace>(p, TR_MAC_WAIT_FULL_CYC, c_full);
+      trace_put<kTrace>(p, TR_MAC_WAIT_RB_CYC, c_rb);
+      trace_put<kTrace>(p, TR_MAC_COMPUTE_CYC, c_comp);
+      trace_put<kTrace>(p, TR_MAC_STAGES, c_st);
+      trace_put<kTrace>(p, TR_MAC_SCHED_CYC, c_sched);
+      trace_put<kTrace>(p, TR_MAC_REDUCE_CYC, c_red);
+    }
+    // tell the epilogue warp to stop (bounded)
+    if (warp_wait(&sm.rb_empty[ub], ubphase ^ 1u, p, lane)) {
+      if (mw == 0 && lane == 0) sm.rb_unit[ub] = -1;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.rb_full[ub]);
+    }
+  } else {
+    // =========================== epilogue warp ===========================
+    int ub = 0;
+    uint32_t ubphase = 0;
+    unsigned long long c_busy = 0;
+    for (;;) {
+      if (!warp_wait(&sm.rb_full[ub], ubphase, p, lane)) break;
+      const int u = sm.rb_unit[ub];
+      if (u < 0 || abort_seen(p)) {
+        if (lane == 0 && kTrace) {
+          trace_stamp<kTrace>(p, TR_EPI_END);
+          trace_put<kTrace>(p, TR_EPI_BUSY_CYC, c_busy);
+        }
+        break;
+      }
+      const UnitDesc d = decode_unit(sh, sm.sc, u);
+      const long long t0 = tclock<kTrace>();
+      epi_finish(p, sm, d, u, sm.rb[ub], lane);
+      c_busy += (unsigned long long)(tclock<kTrace>() - t0);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.rb_empty[ub]);
+      if (++ub == kRB) {
+        ub = 0;
+        ubphase ^= 1u;
+      }
     }
   }
 
   __syncthreads();
   if (tid == 0) {
+    trace_stamp<kTrace>(p, TR_EXIT);
     __threadfence();
     const uint32_t done = atom_add_acq_rel(&p.ctr[CTR_EXIT], 1u);
     if (done == gridDim.x - 1) {
@@ -1020,6 +1422,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
 
 size_t smem_bytes() { return sizeof(Smem) + 1024; }
 int threads_per_cta() { return kThreads; }
-const void* kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel); }
+const void* kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false>); }
+const void* kernel_fn_trace() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true>); }
 
 }  // namespace moe

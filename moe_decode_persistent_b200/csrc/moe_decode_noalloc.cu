@@ -161,7 +161,8 @@ extern "C" int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_d
   CUtensorMap maps[moe::TM_COUNT * kNaMaxLayers];
   for (int l = 0; l < L; ++l) {
     const moe_decode_layer_weights& w = layers[l];
-    if (!w.gamma) return MOE_ERR_INVALID_ARG;
+    if (!w.gamma || (reinterpret_cast<uintptr_t>(w.gamma) & 15u) || (reinterpret_cast<uintptr_t>(w.router_bias) & 3u))
+      return MOE_ERR_INVALID_ARG;
     CUtensorMap* m = maps + l * moe::TM_COUNT;
     if (na_encode(&m[moe::TM_WR], w.w_router, (uint64_t)E, (uint64_t)H) != MOE_OK ||
         na_encode(&m[moe::TM_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H) != MOE_OK ||
