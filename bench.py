@@ -47,6 +47,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline oracle budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--tc-min-batch", type=int, default=None,
+                    help="batch-shape switch: steps of at least this many rows take the tensor-core "
+                         "kernel (0: always the CUDA-core kernel); default: the library's")
     ap.add_argument("--profile-small", action="store_true",
                     help="the batch-1 layer with 64 experts instead of 896 (same per-expert shapes, "
                          "~2.9 GB of weights): the small case for full ncu captures")
@@ -269,6 +272,9 @@ def run_ours(args, wl):
     stream = torch.cuda.current_stream()
     layers = [wl.device_layer(l, device=f"cuda:{local}") for l in range(wl.layers)]
     h = mdp.MoeDecode(wl.H, wl.E, wl.k, wl.I, wl.Is, wl.B, layers, eps=wl.eps, device=local)
+    if args.tc_min_batch is not None:
+        h.set_tc_min_batch(args.tc_min_batch)
+    kernel_path = "tensor_core" if h.step_path(wl.B) == mdp.PATH_TENSOR_CORE else "cuda_core"
     pool_host = wl.x_pool_host(POOL)
     pool = torch.from_numpy(pool_host.view(np.int16)).view(torch.bfloat16).to(f"cuda:{local}")
     y = torch.empty((wl.B, wl.H), dtype=torch.bfloat16, device=f"cuda:{local}")
@@ -352,7 +358,7 @@ def run_ours(args, wl):
         "warmup": W, "ms_per_step": round(max_ms / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded counter-hash weights ~N(0,1/sqrt(fan_in)) and inputs, no trained weights",
-        "config": workload_config(wl, "flushed between timed steps (256 MB write)"),
+        "config": dict(workload_config(wl, "flushed between timed steps (256 MB write)"), kernel_path=kernel_path),
         "us_per_step": round(1e3 * max_ms / K, 2),
         "tokens_per_s": round(world * wl.B * K / (max_ms * 1e-3), 1),
         "unique_experts_mean": float(U.mean()),

@@ -59,6 +59,10 @@ extern "C" {
 #define MOE_ERR_NONFINITE (-7)          /* device status: a router logit was NaN or infinite */
 #define MOE_ERR_NO_MEMORY (-8)          /* workspace allocation failed */
 
+/* Kernel paths of a step (moe_decode_step_path). */
+#define MOE_PATH_CUDA_CORE 0   /* CUDA-core GEMV units of 32 weight rows x 4 token rows */
+#define MOE_PATH_TENSOR_CORE 1 /* tcgen05 tiles of 128 weight rows x all token rows, TMEM accumulators */
+
 /* Layer dimensions, fixed at create time.
  *  hidden        H   (multiple of 32; multiple of 256 or at most 256; at most 16384)
  *  n_experts     E   (multiple of 32, at most 1024)
@@ -162,6 +166,26 @@ int moe_decode_set_trace(moe_decode_handle* h, void* trace);
 
 /* uint64 trace slots of one layer (number of CTAs x 40). */
 int moe_decode_trace_slots(const moe_decode_handle* h);
+
+/* The batch-shape switch (page post.smzdm.com/p/a6zppe4g, section "改了什么：每层
+ * 23 个 kernel 砍到 13 个": small-matrix and split-K kernels chosen by the batch
+ * shape). Steps whose batch is at least min_batch run the tensor-core kernel:
+ * every weight tile is 128 rows (M) and all token rows of the batch, or all slot
+ * rows of one expert, are the MMA's N columns (rounded up to 16), so each selected
+ * expert's weights stream once however many rows chose it, and the products
+ * accumulate in tensor memory. Smaller batches run the CUDA-core kernel (fp32 FMA
+ * GEMV over 4 token rows at a time). min_batch = 0 keeps every step on the
+ * CUDA-core kernel. The tensor-core kernel needs hidden, inter, shared_inter and
+ * n_experts to be multiples of 128 and max_batch <= 64; for other shapes every
+ * step takes the CUDA-core kernel whatever min_batch says. Default min_batch: 1
+ * (the tensor-core kernel measured faster at every batch size, batch 1 included).
+ * Returns MOE_ERR_INVALID_ARG for a null handle or a negative min_batch. */
+int moe_decode_set_tc_min_batch(moe_decode_handle* h, int min_batch);
+
+/* The path a step of `batch` rows takes on this handle: MOE_PATH_CUDA_CORE or
+ * MOE_PATH_TENSOR_CORE (MOE_ERR_INVALID_ARG for a null handle or a batch outside
+ * 1..max_batch). */
+int moe_decode_step_path(const moe_decode_handle* h, int batch);
 
 /* The same decode step for callers that cannot allocate device memory: code on a
  * path where cudaMalloc is not allowed (inside a framework or plugin that owns

@@ -34,6 +34,9 @@ MOE_ERR_NO_MEMORY = -8
 DEBUG_JITTER = 1
 DEBUG_WITHHOLD_NREADY = 2
 
+PATH_CUDA_CORE = 0
+PATH_TENSOR_CORE = 1
+
 
 def nvcc_command(out: str = LIB) -> list[str]:
     return ["nvcc", "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
@@ -102,6 +105,10 @@ def lib():
         L.moe_decode_trace_slots.restype = i
         L.moe_decode_set_debug.argtypes = [vp, u, u]
         L.moe_decode_set_debug.restype = i
+        L.moe_decode_set_tc_min_batch.argtypes = [vp, i]
+        L.moe_decode_set_tc_min_batch.restype = i
+        L.moe_decode_step_path.argtypes = [vp, i]
+        L.moe_decode_step_path.restype = i
         L.moe_decode_destroy.argtypes = [vp]
         L.moe_decode_destroy.restype = None
         L.moe_decode_step_noalloc.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerWeights),
@@ -219,6 +226,17 @@ class MoeDecode:
 
     def set_debug(self, flags: int, wait_ms: int = 2000) -> None:
         _check(lib().moe_decode_set_debug(self.handle, int(flags), int(wait_ms)), "moe_decode_set_debug")
+
+    def set_tc_min_batch(self, min_batch: int) -> None:
+        """Steps of at least min_batch rows take the tensor-core kernel (0: never)."""
+        _check(lib().moe_decode_set_tc_min_batch(self.handle, int(min_batch)), "moe_decode_set_tc_min_batch")
+
+    def step_path(self, batch: int) -> int:
+        """PATH_CUDA_CORE or PATH_TENSOR_CORE: the kernel a step of `batch` rows runs."""
+        r = lib().moe_decode_step_path(self.handle, int(batch))
+        if r < 0:
+            _check(r, "moe_decode_step_path")
+        return r
 
     TRACE_FIELDS = ("start", "nready", "sched", "first_expert", "first_down", "prod_end", "mac_end",
                     "epi_end", "exit", "prod_wait_slot_cyc", "prod_wait_dep_cyc", "prod_grab_cyc",

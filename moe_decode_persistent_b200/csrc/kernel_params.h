@@ -7,6 +7,9 @@
 namespace moe {
 
 // Tensor-map slots of one layer (all 2-D, bf16, row-major [rows][K]).
+// Slots 0-6: CUDA-core path, boxes of 32 rows x up to 256 K columns, no swizzle.
+// Slots 7-16: tensor-core path, 128-byte swizzled boxes of 64 K columns (the
+// K-major operand layout tcgen05.mma reads): weights 128 rows, activations 16 rows.
 enum TensorMapSlot {
   TM_WR = 0,   // W_router  [E][H]
   TM_WG = 1,   // W_gate    [E*I][H]
@@ -15,7 +18,17 @@ enum TensorMapSlot {
   TM_WSG = 4,  // Ws_gate   [Is][H]
   TM_WSU = 5,  // Ws_up     [Is][H]
   TM_WSD = 6,  // Ws_down   [H][Is]
-  TM_COUNT = 7
+  TM_T_WR = 7,
+  TM_T_WG = 8,
+  TM_T_WU = 9,
+  TM_T_WD = 10,
+  TM_T_WSG = 11,
+  TM_T_WSU = 12,
+  TM_T_WSD = 13,
+  TM_T_AN = 14,   // normalised rows n  [max_batch][H]
+  TM_T_AHS = 15,  // shared SwiGLU rows [max_batch][Is]
+  TM_T_AHE = 16,  // expert SwiGLU rows [slots][I]
+  TM_COUNT = 17
 };
 
 // Global counters of one step (reset by the last CTA of every launch).
@@ -37,11 +50,31 @@ constexpr int kDownPairsPerSplit = 2;  // (expert, row-group) pairs per down spl
 constexpr int kPartialFloats = 2 * kBoxRows * kActGroup;  // floats per unit partial
 constexpr int kMaxE = 1024;
 constexpr int kMaxSlots = 1024;        // batch * top_k
+constexpr int kMaxTopK = 32;
+
+// Tensor-core path geometry.
+constexpr int kTcRows = 128;      // M of one tcgen05 tile (weight rows)
+constexpr int kTcAtomK = 64;      // K elements of one 128-byte swizzle atom
+constexpr int kTcActRows = 16;    // activation rows per TMA box (MMA N granule)
+constexpr int kTcMaxN = 64;       // token columns of one tile (max batch)
+constexpr int kTcSharedSplits = 4;
+constexpr int kTcExpertSplits = 4;
+
+// K splits of a router tile pair on the tensor-core path: many short units when the
+// batch is small (the router is on the critical path and its fix-up is cheap), fewer
+// as the batch grows (the fix-up reads splits x batch x 256 partial sums).
+__host__ __device__ inline int tc_router_splits(int B, int nk_atoms) {
+  const int s = B <= 8 ? 28 : B <= 16 ? 14 : B <= 32 ? 8 : 4;
+  return s < nk_atoms ? s : nk_atoms;
+}
+__host__ __device__ inline int tc_clamp_splits(int s, int nk_atoms) { return s < nk_atoms ? s : nk_atoms; }
 
 struct Params {
   // shapes of this step
   int H, E, I, Is, B, k;
   float eps;
+  int tc;          // 1: tensor-core path (tcgen05 tiles), 0: CUDA-core path
+  int RS, SS, ES;  // tensor-core path: K splits of router / shared gate-up / expert gate-up units
   // activations
   const uint16_t* x;  // bf16 [B][H]
   uint16_t* y;        // bf16 [B][H]
@@ -57,7 +90,12 @@ struct Params {
   float* logits;         // fp32 [maxB][E]
   uint16_t* hs;          // bf16 [maxB][Is]
   uint16_t* he;          // bf16 [maxSlots][I]
-  float* partial;        // fp32 [max_units][kPartialFloats]
+  float* partial;        // fp32 [max_units][kPartialFloats] (CUDA-core path)
+  // tensor-core path split-K partial sums (fp32)
+  float* rpart;          // [RS][B][E]
+  float* spart;          // [SS][B][Is/128][256]
+  float* epart;          // [ES][B*k][I/128][256]
+  float* dpart;          // [B*k + B][H]: down outputs of expert slot rows, then shared rows
   uint32_t* ctr;         // [CTR_COUNT]
   uint32_t* tickets;     // [max_tiles]
   uint32_t* pair_done;   // [kMaxSlots]

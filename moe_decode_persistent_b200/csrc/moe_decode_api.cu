@@ -14,6 +14,10 @@ size_t smem_bytes();
 int threads_per_cta();
 const void* kernel_fn();
 const void* kernel_fn_trace();
+size_t tc_smem_bytes();
+int tc_threads_per_cta();
+const void* tc_kernel_fn();
+const void* tc_kernel_fn_trace();
 }  // namespace moe
 
 using moe::Params;
@@ -36,6 +40,10 @@ struct moe_decode_handle {
   uint16_t* hs;
   uint16_t* he;
   float* partial;
+  float* rpart;
+  float* spart;
+  float* epart;
+  float* dpart;
   uint32_t* ctr;
   uint32_t* tickets;
   uint32_t* pair_done;
@@ -44,6 +52,8 @@ struct moe_decode_handle {
   uint16_t* x_stage;     // [max_batch][H] host-step staging
   uint16_t* y_stage;
   unsigned max_units, max_tiles;
+  int tc_capable;    // every dimension a multiple of 128: the tensor-core kernel can run
+  int tc_min_batch;  // batches of at least this many rows take the tensor-core path
   unsigned flags;
   unsigned long long wait_ns;
   unsigned long long* trace;  // nullable [n_layers][num_sms][kTraceSlots]
@@ -55,18 +65,42 @@ static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 static bool tile_dim_ok(int v) { return v >= 32 && v % 32 == 0 && (v % 256 == 0 || v <= 256); }
 
-static int encode_2d(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint64_t rows,
-                     uint64_t cols) {
+// Default batch threshold of the tensor-core path: every batch size. On the measured
+// 7168-wide layers the tensor-core kernel was faster at batch 1 as well (179 vs
+// 211 us per step): it takes the weight tiles straight from shared memory into the
+// MMA, where the CUDA-core kernel spends issue slots on unpacking and FMAs.
+static const int kDefaultTcMinBatch = 1;
+
+static int encode_box(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
   if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return MOE_ERR_INVALID_ARG;
-  const uint32_t box_cols = cols < (uint64_t)moe::kBoxColsMax ? (uint32_t)cols : (uint32_t)moe::kBoxColsMax;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * 2};
-  cuuint32_t box[2] = {box_cols, (cuuint32_t)moe::kBoxRows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// CUDA-core path boxes: 32 rows x min(cols, 256) columns, no swizzle.
+static int encode_2d(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint64_t rows,
+                     uint64_t cols) {
+  const uint32_t box_cols = cols < (uint64_t)moe::kBoxColsMax ? (uint32_t)cols : (uint32_t)moe::kBoxColsMax;
+  return encode_box(enc, map, base, rows, cols, box_cols, (uint32_t)moe::kBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Tensor-core path boxes: 64 columns (one 128-byte swizzle atom) x `box_rows` rows.
+static int encode_tc(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                     uint32_t box_rows) {
+  return encode_box(enc, map, base, rows, cols, (uint32_t)moe::kTcAtomK, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+static bool tc_shape_ok(const moe_decode_config& c) {
+  const int R = moe::kTcRows;
+  return c.hidden % R == 0 && c.inter % R == 0 && c.shared_inter % R == 0 && c.n_experts % R == 0 &&
+         c.max_batch <= moe::kTcMaxN;
 }
 
 extern "C" {
@@ -126,6 +160,19 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe::kernel_fn(), moe::threads_per_cta(),
                                                     smem);
   if (e != cudaSuccess || per_sm < 1) return MOE_ERR_COOPERATIVE;
+  // the tensor-core kernel: only for shapes whose every dimension is a multiple of 128
+  int tc_ok = tc_shape_ok(c) ? 1 : 0;
+  if (tc_ok) {
+    const size_t tsm = moe::tc_smem_bytes();
+    e = cudaFuncSetAttribute(moe::tc_kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::tc_kernel_fn_trace(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    int tc_per_sm = 0;
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&tc_per_sm, moe::tc_kernel_fn(), moe::tc_threads_per_cta(),
+                                                        tsm);
+    if (e != cudaSuccess || tc_per_sm < 1) return MOE_ERR_COOPERATIVE;
+  }
 
   void* fn = nullptr;
   cudaDriverEntryPointQueryResult q;
@@ -139,12 +186,20 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   h->device = device;
   h->num_sms = sms;
   h->wait_ns = 2000ull * 1000000ull;
+  h->tc_capable = tc_ok;
+  h->tc_min_batch = kDefaultTcMinBatch;
   h->layers = (moe_decode_layer_weights*)malloc(sizeof(moe_decode_layer_weights) * c.n_layers);
   memcpy(h->layers, layers, sizeof(moe_decode_layer_weights) * c.n_layers);
 
   const int H = c.hidden, E = c.n_experts, I = c.inter, Is = c.shared_inter, L = c.n_layers;
   // host tensor maps
   CUtensorMap* maps = (CUtensorMap*)aligned_alloc(64, sizeof(CUtensorMap) * moe::TM_COUNT * L);
+  if (!maps) {
+    free(h->layers);
+    free(h);
+    return MOE_ERR_NO_MEMORY;
+  }
+  memset(maps, 0, sizeof(CUtensorMap) * moe::TM_COUNT * L);
   int rc = MOE_OK;
   for (int l = 0; l < L && rc == MOE_OK; ++l) {
     const moe_decode_layer_weights& w = layers[l];
@@ -156,6 +211,16 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
     rc |= encode_2d(enc, &m[moe::TM_WSG], w.ws_gate, (uint64_t)Is, (uint64_t)H);
     rc |= encode_2d(enc, &m[moe::TM_WSU], w.ws_up, (uint64_t)Is, (uint64_t)H);
     rc |= encode_2d(enc, &m[moe::TM_WSD], w.ws_down, (uint64_t)H, (uint64_t)Is);
+    if (tc_ok) {
+      const uint32_t R = (uint32_t)moe::kTcRows;
+      rc |= encode_tc(enc, &m[moe::TM_T_WR], w.w_router, (uint64_t)E, (uint64_t)H, R);
+      rc |= encode_tc(enc, &m[moe::TM_T_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H, R);
+      rc |= encode_tc(enc, &m[moe::TM_T_WU], w.w_up, (uint64_t)E * I, (uint64_t)H, R);
+      rc |= encode_tc(enc, &m[moe::TM_T_WD], w.w_down, (uint64_t)E * H, (uint64_t)I, R);
+      rc |= encode_tc(enc, &m[moe::TM_T_WSG], w.ws_gate, (uint64_t)Is, (uint64_t)H, R);
+      rc |= encode_tc(enc, &m[moe::TM_T_WSU], w.ws_up, (uint64_t)Is, (uint64_t)H, R);
+      rc |= encode_tc(enc, &m[moe::TM_T_WSD], w.ws_down, (uint64_t)H, (uint64_t)Is, R);
+    }
   }
   if (rc != MOE_OK) {
     free(maps);
@@ -175,6 +240,32 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   h->max_units = (unsigned)(GB * RT * KS + GB * ST * KS + maxP * IT * KS +
                             DT * (GB + (maxP + moe::kDownPairsPerSplit - 1) / moe::kDownPairsPerSplit));
   h->max_tiles = (unsigned)(GB * (RT + ST) + maxP * IT + DT);
+  // tensor-core path: tile pairs of the router and of the down projection, one pair per
+  // unique expert, K splits chosen per batch (tc_router_splits) and fixed otherwise
+  const int nkH = H / moe::kTcAtomK;
+  size_t rpart_floats = 0, spart_floats = 0, epart_floats = 0, dpart_floats = 0;
+  const int tcS = moe::tc_clamp_splits(moe::kTcSharedSplits, nkH);
+  const int tcE = moe::tc_clamp_splits(moe::kTcExpertSplits, nkH);
+  if (tc_ok) {
+    const int RT2 = (E + 2 * moe::kTcRows - 1) / (2 * moe::kTcRows), DT2 = (H + 2 * moe::kTcRows - 1) / (2 * moe::kTcRows);
+    const int TST = Is / moe::kTcRows, TIT = I / moe::kTcRows;
+    const int tcP = maxSlots < E ? maxSlots : E;
+    int maxRS = 1;
+    for (int bb = 1; bb <= maxB; ++bb) {
+      const int rs = moe::tc_router_splits(bb, nkH);
+      if ((size_t)rs * bb > rpart_floats) rpart_floats = (size_t)rs * bb;
+      if (rs > maxRS) maxRS = rs;
+    }
+    rpart_floats *= (size_t)E;
+    spart_floats = (size_t)tcS * maxB * 2 * Is;
+    epart_floats = (size_t)tcE * maxSlots * 2 * I;
+    dpart_floats = (size_t)(maxSlots + maxB) * H;
+    const unsigned tu = (unsigned)(RT2 * maxRS + TST * tcS + tcP * TIT * tcE + DT2 * (1 + tcP));
+    const unsigned tt = (unsigned)(RT2 + TST + tcP * TIT + DT2);
+    if (tu > h->max_units) h->max_units = tu;
+    if (tt > h->max_tiles) h->max_tiles = tt;
+  }
+  const int actRows = (maxB + moe::kTcActRows - 1) / moe::kTcActRows * moe::kTcActRows;
 
   size_t off = 0;
   auto carve = [&](size_t bytes) {
@@ -182,11 +273,15 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
     off = align_up(off + bytes, 256);
     return o;
   };
-  const size_t o_n = carve((size_t)maxB * H * 2);
+  const size_t o_n = carve((size_t)actRows * H * 2);
   const size_t o_logits = carve((size_t)maxB * E * 4);
-  const size_t o_hs = carve((size_t)maxB * Is * 2);
+  const size_t o_hs = carve((size_t)actRows * Is * 2);
   const size_t o_he = carve((size_t)moe::kMaxSlots * I * 2);
   const size_t o_part = carve((size_t)h->max_units * moe::kPartialFloats * 4);
+  const size_t o_rpart = carve(rpart_floats * 4);
+  const size_t o_spart = carve(spart_floats * 4);
+  const size_t o_epart = carve(epart_floats * 4);
+  const size_t o_dpart = carve(dpart_floats * 4);
   const size_t o_ctr = carve(moe::CTR_COUNT * 4);
   const size_t o_tix = carve((size_t)h->max_tiles * 4);
   const size_t o_pd = carve(moe::kMaxSlots * 4);
@@ -208,6 +303,10 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   h->hs = (uint16_t*)(b + o_hs);
   h->he = (uint16_t*)(b + o_he);
   h->partial = (float*)(b + o_part);
+  h->rpart = (float*)(b + o_rpart);
+  h->spart = (float*)(b + o_spart);
+  h->epart = (float*)(b + o_epart);
+  h->dpart = (float*)(b + o_dpart);
   h->ctr = (uint32_t*)(b + o_ctr);
   h->tickets = (uint32_t*)(b + o_tix);
   h->pair_done = (uint32_t*)(b + o_pd);
@@ -216,6 +315,23 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   h->x_stage = (uint16_t*)(b + o_xs);
   h->y_stage = (uint16_t*)(b + o_ys);
   h->d_tmaps = (CUtensorMap*)(b + o_maps);
+  if (tc_ok) {
+    // activation operands of the tensor-core path (the same buffers in every layer)
+    const uint32_t AR = (uint32_t)moe::kTcActRows;
+    for (int l = 0; l < L && rc == MOE_OK; ++l) {
+      CUtensorMap* m = maps + l * moe::TM_COUNT;
+      rc |= encode_tc(enc, &m[moe::TM_T_AN], h->n, (uint64_t)actRows, (uint64_t)H, AR);
+      rc |= encode_tc(enc, &m[moe::TM_T_AHS], h->hs, (uint64_t)actRows, (uint64_t)Is, AR);
+      rc |= encode_tc(enc, &m[moe::TM_T_AHE], h->he, (uint64_t)moe::kMaxSlots, (uint64_t)I, AR);
+    }
+    if (rc != MOE_OK) {
+      cudaFree(h->ws);
+      free(maps);
+      free(h->layers);
+      free(h);
+      return MOE_ERR_CUDA;
+    }
+  }
   // counters, tickets, flags and status start at zero; activations zeroed for hygiene
   e = cudaMemset(h->ws, 0, off);
   if (e == cudaSuccess)
@@ -232,10 +348,16 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   return MOE_OK;
 }
 
+static bool use_tc(const moe_decode_handle* h, int batch) {
+  return h->tc_capable && h->tc_min_batch > 0 && batch >= h->tc_min_batch;
+}
+
 static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, int batch, int top_k,
                          cudaStream_t stream, const moe_decode_debug* dbg) {
   const moe_decode_config& c = h->cfg;
   const int L = c.n_layers;
+  const bool tc = use_tc(h, batch);
+  const int nkH = c.hidden / moe::kTcAtomK;
   for (int l = 0; l < L; ++l) {
     Params p;
     memset(&p, 0, sizeof p);
@@ -268,6 +390,16 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     p.hs = h->hs;
     p.he = h->he;
     p.partial = h->partial;
+    p.tc = tc ? 1 : 0;
+    if (tc) {
+      p.RS = moe::tc_router_splits(batch, nkH);
+      p.SS = moe::tc_clamp_splits(moe::kTcSharedSplits, nkH);
+      p.ES = moe::tc_clamp_splits(moe::kTcExpertSplits, nkH);
+      p.rpart = h->rpart;
+      p.spart = h->spart;
+      p.epart = h->epart;
+      p.dpart = h->dpart;
+    }
     p.ctr = h->ctr;
     p.tickets = h->tickets;
     p.pair_done = h->pair_done;
@@ -284,9 +416,11 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     p.wait_ns = h->wait_ns;
     p.trace = h->trace ? h->trace + (size_t)l * h->num_sms * moe::kTraceSlots : nullptr;
     void* args[] = {&p};
-    const void* fn = h->trace ? moe::kernel_fn_trace() : moe::kernel_fn();
-    cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(h->num_sms), dim3(moe::threads_per_cta()),
-                                                args, moe::smem_bytes(), stream);
+    const void* fn = tc ? (h->trace ? moe::tc_kernel_fn_trace() : moe::tc_kernel_fn())
+                        : (h->trace ? moe::kernel_fn_trace() : moe::kernel_fn());
+    const int threads = tc ? moe::tc_threads_per_cta() : moe::threads_per_cta();
+    const size_t smem = tc ? moe::tc_smem_bytes() : moe::smem_bytes();
+    cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(h->num_sms), dim3(threads), args, smem, stream);
     if (e == cudaErrorCooperativeLaunchTooLarge) return MOE_ERR_COOPERATIVE;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
@@ -344,6 +478,17 @@ int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms)
   h->flags = flags;
   h->wait_ns = (unsigned long long)wait_ms * 1000000ull;
   return MOE_OK;
+}
+
+int moe_decode_set_tc_min_batch(moe_decode_handle* h, int min_batch) {
+  if (!h || min_batch < 0) return MOE_ERR_INVALID_ARG;
+  h->tc_min_batch = min_batch;
+  return MOE_OK;
+}
+
+int moe_decode_step_path(const moe_decode_handle* h, int batch) {
+  if (!h || batch < 1 || batch > h->cfg.max_batch) return MOE_ERR_INVALID_ARG;
+  return use_tc(h, batch) ? MOE_PATH_TENSOR_CORE : MOE_PATH_CUDA_CORE;
 }
 
 int moe_decode_trace_slots(const moe_decode_handle* h) {

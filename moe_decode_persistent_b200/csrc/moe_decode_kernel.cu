@@ -65,6 +65,26 @@ constexpr int kSlotBytes = 2 * kBoxBytesMax + 2 * kActSegBytes;   // 36 KB
 constexpr int kStages = 5;
 constexpr int kKSplits = 4;
 constexpr int kRB = 4;  // MAC -> epilogue result buffers
+constexpr int kCcRingBytes = kStages * kSlotBytes;
+
+// Tensor-core path: warp 0 producer, warps 1-8 RMSNorm + routing schedule, warp 9
+// MMA issuer (owns tensor memory), warps 10-13 tensor-memory epilogue (one warp per
+// 32-lane quadrant: warp w reads lanes 32 (w % 4) .. 32 (w % 4) + 31).
+constexpr int kTcMmaWarp = kMacWarps + 1;
+constexpr int kTcEpiWarp0 = kMacWarps + 2;
+constexpr int kTcEpiWarps = 4;
+constexpr int kTcThreads = 32 * (kTcEpiWarp0 + kTcEpiWarps);       // 448
+constexpr int kTcTileBytes = kTcRows * kTcAtomK * 2;               // 16 KB: 128 rows x 64 K
+constexpr int kTcActBytes = kTcMaxN * kTcAtomK * 2;                // 8 KB: <= 64 rows x 64 K
+constexpr int kTcSlotBytes = 2 * kTcTileBytes + kTcActBytes;       // 40 KB
+constexpr int kTcStages = 4;
+constexpr int kTcRingBytes = kTcStages * kTcSlotBytes;
+constexpr int kTcAccBufs = 4;       // accumulator buffers in tensor memory
+constexpr int kTcAccCols = 128;     // columns per buffer: tile 0 at +0, tile 1 at +64
+constexpr int kTmemCols = kTcAccBufs * kTcAccCols;  // 512 (a power of two >= 32)
+
+static_assert(kTcSlotBytes % 1024 == 0 && kTcTileBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(kCcRingBytes % 1024 == 0 && kTcRingBytes % 1024 == 0, "ring keeps the state block aligned");
 
 enum UnitType { UT_ROUTER = 0, UT_SHARED = 1, UT_EXPERT = 2, UT_DOWN_SHARED = 3, UT_DOWN_EXPERT = 4 };
 enum HeaderKind { HK_STAGE = 0, HK_SCHED = 1, HK_END = 2 };
@@ -80,8 +100,13 @@ struct StageHeader {
 };
 
 constexpr int kInfoKpair = 1 << 2, kInfoSegEnd = 1 << 6, kInfoUnitEnd = 1 << 7, kInfoFirst = 1 << 9;
+// Tensor-core stages: bits 0-1 weight tiles, 2-4 activation boxes of 16 rows (N / 16),
+// 5 first stage of the unit (overwrite the accumulator), 6 last stage of the unit.
+constexpr int kTcInfoFirst = 1 << 5, kTcInfoLast = 1 << 6;
 
 // Layout constants of one step (identical in every CTA).
+// On the tensor-core path RT and DT count tile pairs (256 rows), ST and IT 128-row
+// tiles, and the nkb* fields 64-column K atoms.
 struct Shape {
   int B, k, GB;
   int boxH, boxI, boxIs, nkbH, nkbI, nkbIs;
@@ -89,6 +114,8 @@ struct Shape {
   int RS, SS, ES;
   int NR, NS;
   int spp;  // stages per (expert, row group) pair of a down unit
+  int NA;   // tensor-core path: token columns of n- and hs-based tiles (B rounded up to 16)
+  int router_target, hs_target, pair_target;  // tiles that publish logits / h_s / one pair's h
 };
 
 // Routing schedule (identical in every CTA once built).
@@ -102,18 +129,28 @@ struct Sched {
   uint8_t pair_group[kMaxSlots];  // row group of pair p
   uint8_t row_of[kMaxSlots];      // token row of slot row r
   float w_of[kMaxSlots];          // routing weight of slot row r
+  int16_t slot_of[kMaxSlots];     // slot row of (token b, choice j) at b * k + j
 };
 
+// Per-CTA state. The stage ring (kCcRingBytes or kTcRingBytes) sits in front of it in
+// dynamic shared memory, 1024-byte aligned.
+constexpr int kMaxRingStages = kStages > kTcStages ? kStages : kTcStages;
 struct Smem {
-  uint8_t ring[kStages][kSlotBytes];
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  uint64_t full[kMaxRingStages];
+  uint64_t empty[kMaxRingStages];
   uint64_t sched_bar;       // schedule built (MAC warps -> producer)
   uint64_t mac_bar;         // MAC-warp rendezvous (bounded)
   uint64_t rb_full[kRB];    // MAC warps -> epilogue warp
   uint64_t rb_empty[kRB];   // epilogue warp -> MAC warps
-  StageHeader hdr[kStages];
+  uint64_t acc_full[kTcAccBufs];   // tensor-core path: MMA warp -> epilogue warps
+  uint64_t acc_empty[kTcAccBufs];  // epilogue warps -> MMA warp
+  uint64_t mma_bar;                // MMA warp: its last MMAs completed (drain)
+  uint64_t epi_bar;                // rendezvous of the tensor-core epilogue warps (bounded)
+  StageHeader hdr[kMaxRingStages];
   int rb_unit[kRB];         // unit id of the buffer, or -1 (stop)
+  int acc_unit[kTcAccBufs]; // unit id of the accumulator buffer, or -1 (stop)
+  uint32_t tmem_base;
+  int epi_last;             // tensor-core epilogue: this unit's split completed its tile
   int bcast;
   int bcast2;
   int nuniq;
@@ -134,9 +171,11 @@ struct Smem {
   } u;
 };
 
-static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget of one CTA");
+static_assert(kCcRingBytes + sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget of one CTA");
+static_assert(kTcRingBytes + sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget of one CTA");
 static_assert(offsetof(Smem, rb) % 16 == 0 && offsetof(Smem, fin) % 16 == 0, "float4 views of rb / fin");
-static_assert(offsetof(Smem, full) % 8 == 0 && offsetof(Smem, rb_full) % 8 == 0, "mbarrier alignment");
+static_assert(offsetof(Smem, full) % 8 == 0 && offsetof(Smem, rb_full) % 8 == 0 &&
+              offsetof(Smem, acc_full) % 8 == 0, "mbarrier alignment");
 static_assert(kSlotBytes % 1024 == 0 && kBoxBytesMax % 128 == 0 && kActSegBytes % 16 == 0,
               "TMA / bulk-copy destinations");
 static_assert(kRowsPerWarp == 4 && kActGroup == 4, "MAC lane mapping assumes 4 rows x 4 row slots");
@@ -300,6 +339,39 @@ __device__ void make_shape(const Params& p, Shape& s) {
   s.NR = s.GB * s.RT * s.RS;
   s.NS = s.GB * s.ST * s.SS;
   s.spp = (s.nkbI + 1) / 2;
+  s.NA = 0;
+  s.router_target = s.GB * s.RT;
+  s.hs_target = s.GB * s.ST;
+  s.pair_target = s.IT;
+}
+
+// Tensor-core path: router and down units cover a pair of 128-row tiles (the second
+// absent when the rows end half-way), shared and expert gate/up units a 128-row tile
+// of the gate matrix with the same rows of the up matrix. Every token row of the batch
+// is one MMA column (N = B rounded up to 16) except on down-expert units, whose
+// columns are the expert's own slot rows.
+__device__ void make_shape_tc(const Params& p, Shape& s) {
+  s.B = p.B;
+  s.k = p.k;
+  s.GB = 1;
+  s.NA = (p.B + kTcActRows - 1) / kTcActRows * kTcActRows;
+  s.boxH = s.boxI = s.boxIs = kTcAtomK;
+  s.nkbH = p.H / kTcAtomK;
+  s.nkbI = p.I / kTcAtomK;
+  s.nkbIs = p.Is / kTcAtomK;
+  s.RT = (p.E + 2 * kTcRows - 1) / (2 * kTcRows);
+  s.ST = p.Is / kTcRows;
+  s.IT = p.I / kTcRows;
+  s.DT = (p.H + 2 * kTcRows - 1) / (2 * kTcRows);
+  s.RS = p.RS;
+  s.SS = p.SS;
+  s.ES = p.ES;
+  s.NR = s.RT * s.RS;
+  s.NS = s.ST * s.SS;
+  s.spp = 0;
+  s.router_target = s.RT;
+  s.hs_target = s.ST;
+  s.pair_target = s.IT;
 }
 
 __device__ __forceinline__ void split_range(int nkb, int nsplit, int s, int& kb0, int& nkb_s) {
@@ -361,6 +433,62 @@ __device__ UnitDesc decode_unit(const Shape& sh, const Sched& sc, int u) {
       d.nstages = d.npair * sh.spp;
     }
   }
+  return d;
+}
+
+// Tensor-core path unit enumeration (queue order): router (tile pair, K split),
+// shared gate/up (tile, K split), expert gate/up ((unique expert, tile), K split),
+// down (source, tile pair) with source 0 the shared expert and source 1 + i the
+// unique expert i. Down units carry no K split; their tile pair is finished by the
+// last of its B-independent 1 + U sources.
+__device__ UnitDesc decode_unit_tc(const Shape& sh, const Sched& sc, int u) {
+  UnitDesc d;
+  d.npair = 0;
+  d.pair = 0;
+  d.g = 0;
+  if (u < sh.NR) {
+    d.type = UT_ROUTER;
+    d.tile = u / sh.RS;
+    d.split = u % sh.RS;
+    d.nsplit = sh.RS;
+    d.ticket = d.tile;
+    split_range(sh.nkbH, sh.RS, d.split, d.kb0, d.nkb);
+  } else if (u < sh.NR + sh.NS) {
+    const int v = u - sh.NR;
+    d.type = UT_SHARED;
+    d.tile = v / sh.SS;
+    d.split = v % sh.SS;
+    d.nsplit = sh.SS;
+    d.ticket = sh.RT + d.tile;
+    split_range(sh.nkbH, sh.SS, d.split, d.kb0, d.nkb);
+  } else if (u < sh.NR + sh.NS + sc.NE) {
+    const int v = u - sh.NR - sh.NS;
+    d.type = UT_EXPERT;
+    d.split = v % sh.ES;
+    d.tile = (v / sh.ES) % sh.IT;
+    d.pair = v / (sh.ES * sh.IT);
+    d.nsplit = sh.ES;
+    d.ticket = sh.RT + sh.ST + d.pair * sh.IT + d.tile;
+    split_range(sh.nkbH, sh.ES, d.split, d.kb0, d.nkb);
+  } else {
+    const int v = u - sh.NR - sh.NS - sc.NE;
+    const int src = v / sh.DT;
+    d.tile = v % sh.DT;
+    d.split = src;
+    d.nsplit = sc.down_splits;
+    d.ticket = sh.RT + sh.ST + sc.P * sh.IT + d.tile;
+    d.kb0 = 0;
+    if (src == 0) {
+      d.type = UT_DOWN_SHARED;
+      d.nkb = sh.nkbIs;
+    } else {
+      d.type = UT_DOWN_EXPERT;
+      d.pair = src - 1;
+      d.npair = 1;
+      d.nkb = sh.nkbI;
+    }
+  }
+  d.nstages = d.nkb;
   return d;
 }
 
@@ -714,15 +842,18 @@ __device__ void warp_topk_row(const Params& p, Smem& sm, int b, int lane) {
   }
 }
 
-// Builds sm.sc from the final logits. Called by all MAC warps; false on abort.
-template <bool kTrace>
+// Builds sm.sc from the final logits. Called by all MAC warps; false on abort. On the
+// CUDA-core path an expert's rows form pairs of up to kActGroup rows; on the
+// tensor-core path all of an expert's rows (at most the batch, <= 64) form one pair.
+template <bool kTrace, bool kTC>
 __device__ bool build_schedule(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
+  constexpr int kGroup = kTC ? kMaxSlots : kActGroup;
   const Shape& sh = sm.sh;
   Sched& sc = sm.sc;
   const int mtid = mw * 32 + lane;
   if (mw == 0) {
     int ok = 1;
-    if (lane == 0) ok = wait_counter(&p.ctr[CTR_ROUTER], (uint32_t)(sh.GB * sh.RT), p) ? 1 : 0;
+    if (lane == 0) ok = wait_counter(&p.ctr[CTR_ROUTER], (uint32_t)sh.router_target, p) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (lane == 0) sm.bcast = ok;
   }
@@ -772,7 +903,7 @@ __device__ bool build_schedule(const Params& p, Smem& sm, int mw, int lane, uint
     for (int i0 = 0; i0 < U; i0 += 32) {
       const int i = i0 + lane;
       const int c = i < U ? sc.slot_cnt[i] : 0;
-      const int gcount = (c + kActGroup - 1) / kActGroup;
+      const int gcount = (c + kGroup - 1) / kGroup;
       int cs = c, gs = gcount;  // inclusive scans
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -800,7 +931,7 @@ __device__ bool build_schedule(const Params& p, Smem& sm, int mw, int lane, uint
       sc.slot_base[U] = (int16_t)rbase;
       sc.P = pbase;
       sc.NE = pbase * sh.IT * sh.ES;
-      sc.down_splits = sh.GB + (pbase + kDownPairsPerSplit - 1) / kDownPairsPerSplit;
+      sc.down_splits = kTC ? 1 + pbase : sh.GB + (pbase + kDownPairsPerSplit - 1) / kDownPairsPerSplit;
       sc.ND = sh.DT * sc.down_splits;
       sc.total = sh.NR + sh.NS + sc.NE + sc.ND;
       const unsigned tiles = (unsigned)(sh.GB * (sh.RT + sh.ST) + pbase * sh.IT + sh.DT);
@@ -821,7 +952,10 @@ __device__ bool build_schedule(const Params& p, Smem& sm, int mw, int lane, uint
       m &= m - 1ull;
       float w = 0.0f;
       for (int j = 0; j < p.k; ++j)
-        if (sm.u.t.topk_idx[b * p.k + j] == e) w = sm.u.t.topk_w[b * p.k + j];
+        if (sm.u.t.topk_idx[b * p.k + j] == e) {
+          w = sm.u.t.topk_w[b * p.k + j];
+          sc.slot_of[b * p.k + j] = (int16_t)r;
+        }
       sc.row_of[r] = (uint8_t)b;
       sc.w_of[r] = w;
       ++r;
@@ -1014,226 +1148,86 @@ __device__ void epi_finish(const Params& p, Smem& sm, const UnitDesc& d, int u,
   }
 }
 
-// ---- the kernel ----------------------------------------------------------------------------------
+// ---- producer warp (both paths) ------------------------------------------------------------------
 
-template <bool kTrace>
-__global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __grid_constant__ Params p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
-  const int tid = threadIdx.x;
-  const int warp_id = tid / 32;
-  const int lane = tid % 32;
+// Ring position and the producer's waits. A slot's pending record is the phase of its
+// last TMA stage that no later use of the slot has shown to be complete.
+struct Producer {
+  const Params& p;
+  Smem& sm;
+  int lane;
+  int nst;  // ring stages
+  int slot;
+  uint32_t phase;
+  uint32_t pend_mask, pend_parity;
 
-  if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kMacWarps);
-    }
-    for (int b = 0; b < kRB; ++b) {
-      mbar_init(&sm.rb_full[b], kMacWarps);
-      mbar_init(&sm.rb_empty[b], 1);
-    }
-    mbar_init(&sm.sched_bar, 1);
-    mbar_init(&sm.mac_bar, kMacWarps);
-    make_shape(p, sm.sh);
-    for (int w = 0; w < kMaxSlots / 32; ++w) sm.known_done[w] = 0u;
-    if (kTrace) {
-      for (int t = 0; t < kTraceSlots; ++t) p.trace[(size_t)blockIdx.x * kTraceSlots + t] = 0ull;
-      trace_stamp<kTrace>(p, TR_START);
-    }
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  __device__ Producer(const Params& p_, Smem& sm_, int lane_, int nst_)
+      : p(p_), sm(sm_), lane(lane_), nst(nst_), slot(0), phase(0u), pend_mask(0u), pend_parity(0u) {}
+
+  __device__ int grab() {
+    int v = 0;
+    if (lane == 0) v = (int)atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
+    return __shfl_sync(0xffffffffu, v, 0);
   }
-  __syncthreads();
-  const Shape& sh = sm.sh;
+  __device__ void advance() {
+    if (++slot == nst) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+  __device__ void mark_pending() {
+    pend_mask |= 1u << slot;
+    pend_parity = (pend_parity & ~(1u << slot)) | (phase << slot);
+  }
+  __device__ bool wait_bar(uint64_t* bar, uint32_t parity) {
+    int r = 1;
+    if (lane == 0) r = wait_mbar(bar, parity, p) ? 1 : 0;
+    r = __shfl_sync(0xffffffffu, r, 0);
+    __syncwarp();
+    return r != 0;
+  }
+  // Waits for a free slot; the slot's previous stage has then been consumed.
+  __device__ bool wait_slot() {
+    const bool ok = wait_bar(&sm.empty[slot], phase ^ 1u);
+    return ok;
+  }
+  __device__ bool wait_dep(const uint32_t* c, uint32_t target) {
+    int r = 1;
+    if (lane == 0) {
+      r = wait_counter(c, target, p) ? 1 : 0;
+      fence_proxy_async_global();
+    }
+    r = __shfl_sync(0xffffffffu, r, 0);
+    __syncwarp();
+    return r != 0;
+  }
+  // (expert, row group) pair pr complete? One acquire round trip polls 32 pairs.
+  __device__ bool wait_pair(int pr) {
+    const Shape& sh = sm.sh;
+    if ((sm.known_done[pr >> 5] >> (pr & 31)) & 1u) return true;
+    const int q = pr + lane;
+    const bool done = q < sm.sc.P && ld_acquire_gpu(&p.pair_done[q]) >= (uint32_t)sh.pair_target;
+    const uint32_t bal = __ballot_sync(0xffffffffu, done);
+    if (lane == 0) {
+      for (int i = 0; i < 32; ++i)
+        if ((bal >> i) & 1u) sm.known_done[(pr + i) >> 5] |= 1u << ((pr + i) & 31);
+    }
+    __syncwarp();
+    bool r = (bal & 1u) != 0u;
+    if (!r) {
+      r = wait_dep(&p.pair_done[pr], (uint32_t)sh.pair_target);
+      if (r && lane == 0) sm.known_done[pr >> 5] |= 1u << (pr & 31);
+      __syncwarp();
+    } else if (lane == 0) {
+      fence_proxy_async_global();
+    }
+    return r;
+  }
 
-  if (warp_id == 0) {
-    // =========================== producer warp ===========================
-    const uint64_t pol = policy_evict_first();
-    if (lane == 0)
-      for (int t = 0; t < TM_COUNT; ++t) prefetch_tensormap(&p.tmaps[t]);
-    int slot = 0;
-    uint32_t phase = 0;
-    // slots whose last TMA stage no later use has shown complete, and that stage's parity
-    uint32_t pend_mask = 0u, pend_parity = 0u;
-    bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
-    const int pre = sh.NR + sh.NS;
-    auto grab = [&]() -> int {
-      int v = 0;
-      if (lane == 0) v = (int)atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
-      return __shfl_sync(0xffffffffu, v, 0);
-    };
-    auto advance = [&]() {
-      if (++slot == kStages) {
-        slot = 0;
-        phase ^= 1u;
-      }
-    };
-    auto wait_bar = [&](uint64_t* bar, uint32_t parity) -> bool {
-      int r = 1;
-      if (lane == 0) r = wait_mbar(bar, parity, p) ? 1 : 0;
-      r = __shfl_sync(0xffffffffu, r, 0);
-      __syncwarp();
-      return r != 0;
-    };
-    auto wait_dep = [&](const uint32_t* c, uint32_t target) -> bool {
-      int r = 1;
-      if (lane == 0) {
-        r = wait_counter(c, target, p) ? 1 : 0;
-        fence_proxy_async_global();
-      }
-      r = __shfl_sync(0xffffffffu, r, 0);
-      __syncwarp();
-      return r != 0;
-    };
-    // (expert, row group) pair pr complete? One acquire round trip polls 32 pairs.
-    auto wait_pair = [&](int pr) -> bool {
-      if ((sm.known_done[pr >> 5] >> (pr & 31)) & 1u) return true;
-      const int q = pr + lane;
-      const bool done = q < sm.sc.P && ld_acquire_gpu(&p.pair_done[q]) >= (uint32_t)sh.IT;
-      const uint32_t bal = __ballot_sync(0xffffffffu, done);
-      if (lane == 0) {
-        for (int i = 0; i < 32; ++i)
-          if ((bal >> i) & 1u) sm.known_done[(pr + i) >> 5] |= 1u << ((pr + i) & 31);
-      }
-      __syncwarp();
-      bool r = (bal & 1u) != 0u;
-      if (!r) {
-        r = wait_dep(&p.pair_done[pr], (uint32_t)sh.IT);
-        if (r && lane == 0) sm.known_done[pr >> 5] |= 1u << (pr & 31);
-        __syncwarp();
-      } else if (lane == 0) {
-        fence_proxy_async_global();
-      }
-      return r;
-    };
-    int u = grab();
-    bool first_expert = true, first_down = true;
-    unsigned long long c_slot = 0, c_dep = 0, c_grab = 0, c_issue = 0, c_stages = 0, c_units = 0;
-    unsigned long long c_setup = 0, c_schedw = 0;
-    const long long tploop0 = tclock<kTrace>();
-    while (ok) {
-      if (u >= pre && !sched_ready) {
-        ok = wait_bar(&sm.empty[slot], phase ^ 1u);
-        if (!ok) break;
-        pend_mask &= ~(1u << slot);  // the slot's previous stage was consumed
-        if (lane == 0) {
-          sm.hdr[slot].kind = HK_SCHED;
-          mbar_arrive(&sm.full[slot]);
-        }
-        __syncwarp();
-        advance();
-        const long long tw0 = tclock<kTrace>();
-        ok = wait_bar(&sm.sched_bar, 0u);
-        c_schedw += (unsigned long long)(tclock<kTrace>() - tw0);
-        if (!ok) break;
-        sched_ready = true;
-        if (lane == 0) trace_stamp<kTrace>(p, TR_SCHED);
-      }
-      if (sched_ready && u >= sm.sc.total) break;
-      const long long tu0 = tclock<kTrace>();
-      const UnitDesc d = decode_unit(sh, sm.sc, u);
-      // the next unit's queue ticket is requested now and read after this unit's
-      // stages are issued, so the atomic's round trip overlaps the issue loop
-      uint32_t next_ticket = 0;
-      if (lane == 0) next_ticket = atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
-      if (lane == 0 && kTrace) {
-        if (first_expert && d.type == UT_EXPERT) { trace_stamp<kTrace>(p, TR_FIRST_EXPERT); first_expert = false; }
-        if (first_down && (d.type == UT_DOWN_SHARED || d.type == UT_DOWN_EXPERT)) { trace_stamp<kTrace>(p, TR_FIRST_DOWN); first_down = false; }
-        ++c_units;
-      }
-      if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(blockIdx.x * 7919u + (uint32_t)u) % 3000u);
-      const int nseg_units = d.type == UT_DOWN_EXPERT ? d.npair : 1;
-      c_setup += (unsigned long long)(tclock<kTrace>() - tu0);
-      for (int q = 0; q < nseg_units && ok; ++q) {
-        SegCtx x;
-        const long long tm0 = tclock<kTrace>();
-        make_seg(p, sh, sm.sc, d, q, x);
-        c_setup += (unsigned long long)(tclock<kTrace>() - tm0);
-        const uint32_t box_bytes = (uint32_t)(x.box_cols * kBoxRows * 2);
-        const uint32_t row_bytes = (uint32_t)(x.box_cols * 2);
-        const int step = x.kpair ? 2 : 1;
-        const int info0 = (x.kpair ? kInfoKpair : 0) | (x.c << 3) | (q << 8) | (x.box_cols << 16);
-        for (int kb = x.kb0; kb < x.kb_end && ok; kb += step) {
-          {
-            const long long t0 = tclock<kTrace>();
-            ok = wait_bar(&sm.empty[slot], phase ^ 1u);
-            c_slot += (unsigned long long)(tclock<kTrace>() - t0);
-          }
-          if (!ok) break;
-          const long long ti0 = tclock<kTrace>();
-          const int nbox = x.kpair ? (x.kb_end - kb < 2 ? 1 : 2) : 2;
-          const int nseg = x.kpair ? nbox : 1;
-          const bool seg_end = kb + step >= x.kb_end;
-          uint8_t* dst = sm.ring[slot];
-          uint64_t* fb = &sm.full[slot];
-          pend_mask |= 1u << slot;
-          pend_parity = (pend_parity & ~(1u << slot)) | (phase << slot);
-          if (lane == 0) {
-            StageHeader h;
-            h.kind = HK_STAGE;
-            h.unit = u;
-            h.info = info0 | nbox | (seg_end ? kInfoSegEnd : 0) | (seg_end && q == nseg_units - 1 ? kInfoUnitEnd : 0) |
-                     (kb == x.kb0 && q == 0 ? kInfoFirst : 0);
-            h.wrow = x.wrow;
-            sm.hdr[slot] = h;
-            mbar_arrive_expect_tx(fb, (uint32_t)nbox * box_bytes + (uint32_t)(nseg * x.c) * row_bytes);
-            const int col = kb * x.box_cols;
-            tma_load_2d(dst, x.tm0, col, x.y0, fb, pol);
-            if (nbox == 2) tma_load_2d(dst + kBoxBytesMax, x.tm1, x.kpair ? col + x.box_cols : col, x.y0, fb, pol);
-          }
-          // activations: only after the acquire that publishes them
-          bool dep_ok = true;
-          const long long td0 = tclock<kTrace>();
-          if (kb == x.kb0) {
-            if (x.dep == 0) {
-              if (!n_ok) {
-                dep_ok = n_ok = wait_dep(&p.ctr[CTR_NREADY], (uint32_t)p.B);
-                if (lane == 0) trace_stamp<kTrace>(p, TR_NREADY);
-              }
-            } else if (x.dep == 1) {
-              if (!hs_ok) dep_ok = hs_ok = wait_dep(&p.ctr[CTR_HS], (uint32_t)(sh.GB * sh.ST));
-            } else {
-              dep_ok = wait_pair(x.pair);
-            }
-          }
-          const long long td1 = tclock<kTrace>();
-          c_dep += (unsigned long long)(td1 - td0);
-          if (lane == 0) {
-            uint8_t* act = dst + 2 * kBoxBytesMax;
-            for (int sg = 0; sg < nseg; ++sg) {
-              const int col = (kb + sg) * x.box_cols;
-#pragma unroll
-              for (int j = 0; j < kActGroup; ++j)
-                if (j < x.c) bulk_load(act + sg * kActSegBytes + j * row_bytes, x.abase + x.aoff[j] + col, row_bytes, fb);
-            }
-          }
-          __syncwarp();
-          advance();
-          c_issue += (unsigned long long)(tclock<kTrace>() - ti0) - (unsigned long long)(td1 - td0);
-          ++c_stages;
-          if (!dep_ok) ok = false;
-        }
-      }
-      {
-        const long long t0 = tclock<kTrace>();
-        u = __shfl_sync(0xffffffffu, (int)next_ticket, 0);
-        c_grab += (unsigned long long)(tclock<kTrace>() - t0);
-      }
-    }
-    if (lane == 0 && kTrace) {
-      trace_stamp<kTrace>(p, TR_PROD_END);
-      trace_put<kTrace>(p, TR_PROD_WAIT_SLOT_CYC, c_slot);
-      trace_put<kTrace>(p, TR_PROD_WAIT_DEP_CYC, c_dep);
-      trace_put<kTrace>(p, TR_PROD_GRAB_CYC, c_grab);
-      trace_put<kTrace>(p, TR_PROD_ISSUE_CYC, c_issue);
-      trace_put<kTrace>(p, TR_PROD_STAGES, c_stages);
-      trace_put<kTrace>(p, TR_UNITS, c_units);
-      trace_put<kTrace>(p, TR_PROD_SETUP_CYC, c_setup);
-      trace_put<kTrace>(p, TR_PROD_SCHED_CYC, c_schedw);
-      trace_put<kTrace>(p, TR_PROD_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tploop0));
-    }
-    // tell the MAC warps to stop (bounded)
-    if (wait_bar(&sm.empty[slot], phase ^ 1u)) {
+  // After the last stage: the stop header, the drain of every bulk copy still in
+  // flight, and the L2 prefetch of the next layer's router and shared-expert weights.
+  __device__ void finish() {
+    if (wait_slot()) {
       pend_mask &= ~(1u << slot);
       if (lane == 0) {
         sm.hdr[slot].kind = HK_END;
@@ -1241,18 +1235,14 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
       }
     }
     __syncwarp();
-    // drain: every issued bulk copy must have landed before the CTA exits. A slot's
-    // record is the phase of its last TMA stage that no later use of the slot has
-    // shown to be complete (only possible after an abort).
     if (lane == 0) {
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < nst; ++s) {
         if (!((pend_mask >> s) & 1u)) continue;
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&sm.full[s], (pend_parity >> s) & 1u)) {
           if (globaltimer_ns() - t0 > 50000000ull) break;
         }
       }
-      // L2 prefetch of the next layer's router and shared-expert weights
       for (int r = 0; r < 4; ++r) {
         if (!p.pf_ptr[r] || !p.pf_bytes[r]) continue;
         const unsigned long long tot = p.pf_bytes[r];
@@ -1267,140 +1257,928 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
       }
     }
     __syncwarp();
-  } else if (warp_id <= kMacWarps) {
-    // =========================== MAC warps ===========================
-    const int mw = warp_id - 1;
-    uint32_t mphase = 0;
-    bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
-    int slot = 0;
-    uint32_t phase = 0;
-    int ub = 0;
-    uint32_t ubphase = 0;
-    bool rb_claimed = false;
-    float acc[2][kRowsPerWarp][kActGroup];
-    zero_acc(acc);
-    const long long tloop0 = tclock<kTrace>();
-    unsigned long long c_full = 0, c_rb = 0, c_comp = 0, c_st = 0, c_sched = 0, c_red = 0;
-    while (ok) {
+  }
+};
+
+// CUDA-core path producer: units of 32 weight rows, activation rows by 1-D bulk copies.
+template <bool kTrace>
+__device__ void producer_cc(Producer& pr, uint8_t* ring) {
+  const Params& p = pr.p;
+  Smem& sm = pr.sm;
+  const Shape& sh = sm.sh;
+  const int lane = pr.lane;
+  const uint64_t pol = policy_evict_first();
+  if (lane == 0)
+    for (int t = 0; t < TM_T_WR; ++t) prefetch_tensormap(&p.tmaps[t]);
+  bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
+  const int pre = sh.NR + sh.NS;
+  int u = pr.grab();
+  bool first_expert = true, first_down = true;
+  unsigned long long c_slot = 0, c_dep = 0, c_grab = 0, c_issue = 0, c_stages = 0, c_units = 0;
+  unsigned long long c_setup = 0, c_schedw = 0;
+  const long long tploop0 = tclock<kTrace>();
+  while (ok) {
+    if (u >= pre && !sched_ready) {
+      ok = pr.wait_slot();
+      if (!ok) break;
+      pr.pend_mask &= ~(1u << pr.slot);
+      if (lane == 0) {
+        sm.hdr[pr.slot].kind = HK_SCHED;
+        mbar_arrive(&sm.full[pr.slot]);
+      }
+      __syncwarp();
+      pr.advance();
+      const long long tw0 = tclock<kTrace>();
+      ok = pr.wait_bar(&sm.sched_bar, 0u);
+      c_schedw += (unsigned long long)(tclock<kTrace>() - tw0);
+      if (!ok) break;
+      sched_ready = true;
+      if (lane == 0) trace_stamp<kTrace>(p, TR_SCHED);
+    }
+    if (sched_ready && u >= sm.sc.total) break;
+    const long long tu0 = tclock<kTrace>();
+    const UnitDesc d = decode_unit(sh, sm.sc, u);
+    // the next unit's queue ticket is requested now and read after this unit's
+    // stages are issued, so the atomic's round trip overlaps the issue loop
+    uint32_t next_ticket = 0;
+    if (lane == 0) next_ticket = atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
+    if (lane == 0 && kTrace) {
+      if (first_expert && d.type == UT_EXPERT) { trace_stamp<kTrace>(p, TR_FIRST_EXPERT); first_expert = false; }
+      if (first_down && (d.type == UT_DOWN_SHARED || d.type == UT_DOWN_EXPERT)) { trace_stamp<kTrace>(p, TR_FIRST_DOWN); first_down = false; }
+      ++c_units;
+    }
+    if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(blockIdx.x * 7919u + (uint32_t)u) % 3000u);
+    const int nseg_units = d.type == UT_DOWN_EXPERT ? d.npair : 1;
+    c_setup += (unsigned long long)(tclock<kTrace>() - tu0);
+    for (int q = 0; q < nseg_units && ok; ++q) {
+      SegCtx x;
+      const long long tm0 = tclock<kTrace>();
+      make_seg(p, sh, sm.sc, d, q, x);
+      c_setup += (unsigned long long)(tclock<kTrace>() - tm0);
+      const uint32_t box_bytes = (uint32_t)(x.box_cols * kBoxRows * 2);
+      const uint32_t row_bytes = (uint32_t)(x.box_cols * 2);
+      const int step = x.kpair ? 2 : 1;
+      const int info0 = (x.kpair ? kInfoKpair : 0) | (x.c << 3) | (q << 8) | (x.box_cols << 16);
+      for (int kb = x.kb0; kb < x.kb_end && ok; kb += step) {
+        {
+          const long long t0 = tclock<kTrace>();
+          ok = pr.wait_slot();
+          c_slot += (unsigned long long)(tclock<kTrace>() - t0);
+        }
+        if (!ok) break;
+        const long long ti0 = tclock<kTrace>();
+        const int nbox = x.kpair ? (x.kb_end - kb < 2 ? 1 : 2) : 2;
+        const int nseg = x.kpair ? nbox : 1;
+        const bool seg_end = kb + step >= x.kb_end;
+        uint8_t* dst = ring + pr.slot * kSlotBytes;
+        uint64_t* fb = &sm.full[pr.slot];
+        pr.mark_pending();
+        if (lane == 0) {
+          StageHeader h;
+          h.kind = HK_STAGE;
+          h.unit = u;
+          h.info = info0 | nbox | (seg_end ? kInfoSegEnd : 0) | (seg_end && q == nseg_units - 1 ? kInfoUnitEnd : 0) |
+                   (kb == x.kb0 && q == 0 ? kInfoFirst : 0);
+          h.wrow = x.wrow;
+          sm.hdr[pr.slot] = h;
+          mbar_arrive_expect_tx(fb, (uint32_t)nbox * box_bytes + (uint32_t)(nseg * x.c) * row_bytes);
+          const int col = kb * x.box_cols;
+          tma_load_2d(dst, x.tm0, col, x.y0, fb, pol);
+          if (nbox == 2) tma_load_2d(dst + kBoxBytesMax, x.tm1, x.kpair ? col + x.box_cols : col, x.y0, fb, pol);
+        }
+        // activations: only after the acquire that publishes them
+        bool dep_ok = true;
+        const long long td0 = tclock<kTrace>();
+        if (kb == x.kb0) {
+          if (x.dep == 0) {
+            if (!n_ok) {
+              dep_ok = n_ok = pr.wait_dep(&p.ctr[CTR_NREADY], (uint32_t)p.B);
+              if (lane == 0) trace_stamp<kTrace>(p, TR_NREADY);
+            }
+          } else if (x.dep == 1) {
+            if (!hs_ok) dep_ok = hs_ok = pr.wait_dep(&p.ctr[CTR_HS], (uint32_t)sh.hs_target);
+          } else {
+            dep_ok = pr.wait_pair(x.pair);
+          }
+        }
+        const long long td1 = tclock<kTrace>();
+        c_dep += (unsigned long long)(td1 - td0);
+        if (lane == 0) {
+          uint8_t* act = dst + 2 * kBoxBytesMax;
+          for (int sg = 0; sg < nseg; ++sg) {
+            const int col = (kb + sg) * x.box_cols;
+#pragma unroll
+            for (int j = 0; j < kActGroup; ++j)
+              if (j < x.c) bulk_load(act + sg * kActSegBytes + j * row_bytes, x.abase + x.aoff[j] + col, row_bytes, fb);
+          }
+        }
+        __syncwarp();
+        pr.advance();
+        c_issue += (unsigned long long)(tclock<kTrace>() - ti0) - (unsigned long long)(td1 - td0);
+        ++c_stages;
+        if (!dep_ok) ok = false;
+      }
+    }
+    {
+      const long long t0 = tclock<kTrace>();
+      u = __shfl_sync(0xffffffffu, (int)next_ticket, 0);
+      c_grab += (unsigned long long)(tclock<kTrace>() - t0);
+    }
+  }
+  if (lane == 0 && kTrace) {
+    trace_stamp<kTrace>(p, TR_PROD_END);
+    trace_put<kTrace>(p, TR_PROD_WAIT_SLOT_CYC, c_slot);
+    trace_put<kTrace>(p, TR_PROD_WAIT_DEP_CYC, c_dep);
+    trace_put<kTrace>(p, TR_PROD_GRAB_CYC, c_grab);
+    trace_put<kTrace>(p, TR_PROD_ISSUE_CYC, c_issue);
+    trace_put<kTrace>(p, TR_PROD_STAGES, c_stages);
+    trace_put<kTrace>(p, TR_UNITS, c_units);
+    trace_put<kTrace>(p, TR_PROD_SETUP_CYC, c_setup);
+    trace_put<kTrace>(p, TR_PROD_SCHED_CYC, c_schedw);
+    trace_put<kTrace>(p, TR_PROD_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tploop0));
+  }
+  pr.finish();
+}
+
+// Tensor-core path: one unit's tensor maps, rows and activation operand.
+struct TcSeg {
+  const CUtensorMap* tw0;  // weight tile 0 (accumulator columns +0)
+  const CUtensorMap* tw1;  // weight tile 1 (accumulator columns +64)
+  const CUtensorMap* ta;   // activation operand
+  int y0, y1, nbox;
+  int N;     // MMA N: activation rows loaded (multiple of 16)
+  int arow;  // first activation row
+  int dep;   // 0: normalised rows, 1: shared h, 2: the expert's h
+  int pair;
+};
+
+__device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, const Sched& sc, const UnitDesc& d,
+                                            TcSeg& x) {
+  x.pair = d.pair;
+  x.arow = 0;
+  x.N = sh.NA;
+  x.ta = &p.tmaps[TM_T_AN];
+  x.dep = 0;
+  switch (d.type) {
+    case UT_ROUTER:
+      x.tw0 = x.tw1 = &p.tmaps[TM_T_WR];
+      x.y0 = d.tile * 2 * kTcRows;
+      x.y1 = x.y0 + kTcRows;
+      x.nbox = x.y1 < p.E ? 2 : 1;
+      break;
+    case UT_SHARED:
+      x.tw0 = &p.tmaps[TM_T_WSG];
+      x.tw1 = &p.tmaps[TM_T_WSU];
+      x.y0 = x.y1 = d.tile * kTcRows;
+      x.nbox = 2;
+      break;
+    case UT_EXPERT: {
+      // every token row is an MMA column; the epilogue keeps the expert's own rows
+      const int e = sc.slot_expert[sc.pair_slot[d.pair]];
+      x.tw0 = &p.tmaps[TM_T_WG];
+      x.tw1 = &p.tmaps[TM_T_WU];
+      x.y0 = x.y1 = e * p.I + d.tile * kTcRows;
+      x.nbox = 2;
+      break;
+    }
+    case UT_DOWN_SHARED:
+      x.tw0 = x.tw1 = &p.tmaps[TM_T_WSD];
+      x.y0 = d.tile * 2 * kTcRows;
+      x.y1 = x.y0 + kTcRows;
+      x.nbox = x.y1 < p.H ? 2 : 1;
+      x.ta = &p.tmaps[TM_T_AHS];
+      x.dep = 1;
+      break;
+    default: {
+      // the expert's slot rows of h are contiguous: they are the MMA columns
+      const int i = sc.pair_slot[d.pair];
+      const int e = sc.slot_expert[i];
+      x.tw0 = x.tw1 = &p.tmaps[TM_T_WD];
+      x.y0 = e * p.H + d.tile * 2 * kTcRows;
+      x.y1 = x.y0 + kTcRows;
+      x.nbox = d.tile * 2 * kTcRows + kTcRows < p.H ? 2 : 1;
+      x.ta = &p.tmaps[TM_T_AHE];
+      x.arow = sc.slot_base[i];
+      x.N = (sc.slot_cnt[i] + kTcActRows - 1) / kTcActRows * kTcActRows;
+      x.dep = 2;
+      break;
+    }
+  }
+}
+
+// Tensor-core path producer: per 64-column K atom one stage of up to two 128-row weight
+// tiles and the activation operand (N rows, boxes of 16), all 128-byte swizzled.
+template <bool kTrace>
+__device__ void producer_tc(Producer& pr, uint8_t* ring) {
+  const Params& p = pr.p;
+  Smem& sm = pr.sm;
+  const Shape& sh = sm.sh;
+  const int lane = pr.lane;
+  const uint64_t pol = policy_evict_first();
+  if (lane == 0)
+    for (int t = TM_T_WR; t < TM_COUNT; ++t) prefetch_tensormap(&p.tmaps[t]);
+  bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
+  const int pre = sh.NR + sh.NS;
+  int u = pr.grab();
+  bool first_expert = true, first_down = true;
+  unsigned long long c_slot = 0, c_dep = 0, c_grab = 0, c_issue = 0, c_stages = 0, c_units = 0;
+  unsigned long long c_setup = 0, c_schedw = 0;
+  const long long tploop0 = tclock<kTrace>();
+  while (ok) {
+    if (u >= pre && !sched_ready) {
+      const long long tw0 = tclock<kTrace>();
+      ok = pr.wait_bar(&sm.sched_bar, 0u);
+      c_schedw += (unsigned long long)(tclock<kTrace>() - tw0);
+      if (!ok) break;
+      sched_ready = true;
+      if (lane == 0) trace_stamp<kTrace>(p, TR_SCHED);
+    }
+    if (sched_ready && u >= sm.sc.total) break;
+    const long long tu0 = tclock<kTrace>();
+    const UnitDesc d = decode_unit_tc(sh, sm.sc, u);
+    uint32_t next_ticket = 0;
+    if (lane == 0) next_ticket = atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
+    if (lane == 0 && kTrace) {
+      if (first_expert && d.type == UT_EXPERT) { trace_stamp<kTrace>(p, TR_FIRST_EXPERT); first_expert = false; }
+      if (first_down && (d.type == UT_DOWN_SHARED || d.type == UT_DOWN_EXPERT)) { trace_stamp<kTrace>(p, TR_FIRST_DOWN); first_down = false; }
+      ++c_units;
+    }
+    if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(blockIdx.x * 7919u + (uint32_t)u) % 3000u);
+    TcSeg x;
+    make_seg_tc(p, sh, sm.sc, d, x);
+    c_setup += (unsigned long long)(tclock<kTrace>() - tu0);
+    const uint32_t tx = (uint32_t)(x.nbox * kTcTileBytes + x.N * kTcAtomK * 2);
+    const int info0 = x.nbox | ((x.N / kTcActRows) << 2);
+    const int ka_end = d.kb0 + d.nkb;
+    for (int ka = d.kb0; ka < ka_end && ok; ++ka) {
       {
         const long long t0 = tclock<kTrace>();
-        const bool got = warp_wait(&sm.full[slot], phase, p, lane);
-        c_full += (unsigned long long)(tclock<kTrace>() - t0);
-        if (!got) break;
+        ok = pr.wait_slot();
+        c_slot += (unsigned long long)(tclock<kTrace>() - t0);
       }
-      const StageHeader hd = sm.hdr[slot];
-      if (hd.kind == HK_END) {
-        if (mw == 0 && lane == 0) trace_stamp<kTrace>(p, TR_MAC_END);
-        break;
+      if (!ok) break;
+      const long long ti0 = tclock<kTrace>();
+      uint8_t* dst = ring + pr.slot * kTcSlotBytes;
+      uint64_t* fb = &sm.full[pr.slot];
+      pr.mark_pending();
+      const int col = ka * kTcAtomK;
+      if (lane == 0) {
+        StageHeader h;
+        h.kind = HK_STAGE;
+        h.unit = u;
+        h.info = info0 | (ka == d.kb0 ? kTcInfoFirst : 0) | (ka == ka_end - 1 ? kTcInfoLast : 0);
+        h.wrow = -1;
+        sm.hdr[pr.slot] = h;
+        mbar_arrive_expect_tx(fb, tx);
+        tma_load_2d(dst, x.tw0, col, x.y0, fb, pol);
+        if (x.nbox == 2) tma_load_2d(dst + kTcTileBytes, x.tw1, col, x.y1, fb, pol);
       }
-      if (hd.kind == HK_SCHED) {
-        const long long ts0 = tclock<kTrace>();
-        ok = build_schedule<kTrace>(p, sm, mw, lane, mphase);
-        c_sched += (unsigned long long)(tclock<kTrace>() - ts0);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.empty[slot]);
-        if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
-        if (++slot == kStages) {
-          slot = 0;
-          phase ^= 1u;
+      bool dep_ok = true;
+      const long long td0 = tclock<kTrace>();
+      if (ka == d.kb0) {
+        if (x.dep == 0) {
+          if (!n_ok) {
+            dep_ok = n_ok = pr.wait_dep(&p.ctr[CTR_NREADY], (uint32_t)p.B);
+            if (lane == 0) trace_stamp<kTrace>(p, TR_NREADY);
+          }
+        } else if (x.dep == 1) {
+          if (!hs_ok) dep_ok = hs_ok = pr.wait_dep(&p.ctr[CTR_HS], (uint32_t)sh.hs_target);
+        } else {
+          dep_ok = pr.wait_pair(x.pair);
         }
-        continue;
       }
-      const int info = hd.info;
-      const int kpair = (info & kInfoKpair) ? 1 : 0;
-      const int nbox = info & 3;
-      const int c = (info >> 3) & 7;
-      const int box_cols = info >> 16;
-      if (info & kInfoFirst) {
-        zero_acc(acc);
-        rb_claimed = false;
-        if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(hd.unit * 131u + mw * 7u + blockIdx.x) % 1500u);
-        __syncwarp();
+      const long long td1 = tclock<kTrace>();
+      c_dep += (unsigned long long)(td1 - td0);
+      if (lane == 0) {
+        uint8_t* act = dst + 2 * kTcTileBytes;
+        for (int q = 0; q < x.N / kTcActRows; ++q)
+          tma_load_2d_plain(act + q * kTcActRows * kTcAtomK * 2, x.ta, col, x.arow + q * kTcActRows, fb);
       }
-      const long long tc0 = tclock<kTrace>();
-      mac_dispatch(sm.ring[slot], kpair, nbox, box_cols, c, acc, mw, lane);
       __syncwarp();
-      c_comp += (unsigned long long)(tclock<kTrace>() - tc0);
-      ++c_st;
+      pr.advance();
+      c_issue += (unsigned long long)(tclock<kTrace>() - ti0) - (unsigned long long)(td1 - td0);
+      ++c_stages;
+      if (!dep_ok) ok = false;
+    }
+    {
+      const long long t0 = tclock<kTrace>();
+      u = __shfl_sync(0xffffffffu, (int)next_ticket, 0);
+      c_grab += (unsigned long long)(tclock<kTrace>() - t0);
+    }
+  }
+  if (lane == 0 && kTrace) {
+    trace_stamp<kTrace>(p, TR_PROD_END);
+    trace_put<kTrace>(p, TR_PROD_WAIT_SLOT_CYC, c_slot);
+    trace_put<kTrace>(p, TR_PROD_WAIT_DEP_CYC, c_dep);
+    trace_put<kTrace>(p, TR_PROD_GRAB_CYC, c_grab);
+    trace_put<kTrace>(p, TR_PROD_ISSUE_CYC, c_issue);
+    trace_put<kTrace>(p, TR_PROD_STAGES, c_stages);
+    trace_put<kTrace>(p, TR_UNITS, c_units);
+    trace_put<kTrace>(p, TR_PROD_SETUP_CYC, c_setup);
+    trace_put<kTrace>(p, TR_PROD_SCHED_CYC, c_schedw);
+    trace_put<kTrace>(p, TR_PROD_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tploop0));
+  }
+  pr.finish();
+}
+
+// ---- CUDA-core path: MAC warps and the epilogue warp ------------------------------------------
+
+template <bool kTrace>
+__device__ void mac_warps_cc(const Params& p, Smem& sm, uint8_t* ring, int mw, int lane) {
+  uint32_t mphase = 0;
+  bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
+  int slot = 0;
+  uint32_t phase = 0;
+  int ub = 0;
+  uint32_t ubphase = 0;
+  bool rb_claimed = false;
+  float acc[2][kRowsPerWarp][kActGroup];
+  zero_acc(acc);
+  const long long tloop0 = tclock<kTrace>();
+  unsigned long long c_full = 0, c_rb = 0, c_comp = 0, c_st = 0, c_sched = 0, c_red = 0;
+  while (ok) {
+    {
+      const long long t0 = tclock<kTrace>();
+      const bool got = warp_wait(&sm.full[slot], phase, p, lane);
+      c_full += (unsigned long long)(tclock<kTrace>() - t0);
+      if (!got) break;
+    }
+    const StageHeader hd = sm.hdr[slot];
+    if (hd.kind == HK_END) {
+      if (mw == 0 && lane == 0) trace_stamp<kTrace>(p, TR_MAC_END);
+      break;
+    }
+    if (hd.kind == HK_SCHED) {
+      const long long ts0 = tclock<kTrace>();
+      ok = build_schedule<kTrace, false>(p, sm, mw, lane, mphase);
+      c_sched += (unsigned long long)(tclock<kTrace>() - ts0);
+      __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[slot]);
+      if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
       if (++slot == kStages) {
         slot = 0;
         phase ^= 1u;
       }
-      const bool unit_end = (info & kInfoUnitEnd) != 0;
-      const bool seg_end = (info & kInfoSegEnd) != 0;
-      const long long tr0 = tclock<kTrace>();
-      if (seg_end) {
-        if (!rb_claimed) {
-          const long long t0 = tclock<kTrace>();
-          const bool got = warp_wait(&sm.rb_empty[ub], ubphase ^ 1u, p, lane);
-          c_rb += (unsigned long long)(tclock<kTrace>() - t0);
-          if (!got) break;
-          rb_claimed = true;
-        }
-        if (hd.wrow >= 0) {
-          reduce_to(acc, 1, sm.rb[ub], (info >> 8) & 1, &sm.sc.w_of[hd.wrow], c, mw, lane);
-          zero_acc(acc);
-        } else {
-          reduce_to(acc, kpair ? 1 : 2, sm.rb[ub], 0, nullptr, c, mw, lane);
-        }
-      }
-      if (unit_end) {
-        if (mw == 0 && lane == 0) sm.rb_unit[ub] = hd.unit;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.rb_full[ub]);
-        if (++ub == kRB) {
-          ub = 0;
-          ubphase ^= 1u;
-        }
-        rb_claimed = false;
-      }
-      if (seg_end || unit_end) c_red += (unsigned long long)(tclock<kTrace>() - tr0);
+      continue;
     }
-    if (mw == 0 && lane == 0 && kTrace) {
-      trace_put<kTrace>(p, TR_MAC_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tloop0));
-      trace_put<kTrace>(p, TR_MAC_WAIT_FULL_CYC, c_full);
-      trace_put<kTrace>(p, TR_MAC_WAIT_RB_CYC, c_rb);
-      trace_put<kTrace>(p, TR_MAC_COMPUTE_CYC, c_comp);
-      trace_put<kTrace>(p, TR_MAC_STAGES, c_st);
-      trace_put<kTrace>(p, TR_MAC_SCHED_CYC, c_sched);
-      trace_put<kTrace>(p, TR_MAC_REDUCE_CYC, c_red);
+    const int info = hd.info;
+    const int kpair = (info & kInfoKpair) ? 1 : 0;
+    const int nbox = info & 3;
+    const int c = (info >> 3) & 7;
+    const int box_cols = info >> 16;
+    if (info & kInfoFirst) {
+      zero_acc(acc);
+      rb_claimed = false;
+      if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(hd.unit * 131u + mw * 7u + blockIdx.x) % 1500u);
+      __syncwarp();
     }
-    // tell the epilogue warp to stop (bounded)
-    if (warp_wait(&sm.rb_empty[ub], ubphase ^ 1u, p, lane)) {
-      if (mw == 0 && lane == 0) sm.rb_unit[ub] = -1;
+    const long long tc0 = tclock<kTrace>();
+    mac_dispatch(ring + slot * kSlotBytes, kpair, nbox, box_cols, c, acc, mw, lane);
+    __syncwarp();
+    c_comp += (unsigned long long)(tclock<kTrace>() - tc0);
+    ++c_st;
+    if (lane == 0) mbar_arrive(&sm.empty[slot]);
+    if (++slot == kStages) {
+      slot = 0;
+      phase ^= 1u;
+    }
+    const bool unit_end = (info & kInfoUnitEnd) != 0;
+    const bool seg_end = (info & kInfoSegEnd) != 0;
+    const long long tr0 = tclock<kTrace>();
+    if (seg_end) {
+      if (!rb_claimed) {
+        const long long t0 = tclock<kTrace>();
+        const bool got = warp_wait(&sm.rb_empty[ub], ubphase ^ 1u, p, lane);
+        c_rb += (unsigned long long)(tclock<kTrace>() - t0);
+        if (!got) break;
+        rb_claimed = true;
+      }
+      if (hd.wrow >= 0) {
+        reduce_to(acc, 1, sm.rb[ub], (info >> 8) & 1, &sm.sc.w_of[hd.wrow], c, mw, lane);
+        zero_acc(acc);
+      } else {
+        reduce_to(acc, kpair ? 1 : 2, sm.rb[ub], 0, nullptr, c, mw, lane);
+      }
+    }
+    if (unit_end) {
+      if (mw == 0 && lane == 0) sm.rb_unit[ub] = hd.unit;
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.rb_full[ub]);
-    }
-  } else {
-    // =========================== epilogue warp ===========================
-    int ub = 0;
-    uint32_t ubphase = 0;
-    unsigned long long c_busy = 0;
-    for (;;) {
-      if (!warp_wait(&sm.rb_full[ub], ubphase, p, lane)) break;
-      const int u = sm.rb_unit[ub];
-      if (u < 0 || abort_seen(p)) {
-        if (lane == 0 && kTrace) {
-          trace_stamp<kTrace>(p, TR_EPI_END);
-          trace_put<kTrace>(p, TR_EPI_BUSY_CYC, c_busy);
-        }
-        break;
-      }
-      const UnitDesc d = decode_unit(sh, sm.sc, u);
-      const long long t0 = tclock<kTrace>();
-      epi_finish(p, sm, d, u, sm.rb[ub], lane);
-      c_busy += (unsigned long long)(tclock<kTrace>() - t0);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.rb_empty[ub]);
       if (++ub == kRB) {
         ub = 0;
         ubphase ^= 1u;
       }
+      rb_claimed = false;
+    }
+    if (seg_end || unit_end) c_red += (unsigned long long)(tclock<kTrace>() - tr0);
+  }
+  if (mw == 0 && lane == 0 && kTrace) {
+    trace_put<kTrace>(p, TR_MAC_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tloop0));
+    trace_put<kTrace>(p, TR_MAC_WAIT_FULL_CYC, c_full);
+    trace_put<kTrace>(p, TR_MAC_WAIT_RB_CYC, c_rb);
+    trace_put<kTrace>(p, TR_MAC_COMPUTE_CYC, c_comp);
+    trace_put<kTrace>(p, TR_MAC_STAGES, c_st);
+    trace_put<kTrace>(p, TR_MAC_SCHED_CYC, c_sched);
+    trace_put<kTrace>(p, TR_MAC_REDUCE_CYC, c_red);
+  }
+  // tell the epilogue warp to stop (bounded)
+  if (warp_wait(&sm.rb_empty[ub], ubphase ^ 1u, p, lane)) {
+    if (mw == 0 && lane == 0) sm.rb_unit[ub] = -1;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.rb_full[ub]);
+  }
+}
+
+template <bool kTrace>
+__device__ void epilogue_cc(const Params& p, Smem& sm, int lane) {
+  int ub = 0;
+  uint32_t ubphase = 0;
+  unsigned long long c_busy = 0;
+  for (;;) {
+    if (!warp_wait(&sm.rb_full[ub], ubphase, p, lane)) break;
+    const int u = sm.rb_unit[ub];
+    if (u < 0 || abort_seen(p)) {
+      if (lane == 0 && kTrace) {
+        trace_stamp<kTrace>(p, TR_EPI_END);
+        trace_put<kTrace>(p, TR_EPI_BUSY_CYC, c_busy);
+      }
+      break;
+    }
+    const UnitDesc d = decode_unit(sm.sh, sm.sc, u);
+    const long long t0 = tclock<kTrace>();
+    epi_finish(p, sm, d, u, sm.rb[ub], lane);
+    c_busy += (unsigned long long)(tclock<kTrace>() - t0);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.rb_empty[ub]);
+    if (++ub == kRB) {
+      ub = 0;
+      ubphase ^= 1u;
     }
   }
+}
 
+// ---- tensor-core path: MMA warp --------------------------------------------------------------------
+
+// One elected lane issues, per stage, 4 K-steps of 16 for each weight tile into the
+// unit's accumulator buffer, then commits the stage's slot back to the producer
+// (the slot is free once those MMAs have read it). At a unit's last stage the buffer
+// is handed to the epilogue warps: one commit arrive (the MMAs are complete) plus one
+// plain arrive that publishes the unit id.
+template <bool kTrace>
+__device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
+  const uint32_t tmem = sm.tmem_base;
+  int slot = 0;
+  uint32_t phase = 0;
+  int abuf = 0;
+  uint32_t aphase = 0;
+  bool issued = false;
+  unsigned long long c_full = 0, c_acc = 0, c_st = 0, c_issue = 0;
+  const long long tloop0 = tclock<kTrace>();
+  for (;;) {
+    {
+      const long long t0 = tclock<kTrace>();
+      const bool got = warp_wait(&sm.full[slot], phase, p, lane);
+      c_full += (unsigned long long)(tclock<kTrace>() - t0);
+      if (!got) break;
+    }
+    const StageHeader hd = sm.hdr[slot];
+    if (hd.kind == HK_END) {
+      if (lane == 0) trace_stamp<kTrace>(p, TR_MAC_END);
+      break;
+    }
+    const int info = hd.info;
+    const bool first = (info & kTcInfoFirst) != 0;
+    const bool last = (info & kTcInfoLast) != 0;
+    if (first) {
+      const long long t0 = tclock<kTrace>();
+      const bool got = warp_wait(&sm.acc_empty[abuf], aphase ^ 1u, p, lane);
+      c_acc += (unsigned long long)(tclock<kTrace>() - t0);
+      if (!got) break;
+    }
+    tc_fence_after();
+    const long long ti0 = tclock<kTrace>();
+    if (lane == 0) {
+      const uint32_t sbase = smem_u32(ring + slot * kTcSlotBytes);
+      const uint64_t dw0 = sw128_desc(sbase);
+      const uint64_t dw1 = sw128_desc(sbase + kTcTileBytes);
+      const uint64_t da = sw128_desc(sbase + 2 * kTcTileBytes);
+      const int nbox = info & 3;
+      const uint32_t idesc = idesc_bf16_m128((uint32_t)((info >> 2) & 7) * kTcActRows);
+      const uint32_t t0 = tmem + (uint32_t)(abuf * kTcAccCols);
+#pragma unroll
+      for (int ks = 0; ks < kTcAtomK / 16; ++ks) {
+        const uint32_t accum = (first && ks == 0) ? 0u : 1u;
+        tc_mma_bf16(t0, dw0 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
+        if (nbox == 2) tc_mma_bf16(t0 + 64u, dw1 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
+      }
+      tc_commit(&sm.empty[slot]);
+      if (last) {
+        sm.acc_unit[abuf] = hd.unit;
+        tc_commit(&sm.acc_full[abuf]);
+        mbar_arrive(&sm.acc_full[abuf]);
+      }
+    }
+    issued = true;
+    __syncwarp();
+    c_issue += (unsigned long long)(tclock<kTrace>() - ti0);
+    ++c_st;
+    if (last) {
+      if (++abuf == kTcAccBufs) {
+        abuf = 0;
+        aphase ^= 1u;
+      }
+    }
+    if (++slot == kTcStages) {
+      slot = 0;
+      phase ^= 1u;
+    }
+  }
+  if (lane == 0 && kTrace) {
+    trace_put<kTrace>(p, TR_MAC_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tloop0));
+    trace_put<kTrace>(p, TR_MAC_WAIT_FULL_CYC, c_full);
+    trace_put<kTrace>(p, TR_MAC_WAIT_RB_CYC, c_acc);
+    trace_put<kTrace>(p, TR_MAC_COMPUTE_CYC, c_issue);
+    trace_put<kTrace>(p, TR_MAC_STAGES, c_st);
+  }
+  // stop the epilogue warps (bounded)
+  if (warp_wait(&sm.acc_empty[abuf], aphase ^ 1u, p, lane)) {
+    if (lane == 0) {
+      sm.acc_unit[abuf] = -1;
+      mbar_arrive(&sm.acc_full[abuf]);
+      mbar_arrive(&sm.acc_full[abuf]);
+    }
+  }
+  __syncwarp();
+  // every MMA this warp issued completes before the CTA gives up its shared and tensor memory
+  if (issued && lane == 0) {
+    tc_commit(&sm.mma_bar);
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(&sm.mma_bar, 0u)) {
+      if (globaltimer_ns() - t0 > 50000000ull) break;
+    }
+  }
+  __syncwarp();
+}
+
+// ---- tensor-core path: epilogue warps --------------------------------------------------------------
+
+// Rendezvous of the 4 epilogue warps (an mbarrier with bounded waits, so a warp that
+// gives up never leaves the others blocked).
+__device__ __forceinline__ bool epi_sync(Smem& sm, uint32_t& phase, const Params& p, int lane) {
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&sm.epi_bar);
+  const bool ok = warp_wait(&sm.epi_bar, phase, p, lane);
+  phase ^= 1u;
+  return ok;
+}
+
+// Loads accumulator columns [j0, j0 + 16) of both tiles of the buffer (lane quadrant of
+// the calling warp). `two` is warp-uniform.
+__device__ __forceinline__ void tmem_cols16(uint32_t ta, int j0, bool two, uint32_t (&v0)[16], uint32_t (&v1)[16]) {
+  tmem_ld16(ta + (uint32_t)j0, v0);
+  if (two) tmem_ld16(ta + 64u + (uint32_t)j0, v1);
+  tmem_ld_wait();
+  tmem_regs_after_wait(v0);
+  if (two) tmem_regs_after_wait(v1);
+}
+
+// The fix-up of a tile whose splits are all done: fixed split order, so the sums do
+// not depend on which split finished last. Thread et (0..127) owns tile row et.
+__device__ void fixup_tc(const Params& p, const Smem& sm, const UnitDesc& d, int et) {
+  const Shape& sh = sm.sh;
+  const Sched& sc = sm.sc;
+  const int B = sh.B;
+  switch (d.type) {
+    case UT_ROUTER:
+      for (int a = 0; a < 2; ++a) {
+        const int e = d.tile * 2 * kTcRows + a * kTcRows + et;
+        if (e >= p.E) continue;
+        const float bias = p.bias ? p.bias[e] : 0.0f;
+        for (int b = 0; b < B; ++b) {
+          const float* src = p.rpart + (size_t)b * p.E + e;
+          const size_t stride = (size_t)B * p.E;
+          float s = 0.0f;
+          int sp = 0;
+          for (; sp + 4 <= d.nsplit; sp += 4) {
+            const float v0 = __ldcg(src + sp * stride), v1 = __ldcg(src + (sp + 1) * stride);
+            const float v2 = __ldcg(src + (sp + 2) * stride), v3 = __ldcg(src + (sp + 3) * stride);
+            s += v0;
+            s += v1;
+            s += v2;
+            s += v3;
+          }
+          for (; sp < d.nsplit; ++sp) s += __ldcg(src + sp * stride);
+          const float v = s + bias;
+          p.logits[(size_t)b * p.E + e] = v;
+          if (p.dbg_logits) p.dbg_logits[(size_t)b * p.E + e] = v;
+        }
+      }
+      break;
+    case UT_SHARED:
+      for (int b = 0; b < B; ++b) {
+        float g = 0.0f, u = 0.0f;
+        for (int sp = 0; sp < d.nsplit; ++sp) {
+          const float* src = p.spart + (((size_t)sp * B + b) * sh.ST + d.tile) * (2 * kTcRows);
+          g += __ldcg(src + et);
+          u += __ldcg(src + kTcRows + et);
+        }
+        p.hs[(size_t)b * p.Is + d.tile * kTcRows + et] = f2bf(silu(g) * u);
+      }
+      break;
+    case UT_EXPERT: {
+      const int i = sc.pair_slot[d.pair];
+      const int r0 = sc.slot_base[i], cnt = sc.slot_cnt[i];
+      for (int j = 0; j < cnt; ++j) {
+        float g = 0.0f, u = 0.0f;
+        for (int sp = 0; sp < d.nsplit; ++sp) {
+          const float* src = p.epart + (((size_t)sp * sc.S + r0 + j) * sh.IT + d.tile) * (2 * kTcRows);
+          g += __ldcg(src + et);
+          u += __ldcg(src + kTcRows + et);
+        }
+        p.he[(size_t)(r0 + j) * p.I + d.tile * kTcRows + et] = f2bf(silu(g) * u);
+      }
+      break;
+    }
+    default:
+      // y = bf16(x + s + sum_j w_j d_j): shared part first, then the row's choices in
+      // top-k order
+      for (int a = 0; a < 2; ++a) {
+        const int h = d.tile * 2 * kTcRows + a * kTcRows + et;
+        if (h >= p.H) continue;
+        for (int b = 0; b < B; ++b) {
+          float acc = __ldcg(p.dpart + (size_t)(sc.S + b) * p.H + h);
+          const int16_t* so = &sc.slot_of[b * sh.k];
+          int j = 0;
+          for (; j + 4 <= sh.k; j += 4) {
+            const int r0 = so[j], r1 = so[j + 1], r2 = so[j + 2], r3 = so[j + 3];
+            const float v0 = __ldcg(p.dpart + (size_t)r0 * p.H + h);
+            const float v1 = __ldcg(p.dpart + (size_t)r1 * p.H + h);
+            const float v2 = __ldcg(p.dpart + (size_t)r2 * p.H + h);
+            const float v3 = __ldcg(p.dpart + (size_t)r3 * p.H + h);
+            acc = fmaf(sc.w_of[r0], v0, acc);
+            acc = fmaf(sc.w_of[r1], v1, acc);
+            acc = fmaf(sc.w_of[r2], v2, acc);
+            acc = fmaf(sc.w_of[r3], v3, acc);
+          }
+          for (; j < sh.k; ++j) {
+            const int r = so[j];
+            acc = fmaf(sc.w_of[r], __ldcg(p.dpart + (size_t)r * p.H + h), acc);
+          }
+          const float xv = bf2f(p.x[(size_t)b * p.H + h]);
+          p.y[(size_t)b * p.H + h] = f2bf(xv + acc);
+        }
+      }
+      break;
+  }
+}
+
+template <bool kTrace>
+__device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
+  const Shape& sh = sm.sh;
+  const int quad = warp_id & 3;
+  const int row = quad * 32 + lane;                        // accumulator lane = tile row
+  const int et = (warp_id - kTcEpiWarp0) * 32 + lane;       // 0..127 for the fix-ups
+  const uint32_t tq = sm.tmem_base + ((uint32_t)(quad * 32) << 16);
+  int abuf = 0;
+  uint32_t aphase = 0, ephase = 0;
+  unsigned long long c_busy = 0;
+  for (;;) {
+    if (!warp_wait(&sm.acc_full[abuf], aphase, p, lane)) break;
+    const int u = sm.acc_unit[abuf];
+    if (u < 0) {
+      if (lane == 0 && kTrace && warp_id == kTcEpiWarp0) {
+        trace_stamp<kTrace>(p, TR_EPI_END);
+        trace_put<kTrace>(p, TR_EPI_BUSY_CYC, c_busy);
+      }
+      break;
+    }
+    tc_fence_after();
+    const long long tb0 = tclock<kTrace>();
+    const Sched& sc = sm.sc;
+    const UnitDesc d = decode_unit_tc(sh, sc, u);
+    const uint32_t ta = tq + (uint32_t)(abuf * kTcAccCols);
+    const bool direct = d.nsplit == 1 && d.type <= UT_EXPERT;
+    uint32_t v0[16], v1[16];
+    switch (d.type) {
+      case UT_ROUTER: {
+        const int e0 = d.tile * 2 * kTcRows + row, e1 = e0 + kTcRows;
+        const bool two = d.tile * 2 * kTcRows + kTcRows < p.E;
+        float* dst = direct ? p.logits : p.rpart + (size_t)d.split * sh.B * p.E;
+        const float b0 = direct && p.bias ? p.bias[e0] : 0.0f;
+        const float b1 = direct && p.bias && two ? p.bias[e1] : 0.0f;
+        for (int j0 = 0; j0 < sh.B; j0 += 16) {
+          tmem_cols16(ta, j0, two, v0, v1);
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int b = j0 + jj;
+            if (b < sh.B) {
+              const float a0 = __uint_as_float(v0[jj]) + b0;
+              dst[(size_t)b * p.E + e0] = a0;
+              if (direct && p.dbg_logits) p.dbg_logits[(size_t)b * p.E + e0] = a0;
+              if (two) {
+                const float a1 = __uint_as_float(v1[jj]) + b1;
+                dst[(size_t)b * p.E + e1] = a1;
+                if (direct && p.dbg_logits) p.dbg_logits[(size_t)b * p.E + e1] = a1;
+              }
+            }
+          }
+        }
+        break;
+      }
+      case UT_SHARED: {
+        for (int j0 = 0; j0 < sh.B; j0 += 16) {
+          tmem_cols16(ta, j0, true, v0, v1);
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int b = j0 + jj;
+            if (b < sh.B) {
+              const float g = __uint_as_float(v0[jj]), uu = __uint_as_float(v1[jj]);
+              if (direct) {
+                p.hs[(size_t)b * p.Is + d.tile * kTcRows + row] = f2bf(silu(g) * uu);
+              } else {
+                float* dst = p.spart + (((size_t)d.split * sh.B + b) * sh.ST + d.tile) * (2 * kTcRows);
+                dst[row] = g;
+                dst[kTcRows + row] = uu;
+              }
+            }
+          }
+        }
+        break;
+      }
+      case UT_EXPERT: {
+        // the expert's rows are scattered token columns: one column load per row
+        const int i = sc.pair_slot[d.pair];
+        const int r0 = sc.slot_base[i], cnt = sc.slot_cnt[i];
+        for (int j0 = 0; j0 < cnt; j0 += 8) {
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j = j0 + jj < cnt ? j0 + jj : j0;
+            const uint32_t col = (uint32_t)sc.row_of[r0 + j];
+            tmem_ld1(ta + col, v0[jj]);
+            tmem_ld1(ta + 64u + col, v1[jj]);
+          }
+          tmem_ld_wait();
+          tmem_regs_after_wait(v0);
+          tmem_regs_after_wait(v1);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j = j0 + jj;
+            if (j < cnt) {
+              const float g = __uint_as_float(v0[jj]), uu = __uint_as_float(v1[jj]);
+              if (direct) {
+                p.he[(size_t)(r0 + j) * p.I + d.tile * kTcRows + row] = f2bf(silu(g) * uu);
+              } else {
+                float* dst = p.epart + (((size_t)d.split * sc.S + r0 + j) * sh.IT + d.tile) * (2 * kTcRows);
+                dst[row] = g;
+                dst[kTcRows + row] = uu;
+              }
+            }
+          }
+        }
+        break;
+      }
+      default: {
+        // down: unweighted partial rows of the source (expert slot rows, or S + b for
+        // the shared expert); the tile's last source combines them
+        const bool shared = d.type == UT_DOWN_SHARED;
+        const int i = shared ? 0 : sc.pair_slot[d.pair];
+        const int r0 = shared ? sc.S : sc.slot_base[i];
+        const int cnt = shared ? sh.B : sc.slot_cnt[i];
+        const int h0 = d.tile * 2 * kTcRows + row, h1 = h0 + kTcRows;
+        const bool two = d.tile * 2 * kTcRows + kTcRows < p.H;
+        for (int j0 = 0; j0 < cnt; j0 += 16) {
+          tmem_cols16(ta, j0, two, v0, v1);
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            const int j = j0 + jj;
+            if (j < cnt) {
+              float* dst = p.dpart + (size_t)(r0 + j) * p.H;
+              dst[h0] = __uint_as_float(v0[jj]);
+              if (two) dst[h1] = __uint_as_float(v1[jj]);
+            }
+          }
+        }
+        break;
+      }
+    }
+    // accumulator buffer back to the MMA warp
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.acc_empty[abuf]);
+    if (++abuf == kTcAccBufs) {
+      abuf = 0;
+      aphase ^= 1u;
+    }
+    bool finished = direct;
+    if (!direct) {
+      // split-K / multi-source tile: count this split in, the last one does the fix-up
+      __threadfence();
+      if (!epi_sync(sm, ephase, p, lane)) break;
+      if (et == 0) {
+        const uint32_t old = atom_add_acq_rel(&p.tickets[d.ticket], 1u);
+        const int last = old == (uint32_t)(d.nsplit - 1);
+        if (last) st_relaxed_gpu(&p.tickets[d.ticket], 0u);
+        sm.epi_last = last;
+      }
+      if (!epi_sync(sm, ephase, p, lane)) break;
+      finished = sm.epi_last != 0;
+      if (finished) fixup_tc(p, sm, d, et);
+    }
+    uint32_t* done = done_counter(p, d);
+    if (finished && done) {
+      fence_proxy_async_global();
+      __threadfence();
+      if (!epi_sync(sm, ephase, p, lane)) break;
+      if (et == 0) red_release_add(done, 1u);
+    }
+    c_busy += (unsigned long long)(tclock<kTrace>() - tb0);
+  }
+}
+
+// ---- the kernel ----------------------------------------------------------------------------------
+
+template <bool kTrace, bool kTC>
+__global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
+    moe_decode_layer_kernel(const __grid_constant__ Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
+  Smem& sm = *reinterpret_cast<Smem*>(ring + (kTC ? kTcRingBytes : kCcRingBytes));
+  constexpr int kNst = kTC ? kTcStages : kStages;
+  const int tid = threadIdx.x;
+  const int warp_id = tid / 32;
+  const int lane = tid % 32;
+
+  if (tid == 0) {
+    for (int s = 0; s < kNst; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kTC ? 1 : kMacWarps);
+    }
+    if constexpr (kTC) {
+      for (int b = 0; b < kTcAccBufs; ++b) {
+        mbar_init(&sm.acc_full[b], 2);
+        mbar_init(&sm.acc_empty[b], kTcEpiWarps);
+      }
+      mbar_init(&sm.mma_bar, 1);
+      mbar_init(&sm.epi_bar, kTcEpiWarps);
+      make_shape_tc(p, sm.sh);
+    } else {
+      for (int b = 0; b < kRB; ++b) {
+        mbar_init(&sm.rb_full[b], kMacWarps);
+        mbar_init(&sm.rb_empty[b], 1);
+      }
+      make_shape(p, sm.sh);
+    }
+    mbar_init(&sm.sched_bar, 1);
+    mbar_init(&sm.mac_bar, kMacWarps);
+    for (int w = 0; w < kMaxSlots / 32; ++w) sm.known_done[w] = 0u;
+    if (kTrace) {
+      for (int t = 0; t < kTraceSlots; ++t) p.trace[(size_t)blockIdx.x * kTraceSlots + t] = 0ull;
+      trace_stamp<kTrace>(p, TR_START);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if constexpr (kTC) {
+    if (warp_id == kTcMmaWarp) {
+      tmem_alloc(&sm.tmem_base, kTmemCols);
+      tmem_relinquish();
+    }
+    tc_fence_before();
+  }
   __syncthreads();
+  if constexpr (kTC) tc_fence_after();
+
+  if (warp_id == 0) {
+    Producer pr(p, sm, lane, kNst);
+    if constexpr (kTC) producer_tc<kTrace>(pr, ring);
+    else producer_cc<kTrace>(pr, ring);
+  } else if (warp_id <= kMacWarps) {
+    if constexpr (kTC) {
+      // RMSNorm of this CTA's rows, then the routing schedule (the MMA and epilogue
+      // warps keep the router and shared-expert tiles moving meanwhile)
+      const int mw = warp_id - 1;
+      uint32_t mphase = 0;
+      bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
+      if (ok) ok = build_schedule<kTrace, true>(p, sm, mw, lane, mphase);
+      if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
+    } else {
+      mac_warps_cc<kTrace>(p, sm, ring, warp_id - 1, lane);
+    }
+  } else if constexpr (!kTC) {
+    epilogue_cc<kTrace>(p, sm, lane);
+  } else if (warp_id == kTcMmaWarp) {
+    mma_warp<kTrace>(p, sm, ring, lane);
+  } else {
+    epilogue_tc<kTrace>(p, sm, warp_id, lane);
+  }
+
+  if constexpr (kTC) tc_fence_before();
+  __syncthreads();
+  if constexpr (kTC) {
+    if (warp_id == kTcMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(sm.tmem_base, kTmemCols);
+    }
+  }
   if (tid == 0) {
     trace_stamp<kTrace>(p, TR_EXIT);
     __threadfence();
@@ -1420,9 +2198,13 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_layer_kernel(const __g
   }
 }
 
-size_t smem_bytes() { return sizeof(Smem) + 1024; }
+size_t smem_bytes() { return kCcRingBytes + sizeof(Smem) + 1024; }
 int threads_per_cta() { return kThreads; }
-const void* kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false>); }
-const void* kernel_fn_trace() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true>); }
+const void* kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false, false>); }
+const void* kernel_fn_trace() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true, false>); }
+size_t tc_smem_bytes() { return kTcRingBytes + sizeof(Smem) + 1024; }
+int tc_threads_per_cta() { return kTcThreads; }
+const void* tc_kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false, true>); }
+const void* tc_kernel_fn_trace() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true, true>); }
 
 }  // namespace moe

@@ -33,11 +33,16 @@ def bf16_ulp(v):
     return 2.0 ** (e - 7)
 
 
-def make_handle(wl, layers, device=0, max_batch=None, top_k_max=None):
+def make_handle(wl, layers, device=0, max_batch=None, top_k_max=None, tc_min_batch=None):
+    """A handle for the workload; tc_min_batch (if given) sets the batch-shape switch:
+    1 sends every step to the tensor-core kernel, 0 every step to the CUDA-core one."""
     import moe_decode_persistent_b200 as mdp
 
-    return mdp.MoeDecode(wl.H, wl.E, top_k_max or wl.k, wl.I, wl.Is, max_batch or wl.B, layers,
-                         eps=wl.eps, device=device)
+    h = mdp.MoeDecode(wl.H, wl.E, top_k_max or wl.k, wl.I, wl.Is, max_batch or wl.B, layers,
+                      eps=wl.eps, device=device)
+    if tc_min_batch is not None:
+        h.set_tc_min_batch(tc_min_batch)
+    return h
 
 
 def run_gpu(handle, wl, x_bits, k=None, n_layers=1, flags=None):
@@ -77,6 +82,33 @@ def oracle_rows(wl, x_bits, rows, n_layers=1, k=None):
     return res
 
 
+def routing_oracle(wl, x_bits, rows, layers, gpu_inputs, k=None):
+    """Per-layer oracle for the routing checks: layer 0 from x, layer l >= 1 from the
+    GPU's own output of layer l - 1 (gpu_inputs[l - 1], all rows), so that each
+    layer's router is judged on the input it actually received."""
+    import dataclasses
+
+    w = dataclasses.replace(wl, k=k) if k else wl
+    res = []
+    for layer in range(layers):
+        xin = x_bits[rows] if layer == 0 else gpu_inputs[layer - 1][rows]
+        res.append(oracle.workload_layer(w, layer, xin))
+    return res
+
+
+def gpu_layer_outputs(wl, device_layers, x_bits, tc_min_batch=None, k=None):
+    """The GPU's output of each layer but the last, from handles over layer prefixes
+    (a step is deterministic, so these equal the intermediates of the full stack)."""
+    outs = []
+    for n in range(1, wl.layers):
+        h = make_handle(wl, device_layers[:n], tc_min_batch=tc_min_batch)
+        o = run_gpu(h, wl, x_bits, k=k, n_layers=n)
+        assert o["status"] == 0
+        outs.append(o["y"])
+        h.close()
+    return outs
+
+
 def check_layer(gpu_layer, orc, rows, k, tag=""):
     """Routing checks of one layer on the given rows. Returns rows whose own oracle
     selection differs from the GPU's by a genuine near-tie (excluded from y checks)."""
@@ -100,6 +132,27 @@ def check_layer(gpu_layer, orc, rows, k, tag=""):
             assert np.ptp(vals) <= 1e-3 * scale[i, 0], f"{tag}: row {b} selection differs beyond a near-tie"
             near_tie.append(b)
     return near_tie
+
+
+def chained_flips(gpu_layers, orc_layers, rows, k, tag=""):
+    """Rows whose selection in a later layer of the chained oracle (fed by its own
+    earlier outputs) differs from the GPU's: allowed only between experts whose
+    chained-oracle logits lie within the logit perturbation that the earlier layers'
+    rounding caused. Their outputs are excluded from the end-to-end comparison."""
+    flips = set()
+    for l in range(1, len(orc_layers)):
+        lg_o = orc_layers[l]["logits"]
+        for i, b in enumerate(rows):
+            got = gpu_layers[l]["idx"][b]
+            if np.array_equal(np.sort(orc_layers[l]["idx"][i]), np.sort(got)):
+                continue
+            lg_g = gpu_layers[l]["logits"][b].astype(np.float64)
+            pert = float(np.max(np.abs(lg_g - lg_o[i])))
+            diff = list(set(orc_layers[l]["idx"][i]) ^ set(got))
+            band = 2.0 * pert + 1e-3 * float(np.max(np.abs(lg_o[i])))
+            assert np.ptp(lg_o[i][diff]) <= band, f"{tag}: layer {l} row {b} selection differs beyond the perturbation"
+            flips.add(i)
+    return flips
 
 
 def check_y(y_gpu_rows, orc_layers, tag="", skip=()):

@@ -81,6 +81,8 @@ def test_null_handle_calls_are_rejected(L):
     assert L.moe_decode_get_status(None, ctypes.byref(v)) == mdp.MOE_ERR_INVALID_ARG
     assert L.moe_decode_set_debug(None, 0, 100) == mdp.MOE_ERR_INVALID_ARG
     assert L.moe_decode_launches_per_step(None) == mdp.MOE_ERR_INVALID_ARG
+    assert L.moe_decode_set_tc_min_batch(None, 1) == mdp.MOE_ERR_INVALID_ARG
+    assert L.moe_decode_step_path(None, 1) == mdp.MOE_ERR_INVALID_ARG
     L.moe_decode_destroy(None)
 
 

@@ -2,9 +2,12 @@
 
 Small workloads run the oracle on every row; they span several tiles, K splits
 and ragged tails (batch not a multiple of the row group, odd k, k = E, k = 1,
-a skewed router, correlated rows, two layers). The five measured workloads run
-at full size with the oracle on sampled rows (rows are independent) plus
-properties checked on every row.
+a skewed router, correlated rows, two layers). Both kernels of the batch-shape
+switch are checked: the CUDA-core kernel on every workload, the tensor-core kernel
+on the workloads whose dimensions are multiples of 128 (half tile pairs, batches
+that are not a multiple of 16, hot experts chosen by every row, k = 32, the
+largest slot count). The five measured workloads run at full size with the oracle
+on sampled rows (rows are independent) plus properties checked on every row.
 """
 import dataclasses
 
@@ -14,7 +17,8 @@ import pytest
 import oracle
 import synth
 
-from harness import bf, check_layer, check_y, make_handle, oracle_rows, run_gpu
+from harness import (bf, chained_flips, check_layer, check_y, gpu_layer_outputs, make_handle, oracle_rows,
+                     routing_oracle, run_gpu)
 
 torch = pytest.importorskip("torch")
 
@@ -33,6 +37,23 @@ SMALL = [
     W("b1_k1", B=1, H=256, E=32, k=1, I=32, Is=32, seed=27),
     W("b7_h2048", B=7, H=2048, E=64, k=5, I=512, Is=768 - 256, seed=28),
 ]
+
+
+# tensor-core shapes: every dimension a multiple of 128
+TC_SMALL = [
+    W("tc_b1_k8", B=1, H=512, E=256, k=8, I=256, Is=256, seed=31),
+    W("tc_ragged_b5_e384", B=5, H=1024, E=384, k=6, I=256, Is=512, seed=32),
+    W("tc_b64_k16", B=64, H=512, E=128, k=16, I=128, Is=256, seed=33),
+    W("tc_zipf_b17", B=17, H=768, E=256, k=8, I=256, Is=512, seed=34, router="zipf"),
+    W("tc_half_pairs_b9_h128", B=9, H=128, E=384, k=5, I=128, Is=128, seed=38),
+    W("tc_corr_2layer_b32", B=32, H=512, E=256, k=8, I=128, Is=128, seed=35, layers=2, rows="correlated",
+      nseq=4, rows_per_seq=8),
+    W("tc_k32_b3_h256", B=3, H=256, E=128, k=32, I=128, Is=128, seed=36),
+    W("tc_b2_h2048", B=2, H=2048, E=128, k=2, I=512, Is=768, seed=37),
+]
+
+
+TC_BY_NAME = {w.name: w for w in TC_SMALL}
 
 
 def _layers(wl):
@@ -54,17 +75,21 @@ def _cuda_only():
     _free()
 
 
-def run_and_check(wl, rows=None, handle=None, layers=None):
+def run_and_check(wl, rows=None, handle=None, layers=None, tc_min_batch=None):
     layers = layers if layers is not None else _layers(wl)
-    h = handle or make_handle(wl, layers)
+    h = handle or make_handle(wl, layers, tc_min_batch=tc_min_batch)
     x = wl.x_host()
     out = run_gpu(h, wl, x, n_layers=wl.layers)
     assert out["status"] == 0, f"device status {out['status']}"
     rows = list(range(wl.B)) if rows is None else rows
     orc = oracle_rows(wl, x, rows, n_layers=wl.layers)
-    skip = set()
+    route = orc
+    if wl.layers > 1:
+        mid = gpu_layer_outputs(wl, layers, x, tc_min_batch=_switch_of(h, wl))
+        route = routing_oracle(wl, x, rows, wl.layers, mid)
+    skip = chained_flips(out["layers"], orc, rows, wl.k, tag=wl.name)
     for l in range(wl.layers):
-        ties = check_layer(out["layers"][l], orc[l], rows, wl.k, tag=f"{wl.name} layer {l}")
+        ties = check_layer(out["layers"][l], route[l], rows, wl.k, tag=f"{wl.name} layer {l}")
         skip |= {rows.index(b) for b in ties}
         idx = out["layers"][l]["idx"]
         assert out["layers"][l]["U"] == len(np.unique(idx)), "unique-expert count"
@@ -74,9 +99,84 @@ def run_and_check(wl, rows=None, handle=None, layers=None):
     return out, err
 
 
+def _switch_of(h, wl):
+    """tc_min_batch that reproduces the path h takes for wl's batch."""
+    import moe_decode_persistent_b200 as mdp
+
+    return 1 if h.step_path(wl.B) == mdp.PATH_TENSOR_CORE else 0
+
+
 @pytest.mark.parametrize("wl", SMALL, ids=[w.name for w in SMALL])
 def test_small_workloads_match_oracle(wl):
     run_and_check(wl)
+
+
+@pytest.mark.parametrize("path", ["tensor_core", "cuda_core"])
+@pytest.mark.parametrize("wl", TC_SMALL, ids=[w.name for w in TC_SMALL])
+def test_tc_shaped_workloads_match_oracle_on_both_paths(wl, path):
+    import moe_decode_persistent_b200 as mdp
+
+    tc = path == "tensor_core"
+    layers = _layers(wl)
+    h = make_handle(wl, layers, tc_min_batch=1 if tc else 0)
+    assert h.step_path(wl.B) == (mdp.PATH_TENSOR_CORE if tc else mdp.PATH_CUDA_CORE)
+    run_and_check(wl, handle=h, layers=layers)
+    h.close()
+
+
+def test_cuda_core_only_shapes_never_take_the_tensor_core_path():
+    import moe_decode_persistent_b200 as mdp
+
+    wl = SMALL[3]  # E = 64: not a multiple of 128
+    layers = _layers(wl)
+    h = make_handle(wl, layers, tc_min_batch=1)
+    assert h.step_path(wl.B) == mdp.PATH_CUDA_CORE
+    h.close()
+
+
+def test_tc_deterministic_and_jitter_invariant():
+    import moe_decode_persistent_b200 as mdp
+
+    wl = TC_BY_NAME["tc_zipf_b17"]
+    layers = _layers(wl)
+    h = make_handle(wl, layers, tc_min_batch=1)
+    x = wl.x_host()
+    a = run_gpu(h, wl, x)
+    b = run_gpu(h, wl, x)
+    h.set_debug(mdp.DEBUG_JITTER)
+    c = run_gpu(h, wl, x)
+    h.set_debug(0)
+    for o in (a, b, c):
+        assert o["status"] == 0
+    assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["y"], c["y"])
+    assert np.array_equal(a["layers"][0]["logits"], c["layers"][0]["logits"])
+    h.close()
+
+
+def test_tc_timeout_is_reported_and_handle_recovers():
+    import moe_decode_persistent_b200 as mdp
+
+    wl = TC_BY_NAME["tc_ragged_b5_e384"]
+    layers = _layers(wl)
+    h = make_handle(wl, layers, tc_min_batch=1)
+    x = wl.x_host()
+    h.set_debug(mdp.DEBUG_WITHHOLD_NREADY, wait_ms=300)
+    bad = run_gpu(h, wl, x)
+    assert bad["status"] == mdp.MOE_ERR_TIMEOUT
+    h.set_debug(0)
+    good = run_and_check(wl, handle=h, layers=layers)[0]
+    assert good["status"] == 0
+    h.close()
+
+
+def test_tc_smaller_batch_and_k_than_configured():
+    wl = TC_BY_NAME["tc_b64_k16"]
+    layers = _layers(wl)
+    h = make_handle(wl, layers, tc_min_batch=1)
+    for B, k in ((3, 4), (16, 8), (33, 16), (63, 1)):
+        sub = dataclasses.replace(wl, B=B, k=k)
+        run_and_check(sub, handle=h, layers=layers)
+    h.close()
 
 
 def test_device_generator_matches_host():
@@ -151,15 +251,16 @@ def test_smaller_batch_and_k_than_configured():
     h.close()
 
 
-FULL = [1, 2, 3, 4]
+FULL = [(1, None), (2, None), (3, None), (4, None), (1, 0), (2, 0), (3, 0), (4, 0)]
 SAMPLE_ROWS = {1: [0], 2: [0, 5], 3: [0, 37, 63], 4: [0, 9, 31]}
 
 
-@pytest.mark.parametrize("cfg", FULL)
-def test_full_size_workload(cfg):
+@pytest.mark.parametrize("cfg,tc_min_batch", FULL,
+                         ids=[f"config{c}-" + {None: "switch", 0: "cuda_core", 1: "tensor_core"}[t] for c, t in FULL])
+def test_full_size_workload(cfg, tc_min_batch):
     wl = synth.WORKLOADS[cfg]
     layers = _layers(wl)
-    h = make_handle(wl, layers)
+    h = make_handle(wl, layers, tc_min_batch=tc_min_batch)
     x = wl.x_host()
     out = run_gpu(h, wl, x, n_layers=wl.layers)
     assert out["status"] == 0
@@ -180,9 +281,13 @@ def test_full_size_workload(cfg):
     # sampled rows: the whole layer stack against the oracle
     rows = SAMPLE_ROWS[cfg]
     orc = oracle_rows(wl, x, rows, n_layers=wl.layers)
-    skip = set()
+    route = orc
+    if wl.layers > 1:
+        mid = gpu_layer_outputs(wl, layers, x, tc_min_batch=_switch_of(h, wl))
+        route = routing_oracle(wl, x, rows, wl.layers, mid)
+    skip = chained_flips(out["layers"], orc, rows, wl.k, tag=wl.name)
     for l in range(wl.layers):
-        ties = check_layer(out["layers"][l], orc[l], rows, wl.k, tag=f"{wl.name} layer {l}")
+        ties = check_layer(out["layers"][l], route[l], rows, wl.k, tag=f"{wl.name} layer {l}")
         skip |= {rows.index(b) for b in ties}
     check_y(out["y"][rows], orc, tag=wl.name, skip=skip)
     h.close()
