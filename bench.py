@@ -52,7 +52,10 @@ def parse_args(argv=None):
                          "kernel (0: always the CUDA-core kernel); default: the library's")
     ap.add_argument("--profile-small", action="store_true",
                     help="the batch-1 layer with 64 experts instead of 896 (same per-expert shapes, "
-                         "~2.9 GB of weights): the small case for full ncu captures")
+                         "~2.9 GB of weights): the small case for full ncu captures of the CUDA-core kernel")
+    ap.add_argument("--profile-small-tc", action="store_true",
+                    help="batch 1, 128 experts of intermediate 512 (~2.9 GB of weights): the small case "
+                         "for full ncu captures of the tensor-core kernel")
     return ap.parse_args(argv)
 
 
@@ -394,6 +397,8 @@ def main(argv=None):
     wl = synth.WORKLOADS[args.config]
     if args.profile_small:
         wl = synth.Workload("b1_h7168_e64_k16_profile", B=1, H=7168, E=64, k=16, I=1024, Is=2048, seed=1)
+    if args.profile_small_tc:
+        wl = synth.Workload("b1_h7168_e128_i512_k16_profile", B=1, H=7168, E=128, k=16, I=512, Is=1024, seed=1)
     if args.impl == "reference":
         run_reference(args, wl)
     else:

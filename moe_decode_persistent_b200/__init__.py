@@ -244,8 +244,8 @@ class MoeDecode:
                     "mac_compute_cyc", "mac_stages", "prod_issue_cyc", "prod_stages", "mac_sched_cyc",
                     "mac_reduce_cyc", "mac_loop_cyc", "prod_setup_cyc", "prod_sched_cyc",
                     "prod_loop_cyc", "router_seen", "sched_built", "topk_done", "topk_synced",
-                    "unique_done", "n_published", "topk_loaded", "topk_selected", "r34", "r35",
-                    "r36", "r37", "r38", "r39")
+                    "unique_done", "n_published", "topk_loaded", "topk_selected", "topk_chosen",
+                    "topk_cyc", "sched_placed", "sched_sorted", "start_clk", "r39")
 
     def trace_slots(self) -> int:
         return lib().moe_decode_trace_slots(self.handle)

@@ -39,6 +39,7 @@ enum Counter {
   CTR_ROUTER = 3,  // router tiles finished (logits published)
   CTR_HS = 4,      // shared gate/up tiles finished
   CTR_ABORT = 5,   // non-zero once any CTA gave up a wait
+  CTR_TOPK = 6,    // tensor-core path: rows whose top-k choices are published
   CTR_COUNT = 8
 };
 
@@ -60,14 +61,24 @@ constexpr int kTcMaxN = 64;       // token columns of one tile (max batch)
 constexpr int kTcSharedSplits = 4;
 constexpr int kTcExpertSplits = 4;
 
-// K splits of a router tile pair on the tensor-core path: many short units when the
-// batch is small (the router is on the critical path and its fix-up is cheap), fewer
-// as the batch grows (the fix-up reads splits x batch x 256 partial sums).
+constexpr int kTcRouterSplits = 28;
+
+// K splits of a router tile pair on the tensor-core path: short units (4 K atoms of
+// the 7168-wide layer), so the router finishes soon after the normalised rows exist;
+// each token row's owner CTA sums its row's partials.
 __host__ __device__ inline int tc_router_splits(int B, int nk_atoms) {
-  const int s = B <= 8 ? 28 : B <= 16 ? 14 : B <= 32 ? 8 : 4;
-  return s < nk_atoms ? s : nk_atoms;
+  (void)B;
+  return kTcRouterSplits < nk_atoms ? kTcRouterSplits : nk_atoms;
 }
 __host__ __device__ inline int tc_clamp_splits(int s, int nk_atoms) { return s < nk_atoms ? s : nk_atoms; }
+
+// K splits of an expert's gate/up tiles on the tensor-core path, by the number of
+// token rows that chose the expert: a hot expert streams as whole-K units (no fix-up
+// of its many rows), a cold one in short units that spread over the SMs.
+__host__ __device__ inline int tc_expert_splits(int rows, int nk_atoms) {
+  const int s = rows >= 16 ? 1 : rows >= 4 ? 2 : kTcExpertSplits;
+  return s < nk_atoms ? s : nk_atoms;
+}
 
 struct Params {
   // shapes of this step
@@ -96,6 +107,10 @@ struct Params {
   float* spart;          // [SS][B][Is/128][256]
   float* epart;          // [ES][B*k][I/128][256]
   float* dpart;          // [B*k + B][H]: down outputs of expert slot rows, then shared rows
+  int* tk_idx;           // [B][k] published top-k experts of each row
+  float* tk_w;           // [B][k] their softmax weights
+  uint32_t* row_tix;     // [H/256 tile pairs][max_batch]: down contributions arrived per row
+  unsigned row_tix_count;
   uint32_t* ctr;         // [CTR_COUNT]
   uint32_t* tickets;     // [max_tiles]
   uint32_t* pair_done;   // [kMaxSlots]
@@ -147,6 +162,12 @@ enum TraceSlot {
   TR_N_PUBLISHED = 31,         // a normalised row published by this CTA (stamp)
   TR_TOPK_LOADED = 32,         // schedule: first top-k row's logits loaded (stamp)
   TR_TOPK_SELECTED = 33,       // schedule: first top-k row's selection rounds done (stamp)
+  TR_TOPK_CHOSEN = 34,         // tensor-core path: owned row's top-k chosen (stamp)
+  TR_TOPK_CYC = 35,            // tensor-core path: cycles of the owned row's top-k selection
+  TR_SCHED_PLACED = 36,        // tensor-core path: unique experts placed (stamp)
+  TR_SCHED_SORTED = 37,        // tensor-core path: pairs sorted and counted (stamp, warp 0)
+  TR_START_CLK = 38,           // clock64 at kernel start (on the tensor-core path the routing
+                               // stamps, slots 26-30, 32-34 and 36-37, are clock64 values)
   kTraceSlots = 40
 };
 

@@ -44,6 +44,10 @@ struct moe_decode_handle {
   float* spart;
   float* epart;
   float* dpart;
+  int* tk_idx;
+  float* tk_w;
+  uint32_t* row_tix;
+  unsigned row_tix_count;
   uint32_t* ctr;
   uint32_t* tickets;
   uint32_t* pair_done;
@@ -243,7 +247,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   // tensor-core path: tile pairs of the router and of the down projection, one pair per
   // unique expert, K splits chosen per batch (tc_router_splits) and fixed otherwise
   const int nkH = H / moe::kTcAtomK;
-  size_t rpart_floats = 0, spart_floats = 0, epart_floats = 0, dpart_floats = 0;
+  size_t rpart_floats = 0, spart_floats = 0, epart_floats = 0, dpart_floats = 0, row_tix_n = 0;
   const int tcS = moe::tc_clamp_splits(moe::kTcSharedSplits, nkH);
   const int tcE = moe::tc_clamp_splits(moe::kTcExpertSplits, nkH);
   if (tc_ok) {
@@ -260,6 +264,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
     spart_floats = (size_t)tcS * maxB * 2 * Is;
     epart_floats = (size_t)tcE * maxSlots * 2 * I;
     dpart_floats = (size_t)(maxSlots + maxB) * H;
+    row_tix_n = (size_t)DT2 * maxB;
     const unsigned tu = (unsigned)(RT2 * maxRS + TST * tcS + tcP * TIT * tcE + DT2 * (1 + tcP));
     const unsigned tt = (unsigned)(RT2 + TST + tcP * TIT + DT2);
     if (tu > h->max_units) h->max_units = tu;
@@ -282,6 +287,9 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   const size_t o_spart = carve(spart_floats * 4);
   const size_t o_epart = carve(epart_floats * 4);
   const size_t o_dpart = carve(dpart_floats * 4);
+  const size_t o_tki = carve((size_t)maxSlots * 4);
+  const size_t o_tkw = carve((size_t)maxSlots * 4);
+  const size_t o_rtix = carve(row_tix_n * 4 + 4);
   const size_t o_ctr = carve(moe::CTR_COUNT * 4);
   const size_t o_tix = carve((size_t)h->max_tiles * 4);
   const size_t o_pd = carve(moe::kMaxSlots * 4);
@@ -307,6 +315,10 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   h->spart = (float*)(b + o_spart);
   h->epart = (float*)(b + o_epart);
   h->dpart = (float*)(b + o_dpart);
+  h->tk_idx = (int*)(b + o_tki);
+  h->tk_w = (float*)(b + o_tkw);
+  h->row_tix = (uint32_t*)(b + o_rtix);
+  h->row_tix_count = (unsigned)row_tix_n;
   h->ctr = (uint32_t*)(b + o_ctr);
   h->tickets = (uint32_t*)(b + o_tix);
   h->pair_done = (uint32_t*)(b + o_pd);
@@ -399,6 +411,10 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
       p.spart = h->spart;
       p.epart = h->epart;
       p.dpart = h->dpart;
+      p.tk_idx = h->tk_idx;
+      p.tk_w = h->tk_w;
+      p.row_tix = h->row_tix;
+      p.row_tix_count = h->row_tix_count;
     }
     p.ctr = h->ctr;
     p.tickets = h->tickets;

@@ -130,6 +130,10 @@ struct Sched {
   uint8_t row_of[kMaxSlots];      // token row of slot row r
   float w_of[kMaxSlots];          // routing weight of slot row r
   int16_t slot_of[kMaxSlots];     // slot row of (token b, choice j) at b * k + j
+  // tensor-core path: pairs are the unique experts, hottest first (stable)
+  int16_t eslot[kMaxE];           // unique slot of expert e (valid for selected experts)
+  int pair_ubase[kMaxSlots + 1];  // first expert gate/up unit of pair p (prefix over pairs)
+  uint8_t pair_es[kMaxSlots];     // K splits of pair p's gate/up tiles
 };
 
 // Per-CTA state. The stage ring (kCcRingBytes or kTcRingBytes) sits in front of it in
@@ -151,6 +155,10 @@ struct Smem {
   int acc_unit[kTcAccBufs]; // unit id of the accumulator buffer, or -1 (stop)
   uint32_t tmem_base;
   int epi_last;             // tensor-core epilogue: this unit's split completed its tile
+  int ncomb;                // tensor-core epilogue: rows whose down combine falls to this unit
+  int16_t comb_rows[kTcMaxN];
+  int cnt_base[kTcMaxN + 2];  // tensor-core schedule: pairs per row count, then their bases
+  uint64_t topk_cand[64];     // tensor-core routing: top-k candidates of the owned row
   int bcast;
   int bcast2;
   int nuniq;
@@ -168,6 +176,7 @@ struct Smem {
       unsigned long long mask[kMaxE];
     } t;                               // schedule construction
     float yacc[kBoxRows][65];          // down-tile fix-up (epilogue warp)
+    uint64_t keys[kMaxE];              // tensor-core path: the owned row's packed top-k keys
   } u;
 };
 
@@ -230,12 +239,17 @@ __device__ __forceinline__ bool abort_seen(const Params& p) {
 
 constexpr uint32_t kSuspendNs = 20000;  // longest single suspension inside a wait
 
-// Bounded wait on an mbarrier phase by one thread (suspended while waiting).
-__device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Params& p) {
+// Bounded wait on an mbarrier phase by one thread (suspended while waiting). Between
+// polls the thread sleeps, doubling up to max_sleep_ns, so a waiting warp takes no
+// issue slots from the warps that work.
+__device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Params& p, uint32_t max_sleep_ns = 128) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  uint32_t ns = 16;
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    __nanosleep(ns);
+    ns = ns * 2 < max_sleep_ns ? ns * 2 : max_sleep_ns;
     if (abort_seen(p)) return false;
     if (globaltimer_ns() - t0 > p.wait_ns) {
       record_abort(p, MOE_ERR_TIMEOUT);
@@ -246,13 +260,19 @@ __device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Params& p) {
 
 // Bounded wait on an mbarrier phase by a whole warp: every lane observes the
 // completion itself, lane 0 alone decides to give up, and the result is uniform.
-__device__ bool warp_wait(uint64_t* bar, uint32_t parity, const Params& p, int lane) {
+// max_sleep_ns > 0: sleep between polls (doubling up to it); 0: poll without sleeping.
+__device__ bool warp_wait(uint64_t* bar, uint32_t parity, const Params& p, int lane, uint32_t max_sleep_ns = 512) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   uint64_t t0 = 0;
   if (lane == 0) t0 = globaltimer_ns();
+  uint32_t ns = 16;
   for (uint32_t it = 0;; ++it) {
     const bool done = mbar_try_wait_sleep(bar, parity, kSuspendNs);
     if (__all_sync(0xffffffffu, done)) return true;
+    if (max_sleep_ns) {
+      __nanosleep(ns);
+      ns = ns * 2 < max_sleep_ns ? ns * 2 : max_sleep_ns;
+    }
     if ((it & 3u) == 3u) {
       int stop = 0;
       if (lane == 0) {
@@ -283,11 +303,11 @@ __device__ bool wait_counter(const uint32_t* c, uint32_t target, const Params& p
   }
 }
 
-// Rendezvous of the 8 MAC warps (an mbarrier with bounded waits).
+// Rendezvous of the 8 MAC warps (an mbarrier with bounded waits, polled without sleeping).
 __device__ __forceinline__ bool mac_sync(Smem& sm, uint32_t& phase, const Params& p, int lane) {
   __syncwarp();
   if (lane == 0) mbar_arrive(&sm.mac_bar);
-  const bool ok = warp_wait(&sm.mac_bar, phase, p, lane);
+  const bool ok = warp_wait(&sm.mac_bar, phase, p, lane, 256);
   phase ^= 1u;
   return ok;
 }
@@ -315,6 +335,12 @@ __device__ __forceinline__ void trace_put(const Params& p, int slot, unsigned lo
 template <bool kTrace>
 __device__ __forceinline__ long long tclock() {
   return kTrace ? clock64() : 0;
+}
+
+// SM-clock stamp (clock64 of this CTA's SM; compare only with TR_START_CLK of the same CTA).
+template <bool kTrace>
+__device__ __forceinline__ void trace_clk(const Params& p, int slot) {
+  if (kTrace) p.trace[(size_t)blockIdx.x * kTraceSlots + slot] = (unsigned long long)clock64();
 }
 
 // ---- shape and unit decoding ---------------------------------------------------------------
@@ -369,7 +395,7 @@ __device__ void make_shape_tc(const Params& p, Shape& s) {
   s.NR = s.RT * s.RS;
   s.NS = s.ST * s.SS;
   s.spp = 0;
-  s.router_target = s.RT;
+  s.router_target = s.NR;  // every router unit publishes its own partial sums
   s.hs_target = s.ST;
   s.pair_target = s.IT;
 }
@@ -462,14 +488,23 @@ __device__ UnitDesc decode_unit_tc(const Shape& sh, const Sched& sc, int u) {
     d.ticket = sh.RT + d.tile;
     split_range(sh.nkbH, sh.SS, d.split, d.kb0, d.nkb);
   } else if (u < sh.NR + sh.NS + sc.NE) {
+    // pair p owns units [pair_ubase[p], pair_ubase[p + 1]): its IT tiles x pair_es[p] splits
     const int v = u - sh.NR - sh.NS;
+    int lo = 0, hi = sc.P - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (sc.pair_ubase[mid] <= v) lo = mid;
+      else hi = mid - 1;
+    }
+    const int es = sc.pair_es[lo];
+    const int w = v - sc.pair_ubase[lo];
     d.type = UT_EXPERT;
-    d.split = v % sh.ES;
-    d.tile = (v / sh.ES) % sh.IT;
-    d.pair = v / (sh.ES * sh.IT);
-    d.nsplit = sh.ES;
-    d.ticket = sh.RT + sh.ST + d.pair * sh.IT + d.tile;
-    split_range(sh.nkbH, sh.ES, d.split, d.kb0, d.nkb);
+    d.pair = lo;
+    d.split = w % es;
+    d.tile = w / es;
+    d.nsplit = es;
+    d.ticket = sh.RT + sh.ST + lo * sh.IT + d.tile;
+    split_range(sh.nkbH, es, d.split, d.kb0, d.nkb);
   } else {
     const int v = u - sh.NR - sh.NS - sc.NE;
     const int src = v / sh.DT;
@@ -842,12 +877,11 @@ __device__ void warp_topk_row(const Params& p, Smem& sm, int b, int lane) {
   }
 }
 
-// Builds sm.sc from the final logits. Called by all MAC warps; false on abort. On the
-// CUDA-core path an expert's rows form pairs of up to kActGroup rows; on the
-// tensor-core path all of an expert's rows (at most the batch, <= 64) form one pair.
-template <bool kTrace, bool kTC>
+// Builds sm.sc from the final logits (CUDA-core path). Called by all MAC warps; false
+// on abort. An expert's rows form (expert, row group) pairs of up to kActGroup rows.
+template <bool kTrace>
 __device__ bool build_schedule(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
-  constexpr int kGroup = kTC ? kMaxSlots : kActGroup;
+  constexpr int kGroup = kActGroup;
   const Shape& sh = sm.sh;
   Sched& sc = sm.sc;
   const int mtid = mw * 32 + lane;
@@ -931,7 +965,7 @@ __device__ bool build_schedule(const Params& p, Smem& sm, int mw, int lane, uint
       sc.slot_base[U] = (int16_t)rbase;
       sc.P = pbase;
       sc.NE = pbase * sh.IT * sh.ES;
-      sc.down_splits = kTC ? 1 + pbase : sh.GB + (pbase + kDownPairsPerSplit - 1) / kDownPairsPerSplit;
+      sc.down_splits = sh.GB + (pbase + kDownPairsPerSplit - 1) / kDownPairsPerSplit;
       sc.ND = sh.DT * sc.down_splits;
       sc.total = sh.NR + sh.NS + sc.NE + sc.ND;
       const unsigned tiles = (unsigned)(sh.GB * (sh.RT + sh.ST) + pbase * sh.IT + sh.DT);
@@ -970,6 +1004,360 @@ __device__ bool build_schedule(const Params& p, Smem& sm, int mw, int lane, uint
   }
   const bool ok = mac_sync(sm, mphase, p, lane);
   if (mtid == 0) trace_stamp<kTrace>(p, TR_SCHED_BUILT);
+  return ok;
+}
+
+// ---- tensor-core path: routing (MAC warps, i.e. warps 1-8) -------------------------------------
+
+__device__ __forceinline__ uint64_t umax64(uint64_t a, uint64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// Inverse of float_key.
+__device__ __forceinline__ float key_float(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+// Packed top-k key of logit t of expert e: (order key << 32) | ~e. The largest packed
+// key is the largest logit with the lowest index among equals; all packed keys
+// differ; 0 (a non-finite logit) is below every finite key.
+__device__ __forceinline__ uint64_t topk_key(float t, int e) {
+  return isfinite(t) ? (((uint64_t)float_key(t) << 32) | (uint64_t)(~(uint32_t)e)) : 0ull;
+}
+
+// Top-k of one row by one warp from its packed keys in shared memory (keys[0..E),
+// E a multiple of 32, k <= 32): the k largest, ties to the lower expert index. The
+// k-th largest of the 32 lane maxima, L, bounds the k-th largest key from below (k
+// lanes hold a key >= L), so the top k are among the keys >= L. Those candidates
+// (usually a few dozen) are gathered, and each one's position in the descending order
+// is its rank, the number of candidates above it. With more than 64 candidates the
+// exact fallback takes k rounds of warp-wide maxima, dropping each winner from keys.
+// This code runs once per launch, usually with its instructions evicted from L2 by
+// the weight stream, so it is kept compact (loops, not unrolled register arrays).
+// Lane j < k returns the j-th choice's packed key. cand: 64 entries.
+__device__ uint64_t warp_topk_keys(uint64_t* keys, int E, int k, int lane, uint64_t* cand) {
+  const int nq = E / 32;
+  uint64_t m = 0ull;
+#pragma unroll 1
+  for (int q = 0; q < nq; ++q) m = umax64(m, keys[q * 32 + lane]);
+  int lrank = 0;
+#pragma unroll 1
+  for (int sl = 0; sl < 32; ++sl) lrank += shfl_u64(m, sl) > m ? 1 : 0;
+  const uint32_t lb = __ballot_sync(0xffffffffu, lrank == k - 1 && m != 0ull);
+  const uint64_t L = lb ? shfl_u64(m, __ffs(lb) - 1) : 1ull;
+  int c = 0;
+#pragma unroll 1
+  for (int q = 0; q < nq; ++q) c += keys[q * 32 + lane] >= L ? 1 : 0;
+  int incl = c;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += t;
+  }
+  const int total = __shfl_sync(0xffffffffu, incl, 31);
+  uint64_t mine = 0ull;
+  if (total <= 64) {
+    int o = incl - c;
+#pragma unroll 1
+    for (int q = 0; q < nq; ++q) {
+      const uint64_t x = keys[q * 32 + lane];
+      if (x >= L) cand[o++] = x;
+    }
+    __syncwarp();
+    const uint64_t x0 = lane < total ? cand[lane] : 0ull;
+    const uint64_t x1 = lane + 32 < total ? cand[lane + 32] : 0ull;
+    int r0 = 0, r1 = 0;
+#pragma unroll 1
+    for (int sl = 0; sl < 32; ++sl) {
+      const uint64_t o0 = shfl_u64(x0, sl), o1 = shfl_u64(x1, sl);
+      r0 += (o0 > x0 ? 1 : 0) + (o1 > x0 ? 1 : 0);
+      r1 += (o0 > x1 ? 1 : 0) + (o1 > x1 ? 1 : 0);
+    }
+    __syncwarp();
+    if (lane < total) cand[r0] = x0;
+    if (lane + 32 < total) cand[r1] = x1;
+    __syncwarp();
+    mine = lane < k ? cand[lane] : 0ull;
+    __syncwarp();
+  } else {
+#pragma unroll 1
+    for (int j = 0; j < k; ++j) {
+      uint64_t best = 0ull;
+#pragma unroll 1
+      for (int q = 0; q < nq; ++q) best = umax64(best, keys[q * 32 + lane]);
+      const uint32_t hi = (uint32_t)(best >> 32);
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, hi);
+      const uint32_t wlo = __reduce_max_sync(0xffffffffu, hi == kmax ? (uint32_t)best : 0u);
+      const uint64_t win = ((uint64_t)kmax << 32) | wlo;
+      if (lane == j) mine = win;
+      const int e = (int)(~wlo);
+      __syncwarp();
+      if (lane == 0 && e >= 0 && e < E) keys[e] = 0ull;
+      __syncwarp();
+    }
+  }
+  return mine;
+}
+
+// The rows this CTA owns (row b is owned by CTA b): once every router unit has
+// published its partial sums, the row's logits are their sum in split order plus the
+// bias; one warp takes the top-k and the softmax over it and publishes the choices.
+template <bool kTrace>
+__device__ bool route_rows_tc(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
+  const Shape& sh = sm.sh;
+  const int mtid = mw * 32 + lane;
+  const int E = p.E;
+  for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+    if (mw == 0) {
+      int ok = 1;
+      if (lane == 0) ok = wait_counter(&p.ctr[CTR_ROUTER], (uint32_t)sh.router_target, p) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (lane == 0) {
+        sm.bcast = ok;
+        sm.bcast2 = 0;  // non-finite logit seen
+      }
+    }
+    if (!mac_sync(sm, mphase, p, lane)) return false;
+    if (!sm.bcast) return false;
+    if (mtid == 0) trace_clk<kTrace>(p, TR_ROUTER_SEEN);
+    const size_t stride4 = (size_t)p.B * E / 4;  // float4 stride between splits
+    const float4* src = reinterpret_cast<const float4*>(p.rpart + (size_t)b * E);
+    bool nonfinite = false;
+    for (int e4 = mtid; e4 < E / 4; e4 += kMacThreads) {
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+      for (int s0 = 0; s0 < sh.RS; s0 += 8) {
+        float4 t[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (s0 + i < sh.RS) t[i] = __ldcg(src + (size_t)(s0 + i) * stride4 + e4);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (s0 + i < sh.RS) {
+            acc.x += t[i].x;
+            acc.y += t[i].y;
+            acc.z += t[i].z;
+            acc.w += t[i].w;
+          }
+        }
+      }
+      if (p.bias) {  // 4-byte aligned: scalar loads
+        acc.x += p.bias[4 * e4];
+        acc.y += p.bias[4 * e4 + 1];
+        acc.z += p.bias[4 * e4 + 2];
+        acc.w += p.bias[4 * e4 + 3];
+      }
+      reinterpret_cast<float4*>(p.logits + (size_t)b * E)[e4] = acc;
+      const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint64_t key = topk_key(a4[i], 4 * e4 + i);
+        if (key == 0ull) nonfinite = true;
+        sm.u.keys[4 * e4 + i] = key;
+        if (p.dbg_logits) p.dbg_logits[(size_t)b * E + 4 * e4 + i] = a4[i];
+      }
+    }
+    if (__any_sync(0xffffffffu, nonfinite) && lane == 0) sm.bcast2 = 1;
+    if (!mac_sync(sm, mphase, p, lane)) return false;
+    if (mtid == 0) trace_clk<kTrace>(p, TR_TOPK_LOADED);
+    if (mw == 0) {
+      const long long tk0 = tclock<kTrace>();
+      const uint64_t mine = warp_topk_keys(sm.u.keys, E, p.k, lane, sm.topk_cand);
+      if (lane == 0 && kTrace) {
+        trace_put<kTrace>(p, TR_TOPK_CYC, (unsigned long long)(tclock<kTrace>() - tk0));
+        trace_clk<kTrace>(p, TR_TOPK_CHOSEN);
+      }
+      if (sm.bcast2 && lane == 0) record_error(p, MOE_ERR_NONFINITE);
+      int e = (int)(~(uint32_t)mine);
+      if (e < 0 || e >= E) e = 0;  // only with a non-finite row (reported)
+      const float val = lane < p.k ? key_float((uint32_t)(mine >> 32)) : 0.0f;
+      const float mx = __shfl_sync(0xffffffffu, val, 0);
+      const float ex = lane < p.k ? expf(val - mx) : 0.0f;
+      float z = ex;
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+      if (lane < p.k) {
+        p.tk_idx[b * p.k + lane] = e;
+        p.tk_w[b * p.k + lane] = ex / z;
+      }
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) {
+        red_release_add(&p.ctr[CTR_TOPK], 1u);
+        trace_clk<kTrace>(p, TR_TOPK_SELECTED);
+      }
+    }
+    if (!mac_sync(sm, mphase, p, lane)) return false;  // sm.u.keys free again
+  }
+  return true;
+}
+
+// Every CTA: the schedule of the tensor-core path from the published choices. Pairs
+// are the unique experts ordered by row count, hottest first (stable in expert order),
+// so the largest units are queued first and the down units that complete rows last
+// are those of experts with few rows. An expert's slot rows keep expert order.
+template <bool kTrace>
+__device__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
+  const Shape& sh = sm.sh;
+  Sched& sc = sm.sc;
+  const int mtid = mw * 32 + lane;
+  const int B = p.B, k = p.k;
+  for (int e = mtid; e < p.E; e += kMacThreads) sm.u.t.mask[e] = 0ull;
+  if (mw == 0) {
+    int ok = 1;
+    if (lane == 0) ok = wait_counter(&p.ctr[CTR_TOPK], (uint32_t)B, p) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (lane == 0) sm.bcast = ok;
+  }
+  if (!mac_sync(sm, mphase, p, lane)) return false;
+  if (!sm.bcast) return false;
+  if (mtid == 0) trace_clk<kTrace>(p, TR_TOPK_SYNCED);
+  for (int t = mtid; t < B * k; t += kMacThreads) {
+    const int e = __ldcg(p.tk_idx + t);
+    const float w = __ldcg(p.tk_w + t);
+    sm.u.t.topk_idx[t] = e;
+    sm.u.t.topk_w[t] = w;
+    atomicOr(&sm.u.t.mask[e], 1ull << (t / k));
+  }
+  if (!mac_sync(sm, mphase, p, lane)) return false;
+  if (mtid == 0) trace_clk<kTrace>(p, TR_TOPK_DONE);
+  // unique experts in ascending id: per-chunk counts, then placement
+  const int nchunk = p.E / 32;
+  for (int ch = mw; ch < nchunk; ch += kMacWarps) {
+    const uint32_t bal = __ballot_sync(0xffffffffu, sm.u.t.mask[ch * 32 + lane] != 0ull);
+    if (lane == 0) sm.chunk_cnt[ch] = (int16_t)__popc(bal);
+  }
+  if (!mac_sync(sm, mphase, p, lane)) return false;
+  {
+    const int cnt = lane < nchunk ? sm.chunk_cnt[lane] : 0;
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += t;
+    }
+    for (int ch = mw; ch < nchunk; ch += kMacWarps) {
+      const int chbase = __shfl_sync(0xffffffffu, incl - cnt, ch);
+      const unsigned long long m = sm.u.t.mask[ch * 32 + lane];
+      const uint32_t bal = __ballot_sync(0xffffffffu, m != 0ull);
+      if (m != 0ull) {
+        const int pos = chbase + __popc(bal & ((1u << lane) - 1u));
+        sc.slot_expert[pos] = (int16_t)(ch * 32 + lane);
+        sc.slot_cnt[pos] = (int16_t)__popcll(m);
+        sc.eslot[ch * 32 + lane] = (int16_t)pos;
+      }
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (mw == 0 && lane == 0) sm.nuniq = total;
+  }
+  if (mtid <= kTcMaxN + 1 && mtid < kMacThreads) sm.cnt_base[mtid] = 0;
+  if (!mac_sync(sm, mphase, p, lane)) return false;
+  if (mtid == 0) trace_clk<kTrace>(p, TR_SCHED_PLACED);
+  if (mw == 0) {
+    const int U = sm.nuniq;
+    // slot bases (slot order)
+    int rbase = 0;
+    for (int i0 = 0; i0 < U; i0 += 32) {
+      const int i = i0 + lane;
+      const int c = i < U ? sc.slot_cnt[i] : 0;
+      int cs = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, cs, off);
+        if (lane >= off) cs += t;
+      }
+      if (i < U) sc.slot_base[i] = (int16_t)(rbase + cs - c);
+      rbase += __shfl_sync(0xffffffffu, cs, 31);
+    }
+    // stable counting sort of the slots by row count, descending
+    for (int i = lane; i < U; i += 32) atomicAdd(&sm.cnt_base[sc.slot_cnt[i]], 1);
+    __syncwarp();
+    {
+      const int c0 = kTcMaxN - 2 * lane, c1 = c0 - 1;  // lane 0: counts 64, 63; lane 31: 2, 1
+      const int h0 = sm.cnt_base[c0], h1 = sm.cnt_base[c1];
+      int incl = h0 + h1;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += t;
+      }
+      __syncwarp();
+      sm.cnt_base[c0] = incl - h0 - h1;
+      sm.cnt_base[c1] = incl - h1;
+    }
+    __syncwarp();
+    for (int i0 = 0; i0 < U; i0 += 32) {
+      const int i = i0 + lane;
+      const int c = i < U ? sc.slot_cnt[i] : 0;
+      const uint32_t m = __match_any_sync(0xffffffffu, c);
+      const int rank = __popc(m & ((1u << lane) - 1u));
+      if (c > 0) sc.pair_slot[sm.cnt_base[c] + rank] = (int16_t)i;
+      __syncwarp();
+      if (c > 0 && lane == __ffs(m) - 1) sm.cnt_base[c] += __popc(m);
+      __syncwarp();
+    }
+    if (lane == 0) trace_clk<kTrace>(p, TR_SCHED_SORTED);
+    // gate/up units per pair and their prefix
+    int ubase = 0;
+    for (int p0 = 0; p0 < U; p0 += 32) {
+      const int pr = p0 + lane;
+      int units = 0;
+      if (pr < U) {
+        const int es = tc_expert_splits(sc.slot_cnt[sc.pair_slot[pr]], sh.nkbH);
+        sc.pair_es[pr] = (uint8_t)es;
+        sc.pair_group[pr] = 0;
+        units = sh.IT * es;
+      }
+      int cs = units;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int t = __shfl_up_sync(0xffffffffu, cs, off);
+        if (lane >= off) cs += t;
+      }
+      if (pr < U) sc.pair_ubase[pr] = ubase + cs - units;
+      ubase += __shfl_sync(0xffffffffu, cs, 31);
+    }
+    if (lane == 0) {
+      sc.U = U;
+      sc.S = rbase;
+      sc.slot_base[U] = (int16_t)rbase;
+      sc.P = U;
+      sc.pair_ubase[U] = ubase;
+      sc.NE = ubase;
+      sc.down_splits = 1 + U;
+      sc.ND = sh.DT * sc.down_splits;
+      sc.total = sh.NR + sh.NS + sc.NE + sc.ND;
+      const unsigned tiles = (unsigned)(sh.RT + sh.ST + U * sh.IT + sh.DT);
+      sm.bcast2 = ((unsigned)sc.total <= p.max_units && tiles <= p.max_tiles && U <= kMaxSlots) ? 1 : 0;
+      if (!sm.bcast2) record_abort(p, MOE_ERR_UNSUPPORTED_SHAPE);
+    }
+  }
+  if (mtid == 0) trace_clk<kTrace>(p, TR_UNIQUE_DONE);
+  if (!mac_sync(sm, mphase, p, lane)) return false;
+  if (!sm.bcast2) return false;
+  // slot rows: an expert's rows in token order; rank of row b among them by popcount
+  for (int t = mtid; t < B * k; t += kMacThreads) {
+    const int b = t / k;
+    const int e = sm.u.t.topk_idx[t];
+    const unsigned long long m = sm.u.t.mask[e];
+    const int r = sc.slot_base[sc.eslot[e]] + __popcll(m & ((1ull << b) - 1ull));
+    sc.row_of[r] = (uint8_t)b;
+    sc.w_of[r] = sm.u.t.topk_w[t];
+    sc.slot_of[t] = (int16_t)r;
+  }
+  if (blockIdx.x == 0) {
+    for (int t = mtid; t < B * k; t += kMacThreads) {
+      if (p.dbg_idx) p.dbg_idx[t] = sm.u.t.topk_idx[t];
+      if (p.dbg_w) p.dbg_w[t] = sm.u.t.topk_w[t];
+    }
+    if (mtid == 0 && p.dbg_nuniq) *p.dbg_nuniq = sc.U;
+  }
+  const bool ok = mac_sync(sm, mphase, p, lane);
+  if (mtid == 0) trace_clk<kTrace>(p, TR_SCHED_BUILT);
   return ok;
 }
 
@@ -1599,7 +1987,7 @@ __device__ void mac_warps_cc(const Params& p, Smem& sm, uint8_t* ring, int mw, i
   while (ok) {
     {
       const long long t0 = tclock<kTrace>();
-      const bool got = warp_wait(&sm.full[slot], phase, p, lane);
+      const bool got = warp_wait(&sm.full[slot], phase, p, lane, 0);
       c_full += (unsigned long long)(tclock<kTrace>() - t0);
       if (!got) break;
     }
@@ -1610,7 +1998,7 @@ __device__ void mac_warps_cc(const Params& p, Smem& sm, uint8_t* ring, int mw, i
     }
     if (hd.kind == HK_SCHED) {
       const long long ts0 = tclock<kTrace>();
-      ok = build_schedule<kTrace, false>(p, sm, mw, lane, mphase);
+      ok = build_schedule<kTrace>(p, sm, mw, lane, mphase);
       c_sched += (unsigned long long)(tclock<kTrace>() - ts0);
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[slot]);
@@ -1648,7 +2036,7 @@ __device__ void mac_warps_cc(const Params& p, Smem& sm, uint8_t* ring, int mw, i
     if (seg_end) {
       if (!rb_claimed) {
         const long long t0 = tclock<kTrace>();
-        const bool got = warp_wait(&sm.rb_empty[ub], ubphase ^ 1u, p, lane);
+        const bool got = warp_wait(&sm.rb_empty[ub], ubphase ^ 1u, p, lane, 0);
         c_rb += (unsigned long long)(tclock<kTrace>() - t0);
         if (!got) break;
         rb_claimed = true;
@@ -1827,7 +2215,7 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
 __device__ __forceinline__ bool epi_sync(Smem& sm, uint32_t& phase, const Params& p, int lane) {
   __syncwarp();
   if (lane == 0) mbar_arrive(&sm.epi_bar);
-  const bool ok = warp_wait(&sm.epi_bar, phase, p, lane);
+  const bool ok = warp_wait(&sm.epi_bar, phase, p, lane, 0);
   phase ^= 1u;
   return ok;
 }
@@ -1842,93 +2230,56 @@ __device__ __forceinline__ void tmem_cols16(uint32_t ta, int j0, bool two, uint3
   if (two) tmem_regs_after_wait(v1);
 }
 
-// The fix-up of a tile whose splits are all done: fixed split order, so the sums do
-// not depend on which split finished last. Thread et (0..127) owns tile row et.
+// The fix-up of a gate/up tile whose splits are all done: fixed split order, so the
+// sums do not depend on which split finished last. Thread et (0..127) owns tile row et.
 __device__ void fixup_tc(const Params& p, const Smem& sm, const UnitDesc& d, int et) {
   const Shape& sh = sm.sh;
   const Sched& sc = sm.sc;
-  const int B = sh.B;
-  switch (d.type) {
-    case UT_ROUTER:
-      for (int a = 0; a < 2; ++a) {
-        const int e = d.tile * 2 * kTcRows + a * kTcRows + et;
-        if (e >= p.E) continue;
-        const float bias = p.bias ? p.bias[e] : 0.0f;
-        for (int b = 0; b < B; ++b) {
-          const float* src = p.rpart + (size_t)b * p.E + e;
-          const size_t stride = (size_t)B * p.E;
-          float s = 0.0f;
-          int sp = 0;
-          for (; sp + 4 <= d.nsplit; sp += 4) {
-            const float v0 = __ldcg(src + sp * stride), v1 = __ldcg(src + (sp + 1) * stride);
-            const float v2 = __ldcg(src + (sp + 2) * stride), v3 = __ldcg(src + (sp + 3) * stride);
-            s += v0;
-            s += v1;
-            s += v2;
-            s += v3;
-          }
-          for (; sp < d.nsplit; ++sp) s += __ldcg(src + sp * stride);
-          const float v = s + bias;
-          p.logits[(size_t)b * p.E + e] = v;
-          if (p.dbg_logits) p.dbg_logits[(size_t)b * p.E + e] = v;
-        }
+  if (d.type == UT_SHARED) {
+    for (int b = 0; b < sh.B; ++b) {
+      float g = 0.0f, u = 0.0f;
+      for (int sp = 0; sp < d.nsplit; ++sp) {
+        const float* src = p.spart + (((size_t)sp * sh.B + b) * sh.ST + d.tile) * (2 * kTcRows);
+        g += __ldcg(src + et);
+        u += __ldcg(src + kTcRows + et);
       }
-      break;
-    case UT_SHARED:
-      for (int b = 0; b < B; ++b) {
-        float g = 0.0f, u = 0.0f;
-        for (int sp = 0; sp < d.nsplit; ++sp) {
-          const float* src = p.spart + (((size_t)sp * B + b) * sh.ST + d.tile) * (2 * kTcRows);
-          g += __ldcg(src + et);
-          u += __ldcg(src + kTcRows + et);
-        }
-        p.hs[(size_t)b * p.Is + d.tile * kTcRows + et] = f2bf(silu(g) * u);
-      }
-      break;
-    case UT_EXPERT: {
-      const int i = sc.pair_slot[d.pair];
-      const int r0 = sc.slot_base[i], cnt = sc.slot_cnt[i];
-      for (int j = 0; j < cnt; ++j) {
-        float g = 0.0f, u = 0.0f;
-        for (int sp = 0; sp < d.nsplit; ++sp) {
-          const float* src = p.epart + (((size_t)sp * sc.S + r0 + j) * sh.IT + d.tile) * (2 * kTcRows);
-          g += __ldcg(src + et);
-          u += __ldcg(src + kTcRows + et);
-        }
-        p.he[(size_t)(r0 + j) * p.I + d.tile * kTcRows + et] = f2bf(silu(g) * u);
-      }
-      break;
+      p.hs[(size_t)b * p.Is + d.tile * kTcRows + et] = f2bf(silu(g) * u);
     }
-    default:
-      // y = bf16(x + s + sum_j w_j d_j): shared part first, then the row's choices in
-      // top-k order
-      for (int a = 0; a < 2; ++a) {
-        const int h = d.tile * 2 * kTcRows + a * kTcRows + et;
-        if (h >= p.H) continue;
-        for (int b = 0; b < B; ++b) {
-          float acc = __ldcg(p.dpart + (size_t)(sc.S + b) * p.H + h);
-          const int16_t* so = &sc.slot_of[b * sh.k];
-          int j = 0;
-          for (; j + 4 <= sh.k; j += 4) {
-            const int r0 = so[j], r1 = so[j + 1], r2 = so[j + 2], r3 = so[j + 3];
-            const float v0 = __ldcg(p.dpart + (size_t)r0 * p.H + h);
-            const float v1 = __ldcg(p.dpart + (size_t)r1 * p.H + h);
-            const float v2 = __ldcg(p.dpart + (size_t)r2 * p.H + h);
-            const float v3 = __ldcg(p.dpart + (size_t)r3 * p.H + h);
-            acc = fmaf(sc.w_of[r0], v0, acc);
-            acc = fmaf(sc.w_of[r1], v1, acc);
-            acc = fmaf(sc.w_of[r2], v2, acc);
-            acc = fmaf(sc.w_of[r3], v3, acc);
-          }
-          for (; j < sh.k; ++j) {
-            const int r = so[j];
-            acc = fmaf(sc.w_of[r], __ldcg(p.dpart + (size_t)r * p.H + h), acc);
-          }
-          const float xv = bf2f(p.x[(size_t)b * p.H + h]);
-          p.y[(size_t)b * p.H + h] = f2bf(xv + acc);
-        }
+  } else {
+    const int i = sc.pair_slot[d.pair];
+    const int r0 = sc.slot_base[i], cnt = sc.slot_cnt[i];
+    for (int j = 0; j < cnt; ++j) {
+      float g = 0.0f, u = 0.0f;
+      for (int sp = 0; sp < d.nsplit; ++sp) {
+        const float* src = p.epart + (((size_t)sp * sc.S + r0 + j) * sh.IT + d.tile) * (2 * kTcRows);
+        g += __ldcg(src + et);
+        u += __ldcg(src + kTcRows + et);
       }
-      break;
+      p.he[(size_t)(r0 + j) * p.I + d.tile * kTcRows + et] = f2bf(silu(g) * u);
+    }
+  }
+}
+
+// Row b of down tile pair t once its k expert contributions and the shared one have
+// all arrived: y = bf16(x + s + sum_j w_j d_j), the shared part first, then the row's
+// choices in top-k order. Thread et owns features t*256 + et and t*256 + 128 + et.
+__device__ void combine_row_tc(const Params& p, const Smem& sm, int t, int b, int et) {
+  const Shape& sh = sm.sh;
+  const Sched& sc = sm.sc;
+  const int16_t* so = &sc.slot_of[b * sh.k];
+  for (int a = 0; a < 2; ++a) {
+    const int h = t * 2 * kTcRows + a * kTcRows + et;
+    if (h >= p.H) continue;
+    float v[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < sh.k) v[j] = __ldcg(p.dpart + (size_t)so[j] * p.H + h);
+    float acc = __ldcg(p.dpart + (size_t)(sc.S + b) * p.H + h);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < sh.k) acc = fmaf(sc.w_of[so[j]], v[j], acc);
+    const float xv = bf2f(p.x[(size_t)b * p.H + h]);
+    p.y[(size_t)b * p.H + h] = f2bf(xv + acc);
   }
 }
 
@@ -1957,29 +2308,22 @@ __device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
     const Sched& sc = sm.sc;
     const UnitDesc d = decode_unit_tc(sh, sc, u);
     const uint32_t ta = tq + (uint32_t)(abuf * kTcAccCols);
-    const bool direct = d.nsplit == 1 && d.type <= UT_EXPERT;
+    const bool direct = d.nsplit == 1 && (d.type == UT_SHARED || d.type == UT_EXPERT);
     uint32_t v0[16], v1[16];
     switch (d.type) {
       case UT_ROUTER: {
         const int e0 = d.tile * 2 * kTcRows + row, e1 = e0 + kTcRows;
         const bool two = d.tile * 2 * kTcRows + kTcRows < p.E;
-        float* dst = direct ? p.logits : p.rpart + (size_t)d.split * sh.B * p.E;
-        const float b0 = direct && p.bias ? p.bias[e0] : 0.0f;
-        const float b1 = direct && p.bias && two ? p.bias[e1] : 0.0f;
+        // this split's partial logits; the row owners sum the splits
+        float* dst = p.rpart + (size_t)d.split * sh.B * p.E;
         for (int j0 = 0; j0 < sh.B; j0 += 16) {
           tmem_cols16(ta, j0, two, v0, v1);
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int b = j0 + jj;
             if (b < sh.B) {
-              const float a0 = __uint_as_float(v0[jj]) + b0;
-              dst[(size_t)b * p.E + e0] = a0;
-              if (direct && p.dbg_logits) p.dbg_logits[(size_t)b * p.E + e0] = a0;
-              if (two) {
-                const float a1 = __uint_as_float(v1[jj]) + b1;
-                dst[(size_t)b * p.E + e1] = a1;
-                if (direct && p.dbg_logits) p.dbg_logits[(size_t)b * p.E + e1] = a1;
-              }
+              dst[(size_t)b * p.E + e0] = __uint_as_float(v0[jj]);
+              if (two) dst[(size_t)b * p.E + e1] = __uint_as_float(v1[jj]);
             }
           }
         }
@@ -2069,27 +2413,52 @@ __device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
       abuf = 0;
       aphase ^= 1u;
     }
-    bool finished = direct;
-    if (!direct) {
-      // split-K / multi-source tile: count this split in, the last one does the fix-up
+    if (d.type == UT_DOWN_SHARED || d.type == UT_DOWN_EXPERT) {
+      // count this source in for each of its rows; the unit that brings a row's last
+      // contribution (k experts + the shared expert) combines that row of the tile
       __threadfence();
       if (!epi_sync(sm, ephase, p, lane)) break;
-      if (et == 0) {
-        const uint32_t old = atom_add_acq_rel(&p.tickets[d.ticket], 1u);
-        const int last = old == (uint32_t)(d.nsplit - 1);
-        if (last) st_relaxed_gpu(&p.tickets[d.ticket], 0u);
-        sm.epi_last = last;
+      const bool shared = d.type == UT_DOWN_SHARED;
+      const int i = shared ? 0 : sc.pair_slot[d.pair];
+      const int cnt = shared ? sh.B : sc.slot_cnt[i];
+      if (et < cnt) {
+        const int b = shared ? et : sc.row_of[sc.slot_base[i] + et];
+        uint32_t* tix = &p.row_tix[d.tile * sh.B + b];
+        const uint32_t old = atom_add_acq_rel(tix, 1u);
+        if (old == (uint32_t)sh.k) {
+          st_relaxed_gpu(tix, 0u);
+          sm.comb_rows[atomicAdd(&sm.ncomb, 1)] = (int16_t)b;
+        }
       }
       if (!epi_sync(sm, ephase, p, lane)) break;
-      finished = sm.epi_last != 0;
-      if (finished) fixup_tc(p, sm, d, et);
-    }
-    uint32_t* done = done_counter(p, d);
-    if (finished && done) {
-      fence_proxy_async_global();
-      __threadfence();
-      if (!epi_sync(sm, ephase, p, lane)) break;
-      if (et == 0) red_release_add(done, 1u);
+      const int ncomb = sm.ncomb;
+      if (ncomb > 0) {
+        for (int ci = 0; ci < ncomb; ++ci) combine_row_tc(p, sm, d.tile, sm.comb_rows[ci], et);
+        if (!epi_sync(sm, ephase, p, lane)) break;
+        if (et == 0) sm.ncomb = 0;  // ordered before the next unit's list by its first rendezvous
+      }
+    } else {
+      bool finished = direct || d.type == UT_ROUTER;
+      if (!finished) {
+        // split-K gate/up tile: count this split in, the last one does the fix-up
+        __threadfence();
+        if (!epi_sync(sm, ephase, p, lane)) break;
+        if (et == 0) {
+          const uint32_t old = atom_add_acq_rel(&p.tickets[d.ticket], 1u);
+          const int last = old == (uint32_t)(d.nsplit - 1);
+          if (last) st_relaxed_gpu(&p.tickets[d.ticket], 0u);
+          sm.epi_last = last;
+        }
+        if (!epi_sync(sm, ephase, p, lane)) break;
+        finished = sm.epi_last != 0;
+        if (finished) fixup_tc(p, sm, d, et);
+      }
+      if (finished) {
+        fence_proxy_async_global();
+        __threadfence();
+        if (!epi_sync(sm, ephase, p, lane)) break;
+        if (et == 0) red_release_add(done_counter(p, d), 1u);
+      }
     }
     c_busy += (unsigned long long)(tclock<kTrace>() - tb0);
   }
@@ -2130,10 +2499,12 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
     }
     mbar_init(&sm.sched_bar, 1);
     mbar_init(&sm.mac_bar, kMacWarps);
+    sm.ncomb = 0;
     for (int w = 0; w < kMaxSlots / 32; ++w) sm.known_done[w] = 0u;
     if (kTrace) {
       for (int t = 0; t < kTraceSlots; ++t) p.trace[(size_t)blockIdx.x * kTraceSlots + t] = 0ull;
       trace_stamp<kTrace>(p, TR_START);
+      trace_clk<kTrace>(p, TR_START_CLK);
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -2158,7 +2529,8 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       const int mw = warp_id - 1;
       uint32_t mphase = 0;
       bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
-      if (ok) ok = build_schedule<kTrace, true>(p, sm, mw, lane, mphase);
+      if (ok) ok = route_rows_tc<kTrace>(p, sm, mw, lane, mphase);
+      if (ok) ok = build_schedule_tc<kTrace>(p, sm, mw, lane, mphase);
       if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
     } else {
       mac_warps_cc<kTrace>(p, sm, ring, warp_id - 1, lane);
@@ -2189,6 +2561,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       if (aborted) {
         for (unsigned t = 0; t < p.max_tiles; ++t) p.tickets[t] = 0u;
         for (int t = 0; t < kMaxSlots; ++t) p.pair_done[t] = 0u;
+        for (unsigned t = 0; t < p.row_tix_count; ++t) p.row_tix[t] = 0u;
       } else {
         for (int t = 0; t < sm.sc.P; ++t) p.pair_done[t] = 0u;
       }
