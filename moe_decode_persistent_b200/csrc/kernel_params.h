@@ -72,6 +72,13 @@ __host__ __device__ inline int tc_router_splits(int B, int nk_atoms) {
 }
 __host__ __device__ inline int tc_clamp_splits(int s, int nk_atoms) { return s < nk_atoms ? s : nk_atoms; }
 
+// K splits of the shared expert's gate/up tiles on the tensor-core path: short units
+// while the batch is small; whole-K units (no fix-up over batch x splits partial sums)
+// once the batch is large.
+__host__ __device__ inline int tc_shared_splits(int B, int nk_atoms) {
+  return tc_clamp_splits(B <= 16 ? kTcSharedSplits : 1, nk_atoms);
+}
+
 // K splits of an expert's gate/up tiles on the tensor-core path, by the number of
 // token rows that chose the expert: a hot expert streams as whole-K units (no fix-up
 // of its many rows), a cold one in short units that spread over the SMs.

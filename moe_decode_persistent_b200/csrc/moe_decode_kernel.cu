@@ -115,6 +115,7 @@ struct Shape {
   int NR, NS;
   int spp;  // stages per (expert, row group) pair of a down unit
   int NA;   // tensor-core path: token columns of n- and hs-based tiles (B rounded up to 16)
+  int pre;  // units queued before the routing schedule (no unit before it needs the schedule)
   int router_target, hs_target, pair_target;  // tiles that publish logits / h_s / one pair's h
 };
 
@@ -237,7 +238,6 @@ __device__ __forceinline__ bool abort_seen(const Params& p) {
   return ld_relaxed_gpu(&p.ctr[CTR_ABORT]) != 0u;
 }
 
-constexpr uint32_t kSuspendNs = 20000;  // longest single suspension inside a wait
 
 // Bounded wait on an mbarrier phase by one thread (suspended while waiting). Between
 // polls the thread sleeps, doubling up to max_sleep_ns, so a waiting warp takes no
@@ -247,7 +247,7 @@ __device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Params& p, uint3
   const uint64_t t0 = globaltimer_ns();
   uint32_t ns = 16;
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if (mbar_try_wait(bar, parity)) return true;
     __nanosleep(ns);
     ns = ns * 2 < max_sleep_ns ? ns * 2 : max_sleep_ns;
     if (abort_seen(p)) return false;
@@ -261,13 +261,13 @@ __device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Params& p, uint3
 // Bounded wait on an mbarrier phase by a whole warp: every lane observes the
 // completion itself, lane 0 alone decides to give up, and the result is uniform.
 // max_sleep_ns > 0: sleep between polls (doubling up to it); 0: poll without sleeping.
-__device__ bool warp_wait(uint64_t* bar, uint32_t parity, const Params& p, int lane, uint32_t max_sleep_ns = 512) {
+__device__ bool warp_wait(uint64_t* bar, uint32_t parity, const Params& p, int lane, uint32_t max_sleep_ns = 256) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   uint64_t t0 = 0;
   if (lane == 0) t0 = globaltimer_ns();
   uint32_t ns = 16;
   for (uint32_t it = 0;; ++it) {
-    const bool done = mbar_try_wait_sleep(bar, parity, kSuspendNs);
+    const bool done = mbar_try_wait(bar, parity);
     if (__all_sync(0xffffffffu, done)) return true;
     if (max_sleep_ns) {
       __nanosleep(ns);
@@ -307,7 +307,7 @@ __device__ bool wait_counter(const uint32_t* c, uint32_t target, const Params& p
 __device__ __forceinline__ bool mac_sync(Smem& sm, uint32_t& phase, const Params& p, int lane) {
   __syncwarp();
   if (lane == 0) mbar_arrive(&sm.mac_bar);
-  const bool ok = warp_wait(&sm.mac_bar, phase, p, lane, 256);
+  const bool ok = warp_wait(&sm.mac_bar, phase, p, lane, 64);
   phase ^= 1u;
   return ok;
 }
@@ -366,6 +366,7 @@ __device__ void make_shape(const Params& p, Shape& s) {
   s.NS = s.GB * s.ST * s.SS;
   s.spp = (s.nkbI + 1) / 2;
   s.NA = 0;
+  s.pre = s.NR + s.NS;
   s.router_target = s.GB * s.RT;
   s.hs_target = s.GB * s.ST;
   s.pair_target = s.IT;
@@ -395,6 +396,7 @@ __device__ void make_shape_tc(const Params& p, Shape& s) {
   s.NR = s.RT * s.RS;
   s.NS = s.ST * s.SS;
   s.spp = 0;
+  s.pre = s.NR + s.NS + s.DT;  // the shared expert's down tiles need only h_s
   s.router_target = s.NR;  // every router unit publishes its own partial sums
   s.hs_target = s.ST;
   s.pair_target = s.IT;
@@ -463,10 +465,10 @@ __device__ UnitDesc decode_unit(const Shape& sh, const Sched& sc, int u) {
 }
 
 // Tensor-core path unit enumeration (queue order): router (tile pair, K split),
-// shared gate/up (tile, K split), expert gate/up ((unique expert, tile), K split),
-// down (source, tile pair) with source 0 the shared expert and source 1 + i the
-// unique expert i. Down units carry no K split; their tile pair is finished by the
-// last of its B-independent 1 + U sources.
+// shared gate/up (tile, K split), shared down (tile pair) -- all before the routing
+// schedule -- then expert gate/up ((pair, tile), K split) and expert down (pair, tile
+// pair). Down units carry no K split; each row of a down tile pair is combined by the
+// unit that brings its last contribution.
 __device__ UnitDesc decode_unit_tc(const Shape& sh, const Sched& sc, int u) {
   UnitDesc d;
   d.npair = 0;
@@ -487,9 +489,17 @@ __device__ UnitDesc decode_unit_tc(const Shape& sh, const Sched& sc, int u) {
     d.nsplit = sh.SS;
     d.ticket = sh.RT + d.tile;
     split_range(sh.nkbH, sh.SS, d.split, d.kb0, d.nkb);
-  } else if (u < sh.NR + sh.NS + sc.NE) {
+  } else if (u < sh.pre) {
+    d.type = UT_DOWN_SHARED;
+    d.tile = u - sh.NR - sh.NS;
+    d.split = 0;
+    d.nsplit = 1;
+    d.ticket = 0;
+    d.kb0 = 0;
+    d.nkb = sh.nkbIs;
+  } else if (u < sh.pre + sc.NE) {
     // pair p owns units [pair_ubase[p], pair_ubase[p + 1]): its IT tiles x pair_es[p] splits
-    const int v = u - sh.NR - sh.NS;
+    const int v = u - sh.pre;
     int lo = 0, hi = sc.P - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -506,22 +516,16 @@ __device__ UnitDesc decode_unit_tc(const Shape& sh, const Sched& sc, int u) {
     d.ticket = sh.RT + sh.ST + lo * sh.IT + d.tile;
     split_range(sh.nkbH, es, d.split, d.kb0, d.nkb);
   } else {
-    const int v = u - sh.NR - sh.NS - sc.NE;
-    const int src = v / sh.DT;
+    const int v = u - sh.pre - sc.NE;
+    d.type = UT_DOWN_EXPERT;
+    d.pair = v / sh.DT;
     d.tile = v % sh.DT;
-    d.split = src;
-    d.nsplit = sc.down_splits;
-    d.ticket = sh.RT + sh.ST + sc.P * sh.IT + d.tile;
+    d.npair = 1;
+    d.split = 0;
+    d.nsplit = 1;
+    d.ticket = 0;
     d.kb0 = 0;
-    if (src == 0) {
-      d.type = UT_DOWN_SHARED;
-      d.nkb = sh.nkbIs;
-    } else {
-      d.type = UT_DOWN_EXPERT;
-      d.pair = src - 1;
-      d.npair = 1;
-      d.nkb = sh.nkbI;
-    }
+    d.nkb = sh.nkbI;
   }
   d.nstages = d.nkb;
   return d;
@@ -1042,15 +1046,15 @@ __device__ __forceinline__ uint64_t topk_key(float t, int e) {
 __device__ uint64_t warp_topk_keys(uint64_t* keys, int E, int k, int lane, uint64_t* cand) {
   const int nq = E / 32;
   uint64_t m = 0ull;
-#pragma unroll 1
+#pragma unroll 4
   for (int q = 0; q < nq; ++q) m = umax64(m, keys[q * 32 + lane]);
   int lrank = 0;
-#pragma unroll 1
+#pragma unroll 4
   for (int sl = 0; sl < 32; ++sl) lrank += shfl_u64(m, sl) > m ? 1 : 0;
   const uint32_t lb = __ballot_sync(0xffffffffu, lrank == k - 1 && m != 0ull);
   const uint64_t L = lb ? shfl_u64(m, __ffs(lb) - 1) : 1ull;
   int c = 0;
-#pragma unroll 1
+#pragma unroll 4
   for (int q = 0; q < nq; ++q) c += keys[q * 32 + lane] >= L ? 1 : 0;
   int incl = c;
 #pragma unroll
@@ -1062,7 +1066,7 @@ __device__ uint64_t warp_topk_keys(uint64_t* keys, int E, int k, int lane, uint6
   uint64_t mine = 0ull;
   if (total <= 64) {
     int o = incl - c;
-#pragma unroll 1
+#pragma unroll 4
     for (int q = 0; q < nq; ++q) {
       const uint64_t x = keys[q * 32 + lane];
       if (x >= L) cand[o++] = x;
@@ -1071,7 +1075,7 @@ __device__ uint64_t warp_topk_keys(uint64_t* keys, int E, int k, int lane, uint6
     const uint64_t x0 = lane < total ? cand[lane] : 0ull;
     const uint64_t x1 = lane + 32 < total ? cand[lane + 32] : 0ull;
     int r0 = 0, r1 = 0;
-#pragma unroll 1
+#pragma unroll 4
     for (int sl = 0; sl < 32; ++sl) {
       const uint64_t o0 = shfl_u64(x0, sl), o1 = shfl_u64(x1, sl);
       r0 += (o0 > x0 ? 1 : 0) + (o1 > x0 ? 1 : 0);
@@ -1084,10 +1088,10 @@ __device__ uint64_t warp_topk_keys(uint64_t* keys, int E, int k, int lane, uint6
     mine = lane < k ? cand[lane] : 0ull;
     __syncwarp();
   } else {
-#pragma unroll 1
+#pragma unroll 4
     for (int j = 0; j < k; ++j) {
       uint64_t best = 0ull;
-#pragma unroll 1
+#pragma unroll 4
       for (int q = 0; q < nq; ++q) best = umax64(best, keys[q * 32 + lane]);
       const uint32_t hi = (uint32_t)(best >> 32);
       const uint32_t kmax = __reduce_max_sync(0xffffffffu, hi);
@@ -1329,8 +1333,8 @@ __device__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, u
       sc.pair_ubase[U] = ubase;
       sc.NE = ubase;
       sc.down_splits = 1 + U;
-      sc.ND = sh.DT * sc.down_splits;
-      sc.total = sh.NR + sh.NS + sc.NE + sc.ND;
+      sc.ND = sh.DT * U;
+      sc.total = sh.pre + sc.NE + sc.ND;
       const unsigned tiles = (unsigned)(sh.RT + sh.ST + U * sh.IT + sh.DT);
       sm.bcast2 = ((unsigned)sc.total <= p.max_units && tiles <= p.max_tiles && U <= kMaxSlots) ? 1 : 0;
       if (!sm.bcast2) record_abort(p, MOE_ERR_UNSUPPORTED_SHAPE);
@@ -1866,7 +1870,7 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
   if (lane == 0)
     for (int t = TM_T_WR; t < TM_COUNT; ++t) prefetch_tensormap(&p.tmaps[t]);
   bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
-  const int pre = sh.NR + sh.NS;
+  const int pre = sh.pre;
   int u = pr.grab();
   bool first_expert = true, first_down = true;
   unsigned long long c_slot = 0, c_dep = 0, c_grab = 0, c_issue = 0, c_stages = 0, c_units = 0;
@@ -1898,18 +1902,11 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
     const uint32_t tx = (uint32_t)(x.nbox * kTcTileBytes + x.N * kTcAtomK * 2);
     const int info0 = x.nbox | ((x.N / kTcActRows) << 2);
     const int ka_end = d.kb0 + d.nkb;
-    for (int ka = d.kb0; ka < ka_end && ok; ++ka) {
-      {
-        const long long t0 = tclock<kTrace>();
-        ok = pr.wait_slot();
-        c_slot += (unsigned long long)(tclock<kTrace>() - t0);
-      }
-      if (!ok) break;
-      const long long ti0 = tclock<kTrace>();
+    // one stage: header, barrier armed for weights + activations, the weight tiles
+    auto issue_weights = [&](int ka) {
       uint8_t* dst = ring + pr.slot * kTcSlotBytes;
       uint64_t* fb = &sm.full[pr.slot];
       pr.mark_pending();
-      const int col = ka * kTcAtomK;
       if (lane == 0) {
         StageHeader h;
         h.kind = HK_STAGE;
@@ -1918,35 +1915,75 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
         h.wrow = -1;
         sm.hdr[pr.slot] = h;
         mbar_arrive_expect_tx(fb, tx);
-        tma_load_2d(dst, x.tw0, col, x.y0, fb, pol);
-        if (x.nbox == 2) tma_load_2d(dst + kTcTileBytes, x.tw1, col, x.y1, fb, pol);
+        tma_load_2d(dst, x.tw0, ka * kTcAtomK, x.y0, fb, pol);
+        if (x.nbox == 2) tma_load_2d(dst + kTcTileBytes, x.tw1, ka * kTcAtomK, x.y1, fb, pol);
       }
-      bool dep_ok = true;
+    };
+    // the activation operand of stage ka into ring slot s (only after its publication)
+    auto issue_act = [&](int ka, int slot) {
+      if (lane == 0) {
+        uint8_t* act = ring + slot * kTcSlotBytes + 2 * kTcTileBytes;
+        uint64_t* fb = &sm.full[slot];
+        for (int q = 0; q < x.N / kTcActRows; ++q)
+          tma_load_2d_plain(act + q * kTcActRows * kTcAtomK * 2, x.ta, ka * kTcAtomK, x.arow + q * kTcActRows, fb);
+      }
+    };
+    bool dep_known = x.dep == 0 ? n_ok
+                   : x.dep == 1 ? hs_ok
+                                : ((sm.known_done[x.pair >> 5] >> (x.pair & 31)) & 1u) != 0u;
+    int ka = d.kb0;
+    if (!dep_known) {
+      // input not yet published: arm stages with their weight tiles first, so the
+      // weights stream while the input is awaited -- a ring's worth for h, one stage
+      // for the normalised rows (at the start of the step the HBM queue must stay short
+      // for the loads of x that the normalisation waits on)
+      const int depth = x.dep == 0 ? 1 : kTcStages;
+      const int pre_end = ka_end < d.kb0 + depth ? ka_end : d.kb0 + depth;
+      const int slot0 = pr.slot;
+      for (; ka < pre_end && ok; ++ka) {
+        const long long t0 = tclock<kTrace>();
+        ok = pr.wait_slot();
+        c_slot += (unsigned long long)(tclock<kTrace>() - t0);
+        if (!ok) break;
+        issue_weights(ka);
+        __syncwarp();
+        pr.advance();
+        ++c_stages;
+      }
+      const int narmed = ka - d.kb0;
+      bool dep_ok = ok;
       const long long td0 = tclock<kTrace>();
-      if (ka == d.kb0) {
+      if (ok) {
         if (x.dep == 0) {
-          if (!n_ok) {
-            dep_ok = n_ok = pr.wait_dep(&p.ctr[CTR_NREADY], (uint32_t)p.B);
-            if (lane == 0) trace_stamp<kTrace>(p, TR_NREADY);
-          }
+          dep_ok = n_ok = pr.wait_dep(&p.ctr[CTR_NREADY], (uint32_t)p.B);
+          if (lane == 0) trace_stamp<kTrace>(p, TR_NREADY);
         } else if (x.dep == 1) {
-          if (!hs_ok) dep_ok = hs_ok = pr.wait_dep(&p.ctr[CTR_HS], (uint32_t)sh.hs_target);
+          dep_ok = hs_ok = pr.wait_dep(&p.ctr[CTR_HS], (uint32_t)sh.hs_target);
         } else {
           dep_ok = pr.wait_pair(x.pair);
         }
       }
-      const long long td1 = tclock<kTrace>();
-      c_dep += (unsigned long long)(td1 - td0);
-      if (lane == 0) {
-        uint8_t* act = dst + 2 * kTcTileBytes;
-        for (int q = 0; q < x.N / kTcActRows; ++q)
-          tma_load_2d_plain(act + q * kTcActRows * kTcAtomK * 2, x.ta, col, x.arow + q * kTcActRows, fb);
+      c_dep += (unsigned long long)(tclock<kTrace>() - td0);
+      // every armed barrier gets its activation bytes, also after a failed wait
+      for (int i = 0; i < narmed; ++i) issue_act(d.kb0 + i, (slot0 + i) % kTcStages);
+      __syncwarp();
+      if (!dep_ok) ok = false;
+    }
+    for (; ka < ka_end && ok; ++ka) {
+      {
+        const long long t0 = tclock<kTrace>();
+        ok = pr.wait_slot();
+        c_slot += (unsigned long long)(tclock<kTrace>() - t0);
       }
+      if (!ok) break;
+      const long long ti0 = tclock<kTrace>();
+      const int slot = pr.slot;
+      issue_weights(ka);
+      issue_act(ka, slot);
       __syncwarp();
       pr.advance();
-      c_issue += (unsigned long long)(tclock<kTrace>() - ti0) - (unsigned long long)(td1 - td0);
+      c_issue += (unsigned long long)(tclock<kTrace>() - ti0);
       ++c_stages;
-      if (!dep_ok) ok = false;
     }
     {
       const long long t0 = tclock<kTrace>();
@@ -2260,26 +2297,42 @@ __device__ void fixup_tc(const Params& p, const Smem& sm, const UnitDesc& d, int
   }
 }
 
-// Row b of down tile pair t once its k expert contributions and the shared one have
-// all arrived: y = bf16(x + s + sum_j w_j d_j), the shared part first, then the row's
-// choices in top-k order. Thread et owns features t*256 + et and t*256 + 128 + et.
-__device__ void combine_row_tc(const Params& p, const Smem& sm, int t, int b, int et) {
+// Rows rows[0..n) of down tile pair t once each has all its k expert contributions and
+// the shared one: y = bf16(x + s + sum_j w_j d_j), the shared part first, then the
+// row's choices in top-k order. Down partial rows: the shared expert's token row b at
+// b, expert slot row r at B + r. 64 threads cover a row's 256 features four at a
+// time (128-bit loads), two rows per pass.
+__device__ void combine_rows_tc(const Params& p, const Smem& sm, int t, const int16_t* rows, int n, int et) {
   const Shape& sh = sm.sh;
   const Sched& sc = sm.sc;
-  const int16_t* so = &sc.slot_of[b * sh.k];
-  for (int a = 0; a < 2; ++a) {
-    const int h = t * 2 * kTcRows + a * kTcRows + et;
-    if (h >= p.H) continue;
-    float v[kMaxTopK];
+  const int h = t * 2 * kTcRows + 4 * (et & 63);
+  if (h >= p.H) return;
+  for (int ci = et >> 6; ci < n; ci += 2) {
+    const int b = rows[ci];
+    const int16_t* so = &sc.slot_of[b * sh.k];
+    float4 acc = __ldcg(reinterpret_cast<const float4*>(p.dpart + (size_t)b * p.H + h));
+    for (int j0 = 0; j0 < sh.k; j0 += 8) {
+      float4 v[8];
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < sh.k) v[j] = __ldcg(p.dpart + (size_t)so[j] * p.H + h);
-    float acc = __ldcg(p.dpart + (size_t)(sc.S + b) * p.H + h);
+      for (int jj = 0; jj < 8; ++jj)
+        if (j0 + jj < sh.k)
+          v[jj] = __ldcg(reinterpret_cast<const float4*>(p.dpart + (size_t)(sh.B + so[j0 + jj]) * p.H + h));
 #pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j)
-      if (j < sh.k) acc = fmaf(sc.w_of[so[j]], v[j], acc);
-    const float xv = bf2f(p.x[(size_t)b * p.H + h]);
-    p.y[(size_t)b * p.H + h] = f2bf(xv + acc);
+      for (int jj = 0; jj < 8; ++jj) {
+        if (j0 + jj < sh.k) {
+          const float w = sc.w_of[so[j0 + jj]];
+          acc.x = fmaf(w, v[jj].x, acc.x);
+          acc.y = fmaf(w, v[jj].y, acc.y);
+          acc.z = fmaf(w, v[jj].z, acc.z);
+          acc.w = fmaf(w, v[jj].w, acc.w);
+        }
+      }
+    }
+    const uint2 xv = *reinterpret_cast<const uint2*>(p.x + (size_t)b * p.H + h);
+    uint2 yv;
+    yv.x = (uint32_t)f2bf(bf2f(xv.x & 0xFFFFu) + acc.x) | ((uint32_t)f2bf(bf2f(xv.x >> 16) + acc.y) << 16);
+    yv.y = (uint32_t)f2bf(bf2f(xv.y & 0xFFFFu) + acc.z) | ((uint32_t)f2bf(bf2f(xv.y >> 16) + acc.w) << 16);
+    *reinterpret_cast<uint2*>(p.y + (size_t)b * p.H + h) = yv;
   }
 }
 
@@ -2292,6 +2345,7 @@ __device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
   const uint32_t tq = sm.tmem_base + ((uint32_t)(quad * 32) << 16);
   int abuf = 0;
   uint32_t aphase = 0, ephase = 0;
+  bool sched_seen = false;
   unsigned long long c_busy = 0;
   for (;;) {
     if (!warp_wait(&sm.acc_full[abuf], aphase, p, lane)) break;
@@ -2382,11 +2436,11 @@ __device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
         break;
       }
       default: {
-        // down: unweighted partial rows of the source (expert slot rows, or S + b for
-        // the shared expert); the tile's last source combines them
+        // down: unweighted partial rows of the source (token rows 0..B-1 for the shared
+        // expert, B + slot row for an expert), combined per row once all have arrived
         const bool shared = d.type == UT_DOWN_SHARED;
         const int i = shared ? 0 : sc.pair_slot[d.pair];
-        const int r0 = shared ? sc.S : sc.slot_base[i];
+        const int r0 = shared ? 0 : sh.B + sc.slot_base[i];
         const int cnt = shared ? sh.B : sc.slot_cnt[i];
         const int h0 = d.tile * 2 * kTcRows + row, h1 = h0 + kTcRows;
         const bool two = d.tile * 2 * kTcRows + kTcRows < p.H;
@@ -2433,7 +2487,12 @@ __device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
       if (!epi_sync(sm, ephase, p, lane)) break;
       const int ncomb = sm.ncomb;
       if (ncomb > 0) {
-        for (int ci = 0; ci < ncomb; ++ci) combine_row_tc(p, sm, d.tile, sm.comb_rows[ci], et);
+        // a shared-expert tile can complete a row before this CTA's schedule exists
+        if (!sched_seen) {
+          if (!warp_wait(&sm.sched_bar, 0u, p, lane)) break;
+          sched_seen = true;
+        }
+        combine_rows_tc(p, sm, d.tile, sm.comb_rows, ncomb, et);
         if (!epi_sync(sm, ephase, p, lane)) break;
         if (et == 0) sm.ncomb = 0;  // ordered before the next unit's list by its first rendezvous
       }
