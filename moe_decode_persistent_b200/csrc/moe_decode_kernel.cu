@@ -246,14 +246,17 @@ __device__ bool wait_mbar(uint64_t* bar, uint32_t parity, const Params& p, uint3
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t ns = 16;
-  for (;;) {
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     __nanosleep(ns);
     ns = ns * 2 < max_sleep_ns ? ns * 2 : max_sleep_ns;
-    if (abort_seen(p)) return false;
-    if (globaltimer_ns() - t0 > p.wait_ns) {
-      record_abort(p, MOE_ERR_TIMEOUT);
-      return false;
+    // the abort flag is a global load (about a microsecond under load): not every poll
+    if ((it & 31u) == 31u) {
+      if (abort_seen(p)) return false;
+      if (globaltimer_ns() - t0 > p.wait_ns) {
+        record_abort(p, MOE_ERR_TIMEOUT);
+        return false;
+      }
     }
   }
 }
@@ -273,7 +276,7 @@ __device__ bool warp_wait(uint64_t* bar, uint32_t parity, const Params& p, int l
       __nanosleep(ns);
       ns = ns * 2 < max_sleep_ns ? ns * 2 : max_sleep_ns;
     }
-    if ((it & 3u) == 3u) {
+    if ((it & 31u) == 31u) {  // the abort flag is a global load: not every poll
       int stop = 0;
       if (lane == 0) {
         if (abort_seen(p)) {
@@ -292,10 +295,10 @@ __device__ bool warp_wait(uint64_t* bar, uint32_t parity, const Params& p, int l
 __device__ bool wait_counter(const uint32_t* c, uint32_t target, const Params& p) {
   if (ld_acquire_gpu(c) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (;;) {
+  for (uint32_t it = 0;; ++it) {
     __nanosleep(64);
     if (ld_acquire_gpu(c) >= target) return true;
-    if (abort_seen(p)) return false;
+    if ((it & 7u) == 7u && abort_seen(p)) return false;
     if (globaltimer_ns() - t0 > p.wait_ns) {
       record_abort(p, MOE_ERR_TIMEOUT);
       return false;
@@ -1204,8 +1207,14 @@ __device__ bool route_rows_tc(const Params& p, Smem& sm, int mw, int lane, uint3
 // are the unique experts ordered by row count, hottest first (stable in expert order),
 // so the largest units are queued first and the down units that complete rows last
 // are those of experts with few rows. An expert's slot rows keep expert order.
+// dry: a pass over synthetic choices (row b takes experts (13 j + b) mod E, distinct
+// for j < 32 as 13 is odd and E a multiple of 128 below 13 * 128) with no global
+// effects, made by CTAs that own no row while they wait for the published choices, so
+// that the real pass runs with its instructions cached (one out-of-line copy of the
+// code serves both passes).
 template <bool kTrace>
-__device__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
+__device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase,
+                                               bool dry) {
   const Shape& sh = sm.sh;
   Sched& sc = sm.sc;
   const int mtid = mw * 32 + lane;
@@ -1213,22 +1222,22 @@ __device__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, u
   for (int e = mtid; e < p.E; e += kMacThreads) sm.u.t.mask[e] = 0ull;
   if (mw == 0) {
     int ok = 1;
-    if (lane == 0) ok = wait_counter(&p.ctr[CTR_TOPK], (uint32_t)B, p) ? 1 : 0;
+    if (lane == 0 && !dry) ok = wait_counter(&p.ctr[CTR_TOPK], (uint32_t)B, p) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (lane == 0) sm.bcast = ok;
   }
   if (!mac_sync(sm, mphase, p, lane)) return false;
   if (!sm.bcast) return false;
-  if (mtid == 0) trace_clk<kTrace>(p, TR_TOPK_SYNCED);
+  if (mtid == 0 && !dry) trace_clk<kTrace>(p, TR_TOPK_SYNCED);
   for (int t = mtid; t < B * k; t += kMacThreads) {
-    const int e = __ldcg(p.tk_idx + t);
-    const float w = __ldcg(p.tk_w + t);
+    const int e = dry ? (13 * (t % k) + t / k) % p.E : __ldcg(p.tk_idx + t);
+    const float w = dry ? 1.0f : __ldcg(p.tk_w + t);
     sm.u.t.topk_idx[t] = e;
     sm.u.t.topk_w[t] = w;
     atomicOr(&sm.u.t.mask[e], 1ull << (t / k));
   }
   if (!mac_sync(sm, mphase, p, lane)) return false;
-  if (mtid == 0) trace_clk<kTrace>(p, TR_TOPK_DONE);
+  if (mtid == 0 && !dry) trace_clk<kTrace>(p, TR_TOPK_DONE);
   // unique experts in ascending id: per-chunk counts, then placement
   const int nchunk = p.E / 32;
   for (int ch = mw; ch < nchunk; ch += kMacWarps) {
@@ -1260,7 +1269,7 @@ __device__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, u
   }
   if (mtid <= kTcMaxN + 1 && mtid < kMacThreads) sm.cnt_base[mtid] = 0;
   if (!mac_sync(sm, mphase, p, lane)) return false;
-  if (mtid == 0) trace_clk<kTrace>(p, TR_SCHED_PLACED);
+  if (mtid == 0 && !dry) trace_clk<kTrace>(p, TR_SCHED_PLACED);
   if (mw == 0) {
     const int U = sm.nuniq;
     // slot bases (slot order)
@@ -1304,7 +1313,7 @@ __device__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, u
       if (c > 0 && lane == __ffs(m) - 1) sm.cnt_base[c] += __popc(m);
       __syncwarp();
     }
-    if (lane == 0) trace_clk<kTrace>(p, TR_SCHED_SORTED);
+    if (lane == 0 && !dry) trace_clk<kTrace>(p, TR_SCHED_SORTED);
     // gate/up units per pair and their prefix
     int ubase = 0;
     for (int p0 = 0; p0 < U; p0 += 32) {
@@ -1337,10 +1346,10 @@ __device__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, u
       sc.total = sh.pre + sc.NE + sc.ND;
       const unsigned tiles = (unsigned)(sh.RT + sh.ST + U * sh.IT + sh.DT);
       sm.bcast2 = ((unsigned)sc.total <= p.max_units && tiles <= p.max_tiles && U <= kMaxSlots) ? 1 : 0;
-      if (!sm.bcast2) record_abort(p, MOE_ERR_UNSUPPORTED_SHAPE);
+      if (!sm.bcast2 && !dry) record_abort(p, MOE_ERR_UNSUPPORTED_SHAPE);
     }
   }
-  if (mtid == 0) trace_clk<kTrace>(p, TR_UNIQUE_DONE);
+  if (mtid == 0 && !dry) trace_clk<kTrace>(p, TR_UNIQUE_DONE);
   if (!mac_sync(sm, mphase, p, lane)) return false;
   if (!sm.bcast2) return false;
   // slot rows: an expert's rows in token order; rank of row b among them by popcount
@@ -1353,7 +1362,7 @@ __device__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, u
     sc.w_of[r] = sm.u.t.topk_w[t];
     sc.slot_of[t] = (int16_t)r;
   }
-  if (blockIdx.x == 0) {
+  if (blockIdx.x == 0 && !dry) {
     for (int t = mtid; t < B * k; t += kMacThreads) {
       if (p.dbg_idx) p.dbg_idx[t] = sm.u.t.topk_idx[t];
       if (p.dbg_w) p.dbg_w[t] = sm.u.t.topk_w[t];
@@ -1361,7 +1370,7 @@ __device__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, u
     if (mtid == 0 && p.dbg_nuniq) *p.dbg_nuniq = sc.U;
   }
   const bool ok = mac_sync(sm, mphase, p, lane);
-  if (mtid == 0) trace_clk<kTrace>(p, TR_SCHED_BUILT);
+  if (mtid == 0 && !dry) trace_clk<kTrace>(p, TR_SCHED_BUILT);
   return ok;
 }
 
@@ -1888,8 +1897,12 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
     if (sched_ready && u >= sm.sc.total) break;
     const long long tu0 = tclock<kTrace>();
     const UnitDesc d = decode_unit_tc(sh, sm.sc, u);
+    // the next unit's ticket is requested now (its round trip overlaps this unit's
+    // issue), except after a router unit: the router units are then spread over the
+    // SMs instead of pairs of them landing on the CTAs that start first
+    const bool early_grab = d.type != UT_ROUTER;
     uint32_t next_ticket = 0;
-    if (lane == 0) next_ticket = atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
+    if (lane == 0 && early_grab) next_ticket = atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
     if (lane == 0 && kTrace) {
       if (first_expert && d.type == UT_EXPERT) { trace_stamp<kTrace>(p, TR_FIRST_EXPERT); first_expert = false; }
       if (first_down && (d.type == UT_DOWN_SHARED || d.type == UT_DOWN_EXPERT)) { trace_stamp<kTrace>(p, TR_FIRST_DOWN); first_down = false; }
@@ -1987,6 +2000,7 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
     }
     {
       const long long t0 = tclock<kTrace>();
+      if (lane == 0 && !early_grab) next_ticket = atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
       u = __shfl_sync(0xffffffffu, (int)next_ticket, 0);
       c_grab += (unsigned long long)(tclock<kTrace>() - t0);
     }
@@ -2589,7 +2603,20 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       uint32_t mphase = 0;
       bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
       if (ok) ok = route_rows_tc<kTrace>(p, sm, mw, lane, mphase);
-      if (ok) ok = build_schedule_tc<kTrace>(p, sm, mw, lane, mphase);
+      if (ok && (int)blockIdx.x >= p.B && p.B <= 16) {
+        // a CTA that owns no row warms the schedule code (a dry pass) in the gap between
+        // the router units finishing and the rows' choices being published (small
+        // batches: there the gap is idle time and the routing path dominates)
+        if (mw == 0) {
+          int r = 1;
+          if (lane == 0) r = wait_counter(&p.ctr[CTR_ROUTER], (uint32_t)sm.sh.router_target, p) ? 1 : 0;
+          r = __shfl_sync(0xffffffffu, r, 0);
+          if (lane == 0) sm.bcast = r;
+        }
+        ok = mac_sync(sm, mphase, p, lane) && sm.bcast;
+        if (ok) ok = build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, true);
+      }
+      if (ok) ok = build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, false);
       if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
     } else {
       mac_warps_cc<kTrace>(p, sm, ring, warp_id - 1, lane);
