@@ -80,6 +80,31 @@ def step_bytes(wl, n_unique_per_layer, batch=None):
     return total
 
 
+def kernel_source_hash():
+    """sha256 over the kernel's sources: counters taken on other sources do not apply."""
+    import hashlib
+
+    hsh = hashlib.sha256()
+    csrc = os.path.join(ROOT, "moe_decode_persistent_b200", "csrc")
+    for name in ("moe_decode_kernel.cu", "kernel_params.h", "ptx.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            hsh.update(f.read())
+    return hsh.hexdigest()
+
+
+def traffic_per_launch(workload):
+    """DRAM bytes per launch from profiles/traffic.json (ncu counters), or None when the
+    workload was not captured or the kernel sources changed since the capture."""
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(tpath):
+        return None
+    with open(tpath) as f:
+        t = json.load(f).get(workload)
+    if t is None or t.get("kernel_sources_sha256") != kernel_source_hash():
+        return None
+    return t.get("bytes_per_launch")
+
+
 def workload_config(wl, flush):
     return {"workload": wl.name, "batch": wl.B, "hidden": wl.H, "experts": wl.E, "top_k": wl.k,
             "expert_inter": wl.I, "shared_inter": wl.Is, "layers": wl.layers,
@@ -349,12 +374,7 @@ def run_ours(args, wl):
 
     peak, peak_kind = measured_peaks()
     achieved = sum(bytes_steps) / (local_ms * 1e-3) / 1e9  # per launch-stream, this rank
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tpath):
-        with open(tpath) as f:
-            t = json.load(f).get(wl.name)
-        traffic = None if t is None else t.get("bytes_per_launch")
+    traffic = traffic_per_launch(wl.name)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,

@@ -161,7 +161,11 @@ int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms)
  * stamps of the router tiles seen finished, of the schedule built, and of the
  * schedule's top-k, top-k rendezvous and unique-expert steps, of a
  * normalised row published by the CTA, and of the first top-k row's logits
- * loaded and selection done (slots 34-39 are reserved). */
+ * loaded and selection done; on the tensor-core kernel also the owned row's
+ * top-k chosen (34) and its cycle count (35), the unique experts placed (36),
+ * the pairs sorted (37), and clock64 at the kernel start (38): there the
+ * routing stamps (slots 26-30, 32-34, 36, 37) are clock64 values of the CTA's
+ * SM, comparable with slot 38 of the same CTA only (slot 39 is reserved). */
 int moe_decode_set_trace(moe_decode_handle* h, void* trace);
 
 /* uint64 trace slots of one layer (number of CTAs x 40). */
