@@ -76,9 +76,21 @@ constexpr int kTcEpiWarps = 4;
 constexpr int kTcThreads = 32 * (kTcEpiWarp0 + kTcEpiWarps);       // 448
 constexpr int kTcTileBytes = kTcRows * kTcAtomK * 2;               // 16 KB: 128 rows x 64 K
 constexpr int kTcActBytes = kTcMaxN * kTcAtomK * 2;                // 8 KB: <= 64 rows x 64 K
-constexpr int kTcSlotBytes = 2 * kTcTileBytes + kTcActBytes;       // 40 KB
-constexpr int kTcStages = 4;
-constexpr int kTcRingBytes = kTcStages * kTcSlotBytes;
+constexpr int kTcSlotBytes = 2 * kTcTileBytes + kTcActBytes;       // 40 KB: a slot for 64 token columns
+constexpr int kTcRingBytes = 180 * 1024;
+// The slot holds the two weight tiles and N x 128 bytes of activations (N = the step's
+// token columns, rounded up to 16): the ring fits 5 stages up to 32 columns, 4 above.
+// Measured: the fifth stage speeds the streaming-dominated steps (batch 8: 864 -> 854
+// us) and slows the routing-dominated ones (batch 1: 170 -> 172.5 us, the deeper HBM
+// queues delay the routing's loads), so batches of at most 4 rows keep 4 stages.
+constexpr int kTcStagesMax = 5;
+__host__ __device__ constexpr int tc_slot_bytes(int na) { return 2 * kTcTileBytes + ((na * kTcAtomK * 2 + 1023) / 1024) * 1024; }
+__host__ __device__ constexpr int tc_stages(int na, int batch) {
+  return batch <= 4 ? 4
+       : kTcRingBytes / tc_slot_bytes(na) < kTcStagesMax ? kTcRingBytes / tc_slot_bytes(na) : kTcStagesMax;
+}
+static_assert(tc_stages(16, 1) == 4 && tc_stages(16, 8) == 5 && tc_stages(32, 32) == 5 && tc_stages(64, 64) == 4,
+              "ring depths");
 constexpr int kTcAccBufs = 4;       // accumulator buffers in tensor memory
 constexpr int kTcAccCols = 128;     // columns per buffer: tile 0 at +0, tile 1 at +64
 constexpr int kTmemCols = kTcAccBufs * kTcAccCols;  // 512 (a power of two >= 32)
@@ -115,6 +127,7 @@ struct Shape {
   int NR, NS;
   int spp;  // stages per (expert, row group) pair of a down unit
   int NA;   // tensor-core path: token columns of n- and hs-based tiles (B rounded up to 16)
+  int nst, slot_bytes;  // ring stages and slot size
   int pre;  // units queued before the routing schedule (no unit before it needs the schedule)
   int router_target, hs_target, pair_target;  // tiles that publish logits / h_s / one pair's h
 };
@@ -139,7 +152,7 @@ struct Sched {
 
 // Per-CTA state. The stage ring (kCcRingBytes or kTcRingBytes) sits in front of it in
 // dynamic shared memory, 1024-byte aligned.
-constexpr int kMaxRingStages = kStages > kTcStages ? kStages : kTcStages;
+constexpr int kMaxRingStages = kStages > kTcStagesMax ? kStages : kTcStagesMax;
 struct Smem {
   uint64_t full[kMaxRingStages];
   uint64_t empty[kMaxRingStages];
@@ -369,6 +382,8 @@ __device__ void make_shape(const Params& p, Shape& s) {
   s.NS = s.GB * s.ST * s.SS;
   s.spp = (s.nkbI + 1) / 2;
   s.NA = 0;
+  s.nst = kStages;
+  s.slot_bytes = kSlotBytes;
   s.pre = s.NR + s.NS;
   s.router_target = s.GB * s.RT;
   s.hs_target = s.GB * s.ST;
@@ -385,6 +400,8 @@ __device__ void make_shape_tc(const Params& p, Shape& s) {
   s.k = p.k;
   s.GB = 1;
   s.NA = (p.B + kTcActRows - 1) / kTcActRows * kTcActRows;
+  s.slot_bytes = tc_slot_bytes(s.NA);
+  s.nst = tc_stages(s.NA, p.B);
   s.boxH = s.boxI = s.boxIs = kTcAtomK;
   s.nkbH = p.H / kTcAtomK;
   s.nkbI = p.I / kTcAtomK;
@@ -1917,7 +1934,7 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
     const int ka_end = d.kb0 + d.nkb;
     // one stage: header, barrier armed for weights + activations, the weight tiles
     auto issue_weights = [&](int ka) {
-      uint8_t* dst = ring + pr.slot * kTcSlotBytes;
+      uint8_t* dst = ring + pr.slot * sh.slot_bytes;
       uint64_t* fb = &sm.full[pr.slot];
       pr.mark_pending();
       if (lane == 0) {
@@ -1935,7 +1952,7 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
     // the activation operand of stage ka into ring slot s (only after its publication)
     auto issue_act = [&](int ka, int slot) {
       if (lane == 0) {
-        uint8_t* act = ring + slot * kTcSlotBytes + 2 * kTcTileBytes;
+        uint8_t* act = ring + slot * sh.slot_bytes + 2 * kTcTileBytes;
         uint64_t* fb = &sm.full[slot];
         for (int q = 0; q < x.N / kTcActRows; ++q)
           tma_load_2d_plain(act + q * kTcActRows * kTcAtomK * 2, x.ta, ka * kTcAtomK, x.arow + q * kTcActRows, fb);
@@ -1950,7 +1967,7 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
       // weights stream while the input is awaited -- a ring's worth for h, one stage
       // for the normalised rows (at the start of the step the HBM queue must stay short
       // for the loads of x that the normalisation waits on)
-      const int depth = x.dep == 0 ? 1 : kTcStages;
+      const int depth = x.dep == 0 ? 1 : pr.nst;
       const int pre_end = ka_end < d.kb0 + depth ? ka_end : d.kb0 + depth;
       const int slot0 = pr.slot;
       for (; ka < pre_end && ok; ++ka) {
@@ -1978,7 +1995,7 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
       }
       c_dep += (unsigned long long)(tclock<kTrace>() - td0);
       // every armed barrier gets its activation bytes, also after a failed wait
-      for (int i = 0; i < narmed; ++i) issue_act(d.kb0 + i, (slot0 + i) % kTcStages);
+      for (int i = 0; i < narmed; ++i) issue_act(d.kb0 + i, (slot0 + i) % pr.nst);
       __syncwarp();
       if (!dep_ok) ok = false;
     }
@@ -2197,7 +2214,7 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
     tc_fence_after();
     const long long ti0 = tclock<kTrace>();
     if (lane == 0) {
-      const uint32_t sbase = smem_u32(ring + slot * kTcSlotBytes);
+      const uint32_t sbase = smem_u32(ring + slot * sm.sh.slot_bytes);
       const uint64_t dw0 = sw128_desc(sbase);
       const uint64_t dw1 = sw128_desc(sbase + kTcTileBytes);
       const uint64_t da = sw128_desc(sbase + 2 * kTcTileBytes);
@@ -2227,7 +2244,7 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
         aphase ^= 1u;
       }
     }
-    if (++slot == kTcStages) {
+    if (++slot == sm.sh.nst) {
       slot = 0;
       phase ^= 1u;
     }
@@ -2545,7 +2562,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
   Smem& sm = *reinterpret_cast<Smem*>(ring + (kTC ? kTcRingBytes : kCcRingBytes));
-  constexpr int kNst = kTC ? kTcStages : kStages;
+  constexpr int kNst = kTC ? kTcStagesMax : kStages;  // barriers initialised (the TC ring uses sh.nst)
   const int tid = threadIdx.x;
   const int warp_id = tid / 32;
   const int lane = tid % 32;
@@ -2592,7 +2609,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
   if constexpr (kTC) tc_fence_after();
 
   if (warp_id == 0) {
-    Producer pr(p, sm, lane, kNst);
+    Producer pr(p, sm, lane, sm.sh.nst);
     if constexpr (kTC) producer_tc<kTrace>(pr, ring);
     else producer_cc<kTrace>(pr, ring);
   } else if (warp_id <= kMacWarps) {
