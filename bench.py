@@ -383,6 +383,8 @@ def run_ours(args, wl):
         "data": "synthetic: seeded counter-hash weights ~N(0,1/sqrt(fan_in)) and inputs, no trained weights",
         "config": dict(workload_config(wl, "flushed between timed steps (256 MB write)"), kernel_path=kernel_path),
         "us_per_step": round(1e3 * max_ms / K, 2),
+        "us_per_step_median": round(1e3 * float(np.median(step_ms)), 2),
+        "us_per_step_p90": round(1e3 * float(np.percentile(step_ms, 90)), 2),
         "tokens_per_s": round(world * wl.B * K / (max_ms * 1e-3), 1),
         "unique_experts_mean": float(U.mean()),
         "bytes_per_step_mean": float(np.mean(bytes_steps)),

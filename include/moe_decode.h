@@ -56,7 +56,8 @@ extern "C" {
 #define MOE_ERR_COOPERATIVE (-4)        /* cooperative launch unsupported or grid not co-resident */
 #define MOE_ERR_CUDA (-5)               /* a CUDA runtime/driver call failed */
 #define MOE_ERR_TIMEOUT (-6)            /* device status: a bounded wait ran out */
-#define MOE_ERR_NONFINITE (-7)          /* device status: a router logit was NaN or infinite */
+#define MOE_ERR_NONFINITE (-7)          /* device status: a router logit was NaN or infinite
+                                           (the tensor-core kernel abandons the step: y undefined) */
 #define MOE_ERR_NO_MEMORY (-8)          /* workspace allocation failed */
 
 /* Kernel paths of a step (moe_decode_step_path). */

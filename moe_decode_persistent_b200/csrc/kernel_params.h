@@ -92,7 +92,7 @@ struct Params {
   int H, E, I, Is, B, k;
   float eps;
   int tc;          // 1: tensor-core path (tcgen05 tiles), 0: CUDA-core path
-  int RS, SS, ES;  // tensor-core path: K splits of router / shared gate-up / expert gate-up units
+  int RS, SS;      // tensor-core path: K splits of router / shared gate-up units (experts: by row count)
   // activations
   const uint16_t* x;  // bf16 [B][H]
   uint16_t* y;        // bf16 [B][H]

@@ -406,7 +406,6 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     if (tc) {
       p.RS = moe::tc_router_splits(batch, nkH);
       p.SS = moe::tc_shared_splits(batch, nkH);
-      p.ES = moe::tc_clamp_splits(moe::kTcExpertSplits, nkH);
       p.rpart = h->rpart;
       p.spart = h->spart;
       p.epart = h->epart;

@@ -1,4 +1,4 @@
-// moe_decode_kernel.cu - the persistent sm_100a kernel of one MoE decode-layer step.
+// moe_decode_kernel.cu - the persistent sm_100a kernels of one MoE decode-layer step.
 //
 // One launch per layer, one CTA per SM (cooperative launch, all CTAs
 // co-resident). The pages this follows replace a chain of per-layer kernels by
@@ -6,43 +6,45 @@
 // 1.68倍", section "为什么解码阶段适合Megakernel"; page post.smzdm.com/p/a6zppe4g,
 // section "改了什么：每层 23 个 kernel 砍到 13 个": 23 -> 13 kernels per layer).
 //
-// Roles inside a CTA (10 warps)
-//   warp 0      producer: takes units of work from a global queue and streams their
-//               weight tiles (2-D TMA boxes of 32 rows x up to 256 K columns, two
-//               boxes per stage) plus the matching activation rows (1-D bulk copies)
-//               into a kStages-deep shared-memory ring, completed on mbarriers.
-//   warps 1..8  MAC warps: CUDA-core GEMV over each stage (each warp owns 4 weight
-//               rows of a box, each lane 8 K columns), fp32 accumulation in
-//               registers across a unit's stages, warp-shuffle reductions into a
-//               shared-memory result buffer.
-//   warp 9      epilogue warp: per finished unit, the split-K partial, the tile's
-//               ticket, the fixed-order fix-up of the tile's last split and the
-//               unit's outputs (logits, SwiGLU rows, or the combined layer output),
-//               then the release that publishes them. The MAC warps never wait on
-//               global round trips.
+// Two instances of moe_decode_layer_kernel<trace, tc> implement the step; the host
+// picks one per step (the batch-shape switch):
 //
-// Units of work (queue order)
-//   router    (row group g, tile of 32 experts, K split)        -> logits
-//   shared    (row group g, tile of 32 rows of Ws_gate/Ws_up, K split) -> h_s
-//   -- every CTA then builds the same routing schedule from the final logits:
-//      warp-level top-k per row, softmax over the selected logits, the
-//      expert -> rows map and the list of unique experts (each selected expert's
-//      weights are streamed once per step however many rows chose it).
-//   expert    ((expert, row group) pair, tile of 32 rows of W_gate/W_up, K split) -> h_e
-//   down      (tile of 32 output features; split = one shared row group, or up to
-//              two (expert, row group) pairs) -> y, combined by the tile's last split
-// The shared expert's gate/up units run while the router resolves (page
-// post.smzdm.com/p/a6zppe4g, same section: the shared expert moved beside the
-// router computation). The next layer's router and shared weights are
-// prefetched into L2 by CTAs that run out of work (same section, the last item).
+// Tensor-core kernel (tc = true, 14 warps)
+//   warp 0      producer: takes units of work from a global queue and streams, per
+//               64-column K atom, up to two 128-row weight tiles and the activation
+//               operand (all 128-byte swizzled TMA boxes) into a shared-memory ring.
+//   warps 1-8   routing: RMSNorm of the CTA's rows; for the row the CTA owns, the sum
+//               of the router's K-split partials, the top-k and the softmax, published;
+//               then the schedule every CTA builds from the published choices.
+//   warp 9      MMA issuer: owns 512 tensor-memory columns; one lane issues
+//               tcgen05.mma (M = 128 weight rows, N = the token rows, K = 16, bf16,
+//               fp32 accumulate) per stage and commits the slot back to the producer.
+//   warps 10-13 epilogue: read the accumulators (tcgen05.ld, one warp per lane
+//               quadrant) and finish the unit: split-K partials and fix-ups, SwiGLU,
+//               down partials and the per-row combine with the residual.
 //
-// Memory ordering: data produced inside the kernel (normalised rows, logits,
-// h, partials) is read only after an acquire on the counter that publishes it,
-// and never through the non-coherent path; only static weights are loaded
-// ahead of a wait (the pages' review finding: page "vLLM 合併 Kimi K3 專用解碼…",
-// section "AI 寫的 GPU 核心 vLLM 怎麼驗證正確"). Every wait, between CTAs and
-// between warps of a CTA, is bounded; when one runs out the kernel records
-// MOE_ERR_TIMEOUT, all CTAs unwind, drain their bulk copies and exit.
+// CUDA-core kernel (tc = false, 10 warps)
+//   warp 0      producer: 32-row weight boxes and the activation rows (1-D bulk copies).
+//   warps 1-8   MAC warps: fp32-FMA GEMV over each stage (each warp 4 weight rows of a
+//               box, each lane 8 K columns), warp-shuffle reductions; RMSNorm and the
+//               routing schedule (every CTA computes every row's top-k).
+//   warp 9      epilogue: split-K partials, tickets, fixed-order fix-ups, outputs.
+//
+// Units of work (queue order): router, shared gate/up (and, on the tensor-core path,
+// the shared expert's down tiles) -- all streamed while the routing resolves (page
+// post.smzdm.com/p/a6zppe4g, same section: the shared expert moved beside the router
+// computation) -- then expert gate/up and down units over the unique selected experts
+// only (each selected expert's weights stream once however many rows chose it). The
+// next layer's router and shared weights are prefetched into L2 by CTAs that run out of
+// work (same section, the last item).
+//
+// Memory ordering: data produced inside the kernel (normalised rows, logits, h,
+// partials, published choices) is read only after an acquire on the counter that
+// publishes it, and never through the non-coherent path; only static weights are
+// loaded ahead of a wait (the pages' review finding: page "vLLM 合併 Kimi K3 專用解碼…",
+// section "AI 寫的 GPU 核心 vLLM 怎麼驗證正確"). Every wait, between CTAs and between
+// warps of a CTA, is bounded; when one runs out the kernel records MOE_ERR_TIMEOUT, all
+// CTAs unwind, drain their bulk copies and MMAs, and exit.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -412,7 +414,7 @@ __device__ void make_shape_tc(const Params& p, Shape& s) {
   s.DT = (p.H + 2 * kTcRows - 1) / (2 * kTcRows);
   s.RS = p.RS;
   s.SS = p.SS;
-  s.ES = p.ES;
+  s.ES = 0;  // per expert: sc.pair_es
   s.NR = s.RT * s.RS;
   s.NS = s.ST * s.SS;
   s.spp = 0;
@@ -1195,7 +1197,10 @@ __device__ bool route_rows_tc(const Params& p, Smem& sm, int mw, int lane, uint3
         trace_put<kTrace>(p, TR_TOPK_CYC, (unsigned long long)(tclock<kTrace>() - tk0));
         trace_clk<kTrace>(p, TR_TOPK_CHOSEN);
       }
-      if (sm.bcast2 && lane == 0) record_error(p, MOE_ERR_NONFINITE);
+      // a non-finite logit ends the step: with fewer than k finite logits the row's
+      // choices would not be k distinct experts, which the schedule's per-row
+      // bookkeeping assumes (the abort path resets every ticket for the next step)
+      if (sm.bcast2 && lane == 0) record_abort(p, MOE_ERR_NONFINITE);
       int e = (int)(~(uint32_t)mine);
       if (e < 0 || e >= E) e = 0;  // only with a non-finite row (reported)
       const float val = lane < p.k ? key_float((uint32_t)(mine >> 32)) : 0.0f;
@@ -1224,6 +1229,70 @@ __device__ bool route_rows_tc(const Params& p, Smem& sm, int mw, int lane, uint3
 // are the unique experts ordered by row count, hottest first (stable in expert order),
 // so the largest units are queued first and the down units that complete rows last
 // are those of experts with few rows. An expert's slot rows keep expert order.
+// The schedule of a one-row step: the row's k choices are k distinct experts with one
+// row each, so the unique experts are the choices in ascending id (each one's slot is
+// its rank among them) and the hottest-first order is that same order. One warp
+// builds it (the general builder's result, without its masks, scans and rendezvous).
+template <bool kTrace>
+__device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
+  const Shape& sh = sm.sh;
+  Sched& sc = sm.sc;
+  const int k = p.k;
+  if (mw == 0) {
+    int ok = 1;
+    if (lane == 0) ok = wait_counter(&p.ctr[CTR_TOPK], 1u, p) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (lane == 0) sm.bcast = ok;
+    if (ok) {
+      if (lane == 0) trace_clk<kTrace>(p, TR_TOPK_SYNCED);
+      const int e = lane < k ? __ldcg(p.tk_idx + lane) : 0x7fffffff;
+      const float w = lane < k ? __ldcg(p.tk_w + lane) : 0.0f;
+      int r = 0;
+#pragma unroll 4
+      for (int sl = 0; sl < 32; ++sl) r += __shfl_sync(0xffffffffu, e, sl) < e ? 1 : 0;
+      const int es = tc_expert_splits(1, sh.nkbH);
+      if (lane < k) {
+        sm.u.t.topk_idx[lane] = e;
+        sm.u.t.topk_w[lane] = w;
+        sc.slot_expert[r] = (int16_t)e;
+        sc.slot_cnt[r] = 1;
+        sc.slot_base[r] = (int16_t)r;
+        sc.eslot[e] = (int16_t)r;
+        sc.pair_slot[r] = (int16_t)r;
+        sc.pair_group[r] = 0;
+        sc.pair_es[r] = (uint8_t)es;
+        sc.pair_ubase[r] = r * sh.IT * es;
+        sc.row_of[r] = 0;
+        sc.w_of[r] = w;
+        sc.slot_of[lane] = (int16_t)r;
+      }
+      if (lane == 0) {
+        sc.U = k;
+        sc.S = k;
+        sc.P = k;
+        sc.slot_base[k] = (int16_t)k;
+        sc.pair_ubase[k] = k * sh.IT * es;
+        sc.NE = k * sh.IT * es;
+        sc.down_splits = 1 + k;
+        sc.ND = sh.DT * k;
+        sc.total = sh.pre + sc.NE + sc.ND;
+        const unsigned tiles = (unsigned)(sh.RT + sh.ST + k * sh.IT + sh.DT);
+        sm.bcast2 = ((unsigned)sc.total <= p.max_units && tiles <= p.max_tiles) ? 1 : 0;
+        if (!sm.bcast2) record_abort(p, MOE_ERR_UNSUPPORTED_SHAPE);
+      }
+      __syncwarp();
+      if (blockIdx.x == 0 && lane < k) {
+        if (p.dbg_idx) p.dbg_idx[lane] = e;
+        if (p.dbg_w) p.dbg_w[lane] = w;
+      }
+      if (blockIdx.x == 0 && lane == 0 && p.dbg_nuniq) *p.dbg_nuniq = k;
+    }
+  }
+  const bool ok = mac_sync(sm, mphase, p, lane) && sm.bcast && sm.bcast2;
+  if (mw == 0 && lane == 0) trace_clk<kTrace>(p, TR_SCHED_BUILT);
+  return ok;
+}
+
 // dry: a pass over synthetic choices (row b takes experts (13 j + b) mod E, distinct
 // for j < 32 as 13 is odd and E a multiple of 128 below 13 * 128) with no global
 // effects, made by CTAs that own no row while they wait for the published choices, so
@@ -2620,7 +2689,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       uint32_t mphase = 0;
       bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
       if (ok) ok = route_rows_tc<kTrace>(p, sm, mw, lane, mphase);
-      if (ok && (int)blockIdx.x >= p.B && p.B <= 16) {
+      if (ok && (int)blockIdx.x >= p.B && p.B > 1 && p.B <= 16) {
         // a CTA that owns no row warms the schedule code (a dry pass) in the gap between
         // the router units finishing and the rows' choices being published (small
         // batches: there the gap is idle time and the routing path dominates)
@@ -2633,7 +2702,8 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
         ok = mac_sync(sm, mphase, p, lane) && sm.bcast;
         if (ok) ok = build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, true);
       }
-      if (ok) ok = build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, false);
+      if (ok) ok = p.B == 1 ? build_schedule_b1<kTrace>(p, sm, mw, lane, mphase)
+                            : build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, false);
       if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
     } else {
       mac_warps_cc<kTrace>(p, sm, ring, warp_id - 1, lane);

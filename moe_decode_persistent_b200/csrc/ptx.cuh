@@ -42,21 +42,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Same test, but a thread whose phase is not complete is suspended (for at most
-// `suspend_ns`) until the phase completes instead of returning at once, so waiting
-// warps do not compete for issue slots with working warps.
-__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
-      : "memory");
-  return ok != 0;
-}
-
 // ---- bulk copies ------------------------------------------------------------------
 // 2-D tiled TMA load of box (x = innermost coordinate, y = row) into shared memory,
 // completion counted on `bar` (bytes). `policy` is an L2 cache-policy descriptor.

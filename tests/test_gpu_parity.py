@@ -169,11 +169,27 @@ def test_tc_timeout_is_reported_and_handle_recovers():
     h.close()
 
 
+@pytest.mark.parametrize("path", ["tensor_core", "cuda_core"])
+def test_nonfinite_input_is_reported_and_handle_recovers(path):
+    import moe_decode_persistent_b200 as mdp
+
+    wl = TC_BY_NAME["tc_ragged_b5_e384"]
+    layers = _layers(wl)
+    h = make_handle(wl, layers, tc_min_batch=1 if path == "tensor_core" else 0)
+    x = wl.x_host().copy()
+    x[2, 17] = 0x7FC0  # a bf16 NaN: row 2's normalised row and logits become NaN
+    bad = run_gpu(h, wl, x)
+    assert bad["status"] == mdp.MOE_ERR_NONFINITE
+    good = run_and_check(wl, handle=h, layers=layers)[0]
+    assert good["status"] == 0
+    h.close()
+
+
 def test_tc_smaller_batch_and_k_than_configured():
     wl = TC_BY_NAME["tc_b64_k16"]
     layers = _layers(wl)
     h = make_handle(wl, layers, tc_min_batch=1)
-    for B, k in ((3, 4), (16, 8), (33, 16), (63, 1)):
+    for B, k in ((1, 16), (3, 4), (16, 8), (33, 16), (63, 1)):
         sub = dataclasses.replace(wl, B=B, k=k)
         run_and_check(sub, handle=h, layers=layers)
     h.close()
