@@ -1293,18 +1293,19 @@ __device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, u
   return ok;
 }
 
-// dry: a pass over synthetic choices (row b takes experts (13 j + b) mod E, distinct
-// for j < 32 as 13 is odd and E a multiple of 128 below 13 * 128) with no global
-// effects, made by CTAs that own no row while they wait for the published choices, so
-// that the real pass runs with its instructions cached (one out-of-line copy of the
-// code serves both passes).
+// dry: a pass over synthetic choices of at most 4 rows (row b takes experts
+// (13 j + b) mod E, distinct for j < 32 as 13 is odd and E a multiple of 128 below
+// 13 * 128) with no global effects, made by CTAs that own no row while they wait for
+// the published choices, so that the real pass runs with its instructions cached
+// (one out-of-line copy of the code serves both passes).
 template <bool kTrace>
 __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase,
                                                bool dry) {
   const Shape& sh = sm.sh;
   Sched& sc = sm.sc;
   const int mtid = mw * 32 + lane;
-  const int B = p.B, k = p.k;
+  // the dry pass runs the same instructions over at most 4 synthetic rows
+  const int B = dry && p.B > 4 ? 4 : p.B, k = p.k;
   for (int e = mtid; e < p.E; e += kMacThreads) sm.u.t.mask[e] = 0ull;
   if (mw == 0) {
     int ok = 1;
@@ -2689,10 +2690,9 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       uint32_t mphase = 0;
       bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
       if (ok) ok = route_rows_tc<kTrace>(p, sm, mw, lane, mphase);
-      if (ok && (int)blockIdx.x >= p.B && p.B > 1 && p.B <= 16) {
-        // a CTA that owns no row warms the schedule code (a dry pass) in the gap between
-        // the router units finishing and the rows' choices being published (small
-        // batches: there the gap is idle time and the routing path dominates)
+      if (ok && (int)blockIdx.x >= p.B && p.B > 1) {
+        // a CTA that owns no row warms the schedule code (a short dry pass) in the gap
+        // between the router units finishing and the rows' choices being published
         if (mw == 0) {
           int r = 1;
           if (lane == 0) r = wait_counter(&p.ctr[CTR_ROUTER], (uint32_t)sm.sh.router_target, p) ? 1 : 0;
