@@ -164,7 +164,8 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe::kernel_fn(), moe::threads_per_cta(),
                                                     smem);
   if (e != cudaSuccess || per_sm < 1) return MOE_ERR_COOPERATIVE;
-  // the tensor-core kernel: only for shapes whose every dimension is a multiple of 128
+  // the tensor-core kernel: only for shapes whose every dimension is a multiple of 128,
+  // and only if it can be made co-resident; otherwise every step takes the CUDA-core kernel
   int tc_ok = tc_shape_ok(c) ? 1 : 0;
   if (tc_ok) {
     const size_t tsm = moe::tc_smem_bytes();
@@ -175,7 +176,10 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&tc_per_sm, moe::tc_kernel_fn(), moe::tc_threads_per_cta(),
                                                         tsm);
-    if (e != cudaSuccess || tc_per_sm < 1) return MOE_ERR_COOPERATIVE;
+    if (e != cudaSuccess || tc_per_sm < 1) {
+      (void)cudaGetLastError();  // clear the runtime's last-error state left by the failed query
+      tc_ok = 0;
+    }
   }
 
   void* fn = nullptr;

@@ -1465,32 +1465,24 @@ __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw
 
 template <bool kTrace>
 __device__ bool normalise_rows(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
-  // each MAC thread holds up to kNormVec 16-byte vectors of x and gamma in registers:
-  // one round of independent loads, then both passes from registers
-  constexpr int kNormVec = 8;  // hidden <= 8 * 8 * 256 = 16384
+  // This runs once per launch, first thing, with its instructions usually evicted from
+  // L2 (each new instruction line then comes from DRAM): the loops are kept short
+  // rather than unrolled over register arrays. Pass 1 loads x and gamma (4 vectors in
+  // flight per thread) and sums the squares; pass 2 re-reads both from L1.
   const int mtid = mw * 32 + lane;
   const int nv = p.H / 8;
   const uint4* g4 = reinterpret_cast<const uint4*>(p.gamma);
   for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
     const uint4* x4 = reinterpret_cast<const uint4*>(p.x + (size_t)b * p.H);
-    uint4 xv[kNormVec], gv[kNormVec];
-#pragma unroll
-    for (int i = 0; i < kNormVec; ++i) {
-      const int v = mtid + i * kMacThreads;
-      if (v < nv) {
-        xv[i] = x4[v];
-        gv[i] = g4[v];
-      }
-    }
     float ss = 0.0f;
+#pragma unroll 4
+    for (int v = mtid; v < nv; v += kMacThreads) {
+      const uint4 xv = ld_nc_v4(x4 + v);
+      (void)ld_nc_v4(g4 + v);  // brings gamma into L1 for pass 2 (a volatile load is kept)
+      float f[8];
+      unpack8(xv, f);
 #pragma unroll
-    for (int i = 0; i < kNormVec; ++i) {
-      if (mtid + i * kMacThreads < nv) {
-        float f[8];
-        unpack8(xv[i], f);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) ss = fmaf(f[t], f[t], ss);
-      }
+      for (int t = 0; t < 8; ++t) ss = fmaf(f[t], f[t], ss);
     }
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
@@ -1501,19 +1493,16 @@ __device__ bool normalise_rows(const Params& p, Smem& sm, int mw, int lane, uint
     for (int w = 0; w < kMacWarps; ++w) tot += sm.red_ss[w];
     const float r = 1.0f / sqrtf(tot / (float)p.H + p.eps);
     uint4* n4 = reinterpret_cast<uint4*>(p.n + (size_t)b * p.H);
+#pragma unroll 1
+    for (int v = mtid; v < nv; v += kMacThreads) {
+      float f[8], g[8];
+      unpack8(ld_nc_v4(x4 + v), f);
+      unpack8(ld_nc_v4(g4 + v), g);
+      uint32_t o[4];
 #pragma unroll
-    for (int i = 0; i < kNormVec; ++i) {
-      const int v = mtid + i * kMacThreads;
-      if (v < nv) {
-        float f[8], g[8];
-        unpack8(xv[i], f);
-        unpack8(gv[i], g);
-        uint32_t o[4];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-          o[t] = (uint32_t)f2bf(f[2 * t] * r * g[2 * t]) | ((uint32_t)f2bf(f[2 * t + 1] * r * g[2 * t + 1]) << 16);
-        n4[v] = make_uint4(o[0], o[1], o[2], o[3]);
-      }
+      for (int t = 0; t < 4; ++t)
+        o[t] = (uint32_t)f2bf(f[2 * t] * r * g[2 * t]) | ((uint32_t)f2bf(f[2 * t + 1] * r * g[2 * t + 1]) << 16);
+      n4[v] = make_uint4(o[0], o[1], o[2], o[3]);
     }
     fence_proxy_async_global();
     if (!mac_sync(sm, mphase, p, lane)) return false;
