@@ -56,6 +56,9 @@ def parse_args(argv=None):
     ap.add_argument("--profile-small-tc", action="store_true",
                     help="batch 1, 128 experts of intermediate 512 (~2.9 GB of weights): the small case "
                          "for full ncu captures of the tensor-core kernel")
+    ap.add_argument("--profile-small-b64", action="store_true",
+                    help="batch 64 with the Zipf router, 128 experts of intermediate 512 (~2.9 GB of "
+                         "weights): the small hot-expert case for full ncu captures of the tensor-core kernel")
     return ap.parse_args(argv)
 
 
@@ -430,6 +433,9 @@ def main(argv=None):
         wl = synth.Workload("b1_h7168_e64_k16_profile", B=1, H=7168, E=64, k=16, I=1024, Is=2048, seed=1)
     if args.profile_small_tc:
         wl = synth.Workload("b1_h7168_e128_i512_k16_profile", B=1, H=7168, E=128, k=16, I=512, Is=1024, seed=1)
+    if args.profile_small_b64:
+        wl = synth.Workload("b64_h7168_e128_i512_k16_zipf_profile", B=64, H=7168, E=128, k=16, I=512, Is=1024,
+                            seed=3, router="zipf")
     if args.impl == "reference":
         run_reference(args, wl)
     else:
