@@ -31,7 +31,7 @@ enum TensorMapSlot {
   TM_COUNT = 17
 };
 
-// Global counters of one step (reset by the last CTA of every launch).
+// Global counters of one step (reset by the last CTA of every launch, except the epoch).
 enum Counter {
   CTR_QUEUE = 0,   // next unit of work
   CTR_EXIT = 1,    // CTAs finished
@@ -40,6 +40,7 @@ enum Counter {
   CTR_HS = 4,      // shared gate/up tiles finished
   CTR_ABORT = 5,   // non-zero once any CTA gave up a wait
   CTR_TOPK = 6,    // tensor-core path: rows whose top-k choices are published
+  CTR_EPOCH = 7,   // launches completed on this workspace (never reset): tags the choices
   CTR_COUNT = 8
 };
 
@@ -114,8 +115,8 @@ struct Params {
   float* spart;          // [SS][B][Is/128][256]
   float* epart;          // [ES][B*k][I/128][256]
   float* dpart;          // [B*k + B][H]: down outputs of expert slot rows, then shared rows
-  int* tk_idx;           // [B][k] published top-k experts of each row
-  float* tk_w;           // [B][k] their softmax weights
+  uint64_t* tk_pub;      // [B][k][2] published top-k choices of each row: the words
+                         // (tag << 32 | expert) and (tag << 32 | softmax weight bits)
   uint32_t* row_tix;     // [H/256 tile pairs][max_batch]: down contributions arrived per row
   unsigned row_tix_count;
   uint32_t* ctr;         // [CTR_COUNT]

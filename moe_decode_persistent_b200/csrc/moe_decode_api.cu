@@ -44,8 +44,7 @@ struct moe_decode_handle {
   float* spart;
   float* epart;
   float* dpart;
-  int* tk_idx;
-  float* tk_w;
+  uint64_t* tk_pub;
   uint32_t* row_tix;
   unsigned row_tix_count;
   uint32_t* ctr;
@@ -291,8 +290,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   const size_t o_spart = carve(spart_floats * 4);
   const size_t o_epart = carve(epart_floats * 4);
   const size_t o_dpart = carve(dpart_floats * 4);
-  const size_t o_tki = carve((size_t)maxSlots * 4);
-  const size_t o_tkw = carve((size_t)maxSlots * 4);
+  const size_t o_tkp = carve((size_t)maxSlots * 16);
   const size_t o_rtix = carve(row_tix_n * 4 + 4);
   const size_t o_ctr = carve(moe::CTR_COUNT * 4);
   const size_t o_tix = carve((size_t)h->max_tiles * 4);
@@ -319,8 +317,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   h->spart = (float*)(b + o_spart);
   h->epart = (float*)(b + o_epart);
   h->dpart = (float*)(b + o_dpart);
-  h->tk_idx = (int*)(b + o_tki);
-  h->tk_w = (float*)(b + o_tkw);
+  h->tk_pub = (uint64_t*)(b + o_tkp);
   h->row_tix = (uint32_t*)(b + o_rtix);
   h->row_tix_count = (unsigned)row_tix_n;
   h->ctr = (uint32_t*)(b + o_ctr);
@@ -414,8 +411,7 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
       p.spart = h->spart;
       p.epart = h->epart;
       p.dpart = h->dpart;
-      p.tk_idx = h->tk_idx;
-      p.tk_w = h->tk_w;
+      p.tk_pub = h->tk_pub;
       p.row_tix = h->row_tix;
       p.row_tix_count = h->row_tix_count;
     }

@@ -40,7 +40,9 @@
 //
 // Memory ordering: data produced inside the kernel (normalised rows, logits, h,
 // partials, published choices) is read only after an acquire on the counter that
-// publishes it, and never through the non-coherent path; only static weights are
+// publishes it, and never through the non-coherent path -- except a one-row step's
+// top-k choices, which are polled directly: each is an 8-byte word that carries the
+// launch's tag beside its value, valid once the tag matches; only static weights are
 // loaded ahead of a wait (the pages' review finding: page "vLLM 合併 Kimi K3 專用解碼…",
 // section "AI 寫的 GPU 核心 vLLM 怎麼驗證正確"). Every wait, between CTAs and between
 // warps of a CTA, is bounded; when one runs out the kernel records MOE_ERR_TIMEOUT, all
@@ -319,6 +321,49 @@ __device__ bool wait_counter(const uint32_t* c, uint32_t target, const Params& p
       return false;
     }
   }
+}
+
+// Tag of this launch's published top-k choices: odd, so a zeroed word never carries it,
+// and different in consecutive launches (the epoch counts completed launches).
+__device__ __forceinline__ uint32_t choice_tag(const Params& p) {
+  return (ld_relaxed_gpu(&p.ctr[CTR_EPOCH]) << 1) | 1u;
+}
+
+// Bounded wait of one warp for the k choices of row 0 (lane j < k polls choice j's two
+// tagged words) and their values: a choice is valid once both of its words carry this
+// launch's tag, so the load that observes the publication also brings the data (no flag
+// followed by a second round trip for what it guards). The result is warp-uniform.
+__device__ bool warp_poll_choices(const Params& p, uint32_t tag, int k, int lane, int& e, float& w) {
+  const uint64_t* pub = p.tk_pub + 2 * lane;
+  uint64_t a = 0ull, c = 0ull;
+  bool have = lane >= k;
+  uint64_t t0 = 0;
+  if (lane == 0) t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (!have) {
+      ld_relaxed_gpu_v2(pub, a, c);
+      have = (uint32_t)(a >> 32) == tag && (uint32_t)(c >> 32) == tag;
+    }
+    if (__all_sync(0xffffffffu, have)) break;
+    __nanosleep(32);
+    if ((it & 15u) == 15u) {  // the abort flag is a global load: not every poll
+      int stop = 0;
+      if (lane == 0) {
+        if (abort_seen(p)) {
+          stop = 1;
+        } else if (globaltimer_ns() - t0 > p.wait_ns) {
+          record_abort(p, MOE_ERR_TIMEOUT);
+          stop = 1;
+        }
+      }
+      if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+    }
+  }
+  if (lane < k) {
+    e = (int)(uint32_t)a;
+    w = __uint_as_float((uint32_t)c);
+  }
+  return true;
 }
 
 // Rendezvous of the 8 MAC warps (an mbarrier with bounded waits, polled without sleeping).
@@ -1131,9 +1176,10 @@ __device__ uint64_t warp_topk_keys(uint64_t* keys, int E, int k, int lane, uint6
 
 // The rows this CTA owns (row b is owned by CTA b): once every router unit has
 // published its partial sums, the row's logits are their sum in split order plus the
-// bias; one warp takes the top-k and the softmax over it and publishes the choices.
+// bias; one warp takes the top-k and the softmax over it and publishes the choices
+// (tagged words, then a release of the row count for readers of many rows).
 template <bool kTrace>
-__device__ bool route_rows_tc(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
+__device__ bool route_rows_tc(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase, uint32_t tag) {
   const Shape& sh = sm.sh;
   const int mtid = mw * 32 + lane;
   const int E = p.E;
@@ -1209,10 +1255,9 @@ __device__ bool route_rows_tc(const Params& p, Smem& sm, int mw, int lane, uint3
       float z = ex;
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-      if (lane < p.k) {
-        p.tk_idx[b * p.k + lane] = e;
-        p.tk_w[b * p.k + lane] = ex / z;
-      }
+      if (lane < p.k)
+        st_relaxed_gpu_v2(p.tk_pub + 2 * (b * p.k + lane), ((uint64_t)tag << 32) | (uint32_t)e,
+                          ((uint64_t)tag << 32) | __float_as_uint(ex / z));
       __threadfence();
       __syncwarp();
       if (lane == 0) {
@@ -1234,19 +1279,17 @@ __device__ bool route_rows_tc(const Params& p, Smem& sm, int mw, int lane, uint3
 // its rank among them) and the hottest-first order is that same order. One warp
 // builds it (the general builder's result, without its masks, scans and rendezvous).
 template <bool kTrace>
-__device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase) {
+__device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase, uint32_t tag) {
   const Shape& sh = sm.sh;
   Sched& sc = sm.sc;
   const int k = p.k;
   if (mw == 0) {
-    int ok = 1;
-    if (lane == 0) ok = wait_counter(&p.ctr[CTR_TOPK], 1u, p) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (lane == 0) sm.bcast = ok;
+    int e = 0x7fffffff;
+    float w = 0.0f;
+    const bool ok = warp_poll_choices(p, tag, k, lane, e, w);
+    if (lane == 0) sm.bcast = ok ? 1 : 0;
     if (ok) {
       if (lane == 0) trace_clk<kTrace>(p, TR_TOPK_SYNCED);
-      const int e = lane < k ? __ldcg(p.tk_idx + lane) : 0x7fffffff;
-      const float w = lane < k ? __ldcg(p.tk_w + lane) : 0.0f;
       int r = 0;
 #pragma unroll 4
       for (int sl = 0; sl < 32; ++sl) r += __shfl_sync(0xffffffffu, e, sl) < e ? 1 : 0;
@@ -1317,8 +1360,10 @@ __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw
   if (!sm.bcast) return false;
   if (mtid == 0 && !dry) trace_clk<kTrace>(p, TR_TOPK_SYNCED);
   for (int t = mtid; t < B * k; t += kMacThreads) {
-    const int e = dry ? (13 * (t % k) + t / k) % p.E : __ldcg(p.tk_idx + t);
-    const float w = dry ? 1.0f : __ldcg(p.tk_w + t);
+    ulonglong2 ch = make_ulonglong2(0ull, 0ull);
+    if (!dry) ch = __ldcg(reinterpret_cast<const ulonglong2*>(p.tk_pub) + t);
+    const int e = dry ? (13 * (t % k) + t / k) % p.E : (int)(uint32_t)ch.x;
+    const float w = dry ? 1.0f : __uint_as_float((uint32_t)ch.y);
     sm.u.t.topk_idx[t] = e;
     sm.u.t.topk_w[t] = w;
     atomicOr(&sm.u.t.mask[e], 1ull << (t / k));
@@ -2677,8 +2722,9 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       // warps keep the router and shared-expert tiles moving meanwhile)
       const int mw = warp_id - 1;
       uint32_t mphase = 0;
+      const uint32_t tag = choice_tag(p);
       bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
-      if (ok) ok = route_rows_tc<kTrace>(p, sm, mw, lane, mphase);
+      if (ok) ok = route_rows_tc<kTrace>(p, sm, mw, lane, mphase, tag);
       if (ok && (int)blockIdx.x >= p.B && p.B > 1) {
         // a CTA that owns no row warms the schedule code (a short dry pass) in the gap
         // between the router units finishing and the rows' choices being published
@@ -2691,7 +2737,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
         ok = mac_sync(sm, mphase, p, lane) && sm.bcast;
         if (ok) ok = build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, true);
       }
-      if (ok) ok = p.B == 1 ? build_schedule_b1<kTrace>(p, sm, mw, lane, mphase)
+      if (ok) ok = p.B == 1 ? build_schedule_b1<kTrace>(p, sm, mw, lane, mphase, tag)
                             : build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, false);
       if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
     } else {
@@ -2727,7 +2773,9 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       } else {
         for (int t = 0; t < sm.sc.P; ++t) p.pair_done[t] = 0u;
       }
-      for (int c = 0; c < CTR_COUNT; ++c) p.ctr[c] = 0u;
+      for (int c = 0; c < CTR_COUNT; ++c)
+        if (c != CTR_EPOCH) p.ctr[c] = 0u;
+      p.ctr[CTR_EPOCH] += 1u;  // the next launch's choices carry a new tag
       __threadfence();
     }
   }
