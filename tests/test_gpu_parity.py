@@ -169,6 +169,44 @@ def test_tc_timeout_is_reported_and_handle_recovers():
     h.close()
 
 
+def test_tc_one_row_steps_never_take_an_earlier_steps_choices():
+    """One-row steps read the row's choices from words tagged with the launch's epoch.
+    A run of one-row steps on distinct inputs, interleaved with a multi-row step and an
+    aborted step, must route every step from its own logits (a stale tag would hand a
+    step the previous step's experts)."""
+    import moe_decode_persistent_b200 as mdp
+
+    wl = TC_BY_NAME["tc_ragged_b5_e384"]
+    layers = _layers(wl)
+    h = make_handle(wl, layers, tc_min_batch=1)
+    pool = wl.x_pool_host(7)
+    plan = [(0, 1), (1, 1), (2, 4), (3, 1), ("abort", 1), (4, 1), (5, 1), (6, 1)]
+    prev = None
+    changed = 0
+    for v, B in plan:
+        if v == "abort":
+            h.set_debug(mdp.DEBUG_WITHHOLD_NREADY, wait_ms=300)
+            bad = run_gpu(h, wl, pool[0][:B])
+            h.set_debug(0)
+            assert bad["status"] == mdp.MOE_ERR_TIMEOUT
+            continue
+        x = pool[v][:B].copy()
+        assert h.step_path(B) == mdp.PATH_TENSOR_CORE
+        out = run_gpu(h, wl, x)
+        assert out["status"] == 0, f"input {v}: device status {out['status']}"
+        rows = list(range(B))
+        orc = oracle_rows(wl, x, rows)
+        ties = check_layer(out["layers"][0], orc[0], rows, wl.k, tag=f"input {v}")
+        check_y(out["y"], orc, tag=f"input {v}", skip={rows.index(b) for b in ties})
+        if B == 1:
+            chosen = set(out["layers"][0]["idx"][0].tolist())
+            changed += prev is not None and chosen != prev
+            prev = chosen
+    # consecutive one-row steps chose different experts, so a stale read would have shown
+    assert changed >= 3
+    h.close()
+
+
 @pytest.mark.parametrize("path", ["tensor_core", "cuda_core"])
 def test_nonfinite_input_is_reported_and_handle_recovers(path):
     import moe_decode_persistent_b200 as mdp
