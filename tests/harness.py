@@ -85,7 +85,7 @@ def oracle_rows(wl, x_bits, rows, n_layers=1, k=None):
 def routing_oracle(wl, x_bits, rows, layers, gpu_inputs, k=None):
     """Per-layer oracle for the routing checks: layer 0 from x, layer l >= 1 from the
     GPU's own output of layer l - 1 (gpu_inputs[l - 1], all rows), so that each
-    layer's router is judged on the input it actually received."""
+    layer's router is checked on the input it actually received."""
     import dataclasses
 
     w = dataclasses.replace(wl, k=k) if k else wl
