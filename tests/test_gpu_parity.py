@@ -207,6 +207,36 @@ def test_tc_one_row_steps_never_take_an_earlier_steps_choices():
     h.close()
 
 
+def test_rejected_steps_launch_nothing_and_leave_the_handle_usable():
+    """Calls outside the step's contract -- an empty batch, more rows than configured,
+    top_k of 0 or above the configured maximum, y aliasing x, an output buffer off
+    16-byte alignment -- return MOE_ERR_INVALID_ARG before anything is launched: the
+    buffers keep their contents, the device status stays clear and the next step is
+    correct."""
+    import moe_decode_persistent_b200 as mdp
+
+    wl = TC_BY_NAME["tc_ragged_b5_e384"]
+    layers = _layers(wl)
+    h = make_handle(wl, layers, tc_min_batch=1)
+    x = torch.from_numpy(wl.x_host().view(np.int16)).view(torch.bfloat16).cuda()
+    x_before = x.clone()
+    y = torch.full_like(x, 7.0)
+    y_off = torch.full((x.numel() + 8,), 7.0, dtype=torch.bfloat16, device="cuda")[1:1 + x.numel()].view(x.shape)
+    assert y_off.data_ptr() % 16 != 0
+    cases = [(x, y, 0, wl.k), (x, y, wl.B + 1, wl.k), (x, y, wl.B, 0), (x, y, wl.B, wl.k + 1),
+             (x, x, wl.B, wl.k), (x, y_off, wl.B, wl.k)]
+    for xi, yi, B, k in cases:
+        with pytest.raises(mdp.MoeDecodeError) as err:
+            h.step(xi, yi, B, k)
+        assert err.value.code == mdp.MOE_ERR_INVALID_ARG, (B, k)
+    torch.cuda.synchronize()
+    assert h.status() == 0
+    assert torch.equal(x, x_before)
+    assert bool((y == 7.0).all()) and bool((y_off == 7.0).all())
+    run_and_check(wl, handle=h, layers=layers)
+    h.close()
+
+
 @pytest.mark.parametrize("path", ["tensor_core", "cuda_core"])
 def test_nonfinite_input_is_reported_and_handle_recovers(path):
     import moe_decode_persistent_b200 as mdp
