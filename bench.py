@@ -254,7 +254,7 @@ def run_reference(args, wl):
     value = tot_b / tot_t / 1e9
     cores = len(os.sched_getaffinity(0))
     sample = (f"per step: RMSNorm + router of one row of {wl.name}, then SwiGLU experts (shared, "
-              f"then the row's 16 selected, cycling) for ~{budget:.3f} s; weights pre-generated "
+              f"then the row's {wl.k} selected, cycling) for ~{budget:.3f} s; weights pre-generated "
               f"on the host")
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,

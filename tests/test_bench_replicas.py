@@ -60,3 +60,27 @@ def test_reference_arm_does_no_work_on_other_ranks(monkeypatch, capsys):
     args = argparse.Namespace(steps=1, warmup=0, gpus=2, cpu_seconds=1.0)
     assert bench.run_reference(args, synth.WORKLOADS[1]) is None
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_prints_one_contract_line_on_rank_0(monkeypatch, capsys):
+    """The reference arm times the CPU oracle on a bounded sample and prints the same
+    metric, unit and config as the GPU arm, with its own cpu_baseline and a zero-copy e2e."""
+    import argparse
+    import json
+
+    import bench
+    import synth
+
+    monkeypatch.setenv("RANK", "0")
+    wl = synth.WORKLOADS[0]
+    bench.run_reference(argparse.Namespace(steps=2, warmup=1, gpus=1), wl)
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s"
+    assert d["value"] > 0 and d["steps"] == 2 and d["warmup"] == 1 and d["n_gpus"] == 1
+    assert d["higher_is_better"] is True and d["vs_baseline"] is None and d["dtype"] == "f64"
+    assert d["config"]["workload"] == wl.name
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
