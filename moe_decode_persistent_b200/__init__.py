@@ -143,6 +143,29 @@ def _ptr(t) -> int | None:
     return int(t.data_ptr())
 
 
+_ROW_DTYPES = ("torch.bfloat16", "torch.int16", "torch.uint16")  # bf16 values or their bit patterns
+
+
+def _check_rows(t, name: str, batch: int, hidden: int, device_type: str, what: str) -> None:
+    """A torch tensor given as a row buffer must hold bf16 values (or their bit patterns
+    as int16/uint16), be contiguous, live on `device_type` ("cuda" or "cpu") and hold at
+    least batch x hidden elements; otherwise the call fails with MOE_ERR_INVALID_ARG
+    before reaching the library. Raw pointers (ints) are not inspected."""
+    if t is None or isinstance(t, int):
+        return
+    problem = None
+    if str(t.dtype) not in _ROW_DTYPES:
+        problem = f"dtype {t.dtype}, not bfloat16 (or its bits as int16/uint16)"
+    elif t.device.type != device_type:
+        problem = f"on {t.device.type}, not {device_type}"
+    elif not t.is_contiguous():
+        problem = "not contiguous"
+    elif t.numel() < max(0, batch) * hidden:
+        problem = f"{t.numel()} values for {batch} rows of {hidden}"
+    if problem:
+        raise MoeDecodeError(MOE_ERR_INVALID_ARG, f"{what}: {name} is {problem}")
+
+
 def _stream_handle(stream) -> int | None:
     if stream is None:
         return None
@@ -160,6 +183,8 @@ def step_noalloc(hidden, n_experts, inter, shared_inter, layers, x, y, batch, to
     16, hidden <= 7168, n_experts <= 1024, inter <= 1024, shared_inter <= 2048,
     at most 2 layers. Calls that overlap on the GPU race on the shared scratch.
     """
+    for name, t in (("x", x), ("y", y)):
+        _check_rows(t, name, batch, hidden, "cuda", "moe_decode_step_noalloc")
     cfg = Config(hidden, n_experts, top_k, inter, shared_inter, batch, len(layers), eps)
     arr = (LayerWeights * len(layers))()
     for i, w in enumerate(layers):
@@ -193,12 +218,16 @@ class MoeDecode:
 
     def step(self, x, y, batch, top_k, stream=None, debug=None) -> None:
         """y <- layer stack(x); x, y device bf16 [batch, hidden]; asynchronous on `stream`."""
+        for name, t in (("x", x), ("y", y)):
+            _check_rows(t, name, batch, self.cfg.hidden, "cuda", "moe_decode_step")
         dbg = self._debug(debug)
         _check(lib().moe_decode_step(self.handle, _ptr(x), _ptr(y), int(batch), int(top_k),
                                      _stream_handle(stream), dbg), "moe_decode_step")
 
     def step_host(self, x_host, y_host, batch, top_k, stream=None, debug=None) -> None:
         """Same step on host buffers (pinned torch CPU tensors or host pointers)."""
+        for name, t in (("x_host", x_host), ("y_host", y_host)):
+            _check_rows(t, name, batch, self.cfg.hidden, "cpu", "moe_decode_step_host")
         dbg = self._debug(debug)
         _check(lib().moe_decode_step_host(self.handle, _ptr(x_host), _ptr(y_host), int(batch),
                                           int(top_k), _stream_handle(stream), dbg),

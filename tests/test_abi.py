@@ -96,3 +96,25 @@ def test_product_binding_does_not_import_the_oracle():
     subprocess.run([sys.executable, "-c", code], check=True, cwd=root)
     src = open(os.path.join(root, "moe_decode_persistent_b200", "__init__.py")).read()
     assert "import oracle" not in src and "from oracle" not in src
+
+
+def test_row_buffer_checks_of_the_binding():
+    """Tensors passed as x/y must hold bf16 values or their bit patterns, be contiguous,
+    sit on the expected device and hold batch x hidden elements; violations fail with
+    MOE_ERR_INVALID_ARG before the library is called. Raw pointers pass through."""
+    import torch
+
+    check = mdp._check_rows
+    bf = torch.zeros((4, 64), dtype=torch.bfloat16)
+    for ok in (bf, bf.view(torch.int16), bf.view(torch.uint16), bf[:2], None, 0x1000):
+        check(ok, "x", 2, 64, "cpu", "step")
+    check(bf, "x", 0, 64, "cpu", "step")  # an empty batch is the library's to reject
+    bad = [torch.zeros((4, 64), dtype=torch.float32), torch.zeros((4, 64), dtype=torch.float16),
+           torch.zeros((64, 4), dtype=torch.bfloat16).t(), torch.zeros((1, 64), dtype=torch.bfloat16)]
+    for t in bad:
+        with pytest.raises(mdp.MoeDecodeError) as err:
+            check(t, "x", 2, 64, "cpu", "step")
+        assert err.value.code == mdp.MOE_ERR_INVALID_ARG
+    with pytest.raises(mdp.MoeDecodeError) as err:
+        check(bf, "x", 2, 64, "cuda", "step")  # a host tensor where device memory is expected
+    assert err.value.code == mdp.MOE_ERR_INVALID_ARG
