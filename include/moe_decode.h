@@ -166,7 +166,11 @@ int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms)
  * top-k chosen (34) and its cycle count (35), the unique experts placed (36),
  * the pairs sorted (37), and clock64 at the kernel start (38): there the
  * routing stamps (slots 26-30, 32-34, 36, 37) are clock64 values of the CTA's
- * SM, comparable with slot 38 of the same CTA only (slot 39 is reserved). */
+ * SM, comparable with slot 38 of the same CTA only (slot 39 is reserved).
+ * Traced steps run a separate instance of the kernel whose stamps are global stores
+ * on the routing chain: a traced batch-1 step takes several microseconds longer
+ * than an untraced one, so the stamps bound the time of each hop from above and
+ * step times are compared on untraced steps. */
 int moe_decode_set_trace(moe_decode_handle* h, void* trace);
 
 /* uint64 trace slots of one layer (number of CTAs x 40). */
