@@ -98,6 +98,23 @@ def test_product_binding_does_not_import_the_oracle():
     assert "import oracle" not in src and "from oracle" not in src
 
 
+def test_cuda_sources_and_oracle_share_no_headers():
+    """The CUDA path includes only its own headers and the public ABI header; the oracle
+    includes only its own header: neither side compiles any of the other's code."""
+    import glob
+    import re
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    local = re.compile(r'#include\s+"([^"]+)"')
+    csrc = glob.glob(os.path.join(root, "moe_decode_persistent_b200", "csrc", "*"))
+    for f in csrc:
+        for inc in local.findall(open(f).read()):
+            assert inc in ("kernel_params.h", "moe_decode.h", "ptx.cuh"), (f, inc)
+    for f in glob.glob(os.path.join(root, "oracle", "*.[ch]")):
+        for inc in local.findall(open(f).read()):
+            assert inc == "moe_oracle.h", (f, inc)
+
+
 def test_row_buffer_checks_of_the_binding():
     """Tensors passed as x/y must hold bf16 values or their bit patterns, be contiguous,
     sit on the expected device and hold batch x hidden elements; violations fail with
