@@ -20,16 +20,19 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB = os.path.join(_HERE, "libmoe_oracle.so")
+# the same source compiled with its planted mistakes (the pins' own test only)
+MUTANT_LIB = os.path.join(_HERE, "libmoe_oracle_mutants.so")
 
 OK, EINVAL, EMISSING, ENONFINITE = 0, -1, -2, -3
 
 
 def build(verbose: bool = False) -> None:
-    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-o", LIB,
-           os.path.join(_HERE, "moe_oracle.c"), "-lm"]
-    if verbose:
-        print(" ".join(cmd))
-    subprocess.run(cmd, check=True, cwd=_HERE)
+    src = os.path.join(_HERE, "moe_oracle.c")
+    for out, extra in ((LIB, []), (MUTANT_LIB, ["-DORACLE_MUTANTS"])):
+        cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", *extra, "-o", out, src, "-lm"]
+        if verbose:
+            print(" ".join(cmd))
+        subprocess.run(cmd, check=True, cwd=_HERE)
 
 
 class _Dims(ctypes.Structure):
@@ -45,18 +48,19 @@ class _Weights(ctypes.Structure):
                 ("ws_down", ctypes.c_void_p)]
 
 
-_lib = None
+_libs = {}
+_active = LIB
 
 
-def _L():
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB):
+def _load(path):
+    if path not in _libs:
+        if not os.path.exists(path):
             build()
-        lib = ctypes.CDLL(LIB)
+        lib = ctypes.CDLL(path)
         vp, i, d = ctypes.c_void_p, ctypes.c_int, ctypes.c_double
-        lib.oracle_set_mutant.argtypes = [i]
-        lib.oracle_set_mutant.restype = None
+        if path == MUTANT_LIB:
+            lib.oracle_set_mutant.argtypes = [i]
+            lib.oracle_set_mutant.restype = None
         lib.oracle_bf16_round.argtypes = [d]
         lib.oracle_bf16_round.restype = d
         lib.oracle_double_to_bf16_bits.argtypes = [d]
@@ -74,8 +78,15 @@ def _L():
         lib.oracle_layer.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Weights), i, vp,
                                      vp, vp, vp, vp, vp]
         lib.oracle_layer.restype = i
-        _lib = lib
-    return _lib
+        lib.oracle_layer_selected.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Weights), i, vp,
+                                              vp, vp, vp, vp, vp, vp]
+        lib.oracle_layer_selected.restype = i
+        _libs[path] = lib
+    return _libs[path]
+
+
+def _L():
+    return _load(_active)
 
 
 def _c(a, dtype):
@@ -94,8 +105,16 @@ MUTANTS = {
 
 
 def set_mutant(m: int) -> None:
-    """Swap in one planted mistake (tests of the pins only); 0 restores the oracle."""
-    _L().oracle_set_mutant(int(m))
+    """Swap in one planted mistake (tests of the pins only): every later call runs the
+    separately compiled mutant build with mistake m. 0 restores the oracle itself."""
+    global _active
+    if int(m) == 0:
+        if MUTANT_LIB in _libs:
+            _libs[MUTANT_LIB].oracle_set_mutant(0)
+        _active = LIB
+    else:
+        _load(MUTANT_LIB).oracle_set_mutant(int(m))
+        _active = MUTANT_LIB
 
 
 # ---- single stages ---------------------------------------------------------------
@@ -153,17 +172,24 @@ def swiglu(n: np.ndarray, wg_bits, wu_bits, wd_bits) -> np.ndarray:
 
 # ---- whole layer -------------------------------------------------------------------
 
-def layer(dims: dict, weights: dict, x_bits: np.ndarray) -> dict:
+def layer(dims: dict, weights: dict, x_bits: np.ndarray, selection=None) -> dict:
     """Run the oracle on rows x_bits [B, H].
 
     dims: H, E, k, I, Is, eps.  weights: gamma [H], w_router [E,H], router_bias
     [E] or None, experts {e: (W_g [I,H], W_u [I,H], W_d [H,I])} (only the
     experts the rows select need be present), ws_gate [Is,H], ws_up [Is,H],
     ws_down [H,Is]; all bf16 bit arrays. Returns logits, idx, w, y_pre, y.
+
+    selection: None (each row takes the top-k of its logits), or int [B, k] -- each
+    row's k distinct experts given (oracle_layer_selected: the weights are the
+    softmax of the row's own logits over the given set).
     """
     H, E, k = dims["H"], dims["E"], dims["k"]
     x = _c(x_bits, np.uint16).reshape(-1, H)
     B = x.shape[0]
+    sel = None
+    if selection is not None:
+        sel = _c(selection, np.int32).reshape(B, k)
     keep = []  # keep arrays alive across the call
 
     def arr(a, dt):
@@ -194,19 +220,25 @@ def layer(dims: dict, weights: dict, x_bits: np.ndarray) -> dict:
     wts = np.empty((B, k), dtype=np.float64)
     y_pre = np.empty((B, H), dtype=np.float64)
     y = np.empty((B, H), dtype=np.uint16)
-    rc = _L().oracle_layer(ctypes.byref(d), ctypes.byref(w), B, _p(x), _p(logits), _p(idx),
-                           _p(wts), _p(y_pre), _p(y))
+    if sel is None:
+        rc = _L().oracle_layer(ctypes.byref(d), ctypes.byref(w), B, _p(x), _p(logits), _p(idx),
+                               _p(wts), _p(y_pre), _p(y))
+    else:
+        rc = _L().oracle_layer_selected(ctypes.byref(d), ctypes.byref(w), B, _p(x), _p(sel), _p(logits),
+                                        _p(idx), _p(wts), _p(y_pre), _p(y))
     if rc != OK:
         raise RuntimeError(f"oracle_layer failed: {rc}")
     return {"logits": logits, "idx": idx, "w": wts, "y_pre": y_pre, "y": y}
 
 
-def workload_layer(wl, layer_index: int, x_bits: np.ndarray, shared=None, w_router=None) -> dict:
+def workload_layer(wl, layer_index: int, x_bits: np.ndarray, shared=None, w_router=None,
+                   selection=None) -> dict:
     """Oracle of one layer of a ``synth.Workload`` on rows x_bits [B, H].
 
     Only the experts that the rows select are regenerated on the host (one row
     at a time, so host memory stays at 16 experts). ``shared`` and ``w_router``
-    may be passed in to avoid regenerating them for every call.
+    may be passed in to avoid regenerating them for every call. ``selection``
+    (int [B, k], optional) gives each row's experts instead of its top-k.
     """
     dims = dict(H=wl.H, E=wl.E, k=wl.k, I=wl.I, Is=wl.Is, eps=wl.eps)
     gamma = wl.gamma_host(layer_index)
@@ -216,10 +248,14 @@ def workload_layer(wl, layer_index: int, x_bits: np.ndarray, shared=None, w_rout
     x = _c(x_bits, np.uint16).reshape(-1, wl.H)
     outs = []
     for b in range(x.shape[0]):
-        n = rmsnorm(x[b], gamma, wl.eps)
-        sel = topk(router(n, wr, bias), wl.k)
-        experts = {int(e): wl.expert_host(layer_index, int(e)) for e in sel}
+        if selection is None:
+            n = rmsnorm(x[b], gamma, wl.eps)
+            sel = topk(router(n, wr, bias), wl.k)
+            given = None
+        else:
+            sel = given = np.asarray(selection[b], dtype=np.int32).reshape(1, wl.k)
+        experts = {int(e): wl.expert_host(layer_index, int(e)) for e in np.ravel(sel)}
         outs.append(layer(dims, dict(gamma=gamma, w_router=wr, router_bias=bias, experts=experts,
-                                     ws_gate=sg, ws_up=su, ws_down=sd), x[b:b + 1]))
+                                     ws_gate=sg, ws_up=su, ws_down=sd), x[b:b + 1], selection=given))
         del experts
     return {key: np.concatenate([o[key] for o in outs], axis=0) for key in outs[0]}

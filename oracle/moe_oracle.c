@@ -70,12 +70,17 @@ static inline double bf(uint16_t b) { return oracle_bf16_to_double(b); }
 
 static double silu(double v) { return v / (1.0 + exp(-v)); }
 
-/* Planted-mistake switch, used only by the test that proves the pins catch
- * mistakes. 0 (the default) is the oracle; each other value swaps in one
- * plausible error (see ORACLE_MUT_* in moe_oracle.h). */
+/* Planted mistakes exist only in a second build of this file, compiled with
+ * -DORACLE_MUTANTS for the test that proves the pins catch mistakes; there
+ * oracle_set_mutant(m) swaps in one plausible error (ORACLE_MUT_* in
+ * moe_oracle.h). In the oracle itself every MUT() is the constant 0. */
+#ifdef ORACLE_MUTANTS
 static int g_mutant = 0;
 void oracle_set_mutant(int m) { g_mutant = m; }
 #define MUT(m) (g_mutant == (m))
+#else
+#define MUT(m) 0
+#endif
 
 /* ---- stages ---------------------------------------------------------------- */
 
@@ -171,10 +176,48 @@ void oracle_swiglu(int H, int F, const double* n, const uint16_t* wg, const uint
 
 /* ---- whole layer ------------------------------------------------------------ */
 
-int oracle_layer(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
-                 double* logits, int32_t* topk_idx, double* topk_w, double* y_pre, uint16_t* y) {
+/* The output of one row once its selection and weights are known:
+ * y = bf16(x + s + sum_j w[j] E_{S_j}(n)), the shared expert first, then the
+ * selected experts in the order given. Scratch: s, ex, acc (H each). */
+static int combine_row(const oracle_dims* d, const oracle_weights* w, const uint16_t* xb,
+                       const double* n, const int32_t* ib, const double* wb, double* s, double* ex,
+                       double* acc, double* y_pre, uint16_t* y) {
+  const int H = d->H, k = d->k, I = d->I, Is = d->Is;
+  oracle_swiglu(H, Is, n, w->ws_gate, w->ws_up, w->ws_down, s);
+  for (int h = 0; h < H; ++h) {
+    const double res = MUT(ORACLE_MUT_RESIDUAL_N) ? n[h] : bf(xb[h]);
+    acc[h] = res + (MUT(ORACLE_MUT_NO_SHARED) ? 0.0 : s[h]);
+  }
+  for (int j = 0; j < k; ++j) {
+    const int e = ib[j];
+    if (!w->w_gate[e] || !w->w_up[e] || !w->w_down[e]) return ORACLE_EMISSING;
+    oracle_swiglu(H, I, n, w->w_gate[e], w->w_up[e], w->w_down[e], ex);
+    for (int h = 0; h < H; ++h) acc[h] += wb[j] * ex[h];
+  }
+  for (int h = 0; h < H; ++h) {
+    if (y_pre) y_pre[h] = acc[h];
+    if (y) y[h] = oracle_double_to_bf16_bits(acc[h]);
+  }
+  return ORACLE_OK;
+}
+
+/* Both whole-layer entry points. sel == NULL: each row's selection is the top-k
+ * of its logits. Otherwise sel [B][k] gives each row's selection (k distinct
+ * experts); the weights are then the softmax of the row's own logits over it. */
+static int layer_rows(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
+                      const int32_t* sel, double* logits, int32_t* topk_idx, double* topk_w,
+                      double* y_pre, uint16_t* y) {
   const int H = d->H, E = d->E, k = d->k, I = d->I, Is = d->Is;
   if (B < 0 || H < 1 || E < 1 || k < 1 || k > E || I < 1 || Is < 1) return ORACLE_EINVAL;
+  if (sel) {
+    for (int b = 0; b < B; ++b)
+      for (int j = 0; j < k; ++j) {
+        const int e = sel[(size_t)b * k + j];
+        if (e < 0 || e >= E) return ORACLE_EINVAL;
+        for (int i = 0; i < j; ++i)
+          if (sel[(size_t)b * k + i] == e) return ORACLE_EINVAL;
+      }
+  }
   double* n = (double*)malloc(sizeof(double) * (size_t)H);
   double* s = (double*)malloc(sizeof(double) * (size_t)H);
   double* ex = (double*)malloc(sizeof(double) * (size_t)H);
@@ -188,28 +231,34 @@ int oracle_layer(const oracle_dims* d, const oracle_weights* w, int B, const uin
 
     oracle_rmsnorm(H, d->eps, xb, w->gamma, n);
     oracle_router(H, E, n, w->w_router, w->router_bias, lb);
-    if (oracle_topk(E, k, lb, ib) != 0) { rc = ORACLE_ENONFINITE; break; }
+    if (sel) {
+      for (int e = 0; e < E; ++e)
+        if (!isfinite(lb[e])) rc = ORACLE_ENONFINITE;
+      if (rc != ORACLE_OK) break;
+      memcpy(ib, sel + (size_t)b * k, sizeof(int32_t) * (size_t)k);
+    } else if (oracle_topk(E, k, lb, ib) != 0) {
+      rc = ORACLE_ENONFINITE;
+      break;
+    }
     oracle_softmax_selected(k, lb, ib, wb);
-
-    oracle_swiglu(H, Is, n, w->ws_gate, w->ws_up, w->ws_down, s);
-    for (int h = 0; h < H; ++h) {
-      const double res = MUT(ORACLE_MUT_RESIDUAL_N) ? n[h] : bf(xb[h]);
-      acc[h] = res + (MUT(ORACLE_MUT_NO_SHARED) ? 0.0 : s[h]);
-    }
-    for (int j = 0; j < k; ++j) {
-      const int e = ib[j];
-      if (!w->w_gate[e] || !w->w_up[e] || !w->w_down[e]) { rc = ORACLE_EMISSING; break; }
-      oracle_swiglu(H, I, n, w->w_gate[e], w->w_up[e], w->w_down[e], ex);
-      for (int h = 0; h < H; ++h) acc[h] += wb[j] * ex[h];
-    }
-    for (int h = 0; h < H; ++h) {
-      if (y_pre) y_pre[(size_t)b * H + h] = acc[h];
-      if (y) y[(size_t)b * H + h] = oracle_double_to_bf16_bits(acc[h]);
-    }
+    rc = combine_row(d, w, xb, n, ib, wb, s, ex, acc, y_pre ? y_pre + (size_t)b * H : NULL,
+                     y ? y + (size_t)b * H : NULL);
   }
   free(n);
   free(s);
   free(ex);
   free(acc);
   return rc;
+}
+
+int oracle_layer(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
+                 double* logits, int32_t* topk_idx, double* topk_w, double* y_pre, uint16_t* y) {
+  return layer_rows(d, w, B, x, NULL, logits, topk_idx, topk_w, y_pre, y);
+}
+
+int oracle_layer_selected(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
+                          const int32_t* sel, double* logits, int32_t* topk_idx, double* topk_w,
+                          double* y_pre, uint16_t* y) {
+  if (!sel) return ORACLE_EINVAL;
+  return layer_rows(d, w, B, x, sel, logits, topk_idx, topk_w, y_pre, y);
 }

@@ -30,7 +30,9 @@ typedef struct {
   const uint16_t* ws_down;        /* [H][Is] */
 } oracle_weights;
 
-/* Planted mistakes (test of the pins only; 0 = the oracle itself). */
+/* Planted mistakes (test of the pins only; 0 = the oracle itself). They exist only
+ * in the separate build compiled with -DORACLE_MUTANTS (libmoe_oracle_mutants.so),
+ * which alone exports oracle_set_mutant. */
 #define ORACLE_MUT_NONE 0
 #define ORACLE_MUT_NO_N_ROUND 1      /* n not rounded to bf16 */
 #define ORACLE_MUT_NO_H_ROUND 2      /* SwiGLU product not rounded to bf16 */
@@ -62,5 +64,14 @@ void oracle_swiglu(int H, int F, const double* n, const uint16_t* wg, const uint
  * (fp64 before the final rounding; may be NULL), y [B][H] bf16 bits (may be NULL). */
 int oracle_layer(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
                  double* logits, int32_t* topk_idx, double* topk_w, double* y_pre, uint16_t* y);
+
+/* The same layer with each row's selection given instead of chosen: sel [B][k]
+ * holds k distinct experts per row. The logits are still the row's own, and the
+ * weights are the softmax of those logits over the given set (so a given set
+ * equal to the top-k reproduces oracle_layer exactly). topk_idx receives a copy
+ * of sel. ORACLE_EINVAL for a repeated or out-of-range expert. */
+int oracle_layer_selected(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
+                          const int32_t* sel, double* logits, int32_t* topk_idx, double* topk_w,
+                          double* y_pre, uint16_t* y);
 
 #endif

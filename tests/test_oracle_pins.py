@@ -255,9 +255,11 @@ def test_swiglu_gate_and_up_are_not_interchangeable():
 
 # ---- whole layer ------------------------------------------------------------------------------
 
-def closed_form_layer(seed):
+def closed_form_layer(seed, force=None):
     """A tiny layer whose every matrix has one nonzero per row: the whole output
-    has an elementwise closed form."""
+    has an elementwise closed form. force: a list of k distinct experts that
+    replaces the row's top-k (the weights are then the softmax of the row's
+    logits over that list)."""
     rng = np.random.default_rng(seed)
     H, E, k, I, Is, eps = 12, 6, 2, 5, 7, 1e-6
     x = to_bits(rng.standard_normal(H))
@@ -287,7 +289,7 @@ def closed_form_layer(seed):
     r = 1.0 / math.sqrt(np.sum(xf * xf) / H + eps)
     n = np.array([oracle.bf16_round(t) for t in xf * r * bf(gamma)])
     lg = rd * n[rcol] + bias.astype(np.float64)
-    sel = sorted(range(E), key=lambda e: (-lg[e], e))[:k]
+    sel = sorted(range(E), key=lambda e: (-lg[e], e))[:k] if force is None else list(force)
     ws = softmax(lg[sel])
     s = swiglu_closed_form(n, spg, sdg, spu, sdu, spd, sdd)
     y = xf + s
@@ -306,6 +308,47 @@ def test_layer_closed_form(seed):
     np.testing.assert_allclose(got["y_pre"][0], want["y_pre"], rtol=1e-12, atol=1e-12)
     ybits = np.array([oracle.bf16_bits(t) for t in got["y_pre"][0]], np.uint16)
     np.testing.assert_array_equal(got["y"][0], ybits)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_layer_with_given_selection_closed_form(seed):
+    """A selection that is not the top-k: the output is the closed form evaluated on
+    exactly that set, weighted by the softmax of the row's own logits over it."""
+    rng = np.random.default_rng(100 + seed)
+    force = [int(e) for e in rng.permutation(6)[:2]]
+    dims, W, x, want = closed_form_layer(seed, force=force)
+    got = oracle.layer(dims, W, x, selection=np.array([force]))
+    np.testing.assert_array_equal(got["logits"][0], want["logits"])
+    np.testing.assert_array_equal(got["idx"][0], force)
+    np.testing.assert_allclose(got["w"][0], want["w"], rtol=1e-13)
+    np.testing.assert_allclose(got["y_pre"][0], want["y_pre"], rtol=1e-12, atol=1e-12)
+
+
+def test_layer_with_own_selection_equals_layer_bitwise():
+    dims, W = tiny_random_layer(TINY)
+    x = TINY.x_host()
+    own = oracle.layer(dims, W, x)
+    given = oracle.layer(dims, W, x, selection=own["idx"])
+    for key in ("logits", "idx", "w", "y_pre", "y"):
+        assert np.array_equal(own[key], given[key]), key
+
+
+def test_layer_with_given_selection_is_order_free_and_rejects_bad_sets():
+    dims, W = tiny_random_layer(TINY)
+    x = TINY.x_host()
+    own = oracle.layer(dims, W, x)
+    # the same set in reverse order: the same weights per expert, the same output
+    rev = oracle.layer(dims, W, x, selection=own["idx"][:, ::-1])
+    np.testing.assert_allclose(rev["w"], own["w"][:, ::-1], rtol=1e-14)
+    np.testing.assert_allclose(rev["y_pre"], own["y_pre"], rtol=1e-12, atol=1e-13)
+    bad = own["idx"].copy()
+    bad[0, 1] = bad[0, 0]                          # a repeated expert
+    with pytest.raises(RuntimeError):
+        oracle.layer(dims, W, x, selection=bad)
+    bad = own["idx"].copy()
+    bad[1, 0] = TINY.E                             # out of range
+    with pytest.raises(RuntimeError):
+        oracle.layer(dims, W, x, selection=bad)
 
 
 def test_layer_missing_expert_is_an_error():
@@ -424,6 +467,7 @@ PIN_CHECKS = [
     lambda: test_swiglu_closed_form_with_selection_matrices(16, 8),
     test_swiglu_gate_and_up_are_not_interchangeable,
     lambda: [test_layer_closed_form(s) for s in range(8)],
+    lambda: [test_layer_with_given_selection_closed_form(s) for s in range(4)],
     test_layer_zero_routed_down_gives_shared_only,
     test_layer_bias_enters_selection_and_weights,
 ]
@@ -445,3 +489,13 @@ def test_each_planted_mistake_fails_a_pin(mutant):
     finally:
         oracle.set_mutant(0)
     assert failed, f"planted mistake {oracle.MUTANTS[mutant]} was not caught by any pin"
+
+
+def test_shipped_oracle_has_no_mistake_switch():
+    """The planted mistakes live only in the separately compiled mutant build: the
+    oracle library itself exports no switch and carries no mistake branches."""
+    import ctypes
+
+    plain = ctypes.CDLL(oracle.LIB)
+    assert not hasattr(plain, "oracle_set_mutant")
+    assert hasattr(ctypes.CDLL(oracle.MUTANT_LIB), "oracle_set_mutant")
