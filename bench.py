@@ -35,6 +35,7 @@ METRIC = "MoE decode-layer µs/step and HBM GB/s (% of B200 peak) at batch 1–6
 FALLBACK_HBM_GBS = 6650.0
 POOL = 32
 FLUSH_BYTES = 256 << 20
+PER_CONFIG = (1, 2, 3, 4)  # the full-size workloads timed after the headline
 
 
 def parse_args(argv=None):
@@ -47,6 +48,11 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline oracle budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="time only the headline workload (no per_config block)")
+    ap.add_argument("--launch-log", default=None,
+                    help="write every launch's workload, step, layer, unique experts and algorithmic "
+                         "bytes (warm-up included) to this JSON file, to match ncu counters per launch")
     ap.add_argument("--tc-min-batch", type=int, default=None,
                     help="batch-shape switch: steps of at least this many rows take the tensor-core "
                          "kernel (0: always the CUDA-core kernel); default: the library's")
@@ -95,9 +101,9 @@ def kernel_source_hash():
     return hsh.hexdigest()
 
 
-def traffic_per_launch(workload):
-    """DRAM bytes per launch from profiles/traffic.json (ncu counters), or None when the
-    workload was not captured or the kernel sources changed since the capture."""
+def traffic_entry(workload):
+    """The ncu DRAM-traffic record of a workload from profiles/traffic.json, or None when
+    the workload was not captured or the kernel sources changed since the capture."""
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(tpath):
         return None
@@ -105,7 +111,13 @@ def traffic_per_launch(workload):
         t = json.load(f).get(workload)
     if t is None or t.get("kernel_sources_sha256") != kernel_source_hash():
         return None
-    return t.get("bytes_per_launch")
+    return t
+
+
+def traffic_per_launch(workload):
+    """DRAM bytes per launch (ncu counters), or None (see traffic_entry)."""
+    t = traffic_entry(workload)
+    return None if t is None else t.get("bytes_per_launch")
 
 
 def workload_config(wl, flush):
@@ -287,10 +299,105 @@ def aggregate(local_bytes, local_ms, world):
     return float(b.item()), float(t.item())
 
 
+def step_stats(step_ms):
+    a = np.asarray(step_ms, dtype=np.float64) * 1e3  # µs
+    return {"us_per_step": round(float(a.mean()), 2), "us_per_step_p10": round(float(np.percentile(a, 10)), 2),
+            "us_per_step_median": round(float(np.median(a)), 2),
+            "us_per_step_p90": round(float(np.percentile(a, 90)), 2)}
+
+
+class ConfigRun:
+    """One workload on this rank's GPU: its weights (generated on the device), a handle,
+    a pool of POOL seeded input batches resident in HBM and the L2-flush buffer."""
+
+    def __init__(self, wl, device, tc_min_batch=None):
+        import torch
+
+        import moe_decode_persistent_b200 as mdp
+
+        self.wl = wl
+        self.dev = f"cuda:{device}"
+        self.layers = [wl.device_layer(l, device=self.dev) for l in range(wl.layers)]
+        self.h = mdp.MoeDecode(wl.H, wl.E, wl.k, wl.I, wl.Is, wl.B, self.layers, eps=wl.eps, device=device)
+        if tc_min_batch is not None:
+            self.h.set_tc_min_batch(tc_min_batch)
+        self.kernel_path = "tensor_core" if self.h.step_path(wl.B) == mdp.PATH_TENSOR_CORE else "cuda_core"
+        self.pool_host = wl.x_pool_host(POOL)
+        self.pool = torch.from_numpy(self.pool_host.view(np.int16)).view(torch.bfloat16).to(self.dev)
+        self.y = torch.empty((wl.B, wl.H), dtype=torch.bfloat16, device=self.dev)
+        self.flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=self.dev)
+
+    def steps(self, K, W, stream, barrier, host=None, launch_log=None):
+        """W untimed warm-up steps immediately followed (no idle gap, so the clocks stay
+        up) by K timed steps, each preceded by an L2 flush; CUDA events on `stream`
+        bracket every step. host = (x_host, y_host): the host-buffer entry point instead.
+        Returns per-step ms and the unique-expert count of every timed step and layer."""
+        import torch
+
+        wl, h = self.wl, self.h
+        nu = torch.zeros((W + K, wl.layers), dtype=torch.int32, device=self.dev)
+        dbg = lambda i: [dict(n_unique=nu[i, l:l + 1]) for l in range(wl.layers)]
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+
+        def one(i, timed):
+            self.flush.zero_()
+            if timed:
+                ev[i - W][0].record(stream)
+            if host is None:
+                h.step(self.pool[i % POOL], self.y, wl.B, wl.k, stream=stream, debug=dbg(i))
+            else:
+                h.step_host(host[0][i % POOL], host[1], wl.B, wl.k, stream=stream, debug=dbg(i))
+            if timed:
+                ev[i - W][1].record(stream)
+
+        for i in range(W):
+            one(i, False)
+        # the timed region: barrier + synchronize on both sides; the warm-up runs right
+        # before it, so the GPU does not idle (and drop its clocks) in between
+        barrier()
+        torch.cuda.synchronize()
+        wall0 = time.perf_counter()
+        for i in range(W, W + K):
+            one(i, True)
+        torch.cuda.synchronize()
+        barrier()
+        self.wall = time.perf_counter() - wall0
+        status = h.status()
+        if status != 0:
+            import moe_decode_persistent_b200 as mdp
+
+            raise RuntimeError(f"{wl.name}: device status {status}: {mdp.strerror(status)}")
+        U = nu.cpu().numpy()
+        if launch_log is not None:
+            for i in range(W + K):
+                for l in range(wl.layers):
+                    launch_log.append({"workload": wl.name, "step": i, "layer": l, "timed": i >= W,
+                                       "unique_experts": int(U[i, l]),
+                                       "algorithmic_bytes": step_bytes(wl, [int(U[i, l])])})
+        return [a.elapsed_time(b) for a, b in ev], U[W:]
+
+    def close(self):
+        import torch
+
+        self.h.close()
+        del self.layers, self.pool, self.flush, self.y
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+def roofline_entry(wl, achieved, peak, peak_kind):
+    t = traffic_entry(wl.name)
+    return {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4),
+            "traffic": None if t is None else t["bytes_per_launch"],
+            "traffic_over_algorithmic": None if t is None else t.get("traffic_over_algorithmic"),
+            "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                           else "fallback 6.65 TB/s",
+            "kernel": "moe_decode_layer_kernel"}
+
+
 def run_ours(args, wl):
     import torch
-
-    import moe_decode_persistent_b200 as mdp
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -310,106 +417,85 @@ def run_ours(args, wl):
             dist.barrier()
 
     stream = torch.cuda.current_stream()
-    layers = [wl.device_layer(l, device=f"cuda:{local}") for l in range(wl.layers)]
-    h = mdp.MoeDecode(wl.H, wl.E, wl.k, wl.I, wl.Is, wl.B, layers, eps=wl.eps, device=local)
-    if args.tc_min_batch is not None:
-        h.set_tc_min_batch(args.tc_min_batch)
-    kernel_path = "tensor_core" if h.step_path(wl.B) == mdp.PATH_TENSOR_CORE else "cuda_core"
-    pool_host = wl.x_pool_host(POOL)
-    pool = torch.from_numpy(pool_host.view(np.int16)).view(torch.bfloat16).to(f"cuda:{local}")
-    y = torch.empty((wl.B, wl.H), dtype=torch.bfloat16, device=f"cuda:{local}")
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=f"cuda:{local}")
     K, W = args.steps, args.warmup
-    nuniq = torch.zeros((K, wl.layers), dtype=torch.int32, device=f"cuda:{local}")
-
-    def dbg_for(i):
-        return [dict(n_unique=nuniq[i, l:l + 1]) for l in range(wl.layers)]
-
-    for i in range(W):
-        flush.zero_()
-        h.step(pool[i % POOL], y, wl.B, wl.k, stream=stream)
-    torch.cuda.synchronize()
-    if h.status() != 0:
-        raise RuntimeError("device status error during warm-up")
-
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    peak, peak_kind = measured_peaks()
+    launch_log = [] if args.launch_log else None
+    run = ConfigRun(wl, local, args.tc_min_batch)
     sampler = ClockSampler(local)
     sampler.start()
-    barrier()
-    torch.cuda.synchronize()
-    wall0 = time.perf_counter()
-    for i in range(K):
-        flush.zero_()
-        ev[i][0].record(stream)
-        h.step(pool[i % POOL], y, wl.B, wl.k, stream=stream, debug=dbg_for(i))
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    wall = time.perf_counter() - wall0
+    step_ms, U = run.steps(K, W, stream, barrier, launch_log=launch_log)
+    wall = run.wall
     clocks = sampler.stop()
-    status = h.status()
-    if status != 0:
-        raise RuntimeError(f"device status {status}: {mdp.strerror(status)}")
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    U = nuniq.cpu().numpy()
     bytes_steps = [step_bytes(wl, list(U[i])) for i in range(K)]
     local_ms = float(sum(step_ms))
     tot_bytes, max_ms = aggregate(sum(bytes_steps), local_ms, world)
     value = tot_bytes / (max_ms * 1e-3) / 1e9
+    achieved = sum(bytes_steps) / (local_ms * 1e-3) / 1e9  # this rank's launching stream
 
     # end to end through the host-buffer entry point: H2D x, step, D2H y per step
     e2e = None
     if not args.no_e2e:
-        xh = torch.from_numpy(pool_host.view(np.int16)).pin_memory()
+        xh = torch.from_numpy(run.pool_host.view(np.int16)).pin_memory()
         yh = torch.empty((wl.B, wl.H), dtype=torch.int16).pin_memory()
-        for i in range(min(W, 10)):
-            h.step_host(xh[i % POOL], yh, wl.B, wl.k, stream=stream)
-        torch.cuda.synchronize()
-        ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-        barrier()
-        torch.cuda.synchronize()
-        for i in range(K):
-            flush.zero_()
-            ee[i][0].record(stream)
-            h.step_host(xh[i % POOL], yh, wl.B, wl.k, stream=stream, debug=dbg_for(i))
-            ee[i][1].record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        if h.status() != 0:
-            raise RuntimeError("device status error in the end-to-end loop")
-        e_ms = float(sum(a.elapsed_time(b) for a, b in ee))
-        U2 = nuniq.cpu().numpy()
+        e_step, U2 = run.steps(K, min(W, 10), stream, barrier, host=(xh, yh))
+        e_ms = float(sum(e_step))
         e_bytes, e_max = aggregate(sum(step_bytes(wl, list(U2[i])) for i in range(K)), e_ms, world)
         e2e = {"value": round(e_bytes / (e_max * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(xh[0].numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 2),
                "ms_per_step": round(e_max / K, 4)}
-
-    peak, peak_kind = measured_peaks()
-    achieved = sum(bytes_steps) / (local_ms * 1e-3) / 1e9  # per launch-stream, this rank
-    traffic = traffic_per_launch(wl.name)
 
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": W, "ms_per_step": round(max_ms / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded counter-hash weights ~N(0,1/sqrt(fan_in)) and inputs, no trained weights",
-        "config": dict(workload_config(wl, "flushed between timed steps (256 MB write)"), kernel_path=kernel_path),
-        "us_per_step": round(1e3 * max_ms / K, 2),
-        "us_per_step_median": round(1e3 * float(np.median(step_ms)), 2),
-        "us_per_step_p90": round(1e3 * float(np.percentile(step_ms, 90)), 2),
+        "config": dict(workload_config(wl, "flushed between timed steps (256 MB write)"), kernel_path=run.kernel_path),
+        **step_stats(step_ms),
         "tokens_per_s": round(world * wl.B * K / (max_ms * 1e-3), 1),
         "unique_experts_mean": float(U.mean()),
         "bytes_per_step_mean": float(np.mean(bytes_steps)),
         "hbm_frac_of_peak": round(value / world / peak, 4),
-        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": traffic,
-                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6.65 TB/s",
-                     "kernel": "moe_decode_layer_kernel"},
+        "roofline": roofline_entry(wl, achieved, peak, peak_kind),
         "e2e": e2e,
-        "gpu_launches": K * h.launches_per_step(),
+        "gpu_launches": K * run.h.launches_per_step(),
         "clocks": clocks,
         "wall_s_timed_region": round(wall, 4),
     }
+    pool_host = run.pool_host
+    run.close()
+
+    # the other full-size workloads, each on its own weights: µs/step and GB/s over its
+    # own unique-expert bytes, with its own clock record
+    per_config = {}
+    launches = line["gpu_launches"]
+    for c in ([] if args.no_per_config else [c for c in PER_CONFIG if synth.WORKLOADS[c].name != wl.name]):
+        cw = synth.WORKLOADS[c]
+        r = ConfigRun(cw, local, args.tc_min_batch)
+        smp = ClockSampler(local)
+        smp.start()
+        c_ms, cU = r.steps(K, W, stream, barrier, launch_log=launch_log)
+        c_clocks = smp.stop()
+        c_bytes = [step_bytes(cw, list(cU[i])) for i in range(K)]
+        c_local = float(sum(c_ms))
+        c_tot, c_max = aggregate(sum(c_bytes), c_local, world)
+        c_ach = sum(c_bytes) / (c_local * 1e-3) / 1e9
+        per_config[cw.name] = {
+            "config": workload_config(cw, "flushed between timed steps (256 MB write)") | {"kernel_path": r.kernel_path},
+            "value": round(c_tot / (c_max * 1e-3) / 1e9, 2), "unit": "GB/s",
+            **step_stats(c_ms),
+            "tokens_per_s": round(world * cw.B * K / (c_max * 1e-3), 1),
+            "unique_experts_mean": float(cU.mean()), "bytes_per_step_mean": float(np.mean(c_bytes)),
+            "roofline": roofline_entry(cw, c_ach, peak, peak_kind),
+            "gpu_launches": K * r.h.launches_per_step(), "clocks": c_clocks}
+        launches += K * r.h.launches_per_step()
+        r.close()
+    if per_config:
+        line["per_config"] = per_config
+        line["gpu_launches_all_configs"] = launches
+    if args.launch_log and rank == 0:
+        with open(args.launch_log, "w") as f:
+            json.dump(launch_log, f)
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, secs, steps, ninp = cpu_oracle_full_steps(wl, pool_host[:, :1], args.cpu_seconds)
         line["cpu_baseline"] = {
@@ -417,7 +503,6 @@ def run_ours(args, wl):
             "kind": "oracle",
             "sample": f"{steps} full single-row layer steps of {wl.name} over {ninp} distinct pool inputs "
                       f"({secs:.1f} s of oracle time; host weight regeneration not timed)"}
-    h.close()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

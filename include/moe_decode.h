@@ -208,15 +208,19 @@ int moe_decode_step_path(const moe_decode_handle* h, int batch);
  *    not used); beyond them it returns MOE_ERR_UNSUPPORTED_SHAPE.
  *  - cfg, layers, x_in, y_out, batch, top_k and stream mean what they mean for
  *    moe_decode_create and moe_decode_step; the TMA descriptors are built on
- *    every call.
+ *    every call and handed to the GPU by value in a kernel launch's parameters
+ *    (no host buffer is read after the call returns).
  *  - The first call on a device (the current device) sets up that device: it
  *    looks up the scratch array's device address and the kernel's attributes.
  *    Make that first call before any stream capture.
  *  - All calls share the one array and each call clears its counters before it
  *    runs: calls that overlap on the GPU (other streams, other threads) race and
  *    must be serialised by the caller.
- *  - device_status: NULL, or a caller-zeroed device int into which the kernel
- *    records the first device-side MOE_ERR_* of the step (read it after a sync). */
+ *  - device_status (required; NULL is MOE_ERR_INVALID_ARG): a caller-zeroed,
+ *    4-byte aligned device int into which the kernel records the first
+ *    device-side MOE_ERR_* of the step (a wait that ran out, a non-finite router
+ *    logit; read it after a sync). It is the only place such a failure shows:
+ *    the return value covers argument and launch errors only. */
 int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_decode_layer_weights* layers,
                             const void* x_in, void* y_out, int batch, int top_k, void* stream,
                             int* device_status);

@@ -182,6 +182,8 @@ def step_noalloc(hidden, n_experts, inter, shared_inter, layers, x, y, batch, to
     For callers that cannot allocate device memory. Limits: batch <= 4, top_k <=
     16, hidden <= 7168, n_experts <= 1024, inter <= 1024, shared_inter <= 2048,
     at most 2 layers. Calls that overlap on the GPU race on the shared scratch.
+    device_status (required): a zeroed device int32 that receives the first
+    device-side MOE_ERR_* of the step.
     """
     for name, t in (("x", x), ("y", y)):
         _check_rows(t, name, batch, hidden, "cuda", "moe_decode_step_noalloc")

@@ -1758,11 +1758,16 @@ struct Producer {
     }
     __syncwarp();
     if (lane == 0) {
+      // every bulk copy this CTA issued lands before its shared memory is given up;
+      // a copy that never lands is reported like every other wait that runs out
       for (int s = 0; s < nst; ++s) {
         if (!((pend_mask >> s) & 1u)) continue;
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&sm.full[s], (pend_parity >> s) & 1u)) {
-          if (globaltimer_ns() - t0 > 50000000ull) break;
+          if (globaltimer_ns() - t0 > 50000000ull) {
+            record_abort(p, MOE_ERR_TIMEOUT);
+            break;
+          }
         }
       }
       for (int r = 0; r < 4; ++r) {
@@ -1791,7 +1796,10 @@ __device__ void producer_cc(Producer& pr, uint8_t* ring) {
   const int lane = pr.lane;
   const uint64_t pol = policy_evict_first();
   if (lane == 0)
-    for (int t = 0; t < TM_T_WR; ++t) prefetch_tensormap(&p.tmaps[t]);
+    for (int t = 0; t < TM_T_WR; ++t) {
+      fence_tensormap_acquire(&p.tmaps[t]);
+      prefetch_tensormap(&p.tmaps[t]);
+    }
   bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
   const int pre = sh.NR + sh.NS;
   int u = pr.grab();
@@ -1998,7 +2006,10 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
   const int lane = pr.lane;
   const uint64_t pol = policy_evict_first();
   if (lane == 0)
-    for (int t = TM_T_WR; t < TM_COUNT; ++t) prefetch_tensormap(&p.tmaps[t]);
+    for (int t = TM_T_WR; t < TM_COUNT; ++t) {
+      fence_tensormap_acquire(&p.tmaps[t]);
+      prefetch_tensormap(&p.tmaps[t]);
+    }
   bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
   const int pre = sh.pre;
   int u = pr.grab();
@@ -2369,12 +2380,17 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
     }
   }
   __syncwarp();
-  // every MMA this warp issued completes before the CTA gives up its shared and tensor memory
+  // every MMA this warp issued completes before the CTA gives up its shared and tensor
+  // memory. MMAs that never complete are reported; the tensor memory is still freed
+  // (a CTA that kept it would leave its SM's next allocation waiting without bound).
   if (issued && lane == 0) {
     tc_commit(&sm.mma_bar);
     const uint64_t t0 = globaltimer_ns();
     while (!mbar_try_wait(&sm.mma_bar, 0u)) {
-      if (globaltimer_ns() - t0 > 50000000ull) break;
+      if (globaltimer_ns() - t0 > 50000000ull) {
+        record_abort(p, MOE_ERR_TIMEOUT);
+        break;
+      }
     }
   }
   __syncwarp();

@@ -1,13 +1,16 @@
 // moe_decode_noalloc.cu - the decode step for callers that cannot allocate device
 // memory (see moe_decode_step_noalloc in include/moe_decode.h).
 //
-// Some callers cannot call cudaMalloc at all: code that runs inside a captured or
-// replayed CUDA graph's setup path, allocator hooks, plugins hosted by a framework
-// that owns all device memory, or processes whose memory budget is fixed before
-// they start. For them the step's scratch (normalised rows, logits, SwiGLU
+// Some callers cannot call cudaMalloc at all: allocator hooks, plugins hosted by a
+// framework that owns all device memory, or processes whose memory budget is fixed
+// before they start. For them the step's scratch (normalised rows, logits, SwiGLU
 // outputs, split-K partials, counters and the TMA descriptors) lives in one
 // file-scope device array sized for the limits below. Every GPU that loads this
 // library holds the array until the process exits.
+//
+// The descriptors are built on the host at every call and reach the array through
+// the parameters of a small kernel (na_store_maps), which copy them by value at
+// launch: no host buffer is read after the call returns.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -58,15 +61,29 @@ constexpr size_t kOffPartial = kOffHe + na_align((size_t)kNaSlots * kNaMaxInter 
 constexpr size_t kOffIo = kOffPartial + na_align((size_t)kNaUnits * moe::kPartialFloats * 4);
 constexpr size_t kOffMaps = kOffIo + na_align((size_t)(kNaMaxLayers - 1) * kNaMaxBatch * kNaMaxHidden * 2);
 // the regions below must be zero when a step starts; each call clears them
-constexpr size_t kOffZero = kOffMaps + na_align(sizeof(CUtensorMap) * moe::TM_COUNT * kNaMaxLayers);
+constexpr size_t kOffZero = kOffMaps + na_align(sizeof(CUtensorMap) * (moe::TM_WSD + 1) * kNaMaxLayers);
 constexpr size_t kOffCtr = kOffZero;
 constexpr size_t kOffTickets = kOffCtr + na_align(moe::CTR_COUNT * 4);
 constexpr size_t kOffPairDone = kOffTickets + na_align((size_t)kNaTiles * 4);
-constexpr size_t kOffStatus = kOffPairDone + na_align((size_t)moe::kMaxSlots * 4);
-constexpr size_t kScratchBytes = kOffStatus + 256;
+constexpr size_t kScratchBytes = kOffPairDone + na_align((size_t)moe::kMaxSlots * 4);
 constexpr size_t kZeroBytes = kScratchBytes - kOffZero;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
+
+// The CUDA-core kernel's descriptors of up to kNaMaxLayers layers, by value.
+constexpr int kNaMapsPerLayer = moe::TM_WSD + 1;
+struct NaMaps {
+  CUtensorMap m[kNaMapsPerLayer * kNaMaxLayers];
+};
+static_assert(sizeof(NaMaps) + 64 <= 4096, "descriptors fit the kernel parameter space");
+
+// Copies the descriptors of n maps from the kernel parameters into dst (global).
+__global__ void na_store_maps(const __grid_constant__ NaMaps src, int n, CUtensorMap* dst) {
+  const int words = n * (int)(sizeof(CUtensorMap) / 16);
+  const uint4* s4 = reinterpret_cast<const uint4*>(&src.m[0]);
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  for (int i = threadIdx.x; i < words; i += blockDim.x) d4[i] = s4[i];
+}
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -140,7 +157,8 @@ int na_encode(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) 
 extern "C" int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_decode_layer_weights* layers,
                                        const void* x_in, void* y_out, int batch, int top_k, void* stream,
                                        int* device_status) {
-  if (!cfg || !layers || !x_in || !y_out || x_in == y_out) return MOE_ERR_INVALID_ARG;
+  if (!cfg || !layers || !x_in || !y_out || x_in == y_out || !device_status) return MOE_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(device_status) & 3u) return MOE_ERR_INVALID_ARG;
   const moe_decode_config c = *cfg;
   if (c.n_layers < 1 || batch < 1 || top_k < 1 || top_k > c.n_experts || !(c.eps >= 0.0f))
     return MOE_ERR_INVALID_ARG;
@@ -158,12 +176,13 @@ extern "C" int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_d
   if (rc != MOE_OK) return rc;
 
   const int H = c.hidden, E = c.n_experts, I = c.inter, Is = c.shared_inter, L = c.n_layers;
-  CUtensorMap maps[moe::TM_COUNT * kNaMaxLayers];
+  NaMaps maps;
+  memset(&maps, 0, sizeof maps);
   for (int l = 0; l < L; ++l) {
     const moe_decode_layer_weights& w = layers[l];
     if (!w.gamma || (reinterpret_cast<uintptr_t>(w.gamma) & 15u) || (reinterpret_cast<uintptr_t>(w.router_bias) & 3u))
       return MOE_ERR_INVALID_ARG;
-    CUtensorMap* m = maps + l * moe::TM_COUNT;
+    CUtensorMap* m = maps.m + l * kNaMapsPerLayer;
     if (na_encode(&m[moe::TM_WR], w.w_router, (uint64_t)E, (uint64_t)H) != MOE_OK ||
         na_encode(&m[moe::TM_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H) != MOE_OK ||
         na_encode(&m[moe::TM_WU], w.w_up, (uint64_t)E * I, (uint64_t)H) != MOE_OK ||
@@ -175,11 +194,11 @@ extern "C" int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_d
   }
   cudaStream_t s = (cudaStream_t)stream;
   unsigned char* base = st->scratch;
-  // the descriptors are staged by the copy before this call returns; the counters,
-  // tickets and status start at zero
-  if (cudaMemcpyAsync(base + kOffMaps, maps, sizeof(CUtensorMap) * moe::TM_COUNT * L, cudaMemcpyHostToDevice,
-                      s) != cudaSuccess ||
-      cudaMemsetAsync(base + kOffZero, 0, kZeroBytes, s) != cudaSuccess)
+  // the descriptors travel in na_store_maps' parameters (by value, at launch); the
+  // counters and tickets start at zero
+  CUtensorMap* d_maps_w = reinterpret_cast<CUtensorMap*>(base + kOffMaps);
+  na_store_maps<<<1, 128, 0, s>>>(maps, kNaMapsPerLayer * L, d_maps_w);
+  if (cudaGetLastError() != cudaSuccess || cudaMemsetAsync(base + kOffZero, 0, kZeroBytes, s) != cudaSuccess)
     return MOE_ERR_CUDA;
 
   const CUtensorMap* d_maps = reinterpret_cast<const CUtensorMap*>(base + kOffMaps);
@@ -197,7 +216,7 @@ extern "C" int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_d
     p.x = l == 0 ? (const uint16_t*)x_in : io;
     p.y = l == L - 1 ? (uint16_t*)y_out : io;
     const moe_decode_layer_weights& w = layers[l];
-    p.tmaps = d_maps + l * moe::TM_COUNT;
+    p.tmaps = d_maps + l * kNaMapsPerLayer;
     p.gamma = (const uint16_t*)w.gamma;
     p.bias = w.router_bias;
     if (l + 1 < L) {
@@ -219,7 +238,7 @@ extern "C" int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_d
     p.ctr = reinterpret_cast<uint32_t*>(base + kOffCtr);
     p.tickets = reinterpret_cast<uint32_t*>(base + kOffTickets);
     p.pair_done = reinterpret_cast<uint32_t*>(base + kOffPairDone);
-    p.status = device_status ? device_status : reinterpret_cast<int*>(base + kOffStatus);
+    p.status = device_status;
     p.max_units = kNaUnits;
     p.max_tiles = kNaTiles;
     p.wait_ns = 2000ull * 1000000ull;

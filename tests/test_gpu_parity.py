@@ -17,8 +17,7 @@ import pytest
 import oracle
 import synth
 
-from harness import (bf, chained_flips, check_layer, check_y, gpu_layer_outputs, make_handle, oracle_rows,
-                     routing_oracle, run_gpu)
+from harness import bf, check_all, gpu_layer_outputs, make_handle, routing_oracle, run_gpu
 
 torch = pytest.importorskip("torch")
 
@@ -82,18 +81,9 @@ def run_and_check(wl, rows=None, handle=None, layers=None, tc_min_batch=None):
     out = run_gpu(h, wl, x, n_layers=wl.layers)
     assert out["status"] == 0, f"device status {out['status']}"
     rows = list(range(wl.B)) if rows is None else rows
-    orc = oracle_rows(wl, x, rows, n_layers=wl.layers)
-    route = orc
-    if wl.layers > 1:
-        mid = gpu_layer_outputs(wl, layers, x, tc_min_batch=_switch_of(h, wl))
-        route = routing_oracle(wl, x, rows, wl.layers, mid)
-    skip = chained_flips(out["layers"], orc, rows, wl.k, tag=wl.name)
-    for l in range(wl.layers):
-        ties = check_layer(out["layers"][l], route[l], rows, wl.k, tag=f"{wl.name} layer {l}")
-        skip |= {rows.index(b) for b in ties}
-        idx = out["layers"][l]["idx"]
-        assert out["layers"][l]["U"] == len(np.unique(idx)), "unique-expert count"
-    err = check_y(out["y"][rows], orc, tag=wl.name, skip=skip)
+    mid = gpu_layer_outputs(wl, layers, x, tc_min_batch=_switch_of(h, wl)) if wl.layers > 1 else []
+    route = routing_oracle(wl, x, rows, wl.layers, mid)
+    err, _ = check_all(wl, out, x, rows, route, tag=wl.name)
     if handle is None:
         h.close()
     return out, err
@@ -195,9 +185,7 @@ def test_tc_one_row_steps_never_take_an_earlier_steps_choices():
         out = run_gpu(h, wl, x)
         assert out["status"] == 0, f"input {v}: device status {out['status']}"
         rows = list(range(B))
-        orc = oracle_rows(wl, x, rows)
-        ties = check_layer(out["layers"][0], orc[0], rows, wl.k, tag=f"input {v}")
-        check_y(out["y"], orc, tag=f"input {v}", skip={rows.index(b) for b in ties})
+        check_all(wl, out, x, rows, routing_oracle(wl, x, rows, 1, []), tag=f"input {v}")
         if B == 1:
             chosen = set(out["layers"][0]["idx"][0].tolist())
             changed += prev is not None and chosen != prev
@@ -336,42 +324,26 @@ def test_smaller_batch_and_k_than_configured():
 
 
 FULL = [(1, None), (2, None), (3, None), (4, None), (1, 0), (2, 0), (3, 0), (4, 0)]
-SAMPLE_ROWS = {1: [0], 2: [0, 5], 3: [0, 37, 63], 4: [0, 9, 31]}
 
 
 @pytest.mark.parametrize("cfg,tc_min_batch", FULL,
                          ids=[f"config{c}-" + {None: "switch", 0: "cuda_core", 1: "tensor_core"}[t] for c, t in FULL])
 def test_full_size_workload(cfg, tc_min_batch):
+    """A measured workload at full size, every row: indices = the oracle's top-k of the
+    GPU's own logits, softmax weights, logits against the oracle router (each layer on
+    the input it received), and the output of every row against the oracle chain on
+    the GPU's selections."""
     wl = synth.WORKLOADS[cfg]
     layers = _layers(wl)
     h = make_handle(wl, layers, tc_min_batch=tc_min_batch)
     x = wl.x_host()
     out = run_gpu(h, wl, x, n_layers=wl.layers)
     assert out["status"] == 0
-    assert h.launches_per_step() == wl.layers
-    # every row: indices equal the oracle's top-k of the GPU's own logits; weights sum to 1
+    assert h.launches_per_step() == h.launches_per_step_expected()
     for l in range(wl.layers):
-        lay = out["layers"][l]
-        for b in range(wl.B):
-            assert np.array_equal(lay["idx"][b], oracle.topk(lay["logits"][b], wl.k))
-        np.testing.assert_allclose(lay["w"].sum(axis=1), 1.0, atol=1e-5)
-        assert lay["U"] == len(np.unique(lay["idx"]))
-    # every row of layer 0: logits against the oracle router
-    gamma, wr, bias = wl.gamma_host(0), wl.w_router_host(0), wl.bias_host(0)
-    for b in range(wl.B):
-        lo = oracle.router(oracle.rmsnorm(x[b], gamma, wl.eps), wr, bias)
-        lg = out["layers"][0]["logits"][b].astype(np.float64)
-        assert np.max(np.abs(lg - lo)) <= 1e-3 * np.max(np.abs(lo))
-    # sampled rows: the whole layer stack against the oracle
-    rows = SAMPLE_ROWS[cfg]
-    orc = oracle_rows(wl, x, rows, n_layers=wl.layers)
-    route = orc
-    if wl.layers > 1:
-        mid = gpu_layer_outputs(wl, layers, x, tc_min_batch=_switch_of(h, wl))
-        route = routing_oracle(wl, x, rows, wl.layers, mid)
-    skip = chained_flips(out["layers"], orc, rows, wl.k, tag=wl.name)
-    for l in range(wl.layers):
-        ties = check_layer(out["layers"][l], route[l], rows, wl.k, tag=f"{wl.name} layer {l}")
-        skip |= {rows.index(b) for b in ties}
-    check_y(out["y"][rows], orc, tag=wl.name, skip=skip)
+        np.testing.assert_allclose(out["layers"][l]["w"].sum(axis=1), 1.0, atol=1e-5)
+    rows = list(range(wl.B))
+    mid = gpu_layer_outputs(wl, layers, x, tc_min_batch=_switch_of(h, wl)) if wl.layers > 1 else []
+    route = routing_oracle(wl, x, rows, wl.layers, mid)
+    check_all(wl, out, x, rows, route, tag=wl.name)
     h.close()
