@@ -10,8 +10,11 @@ bytes of all ranks / max-over-ranks time); `ms_per_step` is the step time.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config C] [--impl ours|reference]
 
 One step = one moe_decode_step call (one persistent launch per layer) on a
-batch from a pool of 32 seeded inputs, with L2 flushed (256 MB write) between
-timed steps. Under torchrun every rank runs an independent replica (the path
+batch from a pool of 32 seeded inputs. Every step streams more weight bytes than
+the 126 MB L2 holds, and one-layer workloads alternate between two independently
+seeded weight sets, so no step finds the previous step's weights in L2; the
+same steps with a 256 MB L2-flush write between them are reported beside it
+(l2_flushed). Under torchrun every rank runs an independent replica (the path
 does not shard; no data-path collective): weak scaling.
 """
 import argparse
@@ -306,41 +309,59 @@ def step_stats(step_ms):
             "us_per_step_p90": round(float(np.percentile(a, 90)), 2)}
 
 
+L2_PROTOCOL = ("no flush: every step streams more weight bytes than the 126 MB L2, and single-layer "
+               "workloads alternate between two independently seeded weight sets (two layers), so no "
+               "step finds the previous step's weights in L2 (a decode step runs its layers in turn)")
+
+
 class ConfigRun:
-    """One workload on this rank's GPU: its weights (generated on the device), a handle,
-    a pool of POOL seeded input batches resident in HBM and the L2-flush buffer."""
+    """One workload on this rank's GPU: its weights (generated on the device; a one-layer
+    workload gets two independently seeded weight sets, used alternately, like two layers
+    of a model), a handle per set, a pool of POOL seeded input batches resident in HBM,
+    and an L2-flush buffer for the secondary, flushed timing."""
 
     def __init__(self, wl, device, tc_min_batch=None):
+        import dataclasses
+
         import torch
 
         import moe_decode_persistent_b200 as mdp
 
         self.wl = wl
         self.dev = f"cuda:{device}"
-        self.layers = [wl.device_layer(l, device=self.dev) for l in range(wl.layers)]
-        self.h = mdp.MoeDecode(wl.H, wl.E, wl.k, wl.I, wl.Is, wl.B, self.layers, eps=wl.eps, device=device)
-        if tc_min_batch is not None:
-            self.h.set_tc_min_batch(tc_min_batch)
+        variants = [wl] if wl.layers > 1 else [wl, dataclasses.replace(wl, seed=wl.seed + 100)]
+        self.sets = []
+        for v in variants:
+            layers = [v.device_layer(l, device=self.dev) for l in range(wl.layers)]
+            h = mdp.MoeDecode(wl.H, wl.E, wl.k, wl.I, wl.Is, wl.B, layers, eps=wl.eps, device=device)
+            if tc_min_batch is not None:
+                h.set_tc_min_batch(tc_min_batch)
+            self.sets.append((layers, h))
+        self.h = self.sets[0][1]
         self.kernel_path = "tensor_core" if self.h.step_path(wl.B) == mdp.PATH_TENSOR_CORE else "cuda_core"
         self.pool_host = wl.x_pool_host(POOL)
         self.pool = torch.from_numpy(self.pool_host.view(np.int16)).view(torch.bfloat16).to(self.dev)
         self.y = torch.empty((wl.B, wl.H), dtype=torch.bfloat16, device=self.dev)
         self.flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=self.dev)
 
-    def steps(self, K, W, stream, barrier, host=None, launch_log=None):
+    def steps(self, K, W, stream, barrier, host=None, launch_log=None, flush=False):
         """W untimed warm-up steps immediately followed (no idle gap, so the clocks stay
-        up) by K timed steps, each preceded by an L2 flush; CUDA events on `stream`
-        bracket every step. host = (x_host, y_host): the host-buffer entry point instead.
-        Returns per-step ms and the unique-expert count of every timed step and layer."""
+        up) by K timed steps; step i runs weight set i mod (number of sets); CUDA events
+        on `stream` bracket every step. flush: a 256 MB write before every step (the
+        secondary, flushed figure). host = (x_host, y_host): the host-buffer entry point
+        instead. Returns per-step ms and the unique-expert count of every timed step and
+        layer."""
         import torch
 
-        wl, h = self.wl, self.h
+        wl = self.wl
         nu = torch.zeros((W + K, wl.layers), dtype=torch.int32, device=self.dev)
         dbg = lambda i: [dict(n_unique=nu[i, l:l + 1]) for l in range(wl.layers)]
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
 
         def one(i, timed):
-            self.flush.zero_()
+            h = self.sets[i % len(self.sets)][1]
+            if flush:
+                self.flush.zero_()
             if timed:
                 ev[i - W][0].record(stream)
             if host is None:
@@ -362,11 +383,12 @@ class ConfigRun:
         torch.cuda.synchronize()
         barrier()
         self.wall = time.perf_counter() - wall0
-        status = h.status()
-        if status != 0:
-            import moe_decode_persistent_b200 as mdp
+        for _, h in self.sets:
+            status = h.status()
+            if status != 0:
+                import moe_decode_persistent_b200 as mdp
 
-            raise RuntimeError(f"{wl.name}: device status {status}: {mdp.strerror(status)}")
+                raise RuntimeError(f"{wl.name}: device status {status}: {mdp.strerror(status)}")
         U = nu.cpu().numpy()
         if launch_log is not None:
             for i in range(W + K):
@@ -379,8 +401,9 @@ class ConfigRun:
     def close(self):
         import torch
 
-        self.h.close()
-        del self.layers, self.pool, self.flush, self.y
+        for _, h in self.sets:
+            h.close()
+        del self.sets, self.h, self.pool, self.flush, self.y
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
 
@@ -431,6 +454,12 @@ def run_ours(args, wl):
     tot_bytes, max_ms = aggregate(sum(bytes_steps), local_ms, world)
     value = tot_bytes / (max_ms * 1e-3) / 1e9
     achieved = sum(bytes_steps) / (local_ms * 1e-3) / 1e9  # this rank's launching stream
+    # secondary figure: the same steps with a 256 MB write between steps (which also
+    # evicts the kernel's instructions and leaves L2 full of dirty lines to write back)
+    f_ms, fU = run.steps(K, W, stream, barrier, flush=True)
+    f_bytes, f_max = aggregate(sum(step_bytes(wl, list(fU[i])) for i in range(K)), float(sum(f_ms)), world)
+    l2_flushed = {"value": round(f_bytes / (f_max * 1e-3) / 1e9, 2), "unit": "GB/s", **step_stats(f_ms),
+                  "l2": "flushed between timed steps (256 MB write)"}
 
     # end to end through the host-buffer entry point: H2D x, step, D2H y per step
     e2e = None
@@ -449,8 +478,9 @@ def run_ours(args, wl):
         "warmup": W, "ms_per_step": round(max_ms / K, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded counter-hash weights ~N(0,1/sqrt(fan_in)) and inputs, no trained weights",
-        "config": dict(workload_config(wl, "flushed between timed steps (256 MB write)"), kernel_path=run.kernel_path),
+        "config": dict(workload_config(wl, L2_PROTOCOL), kernel_path=run.kernel_path),
         **step_stats(step_ms),
+        "l2_flushed": l2_flushed,
         "tokens_per_s": round(world * wl.B * K / (max_ms * 1e-3), 1),
         "unique_experts_mean": float(U.mean()),
         "bytes_per_step_mean": float(np.mean(bytes_steps)),
@@ -480,7 +510,7 @@ def run_ours(args, wl):
         c_tot, c_max = aggregate(sum(c_bytes), c_local, world)
         c_ach = sum(c_bytes) / (c_local * 1e-3) / 1e9
         per_config[cw.name] = {
-            "config": workload_config(cw, "flushed between timed steps (256 MB write)") | {"kernel_path": r.kernel_path},
+            "config": workload_config(cw, L2_PROTOCOL) | {"kernel_path": r.kernel_path},
             "value": round(c_tot / (c_max * 1e-3) / 1e9, 2), "unit": "GB/s",
             **step_stats(c_ms),
             "tokens_per_s": round(world * cw.B * K / (c_max * 1e-3), 1),

@@ -150,7 +150,7 @@ int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms)
 
 /* Per-CTA timeline of later steps (profiling aid). trace: NULL to switch it off,
  * or a device buffer of n_layers * moe_decode_trace_slots(h) uint64 values,
- * 8-byte aligned, owned by the caller. Per layer and CTA, 40 slots: global-timer
+ * 8-byte aligned, owned by the caller. Per layer and CTA, 48 slots: global-timer
  * stamps (ns) of the kernel start, normalised rows acquired, schedule seen, first
  * expert and first down stage issued, last stage issued, last stage consumed, last
  * epilogue, exit; then clock64 sums of the producer's waits for ring slots, for
@@ -166,14 +166,18 @@ int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms)
  * top-k chosen (34) and its cycle count (35), the unique experts placed (36),
  * the pairs sorted (37), and clock64 at the kernel start (38): there the
  * routing stamps (slots 26-30, 32-34, 36, 37) are clock64 values of the CTA's
- * SM, comparable with slot 38 of the same CTA only (slot 39 is reserved).
+ * SM, comparable with slot 38 of the same CTA only (slot 39 is reserved); then
+ * global-timer stamps of the warp roles starting after the set-up rendezvous (40),
+ * the producer's first weight tile issued (41), and, on the CTA that owns the
+ * first row it normalises, that row's squares summed (42), its sum known to every
+ * routing warp (43) and its normalised values stored (44); slots 45-47 are reserved.
  * Traced steps run a separate instance of the kernel whose stamps are global stores
  * on the routing chain: a traced batch-1 step takes several microseconds longer
  * than an untraced one, so the stamps bound the time of each hop from above and
  * step times are compared on untraced steps. */
 int moe_decode_set_trace(moe_decode_handle* h, void* trace);
 
-/* uint64 trace slots of one layer (number of CTAs x 40). */
+/* uint64 trace slots of one layer (number of CTAs x 48). */
 int moe_decode_trace_slots(const moe_decode_handle* h);
 
 /* The batch-shape switch (page post.smzdm.com/p/a6zppe4g, section "改了什么：每层

@@ -276,7 +276,8 @@ class MoeDecode:
                     "mac_reduce_cyc", "mac_loop_cyc", "prod_setup_cyc", "prod_sched_cyc",
                     "prod_loop_cyc", "router_seen", "sched_built", "topk_done", "topk_synced",
                     "unique_done", "n_published", "topk_loaded", "topk_selected", "topk_chosen",
-                    "topk_cyc", "sched_placed", "sched_sorted", "start_clk", "r39")
+                    "topk_cyc", "sched_placed", "sched_sorted", "start_clk", "r39", "roles",
+                    "first_tma", "norm_summed", "norm_reduced", "norm_stored", "r45", "r46", "r47")
 
     def trace_slots(self) -> int:
         return lib().moe_decode_trace_slots(self.handle)

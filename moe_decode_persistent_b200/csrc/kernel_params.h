@@ -176,7 +176,12 @@ enum TraceSlot {
   TR_SCHED_SORTED = 37,        // tensor-core path: pairs sorted and counted (stamp, warp 0)
   TR_START_CLK = 38,           // clock64 at kernel start (on the tensor-core path the routing
                                // stamps, slots 26-30, 32-34 and 36-37, are clock64 values)
-  kTraceSlots = 40
+  TR_ROLES = 40,               // warp roles start, after the set-up rendezvous (stamp)
+  TR_FIRST_TMA = 41,           // producer issued its first weight tile (stamp)
+  TR_NORM_SUMMED = 42,         // RMSNorm: first row's x and gamma loaded and squares summed (stamp)
+  TR_NORM_REDUCED = 43,        // RMSNorm: the row's sum of squares known to every routing warp (stamp)
+  TR_NORM_STORED = 44,         // RMSNorm: the row's n stored and fenced (stamp)
+  kTraceSlots = 48
 };
 
 constexpr unsigned kFlagJitter = 1u;

@@ -1532,7 +1532,9 @@ __device__ bool normalise_rows(const Params& p, Smem& sm, int mw, int lane, uint
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if (lane == 0) sm.red_ss[mw] = ss;
+    if (mtid == 0 && b == (int)blockIdx.x) trace_stamp<kTrace>(p, TR_NORM_SUMMED);
     if (!mac_sync(sm, mphase, p, lane)) return false;
+    if (mtid == 0 && b == (int)blockIdx.x) trace_stamp<kTrace>(p, TR_NORM_REDUCED);
     float tot = 0.0f;
 #pragma unroll
     for (int w = 0; w < kMacWarps; ++w) tot += sm.red_ss[w];
@@ -1551,6 +1553,7 @@ __device__ bool normalise_rows(const Params& p, Smem& sm, int mw, int lane, uint
     }
     fence_proxy_async_global();
     if (!mac_sync(sm, mphase, p, lane)) return false;
+    if (mtid == 0 && b == (int)blockIdx.x) trace_stamp<kTrace>(p, TR_NORM_STORED);
     if (mtid == 0 && !((p.flags & kFlagWithholdNReady) && b == 0)) red_release_add(&p.ctr[CTR_NREADY], 1u);
     if (mtid == 0) trace_stamp<kTrace>(p, TR_N_PUBLISHED);
   }
@@ -2013,7 +2016,7 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
   bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
   const int pre = sh.pre;
   int u = pr.grab();
-  bool first_expert = true, first_down = true;
+  bool first_expert = true, first_down = true, first_tma = true;
   unsigned long long c_slot = 0, c_dep = 0, c_grab = 0, c_issue = 0, c_stages = 0, c_units = 0;
   unsigned long long c_setup = 0, c_schedw = 0;
   const long long tploop0 = tclock<kTrace>();
@@ -2060,6 +2063,10 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
         h.wrow = -1;
         sm.hdr[pr.slot] = h;
         mbar_arrive_expect_tx(fb, tx);
+        if (kTrace && first_tma) {
+          trace_stamp<kTrace>(p, TR_FIRST_TMA);
+          first_tma = false;
+        }
         tma_load_2d(dst, x.tw0, ka * kTcAtomK, x.y0, fb, pol);
         if (x.nbox == 2) tma_load_2d(dst + kTcTileBytes, x.tw1, ka * kTcAtomK, x.y1, fb, pol);
       }
@@ -2727,6 +2734,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
   }
   __syncthreads();
   if constexpr (kTC) tc_fence_after();
+  if (tid == 0) trace_stamp<kTrace>(p, TR_ROLES);
 
   if (warp_id == 0) {
     Producer pr(p, sm, lane, sm.sh.nst);
