@@ -14,9 +14,9 @@
  * section "为什么解码阶段适合Megakernel"); 896 experts with 16 active per token
  * (page "vLLM 合併 Kimi K3 專用解碼：官方稱 GB300 快 1.5 到 2 倍，423 tok/s 怎麼核對",
  * section "Kimi K3 專用解碼路徑改了什麼"); a batch-shape switch between small-matrix
- * and split-K kernels, router scores, the shared expert beside the routing and an
- * L2 prefetch of the next weights (page post.smzdm.com/p/a6zppe4g, section
- * "改了什么：每层 23 个 kernel 砍到 13 个"). The layer's arithmetic is:
+ * and split-K kernels, router scores and the shared expert beside the routing (page
+ * post.smzdm.com/p/a6zppe4g, section "改了什么：每层 23 个 kernel 砍到 13 个"). The
+ * layer's arithmetic is:
  *
  *   n    = bf16(x * rsqrt(mean(x^2) + eps) * gamma)        (fp32)
  *   l[e] = n . W_r[e] (+ bias[e])                         (fp32 accumulate)
@@ -59,6 +59,9 @@ extern "C" {
 #define MOE_ERR_NONFINITE (-7)          /* device status: a router logit was NaN or infinite
                                            (the tensor-core kernel abandons the step: y undefined) */
 #define MOE_ERR_NO_MEMORY (-8)          /* workspace allocation failed */
+#define MOE_ERR_BOUNDS (-9)             /* device status, bounds-checked build only: an index
+                                           derived from the routing schedule fell outside its
+                                           buffer; the access was skipped and the step abandoned */
 
 /* Kernel paths of a step (moe_decode_step_path). */
 #define MOE_PATH_CUDA_CORE 0   /* CUDA-core GEMV units of 32 weight rows x 4 token rows */
@@ -72,8 +75,10 @@ extern "C" {
  *  shared_inter  Is  shared-expert intermediate (same rule as inter)
  *  max_batch     largest number of token rows per step (1..64)
  *  n_layers      layers run back-to-back by one step (1..8); layer l+1's input is
- *                layer l's output, and layer l prefetches layer l+1's router and
- *                shared-expert weights into L2 while it finishes
+ *                layer l's output. On the tensor-core path all layers run in ONE
+ *                persistent launch: CTAs that run out of layer l's work arm layer
+ *                l+1's first weight tiles, and each row of layer l+1 is normalised as
+ *                soon as all of its layer-l outputs exist
  *  eps           RMSNorm epsilon */
 typedef struct {
   int hidden;
@@ -121,8 +126,9 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
 /* One decode step over all layers. x_in: device bf16 [batch][H]; y_out: device
  * bf16 [batch][H] (may not alias x_in). 1 <= batch <= max_batch, 1 <= top_k <=
  * top_k_max. stream: a cudaStream_t (NULL = legacy default stream). dbg: NULL or
- * an array of n_layers debug records. Launches exactly one kernel per layer;
- * returns MOE_ERR_* for argument errors and launch failures. */
+ * an array of n_layers debug records. Launches one kernel for the whole layer stack
+ * on the tensor-core path, one per layer on the CUDA-core path (see
+ * moe_decode_step_path); returns MOE_ERR_* for argument errors and launch failures. */
 int moe_decode_step(moe_decode_handle* h, const void* x_in, void* y_out, int batch, int top_k,
                     void* stream, const moe_decode_debug* dbg);
 
@@ -139,13 +145,18 @@ int moe_decode_step_host(moe_decode_handle* h, const void* x_host, void* y_host,
  * read itself succeeded. */
 int moe_decode_get_status(moe_decode_handle* h, int* device_status);
 
-/* Number of kernel launches one moe_decode_step makes (= n_layers). */
+/* Number of kernel launches one moe_decode_step of max_batch rows makes: 1 when that
+ * step takes the tensor-core path (the whole layer stack in one launch), n_layers on
+ * the CUDA-core path. */
 int moe_decode_launches_per_step(const moe_decode_handle* h);
 
 /* Sets debug behaviour of later steps (tests only): bit 0 = per-CTA random
  * __nanosleep jitter at unit boundaries; bit 1 = withhold the normalised-row
- * ready signal so that every waiting CTA's bounded wait runs out. wait_ms is the
- * bound of every device-side wait (default 2000 ms). */
+ * ready signal so that every waiting CTA's bounded wait runs out; bit 2 (honoured
+ * by the bounds-checked build, libmoe_decode_checked.so, only) = point row 0's
+ * first choice at the first slot row past the schedule (a row inside the
+ * workspace), which that build's checks must report as MOE_ERR_BOUNDS. wait_ms is
+ * the bound of every device-side wait (default 2000 ms). */
 int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms);
 
 /* Per-CTA timeline of later steps (profiling aid). trace: NULL to switch it off,

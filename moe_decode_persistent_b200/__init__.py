@@ -17,6 +17,9 @@ import subprocess
 _HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(_HERE)
 LIB = os.path.join(_HERE, "libmoe_decode.so")
+# the same sources built with every schedule-derived index range-checked (MOE_BOUNDS_CHECK):
+# a test build, standing in for a memory checker
+CHECKED_LIB = os.path.join(_HERE, "libmoe_decode_checked.so")
 HEADER = os.path.join(ROOT, "include", "moe_decode.h")
 SOURCES = [os.path.join(_HERE, "csrc", f)
            for f in ("moe_decode_kernel.cu", "moe_decode_api.cu", "moe_decode_noalloc.cu")]
@@ -30,26 +33,35 @@ MOE_ERR_CUDA = -5
 MOE_ERR_TIMEOUT = -6
 MOE_ERR_NONFINITE = -7
 MOE_ERR_NO_MEMORY = -8
+MOE_ERR_BOUNDS = -9
 
 DEBUG_JITTER = 1
 DEBUG_WITHHOLD_NREADY = 2
+DEBUG_BAD_SLOT = 4  # bounds-checked build only
 
 PATH_CUDA_CORE = 0
 PATH_TENSOR_CORE = 1
 
 
-def nvcc_command(out: str = LIB) -> list[str]:
+def nvcc_command(out: str = LIB, checked: bool = False) -> list[str]:
     return ["nvcc", "-O3", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
             "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+            *(["-DMOE_BOUNDS_CHECK"] if checked else []),
             "-I" + os.path.join(ROOT, "include"), "-o", out, *SOURCES]
 
 
 def build(verbose: bool = False) -> None:
-    """Compile libmoe_decode.so in-tree for sm_100a."""
-    cmd = nvcc_command()
-    if verbose:
-        print(" ".join(cmd))
-    subprocess.run(cmd, check=True, cwd=_HERE)
+    """Compile libmoe_decode.so and the bounds-checked libmoe_decode_checked.so in-tree
+    for sm_100a (the two nvcc runs in parallel)."""
+    cmds = [nvcc_command(), nvcc_command(CHECKED_LIB, checked=True)]
+    procs = []
+    for cmd in cmds:
+        if verbose:
+            print(" ".join(cmd))
+        procs.append(subprocess.Popen(cmd, cwd=_HERE))
+    for cmd, pr in zip(cmds, procs):
+        if pr.wait() != 0:
+            raise subprocess.CalledProcessError(pr.returncode, cmd)
 
 
 def declared_symbols() -> list[str]:
@@ -78,15 +90,27 @@ class Debug(ctypes.Structure):
 
 
 _lib = None
+_checked_lib = None
 
 
-def lib():
-    """The loaded C-ABI library (raises if it has not been built)."""
-    global _lib
+def lib(checked: bool = False):
+    """The loaded C-ABI library (raises if it has not been built); checked: the
+    bounds-checked build."""
+    global _lib, _checked_lib
+    if checked:
+        if _checked_lib is None:
+            _checked_lib = _load(CHECKED_LIB)
+        return _checked_lib
     if _lib is None:
-        if not os.path.exists(LIB):
-            raise RuntimeError(f"{LIB} is missing: build it with moe_decode_persistent_b200.build()")
-        L = ctypes.CDLL(LIB)
+        _lib = _load(LIB)
+    return _lib
+
+
+def _load(path):
+    if True:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with moe_decode_persistent_b200.build()")
+        L = ctypes.CDLL(path)
         vp, i, u = ctypes.c_void_p, ctypes.c_int, ctypes.c_uint
         L.moe_decode_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerWeights), i,
                                         ctypes.POINTER(vp)]
@@ -116,8 +140,7 @@ def lib():
         L.moe_decode_step_noalloc.restype = i
         L.moe_decode_strerror.argtypes = [i]
         L.moe_decode_strerror.restype = ctypes.c_char_p
-        _lib = L
-    return _lib
+    return L
 
 
 def strerror(code: int) -> str:
@@ -201,11 +224,14 @@ class MoeDecode:
 
     layers: sequence of mappings with keys gamma, w_router, router_bias (or None),
     w_gate, w_up, w_down, ws_gate, ws_up, ws_down (torch tensors or device pointers).
-    The caller keeps those tensors alive for the handle's lifetime.
+    The caller keeps those tensors alive for the handle's lifetime. checked: run the
+    bounds-checked build (libmoe_decode_checked.so), which reports a schedule-derived
+    index outside its buffer as MOE_ERR_BOUNDS instead of accessing it.
     """
 
     def __init__(self, hidden, n_experts, top_k_max, inter, shared_inter, max_batch, layers,
-                 eps=1e-6, device=0):
+                 eps=1e-6, device=0, checked=False):
+        self._lib = lib(checked)  # checked: the bounds-checked test build of the library
         self.cfg = Config(hidden, n_experts, top_k_max, inter, shared_inter, max_batch,
                           len(layers), eps)
         arr = (LayerWeights * len(layers))()
@@ -213,7 +239,7 @@ class MoeDecode:
             arr[i] = LayerWeights(*(_ptr(w.get(name)) for name, _ in LayerWeights._fields_))
         self._weights_keepalive = layers
         h = ctypes.c_void_p()
-        _check(lib().moe_decode_create(ctypes.byref(self.cfg), arr, int(device), ctypes.byref(h)),
+        _check(self._lib.moe_decode_create(ctypes.byref(self.cfg), arr, int(device), ctypes.byref(h)),
                "moe_decode_create")
         self.handle = h
         self.n_layers = len(layers)
@@ -223,7 +249,7 @@ class MoeDecode:
         for name, t in (("x", x), ("y", y)):
             _check_rows(t, name, batch, self.cfg.hidden, "cuda", "moe_decode_step")
         dbg = self._debug(debug)
-        _check(lib().moe_decode_step(self.handle, _ptr(x), _ptr(y), int(batch), int(top_k),
+        _check(self._lib.moe_decode_step(self.handle, _ptr(x), _ptr(y), int(batch), int(top_k),
                                      _stream_handle(stream), dbg), "moe_decode_step")
 
     def step_host(self, x_host, y_host, batch, top_k, stream=None, debug=None) -> None:
@@ -231,7 +257,7 @@ class MoeDecode:
         for name, t in (("x_host", x_host), ("y_host", y_host)):
             _check_rows(t, name, batch, self.cfg.hidden, "cpu", "moe_decode_step_host")
         dbg = self._debug(debug)
-        _check(lib().moe_decode_step_host(self.handle, _ptr(x_host), _ptr(y_host), int(batch),
+        _check(self._lib.moe_decode_step_host(self.handle, _ptr(x_host), _ptr(y_host), int(batch),
                                           int(top_k), _stream_handle(stream), dbg),
                "moe_decode_step_host")
 
@@ -249,22 +275,22 @@ class MoeDecode:
     def status(self) -> int:
         """Device status of the completed steps (MOE_OK or a MOE_ERR_* code); clears it."""
         v = ctypes.c_int(0)
-        _check(lib().moe_decode_get_status(self.handle, ctypes.byref(v)), "moe_decode_get_status")
+        _check(self._lib.moe_decode_get_status(self.handle, ctypes.byref(v)), "moe_decode_get_status")
         return v.value
 
     def launches_per_step(self) -> int:
-        return lib().moe_decode_launches_per_step(self.handle)
+        return self._lib.moe_decode_launches_per_step(self.handle)
 
     def set_debug(self, flags: int, wait_ms: int = 2000) -> None:
-        _check(lib().moe_decode_set_debug(self.handle, int(flags), int(wait_ms)), "moe_decode_set_debug")
+        _check(self._lib.moe_decode_set_debug(self.handle, int(flags), int(wait_ms)), "moe_decode_set_debug")
 
     def set_tc_min_batch(self, min_batch: int) -> None:
         """Steps of at least min_batch rows take the tensor-core kernel (0: never)."""
-        _check(lib().moe_decode_set_tc_min_batch(self.handle, int(min_batch)), "moe_decode_set_tc_min_batch")
+        _check(self._lib.moe_decode_set_tc_min_batch(self.handle, int(min_batch)), "moe_decode_set_tc_min_batch")
 
     def step_path(self, batch: int) -> int:
         """PATH_CUDA_CORE or PATH_TENSOR_CORE: the kernel a step of `batch` rows runs."""
-        r = lib().moe_decode_step_path(self.handle, int(batch))
+        r = self._lib.moe_decode_step_path(self.handle, int(batch))
         if r < 0:
             _check(r, "moe_decode_step_path")
         return r
@@ -280,15 +306,15 @@ class MoeDecode:
                     "first_tma", "norm_summed", "norm_reduced", "norm_stored", "r45", "r46", "r47")
 
     def trace_slots(self) -> int:
-        return lib().moe_decode_trace_slots(self.handle)
+        return self._lib.moe_decode_trace_slots(self.handle)
 
     def set_trace(self, buf) -> None:
         """buf: None, or a device uint64/int64 tensor of n_layers * trace_slots() values."""
-        _check(lib().moe_decode_set_trace(self.handle, _ptr(buf)), "moe_decode_set_trace")
+        _check(self._lib.moe_decode_set_trace(self.handle, _ptr(buf)), "moe_decode_set_trace")
 
     def close(self) -> None:
         if getattr(self, "handle", None):
-            lib().moe_decode_destroy(self.handle)
+            self._lib.moe_decode_destroy(self.handle)
             self.handle = None
 
     def __del__(self):

@@ -31,18 +31,23 @@ enum TensorMapSlot {
   TM_COUNT = 17
 };
 
-// Global counters of one step (reset by the last CTA of every launch, except the epoch).
+// Counters of one layer step (reset by the last CTA of every launch, except the epoch).
+// A launch that runs several layers has one block per layer (Params::ctr) and keeps
+// CTR_EXIT, CTR_ABORT and CTR_EPOCH in the first layer's block (Params::gctr).
 enum Counter {
   CTR_QUEUE = 0,   // next unit of work
-  CTR_EXIT = 1,    // CTAs finished
+  CTR_EXIT = 1,    // CTAs finished (launch-wide)
   CTR_NREADY = 2,  // normalised rows published
   CTR_ROUTER = 3,  // router tiles finished (logits published)
   CTR_HS = 4,      // shared gate/up tiles finished
-  CTR_ABORT = 5,   // non-zero once any CTA gave up a wait
+  CTR_ABORT = 5,   // non-zero once any CTA gave up a wait (launch-wide)
   CTR_TOPK = 6,    // tensor-core path: rows whose top-k choices are published
   CTR_EPOCH = 7,   // launches completed on this workspace (never reset): tags the choices
   CTR_COUNT = 8
 };
+
+// Layers one launch can run back to back (the tensor-core path's fused stack).
+constexpr int kMaxFusedLayers = 8;
 
 // Work-unit limits that size the workspace.
 constexpr int kBoxRows = 32;           // weight rows per TMA box (one output tile)
@@ -101,9 +106,6 @@ struct Params {
   const CUtensorMap* tmaps;  // TM_COUNT maps in global memory
   const uint16_t* gamma;     // bf16 [H]
   const float* bias;         // fp32 [E] or nullptr
-  // next layer's router/shared weights (L2 prefetch), nullptr when last layer
-  const void* pf_ptr[4];
-  unsigned long long pf_bytes[4];
   // workspace
   uint16_t* n;           // bf16 [maxB][H]
   float* logits;         // fp32 [maxB][E]
@@ -119,11 +121,19 @@ struct Params {
                          // (tag << 32 | expert) and (tag << 32 | softmax weight bits)
   uint32_t* row_tix;     // [H/256 tile pairs][max_batch]: down contributions arrived per row
   unsigned row_tix_count;
-  uint32_t* ctr;         // [CTR_COUNT]
+  uint32_t* ctr;         // [CTR_COUNT] this layer's counters
+  uint32_t* gctr;        // the launch's counter block (CTR_EXIT, CTR_ABORT, CTR_EPOCH); == ctr
+                         // when the launch runs one layer
+  int layer;             // index of this layer within its launch (tags its published choices)
+  const uint32_t* rows_in;  // fused stack, layer >= 1: per token row, the previous layer's tile
+                            // pairs of output combined (the row is input once all H/256 are)
+  uint32_t* rows_out;       // fused stack, all layers but the last: this layer's per-row count
   uint32_t* tickets;     // [max_tiles]
   uint32_t* pair_done;   // [kMaxSlots]
   int* status;           // device status word
   unsigned max_units, max_tiles;
+  unsigned cap_slots;       // max_batch x top_k_max: slot rows the workspace holds per split
+  unsigned cap_dpart_rows;  // rows of dpart (slot rows + max_batch)
   // debug outputs (nullable)
   float* dbg_logits;
   int* dbg_idx;
@@ -132,6 +142,12 @@ struct Params {
   unsigned flags;        // bit 0: jitter, bit 1: withhold the n-ready signal
   unsigned long long wait_ns;
   unsigned long long* trace;  // nullable: [gridDim.x][kTraceSlots] timeline (see TraceSlot)
+};
+
+// Parameters of a launch that runs L layers back to back (tensor-core path).
+struct FusedParams {
+  Params layer[kMaxFusedLayers];
+  int L;
 };
 
 // Per-CTA timeline of one launch (global-timer ns stamps; *_CYC slots are clock64 sums).
@@ -186,5 +202,9 @@ enum TraceSlot {
 
 constexpr unsigned kFlagJitter = 1u;
 constexpr unsigned kFlagWithholdNReady = 2u;
+// Bounds-checked build only: after the schedule is built, row 0's first choice points at
+// the first slot row past the schedule (inside the workspace, so an unchecked read
+// stays in bounds); the combine's check must report MOE_ERR_BOUNDS.
+constexpr unsigned kFlagBadSlot = 4u;
 
 }  // namespace moe

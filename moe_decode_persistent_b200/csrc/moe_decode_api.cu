@@ -18,6 +18,8 @@ size_t tc_smem_bytes();
 int tc_threads_per_cta();
 const void* tc_kernel_fn();
 const void* tc_kernel_fn_trace();
+const void* fused_kernel_fn();
+const void* fused_kernel_fn_trace();
 }  // namespace moe
 
 using moe::Params;
@@ -47,9 +49,10 @@ struct moe_decode_handle {
   uint64_t* tk_pub;
   uint32_t* row_tix;
   unsigned row_tix_count;
-  uint32_t* ctr;
+  uint32_t* ctr;         // [n_layers][CTR_COUNT] (a fused launch uses one block per layer)
   uint32_t* tickets;
-  uint32_t* pair_done;
+  uint32_t* pair_done;   // [n_layers][kMaxSlots]
+  uint32_t* rows_done;   // [n_layers][max_batch]: output tile pairs combined per row (fused launch)
   int* status;
   uint16_t* layer_io;    // [n_layers - 1][max_batch][H] intermediate outputs
   uint16_t* x_stage;     // [max_batch][H] host-step staging
@@ -119,6 +122,7 @@ const char* moe_decode_strerror(int code) {
     case MOE_ERR_TIMEOUT: return "device wait timed out";
     case MOE_ERR_NONFINITE: return "non-finite router logit";
     case MOE_ERR_NO_MEMORY: return "workspace allocation failed";
+    case MOE_ERR_BOUNDS: return "schedule-derived index out of bounds (bounds-checked build)";
     default: return "unknown error";
   }
 }
@@ -171,6 +175,10 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
     e = cudaFuncSetAttribute(moe::tc_kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::tc_kernel_fn_trace(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::fused_kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::fused_kernel_fn_trace(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     int tc_per_sm = 0;
     if (e == cudaSuccess)
       e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&tc_per_sm, moe::tc_kernel_fn(), moe::tc_threads_per_cta(),
@@ -292,9 +300,10 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   const size_t o_dpart = carve(dpart_floats * 4);
   const size_t o_tkp = carve((size_t)maxSlots * 16);
   const size_t o_rtix = carve(row_tix_n * 4 + 4);
-  const size_t o_ctr = carve(moe::CTR_COUNT * 4);
+  const size_t o_ctr = carve((size_t)L * moe::CTR_COUNT * 4);
   const size_t o_tix = carve((size_t)h->max_tiles * 4);
-  const size_t o_pd = carve(moe::kMaxSlots * 4);
+  const size_t o_pd = carve((size_t)L * moe::kMaxSlots * 4);
+  const size_t o_rows = carve((size_t)L * maxB * 4);
   const size_t o_status = carve(16);
   const size_t o_io = carve((size_t)(L > 1 ? L - 1 : 1) * maxB * H * 2);
   const size_t o_xs = carve((size_t)maxB * H * 2);
@@ -323,6 +332,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   h->ctr = (uint32_t*)(b + o_ctr);
   h->tickets = (uint32_t*)(b + o_tix);
   h->pair_done = (uint32_t*)(b + o_pd);
+  h->rows_done = (uint32_t*)(b + o_rows);
   h->status = (int*)(b + o_status);
   h->layer_io = (uint16_t*)(b + o_io);
   h->x_stage = (uint16_t*)(b + o_xs);
@@ -365,15 +375,24 @@ static bool use_tc(const moe_decode_handle* h, int batch) {
   return h->tc_capable && h->tc_min_batch > 0 && batch >= h->tc_min_batch;
 }
 
+// A tensor-core step of several layers runs them all in one launch (the fused kernel);
+// otherwise one launch per layer.
+static bool fused_step(const moe_decode_handle* h, int batch) {
+  return use_tc(h, batch) && h->cfg.n_layers > 1;
+}
+
 static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, int batch, int top_k,
                          cudaStream_t stream, const moe_decode_debug* dbg) {
   const moe_decode_config& c = h->cfg;
   const int L = c.n_layers;
   const bool tc = use_tc(h, batch);
+  const bool fused = fused_step(h, batch);
   const int nkH = c.hidden / moe::kTcAtomK;
+  moe::FusedParams f;
+  memset(&f, 0, sizeof f);
+  f.L = L;
   for (int l = 0; l < L; ++l) {
-    Params p;
-    memset(&p, 0, sizeof p);
+    Params& p = f.layer[l];
     p.H = c.hidden;
     p.E = c.n_experts;
     p.I = c.inter;
@@ -387,17 +406,6 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     p.tmaps = h->d_tmaps + l * moe::TM_COUNT;
     p.gamma = (const uint16_t*)w.gamma;
     p.bias = w.router_bias;
-    if (l + 1 < L) {
-      const moe_decode_layer_weights& nx = h->layers[l + 1];
-      p.pf_ptr[0] = nx.w_router;
-      p.pf_bytes[0] = (unsigned long long)c.n_experts * c.hidden * 2;
-      p.pf_ptr[1] = nx.ws_gate;
-      p.pf_bytes[1] = (unsigned long long)c.shared_inter * c.hidden * 2;
-      p.pf_ptr[2] = nx.ws_up;
-      p.pf_bytes[2] = (unsigned long long)c.shared_inter * c.hidden * 2;
-      p.pf_ptr[3] = nx.ws_down;
-      p.pf_bytes[3] = (unsigned long long)c.shared_inter * c.hidden * 2;
-    }
     p.n = h->n;
     p.logits = h->logits;
     p.hs = h->hs;
@@ -415,12 +423,22 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
       p.row_tix = h->row_tix;
       p.row_tix_count = h->row_tix_count;
     }
-    p.ctr = h->ctr;
+    // one layer per launch: every launch uses the first counter block; a fused launch
+    // gives each layer its own block, completion flags and row counts
+    p.ctr = h->ctr + (fused ? (size_t)l * moe::CTR_COUNT : 0);
+    p.gctr = h->ctr;
+    p.layer = fused ? l : 0;
     p.tickets = h->tickets;
-    p.pair_done = h->pair_done;
+    p.pair_done = h->pair_done + (fused ? (size_t)l * moe::kMaxSlots : 0);
+    if (fused) {
+      p.rows_in = l > 0 ? h->rows_done + (size_t)(l - 1) * c.max_batch : nullptr;
+      p.rows_out = l + 1 < L ? h->rows_done + (size_t)l * c.max_batch : nullptr;
+    }
     p.status = h->status;
     p.max_units = h->max_units;
     p.max_tiles = h->max_tiles;
+    p.cap_slots = (unsigned)(c.max_batch * c.top_k_max);
+    p.cap_dpart_rows = (unsigned)(c.max_batch * c.top_k_max + c.max_batch);
     if (dbg) {
       p.dbg_logits = dbg[l].logits;
       p.dbg_idx = dbg[l].topk_idx;
@@ -430,12 +448,21 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     p.flags = h->flags;
     p.wait_ns = h->wait_ns;
     p.trace = h->trace ? h->trace + (size_t)l * h->num_sms * moe::kTraceSlots : nullptr;
+    if (fused) continue;
     void* args[] = {&p};
     const void* fn = tc ? (h->trace ? moe::tc_kernel_fn_trace() : moe::tc_kernel_fn())
                         : (h->trace ? moe::kernel_fn_trace() : moe::kernel_fn());
     const int threads = tc ? moe::tc_threads_per_cta() : moe::threads_per_cta();
     const size_t smem = tc ? moe::tc_smem_bytes() : moe::smem_bytes();
     cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(h->num_sms), dim3(threads), args, smem, stream);
+    if (e == cudaErrorCooperativeLaunchTooLarge) return MOE_ERR_COOPERATIVE;
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  if (fused) {
+    void* args[] = {&f};
+    const void* fn = h->trace ? moe::fused_kernel_fn_trace() : moe::fused_kernel_fn();
+    cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(h->num_sms), dim3(moe::tc_threads_per_cta()), args,
+                                                moe::tc_smem_bytes(), stream);
     if (e == cudaErrorCooperativeLaunchTooLarge) return MOE_ERR_COOPERATIVE;
     if (e != cudaSuccess) return MOE_ERR_CUDA;
   }
@@ -485,7 +512,8 @@ int moe_decode_get_status(moe_decode_handle* h, int* device_status) {
 }
 
 int moe_decode_launches_per_step(const moe_decode_handle* h) {
-  return h ? h->cfg.n_layers : MOE_ERR_INVALID_ARG;
+  if (!h) return MOE_ERR_INVALID_ARG;
+  return fused_step(h, h->cfg.max_batch) ? 1 : h->cfg.n_layers;
 }
 
 int moe_decode_set_debug(moe_decode_handle* h, unsigned flags, unsigned wait_ms) {

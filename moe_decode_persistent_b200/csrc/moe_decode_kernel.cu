@@ -34,9 +34,11 @@
 // the shared expert's down tiles) -- all streamed while the routing resolves (page
 // post.smzdm.com/p/a6zppe4g, same section: the shared expert moved beside the router
 // computation) -- then expert gate/up and down units over the unique selected experts
-// only (each selected expert's weights stream once however many rows chose it). The
-// next layer's router and shared weights are prefetched into L2 by CTAs that run out of
-// work (same section, the last item).
+// only (each selected expert's weights stream once however many rows chose it). A
+// stack of layers runs in one launch on the tensor-core path: CTAs that run out of one
+// layer's work arm the next layer's first weight tiles while the layer drains. (The
+// same section's L2 prefetch of the next layer's weights was measured here and did not
+// pay: it is not done.)
 //
 // Memory ordering: data produced inside the kernel (normalised rows, logits, h,
 // partials, published choices) is read only after an acquire on the counter that
@@ -248,12 +250,27 @@ __device__ __forceinline__ void record_error(const Params& p, int code) {
 
 __device__ __forceinline__ void record_abort(const Params& p, int code) {
   record_error(p, code);
-  atomicExch(&p.ctr[CTR_ABORT], 1u);
+  atomicExch(&p.gctr[CTR_ABORT], 1u);
 }
 
 __device__ __forceinline__ bool abort_seen(const Params& p) {
-  return ld_relaxed_gpu(&p.ctr[CTR_ABORT]) != 0u;
+  return ld_relaxed_gpu(&p.gctr[CTR_ABORT]) != 0u;
 }
+
+// Bounds-checked build (compiled with -DMOE_BOUNDS_CHECK into libmoe_decode_checked.so):
+// every global or shared-memory index that the routing schedule produces is checked
+// before its access; a failed check records MOE_ERR_BOUNDS, raises the abort flag (every
+// CTA unwinds) and the access is skipped. In the product build IDX_OK is `true` and the
+// condition is not evaluated.
+#ifdef MOE_BOUNDS_CHECK
+__device__ __noinline__ bool bounds_fail(const Params& p) {
+  record_abort(p, MOE_ERR_BOUNDS);
+  return false;
+}
+#define IDX_OK(p, cond) ((cond) || ::moe::bounds_fail(p))
+#else
+#define IDX_OK(p, cond) true
+#endif
 
 
 // Bounded wait on an mbarrier phase by one thread (suspended while waiting). Between
@@ -323,10 +340,11 @@ __device__ bool wait_counter(const uint32_t* c, uint32_t target, const Params& p
   }
 }
 
-// Tag of this launch's published top-k choices: odd, so a zeroed word never carries it,
-// and different in consecutive launches (the epoch counts completed launches).
+// Tag of this layer's published top-k choices: odd, so a zeroed word never carries it,
+// and different in consecutive launches (the epoch counts completed launches) and for
+// each layer of one launch.
 __device__ __forceinline__ uint32_t choice_tag(const Params& p) {
-  return (ld_relaxed_gpu(&p.ctr[CTR_EPOCH]) << 1) | 1u;
+  return ((ld_relaxed_gpu(&p.gctr[CTR_EPOCH]) * (uint32_t)kMaxFusedLayers + (uint32_t)p.layer) << 1) | 1u;
 }
 
 // Bounded wait of one warp for the k choices of row 0 (lane j < k polls choice j's two
@@ -730,8 +748,10 @@ __device__ __forceinline__ void make_seg(const Params& p, const Shape& sh, const
       break;
     }
     case UT_EXPERT: {
-      const int e = sc.slot_expert[sc.pair_slot[d.pair]];
-      const int r0 = pair_first_slot_row(sc, d.pair);
+      int e = sc.slot_expert[sc.pair_slot[d.pair]];
+      int r0 = pair_first_slot_row(sc, d.pair);
+      if (!IDX_OK(p, (unsigned)e < (unsigned)p.E && (unsigned)(r0 + kActGroup) <= (unsigned)kMaxSlots))
+        e = r0 = 0;  // reported; the step is abandoned, the copies stay in bounds
       x.tm0 = &p.tmaps[TM_WG];
       x.tm1 = &p.tmaps[TM_WU];
       x.y0 = e * p.I + d.tile * kBoxRows;
@@ -743,7 +763,11 @@ __device__ __forceinline__ void make_seg(const Params& p, const Shape& sh, const
       x.dep = 0;
       x.abase = p.n;
 #pragma unroll
-      for (int j = 0; j < kActGroup; ++j) x.aoff[j] = (uint32_t)(sc.row_of[r0 + (j < x.c ? j : 0)] * p.H);
+      for (int j = 0; j < kActGroup; ++j) {
+        int b = sc.row_of[r0 + (j < x.c ? j : 0)];
+        if (!IDX_OK(p, b < p.B)) b = 0;
+        x.aoff[j] = (uint32_t)(b * p.H);
+      }
       break;
     }
     case UT_DOWN_SHARED:
@@ -761,8 +785,10 @@ __device__ __forceinline__ void make_seg(const Params& p, const Shape& sh, const
       break;
     default: {
       const int pr = d.pair + q;
-      const int e = sc.slot_expert[sc.pair_slot[pr]];
-      const int r0 = pair_first_slot_row(sc, pr);
+      int e = sc.slot_expert[sc.pair_slot[pr]];
+      int r0 = pair_first_slot_row(sc, pr);
+      if (!IDX_OK(p, (unsigned)e < (unsigned)p.E && (unsigned)(r0 + kActGroup) <= (unsigned)kMaxSlots))
+        e = r0 = 0;  // reported; the step is abandoned, the copies stay in bounds
       x.pair = pr;
       x.tm0 = x.tm1 = &p.tmaps[TM_WD];
       x.y0 = e * p.H + d.tile * kBoxRows;
@@ -1050,11 +1076,13 @@ __device__ bool build_schedule(const Params& p, Smem& sm, int mw, int lane, uint
   // token rows and routing weights of every slot row (rows ascending within an expert)
   for (int i = mtid; i < sc.U; i += kMacThreads) {
     const int e = sc.slot_expert[i];
+    if (!IDX_OK(p, (unsigned)e < (unsigned)p.E)) continue;
     unsigned long long m = sm.u.t.mask[e];
     int r = sc.slot_base[i];
     while (m) {
       const int b = __ffsll((long long)m) - 1;
       m &= m - 1ull;
+      if (!IDX_OK(p, (unsigned)r < (unsigned)kMaxSlots)) break;
       float w = 0.0f;
       for (int j = 0; j < p.k; ++j)
         if (sm.u.t.topk_idx[b * p.k + j] == e) {
@@ -1294,6 +1322,10 @@ __device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, u
 #pragma unroll 4
       for (int sl = 0; sl < 32; ++sl) r += __shfl_sync(0xffffffffu, e, sl) < e ? 1 : 0;
       const int es = tc_expert_splits(1, sh.nkbH);
+      if (lane < k && !IDX_OK(p, (unsigned)e < (unsigned)p.E && (unsigned)r < (unsigned)kMaxSlots)) {
+        e = 0;  // reported; the step is abandoned
+        r = lane;
+      }
       if (lane < k) {
         sm.u.t.topk_idx[lane] = e;
         sm.u.t.topk_w[lane] = w;
@@ -1324,6 +1356,10 @@ __device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, u
         if (!sm.bcast2) record_abort(p, MOE_ERR_UNSUPPORTED_SHAPE);
       }
       __syncwarp();
+#ifdef MOE_BOUNDS_CHECK
+      if (lane == 0 && (p.flags & kFlagBadSlot)) sc.slot_of[0] = (int16_t)k;  // the first row past the schedule
+      __syncwarp();
+#endif
       if (blockIdx.x == 0 && lane < k) {
         if (p.dbg_idx) p.dbg_idx[lane] = e;
         if (p.dbg_w) p.dbg_w[lane] = w;
@@ -1362,7 +1398,8 @@ __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw
   for (int t = mtid; t < B * k; t += kMacThreads) {
     ulonglong2 ch = make_ulonglong2(0ull, 0ull);
     if (!dry) ch = __ldcg(reinterpret_cast<const ulonglong2*>(p.tk_pub) + t);
-    const int e = dry ? (13 * (t % k) + t / k) % p.E : (int)(uint32_t)ch.x;
+    int e = dry ? (13 * (t % k) + t / k) % p.E : (int)(uint32_t)ch.x;
+    if (!IDX_OK(p, (unsigned)e < (unsigned)p.E)) e = 0;  // reported; the step is abandoned
     const float w = dry ? 1.0f : __uint_as_float((uint32_t)ch.y);
     sm.u.t.topk_idx[t] = e;
     sm.u.t.topk_w[t] = w;
@@ -1440,7 +1477,8 @@ __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw
       const int c = i < U ? sc.slot_cnt[i] : 0;
       const uint32_t m = __match_any_sync(0xffffffffu, c);
       const int rank = __popc(m & ((1u << lane) - 1u));
-      if (c > 0) sc.pair_slot[sm.cnt_base[c] + rank] = (int16_t)i;
+      if (c > 0 && IDX_OK(p, c <= kTcMaxN && (unsigned)(sm.cnt_base[c] + rank) < (unsigned)kMaxSlots))
+        sc.pair_slot[sm.cnt_base[c] + rank] = (int16_t)i;
       __syncwarp();
       if (c > 0 && lane == __ffs(m) - 1) sm.cnt_base[c] += __popc(m);
       __syncwarp();
@@ -1490,10 +1528,17 @@ __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw
     const int e = sm.u.t.topk_idx[t];
     const unsigned long long m = sm.u.t.mask[e];
     const int r = sc.slot_base[sc.eslot[e]] + __popcll(m & ((1ull << b) - 1ull));
+    if (!IDX_OK(p, (unsigned)r < (unsigned)kMaxSlots)) continue;
     sc.row_of[r] = (uint8_t)b;
     sc.w_of[r] = sm.u.t.topk_w[t];
     sc.slot_of[t] = (int16_t)r;
   }
+#ifdef MOE_BOUNDS_CHECK
+  if (!dry && (p.flags & kFlagBadSlot)) {  // row 0's first choice: the first slot row past the schedule
+    if (!mac_sync(sm, mphase, p, lane)) return false;
+    if (mtid == 0) sc.slot_of[0] = (int16_t)sc.S;
+  }
+#endif
   if (blockIdx.x == 0 && !dry) {
     for (int t = mtid; t < B * k; t += kMacThreads) {
       if (p.dbg_idx) p.dbg_idx[t] = sm.u.t.topk_idx[t];
@@ -1517,12 +1562,24 @@ __device__ bool normalise_rows(const Params& p, Smem& sm, int mw, int lane, uint
   const int mtid = mw * 32 + lane;
   const int nv = p.H / 8;
   const uint4* g4 = reinterpret_cast<const uint4*>(p.gamma);
+  const bool fresh = p.rows_in != nullptr;  // input rows written during this launch
   for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
+    if (fresh) {
+      // the previous layer's output row b is input once all of its tile pairs are combined
+      if (mw == 0) {
+        int ok = 1;
+        if (lane == 0) ok = wait_counter(&p.rows_in[b], (uint32_t)((p.H + 2 * kTcRows - 1) / (2 * kTcRows)), p) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (lane == 0) sm.bcast = ok;
+      }
+      if (!mac_sync(sm, mphase, p, lane)) return false;
+      if (!sm.bcast) return false;
+    }
     const uint4* x4 = reinterpret_cast<const uint4*>(p.x + (size_t)b * p.H);
     float ss = 0.0f;
 #pragma unroll 4
     for (int v = mtid; v < nv; v += kMacThreads) {
-      const uint4 xv = ld_nc_v4(x4 + v);
+      const uint4 xv = fresh ? ld_cg_v4(x4 + v) : ld_nc_v4(x4 + v);
       (void)ld_nc_v4(g4 + v);  // brings gamma into L1 for pass 2 (a volatile load is kept)
       float f[8];
       unpack8(xv, f);
@@ -1543,7 +1600,7 @@ __device__ bool normalise_rows(const Params& p, Smem& sm, int mw, int lane, uint
 #pragma unroll 1
     for (int v = mtid; v < nv; v += kMacThreads) {
       float f[8], g[8];
-      unpack8(ld_nc_v4(x4 + v), f);
+      unpack8(fresh ? ld_cg_v4(x4 + v) : ld_nc_v4(x4 + v), f);
       unpack8(ld_nc_v4(g4 + v), g);
       uint32_t o[4];
 #pragma unroll
@@ -1633,7 +1690,8 @@ __device__ void epi_finish(const Params& p, Smem& sm, const UnitDesc& d, int u,
     const int c = pair_rows(sc, d.pair);
     const int r0 = pair_first_slot_row(sc, d.pair);
     for (int j = 0; j < c; ++j)
-      p.he[(size_t)(r0 + j) * p.I + d.tile * kBoxRows + row] = f2bf(silu(src[0][row][j]) * src[1][row][j]);
+      if (IDX_OK(p, (unsigned)(r0 + j) < (unsigned)kMaxSlots))
+        p.he[(size_t)(r0 + j) * p.I + d.tile * kBoxRows + row] = f2bf(silu(src[0][row][j]) * src[1][row][j]);
   } else {
     // down tile fix-up: y = bf16(x + s + sum_e w_e d_e) in fixed split / pair / row order
     float* yacc = sm.u.yacc[row];
@@ -1655,7 +1713,9 @@ __device__ void epi_finish(const Params& p, Smem& sm, const UnitDesc& d, int u,
           const float vv[4] = {v.x, v.y, v.z, v.w};
           const int c = pair_rows(sc, pr);
           const int r0 = pair_first_slot_row(sc, pr);
-          for (int j = 0; j < c; ++j) yacc[sc.row_of[r0 + j]] += vv[j];
+          for (int j = 0; j < c; ++j)
+            if (IDX_OK(p, (unsigned)(r0 + j) < (unsigned)kMaxSlots && sc.row_of[r0 + j] < sh.B))
+              yacc[sc.row_of[r0 + j]] += vv[j];
         }
       }
     }
@@ -1729,6 +1789,7 @@ struct Producer {
   // (expert, row group) pair pr complete? One acquire round trip polls 32 pairs.
   __device__ bool wait_pair(int pr) {
     const Shape& sh = sm.sh;
+    if (!IDX_OK(p, (unsigned)pr < (unsigned)kMaxSlots)) return false;
     if ((sm.known_done[pr >> 5] >> (pr & 31)) & 1u) return true;
     const int q = pr + lane;
     const bool done = q < sm.sc.P && ld_acquire_gpu(&p.pair_done[q]) >= (uint32_t)sh.pair_target;
@@ -1749,8 +1810,8 @@ struct Producer {
     return r;
   }
 
-  // After the last stage: the stop header, the drain of every bulk copy still in
-  // flight, and the L2 prefetch of the next layer's router and shared-expert weights.
+  // After the last stage: the stop header and the drain of every bulk copy still in
+  // flight.
   __device__ void finish() {
     if (wait_slot()) {
       pend_mask &= ~(1u << slot);
@@ -1773,21 +1834,15 @@ struct Producer {
           }
         }
       }
-      for (int r = 0; r < 4; ++r) {
-        if (!p.pf_ptr[r] || !p.pf_bytes[r]) continue;
-        const unsigned long long tot = p.pf_bytes[r];
-        const unsigned long long lo = (tot * blockIdx.x / gridDim.x) & ~15ull;
-        const unsigned long long hi =
-            blockIdx.x + 1 == gridDim.x ? (tot & ~15ull) : (tot * (blockIdx.x + 1) / gridDim.x) & ~15ull;
-        const uint8_t* base = reinterpret_cast<const uint8_t*>(p.pf_ptr[r]);
-        for (unsigned long long o = lo; o < hi; o += 65536ull) {
-          const unsigned long long n = hi - o < 65536ull ? hi - o : 65536ull;
-          if (n >= 16) prefetch_l2_bulk(base + o, (uint32_t)(n & ~15ull));
-        }
-      }
     }
     __syncwarp();
   }
+};
+
+// Ring position carried by the producer from one layer of a fused launch to the next.
+struct RingState {
+  int slot;
+  uint32_t phase, pend_mask, pend_parity;
 };
 
 // CUDA-core path producer: units of 32 weight rows, activation rows by 1-D bulk copies.
@@ -1799,10 +1854,7 @@ __device__ void producer_cc(Producer& pr, uint8_t* ring) {
   const int lane = pr.lane;
   const uint64_t pol = policy_evict_first();
   if (lane == 0)
-    for (int t = 0; t < TM_T_WR; ++t) {
-      fence_tensormap_acquire(&p.tmaps[t]);
-      prefetch_tensormap(&p.tmaps[t]);
-    }
+    for (int t = 0; t < TM_T_WR; ++t) prefetch_tensormap(&p.tmaps[t]);
   bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
   const int pre = sh.NR + sh.NS;
   int u = pr.grab();
@@ -1967,7 +2019,8 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       break;
     case UT_EXPERT: {
       // every token row is an MMA column; the epilogue keeps the expert's own rows
-      const int e = sc.slot_expert[sc.pair_slot[d.pair]];
+      int e = sc.slot_expert[sc.pair_slot[d.pair]];
+      if (!IDX_OK(p, (unsigned)d.pair < (unsigned)kMaxSlots && (unsigned)e < (unsigned)p.E)) e = 0;
       x.tw0 = &p.tmaps[TM_T_WG];
       x.tw1 = &p.tmaps[TM_T_WU];
       x.y0 = x.y1 = e * p.I + d.tile * kTcRows;
@@ -1984,8 +2037,10 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       break;
     default: {
       // the expert's slot rows of h are contiguous: they are the MMA columns
-      const int i = sc.pair_slot[d.pair];
-      const int e = sc.slot_expert[i];
+      int i = sc.pair_slot[d.pair];
+      if (!IDX_OK(p, (unsigned)i < (unsigned)kMaxE)) i = 0;
+      int e = sc.slot_expert[i];
+      if (!IDX_OK(p, (unsigned)e < (unsigned)p.E && (unsigned)sc.slot_base[i] < (unsigned)kMaxSlots)) e = 0;
       x.tw0 = x.tw1 = &p.tmaps[TM_T_WD];
       x.y0 = e * p.H + d.tile * 2 * kTcRows;
       x.y1 = x.y0 + kTcRows;
@@ -2001,20 +2056,28 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
 
 // Tensor-core path producer: per 64-column K atom one stage of up to two 128-row weight
 // tiles and the activation operand (N rows, boxes of 16), all 128-byte swizzled.
+// last: the launch's last layer (then the stop header and the drain follow); false is
+// returned on abort (after the same stop header and drain).
 template <bool kTrace>
-__device__ void producer_tc(Producer& pr, uint8_t* ring) {
+__device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
   const Params& p = pr.p;
   Smem& sm = pr.sm;
   const Shape& sh = sm.sh;
   const int lane = pr.lane;
   const uint64_t pol = policy_evict_first();
+  // the maps are written before the launch (a host copy, or a preceding kernel on the
+  // no-allocation path): the launch boundary orders them, no proxy fence is needed
+  // (measured: one acquire fence per map cost ~4 us per step)
   if (lane == 0)
-    for (int t = TM_T_WR; t < TM_COUNT; ++t) {
-      fence_tensormap_acquire(&p.tmaps[t]);
-      prefetch_tensormap(&p.tmaps[t]);
-    }
+    for (int t = TM_T_WR; t < TM_COUNT; ++t) prefetch_tensormap(&p.tmaps[t]);
+  if (p.layer > 0) {  // the previous layer's record of completed experts
+    for (int w = lane; w < kMaxSlots / 32; w += 32) sm.known_done[w] = 0u;
+    __syncwarp();
+  }
   bool ok = true, sched_ready = false, n_ok = false, hs_ok = false;
   const int pre = sh.pre;
+  int total = 0;  // this layer's units, once its schedule exists (kept: the schedule may be
+                  // rebuilt for the next layer while this warp still draws tickets)
   int u = pr.grab();
   bool first_expert = true, first_down = true, first_tma = true;
   unsigned long long c_slot = 0, c_dep = 0, c_grab = 0, c_issue = 0, c_stages = 0, c_units = 0;
@@ -2023,13 +2086,14 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
   while (ok) {
     if (u >= pre && !sched_ready) {
       const long long tw0 = tclock<kTrace>();
-      ok = pr.wait_bar(&sm.sched_bar, 0u);
+      ok = pr.wait_bar(&sm.sched_bar, (uint32_t)(p.layer & 1));
       c_schedw += (unsigned long long)(tclock<kTrace>() - tw0);
       if (!ok) break;
       sched_ready = true;
+      total = sm.sc.total;
       if (lane == 0) trace_stamp<kTrace>(p, TR_SCHED);
     }
-    if (sched_ready && u >= sm.sc.total) break;
+    if (sched_ready && u >= total) break;
     const long long tu0 = tclock<kTrace>();
     const UnitDesc d = decode_unit_tc(sh, sm.sc, u);
     // the next unit's ticket is requested now (its round trip overlaps this unit's
@@ -2038,6 +2102,7 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
     const bool early_grab = d.type != UT_ROUTER;
     uint32_t next_ticket = 0;
     if (lane == 0 && early_grab) next_ticket = atom_add_relaxed(&p.ctr[CTR_QUEUE], 1u);
+    const int hunit = (p.layer << 24) | u;  // stage headers name the layer and the unit
     if (lane == 0 && kTrace) {
       if (first_expert && d.type == UT_EXPERT) { trace_stamp<kTrace>(p, TR_FIRST_EXPERT); first_expert = false; }
       if (first_down && (d.type == UT_DOWN_SHARED || d.type == UT_DOWN_EXPERT)) { trace_stamp<kTrace>(p, TR_FIRST_DOWN); first_down = false; }
@@ -2058,7 +2123,7 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
       if (lane == 0) {
         StageHeader h;
         h.kind = HK_STAGE;
-        h.unit = u;
+        h.unit = hunit;
         h.info = info0 | (ka == d.kb0 ? kTcInfoFirst : 0) | (ka == ka_end - 1 ? kTcInfoLast : 0);
         h.wrow = -1;
         sm.hdr[pr.slot] = h;
@@ -2156,7 +2221,8 @@ __device__ void producer_tc(Producer& pr, uint8_t* ring) {
     trace_put<kTrace>(p, TR_PROD_SCHED_CYC, c_schedw);
     trace_put<kTrace>(p, TR_PROD_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tploop0));
   }
-  pr.finish();
+  if (last || !ok) pr.finish();
+  return ok;
 }
 
 // ---- CUDA-core path: MAC warps and the epilogue warp ------------------------------------------
@@ -2444,6 +2510,7 @@ __device__ void fixup_tc(const Params& p, const Smem& sm, const UnitDesc& d, int
     const int i = sc.pair_slot[d.pair];
     const int r0 = sc.slot_base[i], cnt = sc.slot_cnt[i];
     for (int j = 0; j < cnt; ++j) {
+      if (!IDX_OK(p, (unsigned)(r0 + j) < (unsigned)sc.S && (unsigned)sc.S <= p.cap_slots)) break;
       float g = 0.0f, u = 0.0f;
       for (int sp = 0; sp < d.nsplit; ++sp) {
         const float* src = p.epart + (((size_t)sp * sc.S + r0 + j) * sh.IT + d.tile) * (2 * kTcRows);
@@ -2467,7 +2534,13 @@ __device__ void combine_rows_tc(const Params& p, const Smem& sm, int t, const in
   if (h >= p.H) return;
   for (int ci = et >> 6; ci < n; ci += 2) {
     const int b = rows[ci];
+    if (!IDX_OK(p, b < sh.B)) continue;
     const int16_t* so = &sc.slot_of[b * sh.k];
+#ifdef MOE_BOUNDS_CHECK
+    bool bad = false;
+    for (int j = 0; j < sh.k; ++j) bad = bad || (unsigned)so[j] >= (unsigned)sc.S;
+    if (!IDX_OK(p, !bad)) continue;
+#endif
     float4 acc = __ldcg(reinterpret_cast<const float4*>(p.dpart + (size_t)b * p.H + h));
     for (int j0 = 0; j0 < sh.k; j0 += 8) {
       float4 v[8];
@@ -2486,7 +2559,7 @@ __device__ void combine_rows_tc(const Params& p, const Smem& sm, int t, const in
         }
       }
     }
-    const uint2 xv = *reinterpret_cast<const uint2*>(p.x + (size_t)b * p.H + h);
+    const uint2 xv = __ldcg(reinterpret_cast<const uint2*>(p.x + (size_t)b * p.H + h));
     uint2 yv;
     yv.x = (uint32_t)f2bf(bf2f(xv.x & 0xFFFFu) + acc.x) | ((uint32_t)f2bf(bf2f(xv.x >> 16) + acc.y) << 16);
     yv.y = (uint32_t)f2bf(bf2f(xv.y & 0xFFFFu) + acc.z) | ((uint32_t)f2bf(bf2f(xv.y >> 16) + acc.w) << 16);
@@ -2494,8 +2567,10 @@ __device__ void combine_rows_tc(const Params& p, const Smem& sm, int t, const in
   }
 }
 
+// F: the layers of a fused launch (a unit's header names its layer), or nullptr when
+// the launch runs the one layer p0.
 template <bool kTrace>
-__device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
+__device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, const FusedParams* F = nullptr) {
   const Shape& sh = sm.sh;
   const int quad = warp_id & 3;
   const int row = quad * 32 + lane;                        // accumulator lane = tile row
@@ -2503,18 +2578,20 @@ __device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
   const uint32_t tq = sm.tmem_base + ((uint32_t)(quad * 32) << 16);
   int abuf = 0;
   uint32_t aphase = 0, ephase = 0;
-  bool sched_seen = false;
+  int sched_layer = -1;  // the last layer whose schedule this warp has seen
   unsigned long long c_busy = 0;
   for (;;) {
-    if (!warp_wait(&sm.acc_full[abuf], aphase, p, lane)) break;
-    const int u = sm.acc_unit[abuf];
-    if (u < 0) {
+    if (!warp_wait(&sm.acc_full[abuf], aphase, p0, lane)) break;
+    const int hu = sm.acc_unit[abuf];
+    if (hu < 0) {
       if (lane == 0 && kTrace && warp_id == kTcEpiWarp0) {
-        trace_stamp<kTrace>(p, TR_EPI_END);
-        trace_put<kTrace>(p, TR_EPI_BUSY_CYC, c_busy);
+        trace_stamp<kTrace>(p0, TR_EPI_END);
+        trace_put<kTrace>(p0, TR_EPI_BUSY_CYC, c_busy);
       }
       break;
     }
+    const int layer = hu >> 24, u = hu & 0xFFFFFF;
+    const Params& p = F ? F->layer[layer] : p0;
     tc_fence_after();
     const long long tb0 = tclock<kTrace>();
     const Sched& sc = sm.sc;
@@ -2564,12 +2641,15 @@ __device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
       case UT_EXPERT: {
         // the expert's rows are scattered token columns: one column load per row
         const int i = sc.pair_slot[d.pair];
-        const int r0 = sc.slot_base[i], cnt = sc.slot_cnt[i];
+        const int r0 = sc.slot_base[i];
+        int cnt = sc.slot_cnt[i];
+        if (!IDX_OK(p, (unsigned)(r0 + cnt) <= (unsigned)sc.S && (unsigned)sc.S <= p.cap_slots)) cnt = 0;
         for (int j0 = 0; j0 < cnt; j0 += 8) {
 #pragma unroll
           for (int jj = 0; jj < 8; ++jj) {
             const int j = j0 + jj < cnt ? j0 + jj : j0;
-            const uint32_t col = (uint32_t)sc.row_of[r0 + j];
+            uint32_t col = (uint32_t)sc.row_of[r0 + j];
+            if (!IDX_OK(p, col < (uint32_t)sh.NA)) col = 0;
             tmem_ld1(ta + col, v0[jj]);
             tmem_ld1(ta + 64u + col, v1[jj]);
           }
@@ -2599,7 +2679,8 @@ __device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
         const bool shared = d.type == UT_DOWN_SHARED;
         const int i = shared ? 0 : sc.pair_slot[d.pair];
         const int r0 = shared ? 0 : sh.B + sc.slot_base[i];
-        const int cnt = shared ? sh.B : sc.slot_cnt[i];
+        int cnt = shared ? sh.B : sc.slot_cnt[i];
+        if (!IDX_OK(p, (unsigned)(r0 + cnt) <= p.cap_dpart_rows)) cnt = 0;
         const int h0 = d.tile * 2 * kTcRows + row, h1 = h0 + kTcRows;
         const bool two = d.tile * 2 * kTcRows + kTcRows < p.H;
         for (int j0 = 0; j0 < cnt; j0 += 16) {
@@ -2633,25 +2714,30 @@ __device__ void epilogue_tc(const Params& p, Smem& sm, int warp_id, int lane) {
       const bool shared = d.type == UT_DOWN_SHARED;
       const int i = shared ? 0 : sc.pair_slot[d.pair];
       const int cnt = shared ? sh.B : sc.slot_cnt[i];
-      if (et < cnt) {
+      if (et < cnt &&
+          IDX_OK(p, shared || ((unsigned)(sc.slot_base[i] + et) < (unsigned)kMaxSlots &&
+                               sc.row_of[sc.slot_base[i] + et] < sh.B))) {
         const int b = shared ? et : sc.row_of[sc.slot_base[i] + et];
         uint32_t* tix = &p.row_tix[d.tile * sh.B + b];
         const uint32_t old = atom_add_acq_rel(tix, 1u);
         if (old == (uint32_t)sh.k) {
           st_relaxed_gpu(tix, 0u);
-          sm.comb_rows[atomicAdd(&sm.ncomb, 1)] = (int16_t)b;
+          const int slot = atomicAdd(&sm.ncomb, 1);
+          if (IDX_OK(p, slot < kTcMaxN)) sm.comb_rows[slot] = (int16_t)b;
         }
       }
       if (!epi_sync(sm, ephase, p, lane)) break;
-      const int ncomb = sm.ncomb;
+      const int ncomb = sm.ncomb < kTcMaxN ? sm.ncomb : kTcMaxN;
       if (ncomb > 0) {
         // a shared-expert tile can complete a row before this CTA's schedule exists
-        if (!sched_seen) {
-          if (!warp_wait(&sm.sched_bar, 0u, p, lane)) break;
-          sched_seen = true;
+        if (sched_layer < layer) {
+          if (!warp_wait(&sm.sched_bar, (uint32_t)(layer & 1), p, lane)) break;
+          sched_layer = layer;
         }
         combine_rows_tc(p, sm, d.tile, sm.comb_rows, ncomb, et);
+        if (p.rows_out) __threadfence();  // the rows' outputs, then their completion counts
         if (!epi_sync(sm, ephase, p, lane)) break;
+        if (p.rows_out && et < ncomb) red_release_add(&p.rows_out[sm.comb_rows[et]], 1u);
         if (et == 0) sm.ncomb = 0;  // ordered before the next unit's list by its first rendezvous
       }
     } else {
@@ -2786,10 +2872,10 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
   if (tid == 0) {
     trace_stamp<kTrace>(p, TR_EXIT);
     __threadfence();
-    const uint32_t done = atom_add_acq_rel(&p.ctr[CTR_EXIT], 1u);
+    const uint32_t done = atom_add_acq_rel(&p.gctr[CTR_EXIT], 1u);
     if (done == gridDim.x - 1) {
       // last CTA out: reset this step's counters for the next launch
-      const bool aborted = ld_relaxed_gpu(&p.ctr[CTR_ABORT]) != 0u;
+      const bool aborted = ld_relaxed_gpu(&p.gctr[CTR_ABORT]) != 0u;
       if (aborted) {
         for (unsigned t = 0; t < p.max_tiles; ++t) p.tickets[t] = 0u;
         for (int t = 0; t < kMaxSlots; ++t) p.pair_done[t] = 0u;
@@ -2805,6 +2891,139 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
   }
 }
 
+// ---- several layers in one launch (tensor-core path) ---------------------------------------------
+//
+// Layer l + 1 follows layer l inside the same persistent launch: a CTA whose producer
+// has drawn the last of layer l's units moves on to layer l + 1's queue (its router and
+// shared-expert tiles arm their weight stages while layer l drains); each output row of
+// layer l counts its
+// combined tile pairs, and the CTA that owns row b normalises it for layer l + 1 once all
+// have arrived. Every layer keeps its own counters, completion flags and choice tags;
+// the activation buffers are shared, since a layer writes them only after the previous
+// layer's output is complete everywhere, which means no unit of that layer is left.
+// The per-layer kernel count of the pages' decode path (page post.smzdm.com/p/a6zppe4g,
+// section "改了什么：每层 23 个 kernel 砍到 13 个") becomes one launch per step.
+template <bool kTrace>
+__global__ void __launch_bounds__(kTcThreads, 1) moe_decode_fused_kernel(const __grid_constant__ FusedParams F) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
+  Smem& sm = *reinterpret_cast<Smem*>(ring + kTcRingBytes);
+  const Params& p0 = F.layer[0];
+  const int L = F.L;
+  const int tid = threadIdx.x;
+  const int warp_id = tid / 32;
+  const int lane = tid % 32;
+
+  if (tid == 0) {
+    for (int s = 0; s < kTcStagesMax; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < kTcAccBufs; ++b) {
+      mbar_init(&sm.acc_full[b], 2);
+      mbar_init(&sm.acc_empty[b], kTcEpiWarps);
+    }
+    mbar_init(&sm.mma_bar, 1);
+    mbar_init(&sm.epi_bar, kTcEpiWarps);
+    make_shape_tc(p0, sm.sh);  // every layer of the stack has the same shape
+    mbar_init(&sm.sched_bar, 1);  // one phase per layer
+    mbar_init(&sm.mac_bar, kMacWarps);
+    sm.ncomb = 0;
+    for (int w = 0; w < kMaxSlots / 32; ++w) sm.known_done[w] = 0u;
+    if (kTrace) {
+      for (int l = 0; l < L; ++l)
+        for (int t = 0; t < kTraceSlots; ++t) F.layer[l].trace[(size_t)blockIdx.x * kTraceSlots + t] = 0ull;
+      trace_stamp<kTrace>(p0, TR_START);
+      trace_clk<kTrace>(p0, TR_START_CLK);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp_id == kTcMmaWarp) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0) trace_stamp<kTrace>(p0, TR_ROLES);
+
+  if (warp_id == 0) {
+    RingState st{0, 0u, 0u, 0u};
+    for (int l = 0; l < L; ++l) {
+      Producer pr(F.layer[l], sm, lane, sm.sh.nst);
+      pr.slot = st.slot;
+      pr.phase = st.phase;
+      pr.pend_mask = st.pend_mask;
+      pr.pend_parity = st.pend_parity;
+      const bool ok = producer_tc<kTrace>(pr, ring, l == L - 1);
+      st = RingState{pr.slot, pr.phase, pr.pend_mask, pr.pend_parity};
+      if (!ok) break;  // the stop header and the drain are done
+    }
+  } else if (warp_id <= kMacWarps) {
+    const int mw = warp_id - 1;
+    uint32_t mphase = 0;
+    for (int l = 0; l < L; ++l) {
+      const Params& p = F.layer[l];
+      const uint32_t tag = choice_tag(p);
+      bool ok = normalise_rows<kTrace>(p, sm, mw, lane, mphase);
+      if (ok) ok = route_rows_tc<kTrace>(p, sm, mw, lane, mphase, tag);
+      if (ok && (int)blockIdx.x >= p.B && p.B > 1) {
+        if (mw == 0) {
+          int r = 1;
+          if (lane == 0) r = wait_counter(&p.ctr[CTR_ROUTER], (uint32_t)sm.sh.router_target, p) ? 1 : 0;
+          r = __shfl_sync(0xffffffffu, r, 0);
+          if (lane == 0) sm.bcast = r;
+        }
+        ok = mac_sync(sm, mphase, p, lane) && sm.bcast;
+        if (ok) ok = build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, true);
+      }
+      if (ok) ok = p.B == 1 ? build_schedule_b1<kTrace>(p, sm, mw, lane, mphase, tag)
+                            : build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, false);
+      if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
+      if (!ok) break;
+    }
+  } else if (warp_id == kTcMmaWarp) {
+    mma_warp<kTrace>(p0, sm, ring, lane);
+  } else {
+    epilogue_tc<kTrace>(p0, sm, warp_id, lane, &F);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp_id == kTcMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(sm.tmem_base, kTmemCols);
+  }
+  if (tid == 0) {
+    trace_stamp<kTrace>(p0, TR_EXIT);
+    __threadfence();
+    const uint32_t done = atom_add_acq_rel(&p0.gctr[CTR_EXIT], 1u);
+    sm.bcast = done == gridDim.x - 1 ? 1 : 0;
+  }
+  __syncthreads();
+  if (sm.bcast) {
+    // last CTA out: every layer's counters, completion flags and row counts start at zero
+    // for the next launch (and the shared tickets, which an aborted step may leave set)
+    const bool aborted = ld_relaxed_gpu(&p0.gctr[CTR_ABORT]) != 0u;
+    for (int l = 0; l < L; ++l) {
+      const Params& p = F.layer[l];
+      for (int t = tid; t < kMaxSlots; t += kTcThreads) p.pair_done[t] = 0u;
+      if (p.rows_out)
+        for (int t = tid; t < p.B; t += kTcThreads) p.rows_out[t] = 0u;
+      if (tid < CTR_COUNT && !(l == 0 && tid == CTR_EPOCH)) p.ctr[tid] = 0u;
+    }
+    if (aborted) {
+      for (unsigned t = tid; t < p0.max_tiles; t += kTcThreads) p0.tickets[t] = 0u;
+      for (unsigned t = tid; t < p0.row_tix_count; t += kTcThreads) p0.row_tix[t] = 0u;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      p0.gctr[CTR_EPOCH] += 1u;  // the next launch's choices carry new tags
+      __threadfence();
+    }
+  }
+}
+
 size_t smem_bytes() { return kCcRingBytes + sizeof(Smem) + 1024; }
 int threads_per_cta() { return kThreads; }
 const void* kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false, false>); }
@@ -2813,5 +3032,7 @@ size_t tc_smem_bytes() { return kTcRingBytes + sizeof(Smem) + 1024; }
 int tc_threads_per_cta() { return kTcThreads; }
 const void* tc_kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false, true>); }
 const void* tc_kernel_fn_trace() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true, true>); }
+const void* fused_kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_fused_kernel<false>); }
+const void* fused_kernel_fn_trace() { return reinterpret_cast<const void*>(&moe_decode_fused_kernel<true>); }
 
 }  // namespace moe

@@ -219,28 +219,20 @@ extern "C" int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_d
     p.tmaps = d_maps + l * kNaMapsPerLayer;
     p.gamma = (const uint16_t*)w.gamma;
     p.bias = w.router_bias;
-    if (l + 1 < L) {
-      const moe_decode_layer_weights& nx = layers[l + 1];
-      p.pf_ptr[0] = nx.w_router;
-      p.pf_bytes[0] = (unsigned long long)E * H * 2;
-      p.pf_ptr[1] = nx.ws_gate;
-      p.pf_bytes[1] = (unsigned long long)Is * H * 2;
-      p.pf_ptr[2] = nx.ws_up;
-      p.pf_bytes[2] = (unsigned long long)Is * H * 2;
-      p.pf_ptr[3] = nx.ws_down;
-      p.pf_bytes[3] = (unsigned long long)Is * H * 2;
-    }
     p.n = reinterpret_cast<uint16_t*>(base + kOffN);
     p.logits = reinterpret_cast<float*>(base + kOffLogits);
     p.hs = reinterpret_cast<uint16_t*>(base + kOffHs);
     p.he = reinterpret_cast<uint16_t*>(base + kOffHe);
     p.partial = reinterpret_cast<float*>(base + kOffPartial);
     p.ctr = reinterpret_cast<uint32_t*>(base + kOffCtr);
+    p.gctr = p.ctr;  // one layer per launch: the launch-wide counters share the layer's block
     p.tickets = reinterpret_cast<uint32_t*>(base + kOffTickets);
     p.pair_done = reinterpret_cast<uint32_t*>(base + kOffPairDone);
     p.status = device_status;
     p.max_units = kNaUnits;
     p.max_tiles = kNaTiles;
+    p.cap_slots = (unsigned)kNaSlots;
+    p.cap_dpart_rows = (unsigned)(kNaSlots + kNaMaxBatch);
     p.wait_ns = 2000ull * 1000000ull;
     void* args[] = {&p};
     const cudaError_t e = cudaLaunchCooperativeKernel(moe::kernel_fn(), dim3(st->num_sms),

@@ -1,5 +1,5 @@
 // ptx.cuh - thin inline-PTX wrappers for sm_100a used by the persistent kernel:
-// mbarriers, TMA (cp.async.bulk.tensor) and 1-D bulk copies, L2 prefetch,
+// mbarriers, TMA (cp.async.bulk.tensor) and 1-D bulk copies, tensor-map prefetch,
 // proxy fences, gpu-scope acquire/release, the global timer, and the tcgen05
 // tensor-core instructions (tensor-memory allocation, MMA, commit, loads).
 #pragma once
@@ -64,18 +64,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-__device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
-// Makes a tensor map written to global memory through the generic proxy (a host
-// copy, or another kernel's stores) visible to the tensor-map proxy that TMA reads
-// it through; issued once per map before its first use.
-__device__ __forceinline__ void fence_tensormap_acquire(const CUtensorMap* map) {
-  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(reinterpret_cast<uint64_t>(map))
-               : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -108,6 +96,15 @@ __device__ __forceinline__ void fence_proxy_async_global() {
 __device__ __forceinline__ uint4 ld_nc_v4(const void* ptr) {
   uint4 v;
   asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(ptr));
+  return v;
+}
+
+// 16-byte load through L2 (not L1): data another CTA wrote during this kernel.
+__device__ __forceinline__ uint4 ld_cg_v4(const void* ptr) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(ptr));
   return v;

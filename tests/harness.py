@@ -38,13 +38,14 @@ def bf16_ulp(v):
     return 2.0 ** (e - 7)
 
 
-def make_handle(wl, layers, device=0, max_batch=None, top_k_max=None, tc_min_batch=None):
+def make_handle(wl, layers, device=0, max_batch=None, top_k_max=None, tc_min_batch=None, checked=False):
     """A handle for the workload; tc_min_batch (if given) sets the batch-shape switch:
-    1 sends every step to the tensor-core kernel, 0 every step to the CUDA-core one."""
+    1 sends every step to the tensor-core kernel, 0 every step to the CUDA-core one.
+    checked: the bounds-checked build of the library."""
     import moe_decode_persistent_b200 as mdp
 
     h = mdp.MoeDecode(wl.H, wl.E, top_k_max or wl.k, wl.I, wl.Is, max_batch or wl.B, layers,
-                      eps=wl.eps, device=device)
+                      eps=wl.eps, device=device, checked=checked)
     if tc_min_batch is not None:
         h.set_tc_min_batch(tc_min_batch)
     return h

@@ -22,8 +22,17 @@ def test_exports_every_declared_symbol(L):
         assert hasattr(L, name), name
 
 
+def test_bounds_checked_build_exports_the_same_symbols():
+    if not os.path.exists(mdp.CHECKED_LIB):
+        mdp.build()
+    C = mdp.lib(checked=True)
+    for name in mdp.declared_symbols():
+        assert hasattr(C, name), name
+    assert C is not mdp.lib()
+
+
 def test_strerror_is_distinct_per_code(L):
-    codes = [0, -1, -2, -3, -4, -5, -6, -7, -8]
+    codes = [0, -1, -2, -3, -4, -5, -6, -7, -8, -9]
     msgs = [mdp.strerror(c) for c in codes]
     assert len(set(msgs)) == len(codes)
     assert mdp.strerror(-99) == "unknown error"

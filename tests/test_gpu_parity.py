@@ -49,8 +49,12 @@ TC_SMALL = [
       nseq=4, rows_per_seq=8),
     W("tc_k32_b3_h256", B=3, H=256, E=128, k=32, I=128, Is=128, seed=36),
     W("tc_b2_h2048", B=2, H=2048, E=128, k=2, I=512, Is=768, seed=37),
-    # the largest batch routed by router tile pair (two pairs, 32 candidates per row)
     W("tc_b4_k16_e512", B=4, H=512, E=512, k=16, I=128, Is=128, seed=39),
+    # stacks of three layers in one launch: the middle layer both waits for its input
+    # rows and counts its output rows; one row (the one-row routing path) and four
+    W("tc_3layer_b4", B=4, H=512, E=256, k=8, I=128, Is=128, seed=44, layers=3, rows="correlated",
+      nseq=1, rows_per_seq=4),
+    W("tc_3layer_b1", B=1, H=512, E=256, k=8, I=256, Is=256, seed=45, layers=3),
 ]
 
 
@@ -91,6 +95,35 @@ def run_and_check(wl, rows=None, handle=None, layers=None, tc_min_batch=None):
     return out, err
 
 
+def _launches(h, wl):
+    """Launches one step makes: the tensor-core path runs a stack of layers in one launch,
+    the CUDA-core path launches once per layer."""
+    import moe_decode_persistent_b200 as mdp
+
+    return 1 if h.step_path(wl.B) == mdp.PATH_TENSOR_CORE else wl.layers
+
+
+def test_tc_layer_stack_runs_in_one_launch_and_recovers_from_a_timeout():
+    """A three-layer stack on the tensor-core path is one launch per step. A step whose
+    first normalised row is withheld times out in every CTA (status MOE_ERR_TIMEOUT);
+    the counters of every layer are reset by the launch's last CTA, so the next step on
+    the same handle is correct."""
+    import moe_decode_persistent_b200 as mdp
+
+    wl = TC_BY_NAME["tc_3layer_b4"]
+    layers = _layers(wl)
+    h = make_handle(wl, layers, tc_min_batch=1)
+    assert h.step_path(wl.B) == mdp.PATH_TENSOR_CORE and h.launches_per_step() == 1
+    x = wl.x_host()
+    h.set_debug(mdp.DEBUG_WITHHOLD_NREADY, wait_ms=300)
+    bad = run_gpu(h, wl, x, n_layers=wl.layers)
+    assert bad["status"] == mdp.MOE_ERR_TIMEOUT
+    h.set_debug(0)
+    for _ in range(2):
+        run_and_check(wl, handle=h, layers=layers)
+    h.close()
+
+
 def _switch_of(h, wl):
     """tc_min_batch that reproduces the path h takes for wl's batch."""
     import moe_decode_persistent_b200 as mdp
@@ -126,11 +159,11 @@ def test_cuda_core_only_shapes_never_take_the_tensor_core_path():
     h.close()
 
 
-@pytest.mark.parametrize("name", ["tc_zipf_b17", "tc_b4_k16_e512"])
+@pytest.mark.parametrize("name", ["tc_zipf_b17", "tc_b4_k16_e512", "tc_3layer_b4"])
 def test_tc_deterministic_and_jitter_invariant(name):
     """Bitwise the same output under random per-CTA delays: every reduction runs in a
-    fixed order whichever CTA finishes last (the row owners' routing at batch 17, the
-    router tile pairs' routing at batch 4)."""
+    fixed order whichever CTA finishes last, within a layer and across the layers of a
+    stack run in one launch."""
     import moe_decode_persistent_b200 as mdp
 
     wl = TC_BY_NAME[name]
@@ -345,7 +378,7 @@ def test_full_size_workload(cfg, tc_min_batch):
     x = wl.x_host()
     out = run_gpu(h, wl, x, n_layers=wl.layers)
     assert out["status"] == 0
-    assert h.launches_per_step() == wl.layers
+    assert h.launches_per_step() == _launches(h, wl)
     for l in range(wl.layers):
         np.testing.assert_allclose(out["layers"][l]["w"].sum(axis=1), 1.0, atol=1e-5)
     rows = list(range(wl.B))
