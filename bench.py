@@ -56,6 +56,9 @@ def parse_args(argv=None):
     ap.add_argument("--launch-log", default=None,
                     help="write every launch's workload, step, layer, unique experts and algorithmic "
                          "bytes (warm-up included) to this JSON file, to match ncu counters per launch")
+    ap.add_argument("--ingest-traffic", nargs=4, metavar=("NCU_CSV", "LAUNCH_LOG", "WORKLOAD", "COMMAND"),
+                    help="update profiles/traffic.json from an ncu DRAM-bytes capture and the --launch-log "
+                         "of the same command (no GPU work)")
     ap.add_argument("--tc-min-batch", type=int, default=None,
                     help="batch-shape switch: steps of at least this many rows take the tensor-core "
                          "kernel (0: always the CUDA-core kernel); default: the library's")
@@ -121,6 +124,56 @@ def traffic_per_launch(workload):
     """DRAM bytes per launch (ncu counters), or None (see traffic_entry)."""
     t = traffic_entry(workload)
     return None if t is None else t.get("bytes_per_launch")
+
+
+def ingest_traffic(csv_path, log_path, workload, command):
+    """Update profiles/traffic.json from an ncu CSV (dram__bytes_read.sum and
+    dram__bytes_write.sum of the captured moe_decode launches, in launch order) and this
+    bench's --launch-log of the same command: each captured launch is matched to the
+    step it ran (the -s count of skipped launches is read from `command`), and its DRAM
+    bytes are set beside that step's own algorithmic bytes (all layers of the step when
+    one launch runs the whole stack)."""
+    import csv
+    import re
+
+    per_launch = {}
+    with open(csv_path) as f:
+        rows = [r for r in csv.reader(l for l in f if not l.startswith("=="))]
+    head = rows[0]
+    ix = {k: head.index(k) for k in ("ID", "Kernel Name", "Metric Name", "Metric Value")}
+    for r in rows[1:]:
+        if len(r) < len(head) or "moe_decode" not in r[ix["Kernel Name"]]:
+            continue
+        d = per_launch.setdefault(int(r[ix["ID"]]), {"kernel": r[ix["Kernel Name"]]})
+        d[r[ix["Metric Name"]]] = float(r[ix["Metric Value"]].replace(",", ""))
+    with open(log_path) as f:
+        log = [e for e in json.load(f) if e["workload"] == workload]
+    steps = sorted({e["step"] for e in log})
+    skip = int(re.search(r"-s\s+(\d+)", command).group(1))
+    fused = "fused" in next(iter(per_launch.values()))["kernel"]
+    launches = []
+    for n, lid in enumerate(sorted(per_launch)):
+        d = per_launch[lid]
+        traffic = d["dram__bytes_read.sum"] + d["dram__bytes_write.sum"]
+        if fused:  # one launch per step
+            step = steps[skip + n]
+            alg = sum(e["algorithmic_bytes"] for e in log if e["step"] == step)
+        else:  # one launch per layer, in step order
+            e = sorted(log, key=lambda e: (e["step"], e["layer"]))[skip + n]
+            step, alg = e["step"], e["algorithmic_bytes"]
+        launches.append({"step": step, "dram_read": d["dram__bytes_read.sum"],
+                         "dram_write": d["dram__bytes_write.sum"], "traffic": traffic,
+                         "algorithmic_bytes": alg, "ratio": round(traffic / alg, 4)})
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    t = json.load(open(tpath)) if os.path.exists(tpath) else {}
+    t[workload] = {"bytes_per_launch": round(sum(l["traffic"] for l in launches) / len(launches)),
+                   "traffic_over_algorithmic": round(sum(l["traffic"] for l in launches)
+                                                     / sum(l["algorithmic_bytes"] for l in launches), 4),
+                   "launches": launches, "kernel": per_launch[sorted(per_launch)[0]]["kernel"],
+                   "source": command, "kernel_sources_sha256": kernel_source_hash()}
+    with open(tpath, "w") as f:
+        json.dump(t, f, indent=1)
+    return t[workload]
 
 
 def workload_config(wl, flush):
@@ -329,7 +382,9 @@ class ConfigRun:
 
         self.wl = wl
         self.dev = f"cuda:{device}"
-        variants = [wl] if wl.layers > 1 else [wl, dataclasses.replace(wl, seed=wl.seed + 100)]
+        # (the small profiling layers keep one set: a full ncu capture holds ~3 GB)
+        one = wl.layers > 1 or wl.name.endswith("_profile")
+        variants = [wl] if one else [wl, dataclasses.replace(wl, seed=wl.seed + 100)]
         self.sets = []
         for v in variants:
             layers = [v.device_layer(l, device=self.dev) for l in range(wl.layers)]
@@ -543,6 +598,9 @@ def run_ours(args, wl):
 
 def main(argv=None):
     args = parse_args(argv)
+    if args.ingest_traffic:
+        print(json.dumps(ingest_traffic(*args.ingest_traffic), indent=1))
+        return
     wl = synth.WORKLOADS[args.config]
     if args.profile_small:
         wl = synth.Workload("b1_h7168_e64_k16_profile", B=1, H=7168, E=64, k=16, I=1024, Is=2048, seed=1)

@@ -48,3 +48,43 @@ def test_traffic_applies_only_to_the_captured_sources(tmp_path, monkeypatch):
     assert bench.traffic_per_launch("other") is None
     monkeypatch.setattr(bench, "kernel_source_hash", lambda: "changed")
     assert bench.traffic_per_launch("w") is None
+
+
+def test_ingest_traffic_matches_each_captured_launch_to_its_own_step(tmp_path, monkeypatch):
+    """Captured launches (after -s skipped ones) are set beside the algorithmic bytes of
+    the step they ran; a launch that runs a whole layer stack is set beside all of that
+    step's layers."""
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "h")
+    head = '"ID","Kernel Name","Metric Name","Metric Unit","Metric Value"\n'
+
+    def csv_of(kernel, vals):
+        out = head
+        for i, (r, w) in enumerate(vals):
+            out += f'"{i}","{kernel}","dram__bytes_read.sum","byte","{r:,}"\n'
+            out += f'"{i}","{kernel}","dram__bytes_write.sum","byte","{w}"\n'
+        return out
+
+    # one layer: steps 0..4, U differs per step; launches 3 and 4 captured
+    wl = synth.WORKLOADS[2]
+    log = [{"workload": wl.name, "step": s, "layer": 0, "timed": s >= 3, "unique_experts": 100 + s,
+            "algorithmic_bytes": bench.step_bytes(wl, [100 + s])} for s in range(5)]
+    (tmp_path / "log.json").write_text(json.dumps(log))
+    (tmp_path / "a.csv").write_text(csv_of("moe_decode_layer_kernel<false,true>", [(5_000_000_000, 1000),
+                                                                                    (5_100_000_000, 2000)]))
+    t = bench.ingest_traffic(str(tmp_path / "a.csv"), str(tmp_path / "log.json"), wl.name, "ncu -s 3 -c 2 x")
+    assert [l["step"] for l in t["launches"]] == [3, 4]
+    assert t["launches"][0]["algorithmic_bytes"] == bench.step_bytes(wl, [103])
+    assert t["launches"][1]["traffic"] == 5_100_002_000
+    assert t["bytes_per_launch"] == round((5_000_001_000 + 5_100_002_000) / 2)
+    assert bench.traffic_per_launch(wl.name) == t["bytes_per_launch"]
+    # a two-layer stack in one launch per step: both layers' bytes of the step
+    v = synth.WORKLOADS[4]
+    log = [{"workload": v.name, "step": s, "layer": l, "timed": s >= 1, "unique_experts": 80 + l,
+            "algorithmic_bytes": bench.step_bytes(v, [80 + l])} for s in range(3) for l in range(2)]
+    (tmp_path / "log2.json").write_text(json.dumps(log))
+    (tmp_path / "b.csv").write_text(csv_of("moe_decode_fused_kernel<false>", [(7_000_000_000, 0)]))
+    t = bench.ingest_traffic(str(tmp_path / "b.csv"), str(tmp_path / "log2.json"), v.name, "ncu -s 1 -c 1 x")
+    assert t["launches"][0]["step"] == 1
+    assert t["launches"][0]["algorithmic_bytes"] == bench.step_bytes(v, [80, 81])
