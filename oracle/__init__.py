@@ -81,6 +81,10 @@ def _load(path):
         lib.oracle_layer_selected.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Weights), i, vp,
                                               vp, vp, vp, vp, vp, vp]
         lib.oracle_layer_selected.restype = i
+        lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_to_double.restype = d
+        lib.oracle_dequant_e4m3.argtypes = [i, i, vp, vp, vp]
+        lib.oracle_dequant_e4m3.restype = i
         _libs[path] = lib
     return _libs[path]
 
@@ -100,7 +104,7 @@ def _p(a):
 MUTANTS = {
     1: "no_n_round", 2: "no_h_round", 3: "residual_n", 4: "ties_high", 5: "equal_weights",
     6: "no_shared", 7: "silu_on_up", 8: "no_gamma", 9: "down_transposed", 10: "no_bias",
-    11: "eps_outside",
+    11: "eps_outside", 12: "e4m3_bias", 13: "block_transposed",
 }
 
 
@@ -170,6 +174,29 @@ def swiglu(n: np.ndarray, wg_bits, wu_bits, wd_bits) -> np.ndarray:
     return out
 
 
+# ---- FP8 expert weights ----------------------------------------------------------------
+
+def e4m3_value(code: int) -> float:
+    return _L().oracle_e4m3_to_double(int(code))
+
+
+def dequant_e4m3(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """bf16 bits of value(code) * scale of its 128 x 128 block ([rows, cols] codes,
+    [ceil(rows/128), ceil(cols/128)] scales); raises if a product is not a bf16 value."""
+    q = _c(codes, np.uint8)
+    rows, cols = q.shape
+    sc = _c(scales, np.float32)
+    out = np.empty((rows, cols), dtype=np.uint16)
+    if _L().oracle_dequant_e4m3(rows, cols, _p(q), _p(sc), _p(out)) != OK:
+        raise ValueError("oracle_dequant_e4m3: a dequantised weight is not a bf16 value")
+    return out
+
+
+def fp8_expert(fp8: dict):
+    """(W_g, W_u, W_d) bf16 bits of an expert given as {gate, up, down: (codes, scales)}."""
+    return tuple(dequant_e4m3(*fp8[m]) for m in ("gate", "up", "down"))
+
+
 # ---- whole layer -------------------------------------------------------------------
 
 def layer(dims: dict, weights: dict, x_bits: np.ndarray, selection=None) -> dict:
@@ -232,13 +259,14 @@ def layer(dims: dict, weights: dict, x_bits: np.ndarray, selection=None) -> dict
 
 
 def workload_layer(wl, layer_index: int, x_bits: np.ndarray, shared=None, w_router=None,
-                   selection=None) -> dict:
+                   selection=None, fp8: bool = False) -> dict:
     """Oracle of one layer of a ``synth.Workload`` on rows x_bits [B, H].
 
     Only the experts that the rows select are regenerated on the host (one row
     at a time, so host memory stays at 16 experts). ``shared`` and ``w_router``
     may be passed in to avoid regenerating them for every call. ``selection``
-    (int [B, k], optional) gives each row's experts instead of its top-k.
+    (int [B, k], optional) gives each row's experts instead of its top-k. ``fp8``: the
+    experts are the workload's FP8 ones (E4M3 codes and block scales, dequantised).
     """
     dims = dict(H=wl.H, E=wl.E, k=wl.k, I=wl.I, Is=wl.Is, eps=wl.eps)
     gamma = wl.gamma_host(layer_index)
@@ -254,7 +282,8 @@ def workload_layer(wl, layer_index: int, x_bits: np.ndarray, shared=None, w_rout
             given = None
         else:
             sel = given = np.asarray(selection[b], dtype=np.int32).reshape(1, wl.k)
-        experts = {int(e): wl.expert_host(layer_index, int(e)) for e in np.ravel(sel)}
+        experts = {int(e): (fp8_expert(wl.expert_fp8_host(layer_index, int(e))) if fp8
+                            else wl.expert_host(layer_index, int(e))) for e in np.ravel(sel)}
         outs.append(layer(dims, dict(gamma=gamma, w_router=wr, router_bias=bias, experts=experts,
                                      ws_gate=sg, ws_up=su, ws_down=sd), x[b:b + 1], selection=given))
         del experts

@@ -174,6 +174,36 @@ void oracle_swiglu(int H, int F, const double* n, const uint16_t* wg, const uint
   free(u);
 }
 
+/* ---- FP8 expert weights ---------------------------------------------------------- */
+
+/* The value of an FP8 E4M3 code (OCP FP8 "E4M3": 1 sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent field 0 is subnormal, m/8 * 2^-6; S.1111.111 is
+ * NaN; there are no infinities). */
+double oracle_e4m3_to_double(uint8_t code) {
+  const int sgn = (code >> 7) & 1, ex = (code >> 3) & 15, m = code & 7;
+  if (ex == 15 && m == 7) return NAN;
+  const int bias = MUT(ORACLE_MUT_E4M3_BIAS) ? 8 : 7;
+  const double mag = ex == 0 ? ldexp((double)m / 8.0, 1 - bias) : ldexp(1.0 + (double)m / 8.0, ex - bias);
+  return sgn ? -mag : mag;
+}
+
+/* Dequantises a [rows][cols] matrix of E4M3 codes with one scale per 128 x 128 block
+ * (scales [ceil(rows/128)][ceil(cols/128)]): w = value(code) * scale, returned as bf16
+ * bits. The layer with FP8 expert weights is the bf16 layer evaluated on these weights,
+ * so every w must be a bf16 value: ORACLE_EINVAL if one is not (or a code is NaN). */
+int oracle_dequant_e4m3(int rows, int cols, const uint8_t* codes, const float* scales, uint16_t* out) {
+  const int cb = (cols + 127) / 128;
+  for (int r = 0; r < rows; ++r)
+    for (int c = 0; c < cols; ++c) {
+      const size_t blk = MUT(ORACLE_MUT_BLOCK_TRANSPOSED) ? (size_t)(c / 128) * ((rows + 127) / 128) + r / 128
+                                                          : (size_t)(r / 128) * cb + c / 128;
+      const double w = oracle_e4m3_to_double(codes[(size_t)r * cols + c]) * (double)scales[blk];
+      if (!isfinite(w) || oracle_bf16_round(w) != w) return ORACLE_EINVAL;
+      out[(size_t)r * cols + c] = oracle_double_to_bf16_bits(w);
+    }
+  return ORACLE_OK;
+}
+
 /* ---- whole layer ------------------------------------------------------------ */
 
 /* The output of one row once its selection and weights are known:

@@ -45,7 +45,9 @@ typedef struct {
 #define ORACLE_MUT_DOWN_TRANSPOSED 9 /* down projection read transposed */
 #define ORACLE_MUT_NO_BIAS 10        /* router bias dropped */
 #define ORACLE_MUT_EPS_OUTSIDE 11    /* eps added outside the square root */
-#define ORACLE_MUT_COUNT 12
+#define ORACLE_MUT_E4M3_BIAS 12      /* E4M3 exponent bias 8 instead of 7 */
+#define ORACLE_MUT_BLOCK_TRANSPOSED 13 /* FP8 block scales indexed [col block][row block] */
+#define ORACLE_MUT_COUNT 14
 void oracle_set_mutant(int m);
 
 double oracle_bf16_to_double(uint16_t b);
@@ -59,6 +61,12 @@ int oracle_topk(int E, int k, const double* v, int32_t* idx_out);
 void oracle_softmax_selected(int k, const double* logits, const int32_t* idx, double* w_out);
 void oracle_swiglu(int H, int F, const double* n, const uint16_t* wg, const uint16_t* wu,
                    const uint16_t* wd, double* out);
+
+/* FP8 E4M3 code -> value (NaN for the NaN codes). */
+double oracle_e4m3_to_double(uint8_t code);
+/* [rows][cols] E4M3 codes times one scale per 128 x 128 block -> bf16 bits;
+ * ORACLE_EINVAL if a product is not a bf16 value or a code is NaN. */
+int oracle_dequant_e4m3(int rows, int cols, const uint8_t* codes, const float* scales, uint16_t* out);
 
 /* B rows; outputs: logits [B][E], topk_idx [B][k], topk_w [B][k], y_pre [B][H]
  * (fp64 before the final rounding; may be NULL), y [B][H] bf16 bits (may be NULL). */

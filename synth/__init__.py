@@ -38,6 +38,13 @@ KIND_X = 9
 KIND_BIAS_PERM = 10
 KIND_ROW_NOISE = 11
 KIND_ROW_BASE = 12
+KIND_WQ_GATE = 13   # FP8 expert weights: E4M3 codes
+KIND_WQ_UP = 14
+KIND_WQ_DOWN = 15
+KIND_SQ_GATE = 16   # FP8 expert weights: per-block scale exponents
+KIND_SQ_UP = 17
+KIND_SQ_DOWN = 18
+FP8_BLOCK = 128     # scale blocks are FP8_BLOCK x FP8_BLOCK elements
 
 
 def tensor_id(layer: int, kind: int) -> int:
@@ -84,6 +91,12 @@ def _host_lib():
         lib.ms_fill_rows_correlated.restype = None
         lib.ms_router_bias.argtypes = [u64, ctypes.c_uint32, ctypes.c_int, vp]
         lib.ms_router_bias.restype = None
+        lib.ms_fill_e4m3_host.argtypes = [u64, u64, u64, u64, vp]
+        lib.ms_fill_e4m3_host.restype = None
+        lib.ms_e4m3_encode_host.argtypes = [vp, u64, vp]
+        lib.ms_e4m3_encode_host.restype = None
+        lib.ms_block_exps_host.argtypes = [u64, u64, u64, u64, ctypes.c_int, vp]
+        lib.ms_block_exps_host.restype = None
         _host = lib
     return _host
 
@@ -97,6 +110,8 @@ def _cuda_lib():
         u64, f32, vp = ctypes.c_uint64, ctypes.c_float, ctypes.c_void_p
         lib.ms_fill_device.argtypes = [u64, u64, u64, u64, f32, f32, vp, vp]
         lib.ms_fill_device.restype = ctypes.c_int
+        lib.ms_fill_e4m3_device.argtypes = [u64, u64, u64, u64, vp, vp]
+        lib.ms_fill_e4m3_device.restype = ctypes.c_int
         _cuda = lib
     return _cuda
 
@@ -137,6 +152,42 @@ def router_bias(seed: int, layer: int, E: int) -> np.ndarray:
     out = np.empty(E, dtype=np.float32)
     _host_lib().ms_router_bias(seed, layer, E, _ptr(out))
     return out
+
+
+def fill_e4m3_host(seed: int, tid: int, start: int, n: int) -> np.ndarray:
+    """E4M3 codes (uint8) of elements start .. start + n - 1 of tensor tid."""
+    out = np.empty(int(n), dtype=np.uint8)
+    _host_lib().ms_fill_e4m3_host(seed, tid, start, n, _ptr(out))
+    return out
+
+
+def e4m3_encode_host(values) -> np.ndarray:
+    """The generator's encoder: the E4M3 code nearest each fp32 value (ties to even),
+    values clamped to [-448, 448]."""
+    v = np.ascontiguousarray(values, dtype=np.float32).ravel()
+    out = np.empty(v.size, dtype=np.uint8)
+    _host_lib().ms_e4m3_encode_host(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def block_exps_host(seed: int, tid: int, start: int, n: int, s0: int) -> np.ndarray:
+    """Scale exponents (s0 - 1, s0 or s0 + 1) of blocks start .. start + n - 1."""
+    out = np.empty(int(n), dtype=np.int32)
+    _host_lib().ms_block_exps_host(seed, tid, start, n, int(s0), _ptr(out))
+    return out
+
+
+def fp8_s0(fan_in: int) -> int:
+    """Central scale exponent of an FP8 matrix: 2^s0 * (448 / 6) is the power of two
+    nearest 1/sqrt(fan_in), so the dequantised weights have about the bf16 weights'
+    spread."""
+    return int(np.round(np.log2((1.0 / np.sqrt(float(fan_in))) / (448.0 / 6.0))))
+
+
+def fill_e4m3_device(ptr: int, seed: int, tid: int, start: int, n: int, stream: int = 0) -> None:
+    rc = _cuda_lib().ms_fill_e4m3_device(seed, tid, start, n, ctypes.c_void_p(ptr), ctypes.c_void_p(stream))
+    if rc != 0:
+        raise RuntimeError(f"ms_fill_e4m3_device failed with cudaError {rc}")
 
 
 def fill_device(ptr: int, seed: int, tid: int, start: int, n: int, sigma: float, mean: float = 0.0,
@@ -272,6 +323,60 @@ class Workload:
         out["ws_gate"] = out["ws_gate"].view(Is, H)
         out["ws_up"] = out["ws_up"].view(Is, H)
         out["ws_down"] = out["ws_down"].view(H, Is)
+        bias = self.bias_host(layer)
+        out["router_bias"] = None if bias is None else torch.from_numpy(bias).to(device)
+        return out
+
+    # ---- FP8 expert weights (E4M3 codes, one power-of-two scale per 128 x 128 block) ----
+    def fp8_matrices(self):
+        """(name, code kind, scale kind, rows, cols, fan_in) of each expert matrix."""
+        H, I = self.H, self.I
+        return [("gate", KIND_WQ_GATE, KIND_SQ_GATE, I, H, H), ("up", KIND_WQ_UP, KIND_SQ_UP, I, H, H),
+                ("down", KIND_WQ_DOWN, KIND_SQ_DOWN, H, I, I)]
+
+    def fp8_scales_host(self, layer: int, which: str, experts=None) -> np.ndarray:
+        """fp32 scales 2^exponent [len(experts)][rows/128][cols/128] of one matrix kind."""
+        name, _, sk, rows, cols, fan_in = next(m for m in self.fp8_matrices() if m[0] == which)
+        rb, cb = rows // FP8_BLOCK, cols // FP8_BLOCK
+        experts = range(self.E) if experts is None else experts
+        out = np.empty((len(experts), rb, cb), dtype=np.float32)
+        for i, e in enumerate(experts):
+            ex = block_exps_host(self.seed, tensor_id(layer, sk), int(e) * rb * cb, rb * cb, fp8_s0(fan_in))
+            out[i] = np.ldexp(np.float32(1.0), ex).astype(np.float32).reshape(rb, cb)
+        return out
+
+    def expert_fp8_host(self, layer: int, e: int):
+        """{gate, up, down: (E4M3 codes [rows, cols] uint8, fp32 block scales
+        [rows/128, cols/128])} of expert e."""
+        out = {}
+        for name, qk, _, rows, cols, _ in self.fp8_matrices():
+            codes = fill_e4m3_host(self.seed, tensor_id(layer, qk), e * rows * cols, rows * cols)
+            out[name] = (codes.reshape(rows, cols), self.fp8_scales_host(layer, name, [e])[0])
+        return out
+
+    def device_layer_fp8(self, layer: int, device="cuda", stream: int = 0) -> dict:
+        """One layer with FP8 expert weights, generated on the device: gamma, router and
+        shared expert bf16 as in device_layer; w_gate_q, w_up_q, w_down_q uint8 [E, rows,
+        cols] and w_gate_scale, w_up_scale, w_down_scale fp32 [E, rows/128, cols/128]."""
+        import torch
+
+        out = {}
+        for name, kind, numel, sigma, mean in self.device_specs(layer):
+            if name in ("w_gate", "w_up", "w_down"):
+                continue
+            t = torch.empty(int(numel), dtype=torch.bfloat16, device=device)
+            fill_device(t.data_ptr(), self.seed, tensor_id(layer, kind), 0, int(numel), sigma, mean, stream)
+            out[name] = t
+        H, E, Is = self.H, self.E, self.Is
+        out["w_router"] = out["w_router"].view(E, H)
+        out["ws_gate"] = out["ws_gate"].view(Is, H)
+        out["ws_up"] = out["ws_up"].view(Is, H)
+        out["ws_down"] = out["ws_down"].view(H, Is)
+        for name, qk, _, rows, cols, _ in self.fp8_matrices():
+            q = torch.empty((E, rows, cols), dtype=torch.uint8, device=device)
+            fill_e4m3_device(q.data_ptr(), self.seed, tensor_id(layer, qk), 0, E * rows * cols, stream)
+            out[f"w_{name}_q"] = q
+            out[f"w_{name}_scale"] = torch.from_numpy(self.fp8_scales_host(layer, name)).to(device)
         bias = self.bias_host(layer)
         out["router_bias"] = None if bias is None else torch.from_numpy(bias).to(device)
         return out

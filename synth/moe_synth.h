@@ -49,7 +49,13 @@ enum ms_kind {
   MS_KIND_X = 9,
   MS_KIND_BIAS_PERM = 10,
   MS_KIND_ROW_NOISE = 11,
-  MS_KIND_ROW_BASE = 12
+  MS_KIND_ROW_BASE = 12,
+  MS_KIND_WQ_GATE = 13, /* FP8 expert weights: e4m3 codes */
+  MS_KIND_WQ_UP = 14,
+  MS_KIND_WQ_DOWN = 15,
+  MS_KIND_SQ_GATE = 16, /* FP8 expert weights: per-block scale exponents */
+  MS_KIND_SQ_UP = 17,
+  MS_KIND_SQ_DOWN = 18
 };
 
 MS_FN uint64_t ms_tensor_id(uint32_t layer, uint32_t kind) {
@@ -115,6 +121,53 @@ MS_FN float ms_add_rn(float a, float b) {
 /* One generated element: bf16(mean + sigma * z). */
 MS_FN uint16_t ms_value_bf16(uint64_t key, uint64_t i, float sigma, float mean) {
   return ms_bf16_rne(ms_add_rn(mean, ms_mul_rn(sigma, ms_z(key, i))));
+}
+
+/*
+ * FP8 E4M3 inputs (the low-precision expert weights). A code is the E4M3 value
+ * (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; largest finite 448) nearest
+ * to the fp32 value v (ties to even), after v is clamped to [-448, 448]:
+ *   code(i) = e4m3(z(key, i) * (448 / 6))  -- the Irwin-Hall z in [-6, 6] spans the
+ *                                             whole finite range
+ * and every 128 x 128 block b of a matrix has a power-of-two scale 2^(s0 + d(b)),
+ * d(b) = word(key_s, b) mod 3 - 1 (so neighbouring blocks differ). Only input
+ * generation lives here: decoding a code and applying its scale is the layer's
+ * arithmetic, done separately by the oracle and by the GPU kernel.
+ */
+MS_FN uint8_t ms_e4m3_rne(float v) {
+  uint32_t u = ms_f32_bits(v);
+  const uint32_t sign = (u >> 24) & 0x80u;
+  float a = v < 0.0f ? -v : v;
+  if (!(a < 448.0f)) return (uint8_t)(sign | 0x7Eu); /* clamp (and any NaN) to the largest finite */
+  /* quantum of a's binade (normal for a >= 2^-6, else the subnormal spacing 2^-9) */
+  uint32_t ab = ms_f32_bits(a);
+  int e = (int)((ab >> 23) & 0xFFu) - 127;
+  if (e < -6) e = -6;
+  /* a / 2^(e-3), rounded to the nearest integer, ties to even: exact fp32 scaling */
+  union { uint32_t u; float f; } sc;
+  sc.u = (uint32_t)(127 - (e - 3)) << 23;
+  const float t = ms_mul_rn(a, sc.f);            /* in [0, 16) */
+  uint32_t q = (uint32_t)t;                       /* floor */
+  const float frac = t - (float)q;                /* exact */
+  if (frac > 0.5f || (frac == 0.5f && (q & 1u))) ++q;
+  /* value = q * 2^(e-3); q in [0, 16] (16: carried into the next binade) */
+  if (q == 0u) return (uint8_t)sign;
+  if (e == -6 && q < 8u) return (uint8_t)(sign | q); /* subnormal: exponent field 0 */
+  if (q == 16u) {
+    q = 8u;
+    ++e;
+  }
+  return (uint8_t)(sign | ((uint32_t)(e + 7) << 3) | (q - 8u));
+}
+
+/* One generated FP8 code (74.66666412353515625 is the fp32 value nearest 448 / 6). */
+MS_FN uint8_t ms_code_e4m3(uint64_t key, uint64_t i) {
+  return ms_e4m3_rne(ms_mul_rn(ms_z(key, i), 74.66666412353515625f));
+}
+
+/* Scale exponent of block b: s0 - 1, s0 or s0 + 1. */
+MS_FN int ms_block_exp(uint64_t key, uint64_t b, int s0) {
+  return s0 + (int)(ms_word(key, b) % 3ULL) - 1;
 }
 
 #endif /* MOE_SYNTH_H */

@@ -74,3 +74,22 @@ void ms_router_bias(uint64_t seed, uint32_t layer, int E, float* out) {
   for (int r = 0; r < E; ++r) out[perm[r]] = (float)(-2.2 * log((double)(r + 1)));
   free(perm);
 }
+
+/* out[i] = E4M3 code of element start + i of tensor tid (ms_code_e4m3), i < n. */
+void ms_fill_e4m3_host(uint64_t seed, uint64_t tensor_id, uint64_t start, uint64_t n, uint8_t* out) {
+  const uint64_t key = ms_key(seed, tensor_id);
+  int64_t i;
+#pragma omp parallel for schedule(static)
+  for (i = 0; i < (int64_t)n; ++i) out[i] = ms_code_e4m3(key, start + (uint64_t)i);
+}
+
+/* The E4M3 code nearest to each fp32 value (the generator's encoder; tests only). */
+void ms_e4m3_encode_host(const float* v, uint64_t n, uint8_t* out) {
+  for (uint64_t i = 0; i < n; ++i) out[i] = ms_e4m3_rne(v[i]);
+}
+
+/* Scale exponents of blocks start .. start + n - 1 of tensor tid: s0 - 1, s0 or s0 + 1. */
+void ms_block_exps_host(uint64_t seed, uint64_t tensor_id, uint64_t start, uint64_t n, int s0, int32_t* out) {
+  const uint64_t key = ms_key(seed, tensor_id);
+  for (uint64_t i = 0; i < n; ++i) out[i] = ms_block_exp(key, start + i, s0);
+}

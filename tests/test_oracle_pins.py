@@ -459,6 +459,67 @@ def test_layer_bias_enters_selection_and_weights():
         np.testing.assert_allclose(got["w"][b], softmax(lg[sel]), rtol=1e-13)
 
 
+# ---- FP8 expert weights ------------------------------------------------------------------
+
+def test_e4m3_decode_matches_an_independent_table():
+    """Every E4M3 code against torch's float8_e4m3fn conversion (NaN codes included)."""
+    import torch
+
+    codes = np.arange(256, dtype=np.uint8)
+    mine = np.array([oracle.e4m3_value(c) for c in codes])
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(mine), np.isnan(ref))
+    assert np.array_equal(mine[~np.isnan(mine)], ref[~np.isnan(ref)])
+
+
+def test_e4m3_decode_closed_forms():
+    # 1.0, the largest finite, the smallest subnormal and normal, signed zero and one
+    assert oracle.e4m3_value(0x38) == 1.0 and oracle.e4m3_value(0x7E) == 448.0
+    assert oracle.e4m3_value(0x01) == 2.0 ** -9 and oracle.e4m3_value(0x08) == 2.0 ** -6
+    assert oracle.e4m3_value(0x07) == 7 * 2.0 ** -9 and oracle.e4m3_value(0x0F) == 1.875 * 2.0 ** -6
+    assert oracle.e4m3_value(0xB8) == -1.0 and math.copysign(1.0, oracle.e4m3_value(0x80)) == -1.0
+    assert math.isnan(oracle.e4m3_value(0x7F)) and math.isnan(oracle.e4m3_value(0xFF))
+
+
+def test_dequant_applies_each_blocks_own_scale():
+    """Codes of value 1 (and a few others) in a 3 x 2 grid of 128 x 128 blocks whose
+    scales all differ: every weight is its code's value times its own block's scale."""
+    rows, cols = 384, 256
+    codes = np.full((rows, cols), 0x38, dtype=np.uint8)           # 1.0
+    codes[5, 200] = 0x3C                                          # 1.5 in block (0, 1)
+    codes[300, 7] = 0xC6                                          # -3.5 in block (2, 0)
+    scales = np.ldexp(np.float32(1.0), np.array([[0, 3], [-2, 5], [7, -9]])).astype(np.float32)
+    w = synth.bf16_bits_to_f32(oracle.dequant_e4m3(codes, scales)).astype(np.float64)
+    want = np.repeat(np.repeat(scales.astype(np.float64), 128, axis=0), 128, axis=1)
+    want[5, 200] *= 1.5
+    want[300, 7] *= -3.5
+    np.testing.assert_array_equal(w, want)
+
+
+def test_dequant_rejects_weights_bf16_cannot_hold():
+    codes = np.full((128, 128), 0x39, dtype=np.uint8)             # 1.125
+    with pytest.raises(ValueError):
+        oracle.dequant_e4m3(codes, np.array([[1.0 / 3.0]], dtype=np.float32))
+    codes[0, 0] = 0x7F                                            # NaN
+    with pytest.raises(ValueError):
+        oracle.dequant_e4m3(codes, np.array([[1.0]], dtype=np.float32))
+
+
+def test_fp8_layer_is_the_bf16_layer_on_the_dequantised_weights():
+    """The workload's FP8 experts, dequantised, drive the same layer definition: the
+    FP8 oracle layer equals oracle.layer given the dequantised expert matrices."""
+    wl = synth.Workload("pin_fp8", B=2, H=256, E=8, k=2, I=128, Is=128, seed=13)
+    x = wl.x_host()
+    got = oracle.workload_layer(wl, 0, x, fp8=True)
+    dims = dict(H=wl.H, E=wl.E, k=wl.k, I=wl.I, Is=wl.Is, eps=wl.eps)
+    sg, su, sd = wl.shared_host(0)
+    W = dict(gamma=wl.gamma_host(0), w_router=wl.w_router_host(0), router_bias=None, ws_gate=sg, ws_up=su,
+             ws_down=sd, experts={e: oracle.fp8_expert(wl.expert_fp8_host(0, e)) for e in range(wl.E)})
+    want = oracle.layer(dims, W, x)
+    for key in ("logits", "idx", "w", "y"):
+        assert np.array_equal(got[key], want[key]), key
+
+
 PIN_CHECKS = [
     lambda: test_topk_matches_full_stable_sort(16, 4),
     test_softmax_selected_two_experts_is_logistic,
@@ -470,6 +531,8 @@ PIN_CHECKS = [
     lambda: [test_layer_with_given_selection_closed_form(s) for s in range(4)],
     test_layer_zero_routed_down_gives_shared_only,
     test_layer_bias_enters_selection_and_weights,
+    test_e4m3_decode_matches_an_independent_table,
+    test_dequant_applies_each_blocks_own_scale,
 ]
 
 

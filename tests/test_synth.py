@@ -105,3 +105,28 @@ def test_workload_table():
     assert w[2].B == 8 and w[3].B == 64 and w[3].router == "zipf"
     assert w[4].B == 32 and w[4].layers == 2 and w[4].nseq * w[4].rows_per_seq == 32
     assert abs(w[1].weight_bytes_per_layer() / 1e9 - 39.56) < 0.05
+
+
+def test_e4m3_encoder_is_nearest_ties_to_even_as_an_independent_conversion():
+    """The generator's FP8 encoder against torch's float8_e4m3fn conversion on values
+    inside the finite range (the generator clamps to +-448 first), ties included."""
+    import torch
+
+    rng = np.random.default_rng(3)
+    v = np.concatenate([rng.standard_normal(50000) * 100, rng.standard_normal(50000) * 0.01,
+                        np.array([0.0, -0.0, 448.0, -448.0, 2.0 ** -10, 3 * 2.0 ** -10, 1.0625, 1.1875])])
+    v = np.clip(v, -448, 448).astype(np.float32)
+    want = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(synth.e4m3_encode_host(v), want)
+    # out-of-range values clamp to the largest finite code instead of NaN
+    assert list(synth.e4m3_encode_host(np.array([500.0, -1e30], dtype=np.float32))) == [0x7E, 0xFE]
+
+
+def test_fp8_block_scales_are_powers_of_two_around_the_weight_spread():
+    wl = synth.WORKLOADS[1]
+    s = wl.fp8_scales_host(0, "gate", [0, 1])
+    e = np.log2(s)
+    assert np.array_equal(e, np.round(e)) and s.shape == (2, wl.I // 128, wl.H // 128)
+    s0 = synth.fp8_s0(wl.H)
+    assert set(np.unique(e).astype(int)) <= {s0 - 1, s0, s0 + 1}
+    assert len(np.unique(e)) == 3
