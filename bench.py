@@ -39,6 +39,7 @@ FALLBACK_HBM_GBS = 6650.0
 POOL = 32
 FLUSH_BYTES = 256 << 20
 PER_CONFIG = (1, 2, 3, 4)  # the full-size workloads timed after the headline
+PER_CONFIG_FP8 = (1, 2)    # and the same layers with FP8 experts (synth.FP8_WORKLOADS)
 
 
 def parse_args(argv=None):
@@ -47,6 +48,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--config", type=int, default=1, help="workload index (synth.WORKLOADS)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="the workload with FP8 expert weights (synth.FP8_WORKLOADS[config])")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-baseline oracle budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -85,13 +88,14 @@ def measured_peaks():
 
 def step_bytes(wl, n_unique_per_layer, batch=None):
     """Algorithmic bytes of one step: every weight byte the step must read once
-    (router, shared expert, each unique selected expert) plus x, y and gamma."""
+    (router, shared expert, each unique selected expert as stored: bf16, or E4M3 codes
+    and their block scales) plus x, y and gamma."""
     B = wl.B if batch is None else batch
-    H, E, I, Is = wl.H, wl.E, wl.I, wl.Is
+    H, E, Is = wl.H, wl.E, wl.Is
     per_layer_fixed = 2 * (E * H + 3 * Is * H + H) + (4 * E if wl.router == "zipf" else 0)
     total = 0
     for U in n_unique_per_layer:
-        total += per_layer_fixed + int(U) * 3 * I * H * 2 + 2 * B * H * 2
+        total += per_layer_fixed + int(U) * wl.expert_bytes() + 2 * B * H * 2
     return total
 
 
@@ -179,7 +183,7 @@ def ingest_traffic(csv_path, log_path, workload, command):
 def workload_config(wl, flush):
     return {"workload": wl.name, "batch": wl.B, "hidden": wl.H, "experts": wl.E, "top_k": wl.k,
             "expert_inter": wl.I, "shared_inter": wl.Is, "layers": wl.layers,
-            "router": wl.router, "rows": wl.rows, "input_pool": POOL,
+            "router": wl.router, "rows": wl.rows, "expert_weights": wl.experts, "input_pool": POOL,
             "l2": flush, "parallelism": "replicas"}
 
 
@@ -387,8 +391,9 @@ class ConfigRun:
         variants = [wl] if one else [wl, dataclasses.replace(wl, seed=wl.seed + 100)]
         self.sets = []
         for v in variants:
-            layers = [v.device_layer(l, device=self.dev) for l in range(wl.layers)]
-            h = mdp.MoeDecode(wl.H, wl.E, wl.k, wl.I, wl.Is, wl.B, layers, eps=wl.eps, device=device)
+            layers = [v.device_layer_any(l, device=self.dev) for l in range(wl.layers)]
+            h = mdp.MoeDecode(wl.H, wl.E, wl.k, wl.I, wl.Is, wl.B, layers, eps=wl.eps, device=device,
+                              fp8=wl.is_fp8)
             if tc_min_batch is not None:
                 h.set_tc_min_batch(tc_min_batch)
             self.sets.append((layers, h))
@@ -553,8 +558,8 @@ def run_ours(args, wl):
     # own unique-expert bytes, with its own clock record
     per_config = {}
     launches = line["gpu_launches"]
-    for c in ([] if args.no_per_config else [c for c in PER_CONFIG if synth.WORKLOADS[c].name != wl.name]):
-        cw = synth.WORKLOADS[c]
+    others = [synth.WORKLOADS[c] for c in PER_CONFIG] + [synth.FP8_WORKLOADS[c] for c in PER_CONFIG_FP8]
+    for cw in ([] if args.no_per_config else [o for o in others if o.name != wl.name]):
         r = ConfigRun(cw, local, args.tc_min_batch)
         smp = ClockSampler(local)
         smp.start()
@@ -566,6 +571,7 @@ def run_ours(args, wl):
         c_ach = sum(c_bytes) / (c_local * 1e-3) / 1e9
         per_config[cw.name] = {
             "config": workload_config(cw, L2_PROTOCOL) | {"kernel_path": r.kernel_path},
+            "dtype": "fp8 (e4m3) experts, bf16 activations" if cw.is_fp8 else "bf16",
             "value": round(c_tot / (c_max * 1e-3) / 1e9, 2), "unit": "GB/s",
             **step_stats(c_ms),
             "tokens_per_s": round(world * cw.B * K / (c_max * 1e-3), 1),
@@ -601,7 +607,7 @@ def main(argv=None):
     if args.ingest_traffic:
         print(json.dumps(ingest_traffic(*args.ingest_traffic), indent=1))
         return
-    wl = synth.WORKLOADS[args.config]
+    wl = synth.FP8_WORKLOADS[args.config] if args.fp8 else synth.WORKLOADS[args.config]
     if args.profile_small:
         wl = synth.Workload("b1_h7168_e64_k16_profile", B=1, H=7168, E=64, k=16, I=1024, Is=2048, seed=1)
     if args.profile_small_tc:

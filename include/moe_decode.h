@@ -105,6 +105,36 @@ typedef struct {
   const void* ws_down;      /* [H][Is] */
 } moe_decode_layer_weights;
 
+/* Device pointers of one layer whose routed experts are stored in FP8: E4M3 codes
+ * (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; largest finite 448) with one
+ * power-of-two fp32 scale per 128 x 128 block of each expert matrix. A weight is
+ * value(code) * scale of its block, which must be exactly a bf16 value: the layer is
+ * then the bf16 layer on those weights. Every scale must be a power of two (either
+ * sign) in [2^-117, 2^7], the range in which the kernel's in-register decode is exact;
+ * moe_decode_create_fp8 reads the scales once and refuses any other value with
+ * MOE_ERR_INVALID_ARG. Router and shared expert stay bf16. All
+ * pointers 16-byte aligned (router_bias 4-byte aligned). The kernel reads the scale
+ * arrays in whole aligned 16-byte groups, so each scale allocation must stay readable
+ * up to the next 16-byte boundary past its last element (any cudaMalloc or torch
+ * allocation is).
+ * (A more aggressive quantisation format is named on page "Kimi K3推理吞吐提升1.68倍",
+ * intro, only as what the reported gain did not need; the format here is this
+ * library's reading.) */
+typedef struct {
+  const void* gamma;          /* bf16 [H] */
+  const void* w_router;       /* bf16 [E][H] */
+  const float* router_bias;   /* fp32 [E] or NULL */
+  const uint8_t* w_gate;      /* E4M3 [E][I][H] */
+  const float* w_gate_scale;  /* fp32 [E][I/128][H/128] */
+  const uint8_t* w_up;        /* E4M3 [E][I][H] */
+  const float* w_up_scale;    /* fp32 [E][I/128][H/128] */
+  const uint8_t* w_down;      /* E4M3 [E][H][I] */
+  const float* w_down_scale;  /* fp32 [E][H/128][I/128] */
+  const void* ws_gate;        /* bf16 [Is][H] */
+  const void* ws_up;          /* bf16 [Is][H] */
+  const void* ws_down;        /* bf16 [H][Is] */
+} moe_decode_layer_weights_fp8;
+
 /* Optional per-layer debug outputs of a step (device pointers; any may be NULL). */
 typedef struct {
   float* logits;      /* fp32 [B][E]: router logits (bias included) */
@@ -122,6 +152,17 @@ typedef struct moe_decode_handle moe_decode_handle;
  * a handle owned by the caller (free it with moe_decode_destroy). */
 int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weights* layers,
                       int device, moe_decode_handle** out);
+
+/* moe_decode_create for layers with FP8 expert weights (moe_decode_layer_weights_fp8).
+ * Every dimension must be a multiple of 128 (MOE_ERR_UNSUPPORTED_SHAPE otherwise):
+ * steps of such a handle always take the tensor-core path, one launch per layer, and
+ * the expert tiles stream as E4M3 codes (half the bytes of bf16), turned into the bf16
+ * MMA operand in shared memory by the CTA's routing warps once the routing is done.
+ * Copies the scale arrays to the host once to check them (synchronous on `device`):
+ * MOE_ERR_INVALID_ARG for a scale outside the range above or a scale pointer that is
+ * not 16-byte aligned, MOE_ERR_CUDA if the copy fails. */
+int moe_decode_create_fp8(const moe_decode_config* cfg, const moe_decode_layer_weights_fp8* layers, int device,
+                          moe_decode_handle** out);
 
 /* One decode step over all layers. x_in: device bf16 [batch][H]; y_out: device
  * bf16 [batch][H] (may not alias x_in). 1 <= batch <= max_batch, 1 <= top_k <=

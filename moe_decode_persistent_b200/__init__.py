@@ -67,7 +67,7 @@ def build(verbose: bool = False) -> None:
 def declared_symbols() -> list[str]:
     """Function names declared by include/moe_decode.h."""
     text = open(HEADER).read()
-    return sorted(set(re.findall(r"\b(moe_decode_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(moe_decode_[a-z0-9_]+)\s*\(", text)))
 
 
 class Config(ctypes.Structure):
@@ -82,6 +82,19 @@ class LayerWeights(ctypes.Structure):
                 ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
                 ("ws_gate", ctypes.c_void_p), ("ws_up", ctypes.c_void_p),
                 ("ws_down", ctypes.c_void_p)]
+
+
+class LayerWeightsFp8(ctypes.Structure):
+    _fields_ = [("gamma", ctypes.c_void_p), ("w_router", ctypes.c_void_p),
+                ("router_bias", ctypes.c_void_p), ("w_gate", ctypes.c_void_p),
+                ("w_gate_scale", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
+                ("w_up_scale", ctypes.c_void_p), ("w_down", ctypes.c_void_p),
+                ("w_down_scale", ctypes.c_void_p), ("ws_gate", ctypes.c_void_p),
+                ("ws_up", ctypes.c_void_p), ("ws_down", ctypes.c_void_p)]
+
+
+# keys of a layer mapping with FP8 experts (synth.Workload.device_layer_fp8) per field
+_FP8_KEYS = {"w_gate": "w_gate_q", "w_up": "w_up_q", "w_down": "w_down_q"}
 
 
 class Debug(ctypes.Structure):
@@ -115,6 +128,9 @@ def _load(path):
         L.moe_decode_create.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerWeights), i,
                                         ctypes.POINTER(vp)]
         L.moe_decode_create.restype = i
+        L.moe_decode_create_fp8.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerWeightsFp8), i,
+                                            ctypes.POINTER(vp)]
+        L.moe_decode_create_fp8.restype = i
         L.moe_decode_step.argtypes = [vp, vp, vp, i, i, vp, vp]
         L.moe_decode_step.restype = i
         L.moe_decode_step_host.argtypes = [vp, vp, vp, i, i, vp, vp]
@@ -230,17 +246,24 @@ class MoeDecode:
     """
 
     def __init__(self, hidden, n_experts, top_k_max, inter, shared_inter, max_batch, layers,
-                 eps=1e-6, device=0, checked=False):
+                 eps=1e-6, device=0, checked=False, fp8=False):
         self._lib = lib(checked)  # checked: the bounds-checked test build of the library
         self.cfg = Config(hidden, n_experts, top_k_max, inter, shared_inter, max_batch,
                           len(layers), eps)
-        arr = (LayerWeights * len(layers))()
-        for i, w in enumerate(layers):
-            arr[i] = LayerWeights(*(_ptr(w.get(name)) for name, _ in LayerWeights._fields_))
         self._weights_keepalive = layers
         h = ctypes.c_void_p()
-        _check(self._lib.moe_decode_create(ctypes.byref(self.cfg), arr, int(device), ctypes.byref(h)),
-               "moe_decode_create")
+        if fp8:  # layers with FP8 experts: w_gate_q / w_gate_scale ... (moe_decode_create_fp8)
+            arr = (LayerWeightsFp8 * len(layers))()
+            for i, w in enumerate(layers):
+                arr[i] = LayerWeightsFp8(*(_ptr(w.get(_FP8_KEYS.get(name, name))) for name, _ in LayerWeightsFp8._fields_))
+            _check(self._lib.moe_decode_create_fp8(ctypes.byref(self.cfg), arr, int(device), ctypes.byref(h)),
+                   "moe_decode_create_fp8")
+        else:
+            arr = (LayerWeights * len(layers))()
+            for i, w in enumerate(layers):
+                arr[i] = LayerWeights(*(_ptr(w.get(name)) for name, _ in LayerWeights._fields_))
+            _check(self._lib.moe_decode_create(ctypes.byref(self.cfg), arr, int(device), ctypes.byref(h)),
+                   "moe_decode_create")
         self.handle = h
         self.n_layers = len(layers)
 
@@ -303,7 +326,8 @@ class MoeDecode:
                     "prod_loop_cyc", "router_seen", "sched_built", "topk_done", "topk_synced",
                     "unique_done", "n_published", "topk_loaded", "topk_selected", "topk_chosen",
                     "topk_cyc", "sched_placed", "sched_sorted", "start_clk", "r39", "roles",
-                    "first_tma", "norm_summed", "norm_reduced", "norm_stored", "r45", "r46", "r47")
+                    "first_tma", "norm_summed", "norm_reduced", "norm_stored", "conv_wait_cyc", "conv_work_cyc",
+                    "mma_wait_conv_cyc")
 
     def trace_slots(self) -> int:
         return self._lib.moe_decode_trace_slots(self.handle)

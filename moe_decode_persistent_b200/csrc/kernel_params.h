@@ -28,7 +28,11 @@ enum TensorMapSlot {
   TM_T_AN = 14,   // normalised rows n  [max_batch][H]
   TM_T_AHS = 15,  // shared SwiGLU rows [max_batch][Is]
   TM_T_AHE = 16,  // expert SwiGLU rows [slots][I]
-  TM_COUNT = 17
+  // FP8 expert weights (E4M3 codes, one byte each): boxes of 128 rows x 64 codes, no swizzle
+  TM_Q_WG = 17,   // W_gate codes [E*I][H]
+  TM_Q_WU = 18,   // W_up codes   [E*I][H]
+  TM_Q_WD = 19,   // W_down codes [E*H][I]
+  TM_COUNT = 20
 };
 
 // Counters of one layer step (reset by the last CTA of every launch, except the epoch).
@@ -106,6 +110,10 @@ struct Params {
   const CUtensorMap* tmaps;  // TM_COUNT maps in global memory
   const uint16_t* gamma;     // bf16 [H]
   const float* bias;         // fp32 [E] or nullptr
+  int fp8;                   // 1: expert weights are E4M3 codes (TM_Q_*) with block scales below
+  const float* sc_gate;      // fp32 [E][I/128][H/128]: 2^s of each 128 x 128 block
+  const float* sc_up;        // fp32 [E][I/128][H/128]
+  const float* sc_down;      // fp32 [E][H/128][I/128]
   // workspace
   uint16_t* n;           // bf16 [maxB][H]
   float* logits;         // fp32 [maxB][E]
@@ -197,6 +205,9 @@ enum TraceSlot {
   TR_NORM_SUMMED = 42,         // RMSNorm: first row's x and gamma loaded and squares summed (stamp)
   TR_NORM_REDUCED = 43,        // RMSNorm: the row's sum of squares known to every routing warp (stamp)
   TR_NORM_STORED = 44,         // RMSNorm: the row's n stored and fenced (stamp)
+  TR_CONV_WAIT_CYC = 45,       // FP8 converter warp 0 cycles waiting for stages
+  TR_CONV_WORK_CYC = 46,       // FP8 converter warp 0 cycles converting
+  TR_MMA_WAIT_CONV_CYC = 47,   // MMA warp cycles waiting for converted FP8 stages
   kTraceSlots = 48
 };
 

@@ -18,6 +18,8 @@ size_t tc_smem_bytes();
 int tc_threads_per_cta();
 const void* tc_kernel_fn();
 const void* tc_kernel_fn_trace();
+const void* tc_fp8_kernel_fn();
+const void* tc_fp8_kernel_fn_trace();
 const void* fused_kernel_fn();
 const void* fused_kernel_fn_trace();
 }  // namespace moe
@@ -34,6 +36,7 @@ struct moe_decode_handle {
   int device;
   int num_sms;
   moe_decode_layer_weights* layers;
+  moe_decode_layer_weights_fp8* layers_fp8;  // FP8 handles: the layers as given (else nullptr)
   CUtensorMap* d_tmaps;  // [n_layers][TM_COUNT]
   // workspace
   void* ws;              // one allocation, carved below
@@ -97,6 +100,57 @@ static int encode_2d(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint
   return encode_box(enc, map, base, rows, cols, box_cols, (uint32_t)moe::kBoxRows, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
+// FP8 expert codes: boxes of 128 rows x 64 one-byte codes, no swizzle (the routing warps
+// read them and write the swizzled bf16 operand).
+// E4M3 codes [rows][cols], box 64 columns x 128 rows (64 bytes a row), 64-byte swizzled:
+// 16-byte chunk c of box row r lands at chunk c ^ ((r / 2) mod 4) of the row, so the
+// converters, one row per lane, read distinct banks.
+static int encode_fp8(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return MOE_ERR_INVALID_ARG;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols};
+  cuuint32_t box[2] = {(cuuint32_t)moe::kTcAtomK, (cuuint32_t)moe::kTcRows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Every FP8 block scale must be a power of two in [2^-117, 2^7] (either sign): the
+// kernel turns a code into the bf16 value(code) x 2^-120 (exact; a bf16 subnormal for
+// the E4M3 subnormals) and multiplies by scale x 2^120 (a bf16 normal for these scales),
+// so the product is the weight value(code) x scale exactly and never a subnormal.
+static bool fp8_scale_ok(float s) {
+  uint32_t b;
+  memcpy(&b, &s, 4);
+  const int ex = (int)((b >> 23) & 0xFFu) - 127;
+  return (b & 0x7FFFFFu) == 0u && ex >= -117 && ex <= 7 && ((b >> 23) & 0xFFu) != 0u;
+}
+
+static int check_fp8_scales(const moe_decode_layer_weights_fp8* f, int L, int E, int I, int H) {
+  const size_t n = (size_t)E * (I / moe::kTcRows) * (H / moe::kTcRows);
+  float* buf = (float*)malloc(n * sizeof(float));
+  if (!buf) return MOE_ERR_NO_MEMORY;
+  int rc = MOE_OK;
+  for (int l = 0; l < L && rc == MOE_OK; ++l) {
+    const float* arr[3] = {f[l].w_gate_scale, f[l].w_up_scale, f[l].w_down_scale};
+    for (int a = 0; a < 3 && rc == MOE_OK; ++a) {
+      if (cudaMemcpy(buf, arr[a], n * sizeof(float), cudaMemcpyDeviceToHost) != cudaSuccess) {
+        rc = MOE_ERR_CUDA;
+        break;
+      }
+      for (size_t i = 0; i < n; ++i)
+        if (!fp8_scale_ok(buf[i])) {
+          rc = MOE_ERR_INVALID_ARG;
+          break;
+        }
+    }
+  }
+  free(buf);
+  return rc;
+}
+
 // Tensor-core path boxes: 64 columns (one 128-byte swizzle atom) x `box_rows` rows.
 static int encode_tc(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                      uint32_t box_rows) {
@@ -127,8 +181,10 @@ const char* moe_decode_strerror(int code) {
   }
 }
 
-int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weights* layers,
-                      int device, moe_decode_handle** out) {
+// Both create entry points: layers (bf16 experts), or fp8 (FP8 experts; layers then
+// holds the same layers with the expert pointers set to the codes, for the checks).
+static int create_impl(const moe_decode_config* cfg, const moe_decode_layer_weights* layers,
+                       const moe_decode_layer_weights_fp8* fp8, int device, moe_decode_handle** out) {
   if (!cfg || !layers || !out) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   const moe_decode_config c = *cfg;
@@ -170,11 +226,20 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   // the tensor-core kernel: only for shapes whose every dimension is a multiple of 128,
   // and only if it can be made co-resident; otherwise every step takes the CUDA-core kernel
   int tc_ok = tc_shape_ok(c) ? 1 : 0;
+  if (fp8 && !tc_ok) return MOE_ERR_UNSUPPORTED_SHAPE;  // FP8 experts: tensor-core path only
+  if (fp8) {
+    const int rc = check_fp8_scales(fp8, c.n_layers, c.n_experts, c.inter, c.hidden);
+    if (rc != MOE_OK) return rc;
+  }
   if (tc_ok) {
     const size_t tsm = moe::tc_smem_bytes();
     e = cudaFuncSetAttribute(moe::tc_kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::tc_kernel_fn_trace(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::tc_fp8_kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::tc_fp8_kernel_fn_trace(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::fused_kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e == cudaSuccess)
@@ -205,12 +270,17 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   h->tc_min_batch = kDefaultTcMinBatch;
   h->layers = (moe_decode_layer_weights*)malloc(sizeof(moe_decode_layer_weights) * c.n_layers);
   memcpy(h->layers, layers, sizeof(moe_decode_layer_weights) * c.n_layers);
+  if (fp8) {
+    h->layers_fp8 = (moe_decode_layer_weights_fp8*)malloc(sizeof(moe_decode_layer_weights_fp8) * c.n_layers);
+    memcpy(h->layers_fp8, fp8, sizeof(moe_decode_layer_weights_fp8) * c.n_layers);
+  }
 
   const int H = c.hidden, E = c.n_experts, I = c.inter, Is = c.shared_inter, L = c.n_layers;
   // host tensor maps
   CUtensorMap* maps = (CUtensorMap*)aligned_alloc(64, sizeof(CUtensorMap) * moe::TM_COUNT * L);
   if (!maps) {
     free(h->layers);
+    free(h->layers_fp8);
     free(h);
     return MOE_ERR_NO_MEMORY;
   }
@@ -220,18 +290,26 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
     const moe_decode_layer_weights& w = layers[l];
     CUtensorMap* m = maps + l * moe::TM_COUNT;
     rc |= encode_2d(enc, &m[moe::TM_WR], w.w_router, (uint64_t)E, (uint64_t)H);
-    rc |= encode_2d(enc, &m[moe::TM_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H);
-    rc |= encode_2d(enc, &m[moe::TM_WU], w.w_up, (uint64_t)E * I, (uint64_t)H);
-    rc |= encode_2d(enc, &m[moe::TM_WD], w.w_down, (uint64_t)E * H, (uint64_t)I);
+    if (!fp8) {  // (an FP8 handle never takes the CUDA-core path)
+      rc |= encode_2d(enc, &m[moe::TM_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H);
+      rc |= encode_2d(enc, &m[moe::TM_WU], w.w_up, (uint64_t)E * I, (uint64_t)H);
+      rc |= encode_2d(enc, &m[moe::TM_WD], w.w_down, (uint64_t)E * H, (uint64_t)I);
+    }
     rc |= encode_2d(enc, &m[moe::TM_WSG], w.ws_gate, (uint64_t)Is, (uint64_t)H);
     rc |= encode_2d(enc, &m[moe::TM_WSU], w.ws_up, (uint64_t)Is, (uint64_t)H);
     rc |= encode_2d(enc, &m[moe::TM_WSD], w.ws_down, (uint64_t)H, (uint64_t)Is);
     if (tc_ok) {
       const uint32_t R = (uint32_t)moe::kTcRows;
       rc |= encode_tc(enc, &m[moe::TM_T_WR], w.w_router, (uint64_t)E, (uint64_t)H, R);
-      rc |= encode_tc(enc, &m[moe::TM_T_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H, R);
-      rc |= encode_tc(enc, &m[moe::TM_T_WU], w.w_up, (uint64_t)E * I, (uint64_t)H, R);
-      rc |= encode_tc(enc, &m[moe::TM_T_WD], w.w_down, (uint64_t)E * H, (uint64_t)I, R);
+      if (fp8) {
+        rc |= encode_fp8(enc, &m[moe::TM_Q_WG], fp8[l].w_gate, (uint64_t)E * I, (uint64_t)H);
+        rc |= encode_fp8(enc, &m[moe::TM_Q_WU], fp8[l].w_up, (uint64_t)E * I, (uint64_t)H);
+        rc |= encode_fp8(enc, &m[moe::TM_Q_WD], fp8[l].w_down, (uint64_t)E * H, (uint64_t)I);
+      } else {
+        rc |= encode_tc(enc, &m[moe::TM_T_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H, R);
+        rc |= encode_tc(enc, &m[moe::TM_T_WU], w.w_up, (uint64_t)E * I, (uint64_t)H, R);
+        rc |= encode_tc(enc, &m[moe::TM_T_WD], w.w_down, (uint64_t)E * H, (uint64_t)I, R);
+      }
       rc |= encode_tc(enc, &m[moe::TM_T_WSG], w.ws_gate, (uint64_t)Is, (uint64_t)H, R);
       rc |= encode_tc(enc, &m[moe::TM_T_WSU], w.ws_up, (uint64_t)Is, (uint64_t)H, R);
       rc |= encode_tc(enc, &m[moe::TM_T_WSD], w.ws_down, (uint64_t)H, (uint64_t)Is, R);
@@ -240,6 +318,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   if (rc != MOE_OK) {
     free(maps);
     free(h->layers);
+    free(h->layers_fp8);
     free(h);
     return rc < 0 ? MOE_ERR_INVALID_ARG : rc;
   }
@@ -313,6 +392,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   if (e != cudaSuccess) {
     free(maps);
     free(h->layers);
+    free(h->layers_fp8);
     free(h);
     return MOE_ERR_NO_MEMORY;
   }
@@ -351,6 +431,8 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
       cudaFree(h->ws);
       free(maps);
       free(h->layers);
+      free(h->layers_fp8);
+    free(h->layers_fp8);
       free(h);
       return MOE_ERR_CUDA;
     }
@@ -364,6 +446,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   if (e != cudaSuccess) {
     cudaFree(h->ws);
     free(h->layers);
+    free(h->layers_fp8);
     free(h);
     return MOE_ERR_CUDA;
   }
@@ -371,14 +454,38 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   return MOE_OK;
 }
 
+int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weights* layers, int device,
+                      moe_decode_handle** out) {
+  return create_impl(cfg, layers, nullptr, device, out);
+}
+
+int moe_decode_create_fp8(const moe_decode_config* cfg, const moe_decode_layer_weights_fp8* layers, int device,
+                          moe_decode_handle** out) {
+  if (!cfg || !layers || !out || cfg->n_layers < 1 || cfg->n_layers > 8) return MOE_ERR_INVALID_ARG;
+  moe_decode_layer_weights w[8];
+  for (int l = 0; l < cfg->n_layers; ++l) {
+    const moe_decode_layer_weights_fp8& f = layers[l];
+    if (!f.w_gate_scale || !f.w_up_scale || !f.w_down_scale ||
+        ((reinterpret_cast<uintptr_t>(f.w_gate_scale) | reinterpret_cast<uintptr_t>(f.w_up_scale) |
+          reinterpret_cast<uintptr_t>(f.w_down_scale)) & 15u))
+      return MOE_ERR_INVALID_ARG;
+    w[l] = moe_decode_layer_weights{f.gamma, f.w_router, f.router_bias, f.w_gate, f.w_up, f.w_down,
+                                    f.ws_gate, f.ws_up, f.ws_down};
+  }
+  return create_impl(cfg, w, layers, device, out);
+}
+
 static bool use_tc(const moe_decode_handle* h, int batch) {
+  if (h->layers_fp8) return true;  // FP8 experts: the tensor-core kernel only
   return h->tc_capable && h->tc_min_batch > 0 && batch >= h->tc_min_batch;
 }
 
 // A tensor-core step of several layers runs them all in one launch (the fused kernel);
 // otherwise one launch per layer.
 static bool fused_step(const moe_decode_handle* h, int batch) {
-  return use_tc(h, batch) && h->cfg.n_layers > 1;
+  // (an FP8 layer's routing warps convert its expert tiles after the routing, so they
+  // cannot route the next layer meanwhile: FP8 stacks run one launch per layer)
+  return use_tc(h, batch) && h->cfg.n_layers > 1 && !h->layers_fp8;
 }
 
 static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, int batch, int top_k,
@@ -406,6 +513,12 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     p.tmaps = h->d_tmaps + l * moe::TM_COUNT;
     p.gamma = (const uint16_t*)w.gamma;
     p.bias = w.router_bias;
+    if (h->layers_fp8) {
+      p.fp8 = 1;
+      p.sc_gate = h->layers_fp8[l].w_gate_scale;
+      p.sc_up = h->layers_fp8[l].w_up_scale;
+      p.sc_down = h->layers_fp8[l].w_down_scale;
+    }
     p.n = h->n;
     p.logits = h->logits;
     p.hs = h->hs;
@@ -450,8 +563,9 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     p.trace = h->trace ? h->trace + (size_t)l * h->num_sms * moe::kTraceSlots : nullptr;
     if (fused) continue;
     void* args[] = {&p};
-    const void* fn = tc ? (h->trace ? moe::tc_kernel_fn_trace() : moe::tc_kernel_fn())
-                        : (h->trace ? moe::kernel_fn_trace() : moe::kernel_fn());
+    const void* fn = !tc             ? (h->trace ? moe::kernel_fn_trace() : moe::kernel_fn())
+                     : h->layers_fp8 ? (h->trace ? moe::tc_fp8_kernel_fn_trace() : moe::tc_fp8_kernel_fn())
+                                     : (h->trace ? moe::tc_kernel_fn_trace() : moe::tc_kernel_fn());
     const int threads = tc ? moe::tc_threads_per_cta() : moe::threads_per_cta();
     const size_t smem = tc ? moe::tc_smem_bytes() : moe::smem_bytes();
     cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(h->num_sms), dim3(threads), args, smem, stream);
@@ -550,6 +664,7 @@ void moe_decode_destroy(moe_decode_handle* h) {
   cudaSetDevice(h->device);
   cudaFree(h->ws);
   free(h->layers);
+  free(h->layers_fp8);
   free(h);
 }
 

@@ -6,8 +6,8 @@
 // 1.68倍", section "为什么解码阶段适合Megakernel"; page post.smzdm.com/p/a6zppe4g,
 // section "改了什么：每层 23 个 kernel 砍到 13 个": 23 -> 13 kernels per layer).
 //
-// Two instances of moe_decode_layer_kernel<trace, tc> implement the step; the host
-// picks one per step (the batch-shape switch):
+// Instances of moe_decode_layer_kernel<trace, tc, fp8> implement the step; the host
+// picks one per step (the batch-shape switch; fp8 for a handle with FP8 experts):
 //
 // Tensor-core kernel (tc = true, 14 warps)
 //   warp 0      producer: takes units of work from a global queue and streams, per
@@ -22,6 +22,10 @@
 //   warps 10-13 epilogue: read the accumulators (tcgen05.ld, one warp per lane
 //               quadrant) and finish the unit: split-K partials and fix-ups, SwiGLU,
 //               down partials and the per-row combine with the residual.
+//   FP8 experts (fp8 = true): the producer streams the expert tiles as E4M3 codes and
+//               their block scales; once the schedule is built the routing warps turn
+//               each stage into bf16 weights in tensor memory, which the MMA reads as
+//               its A operand (the bf16 instance has none of this code).
 //
 // CUDA-core kernel (tc = false, 10 warps)
 //   warp 0      producer: 32-row weight boxes and the activation rows (1-D bulk copies).
@@ -100,6 +104,14 @@ static_assert(tc_stages(16, 1) == 4 && tc_stages(16, 8) == 5 && tc_stages(32, 32
 constexpr int kTcAccBufs = 4;       // accumulator buffers in tensor memory
 constexpr int kTcAccCols = 128;     // columns per buffer: tile 0 at +0, tile 1 at +64
 constexpr int kTmemCols = kTcAccBufs * kTcAccCols;  // 512 (a power of two >= 32)
+// A layer with FP8 experts keeps 2 accumulator buffers (columns 0-255) and uses columns
+// 256-511 as 4 stages of the MMA's A operand: the converted bf16 weight tiles of an FP8
+// stage (tile j at +32 j; row m in lane m, K elements 2c and 2c + 1 in column c).
+constexpr int kFp8AccBufs = 2;
+constexpr int kFp8AStages = 4;
+constexpr int kFp8ACol0 = kFp8AccBufs * kTcAccCols;
+constexpr int kFp8AStageCols = 2 * kTcAtomK / 2;
+static_assert(kFp8ACol0 + kFp8AStages * kFp8AStageCols <= kTmemCols, "FP8 tensor-memory plan");
 
 static_assert(kTcSlotBytes % 1024 == 0 && kTcTileBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kCcRingBytes % 1024 == 0 && kTcRingBytes % 1024 == 0, "ring keeps the state block aligned");
@@ -121,6 +133,17 @@ constexpr int kInfoKpair = 1 << 2, kInfoSegEnd = 1 << 6, kInfoUnitEnd = 1 << 7, 
 // Tensor-core stages: bits 0-1 weight tiles, 2-4 activation boxes of 16 rows (N / 16),
 // 5 first stage of the unit (overwrite the accumulator), 6 last stage of the unit.
 constexpr int kTcInfoFirst = 1 << 5, kTcInfoLast = 1 << 6;
+// Tensor-core stage whose weight tiles arrive as E4M3 codes (8 KB per tile at the start
+// of the slot, tile 1 at +8 KB; 64 bytes a row, 64-byte swizzled) and are converted by
+// the routing warps into an A stage in tensor memory, which the MMA reads instead of
+// shared memory. With the codes, each tile's block scale lands in the slot at +16 KB
+// (tile j at +16 j: the aligned 16-byte group of the scale array that holds it), both
+// counted on Smem::wfull of the slot (the activations stay on full); the header's wrow
+// holds the scale's position in its group, tile 0 in bits 0-1, tile 1 in bits 2-3.
+constexpr int kTcInfoFp8 = 1 << 7;
+constexpr int kFp8TileBytes = kTcRows * kTcAtomK;  // 8 KB: 128 rows x 64 codes
+constexpr int kFp8ScaleOff = 2 * kFp8TileBytes;    // the scale groups of an FP8 stage in its slot
+constexpr int kCq = 8;                            // entries of the converter queue
 
 // Layout constants of one step (identical in every CTA).
 // On the tensor-core path RT and DT count tile pairs (256 rows), ST and IT 128-row
@@ -170,6 +193,12 @@ struct Smem {
   uint64_t acc_empty[kTcAccBufs];  // epilogue warps -> MMA warp
   uint64_t mma_bar;                // MMA warp: its last MMAs completed (drain)
   uint64_t epi_bar;                // rendezvous of the tensor-core epilogue warps (bounded)
+  uint64_t conv_bar[kTcStagesMax]; // FP8 stage of the slot converted (routing warps -> MMA warp)
+  uint64_t cq_full[kCq];           // converter queue: FP8 stages issued (producer -> routing warps)
+  uint64_t cq_empty[kCq];
+  uint64_t wfull[kTcStagesMax];    // FP8 stage: codes and scales of the slot landed
+  int16_t cq_slot[kCq];            // ring slot of the queued stage (-1: no more stages)
+  uint8_t cq_par[kCq];             // the slot's wfull parity for that stage
   StageHeader hdr[kMaxRingStages];
   int rb_unit[kRB];         // unit id of the buffer, or -1 (stop)
   int acc_unit[kTcAccBufs]; // unit id of the accumulator buffer, or -1 (stop)
@@ -201,6 +230,11 @@ struct Smem {
 };
 
 static_assert(kCcRingBytes + sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget of one CTA");
+// The CUDA-core path's result-buffer barriers (rb_full) serve a tensor-core launch with
+// FP8 experts as its A-stage barriers: the MMAs that read a tensor-memory A stage
+// completed (the two paths never run in one launch).
+static_assert(kFp8AStages <= kRB, "A-stage barriers");
+__device__ __forceinline__ uint64_t* astage_empty(Smem& sm) { return sm.rb_full; }
 static_assert(kTcRingBytes + sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget of one CTA");
 static_assert(offsetof(Smem, rb) % 16 == 0 && offsetof(Smem, fin) % 16 == 0, "float4 views of rb / fin");
 static_assert(offsetof(Smem, full) % 8 == 0 && offsetof(Smem, rb_full) % 8 == 0 &&
@@ -1746,8 +1780,39 @@ struct Producer {
   uint32_t phase;
   uint32_t pend_mask, pend_parity;
 
+  int cq_pos;        // converter queue: next entry and its phase
+  uint32_t cq_phase;
+  uint32_t wpar, wpend;  // FP8: per slot the parity of its next wfull phase; slots used
+
   __device__ Producer(const Params& p_, Smem& sm_, int lane_, int nst_)
-      : p(p_), sm(sm_), lane(lane_), nst(nst_), slot(0), phase(0u), pend_mask(0u), pend_parity(0u) {}
+      : p(p_), sm(sm_), lane(lane_), nst(nst_), slot(0), phase(0u), pend_mask(0u), pend_parity(0u), cq_pos(0),
+        cq_phase(0u), wpar(0u), wpend(0u) {}
+
+  // An FP8 stage in the current slot: the parity of the wfull phase its codes complete.
+  __device__ uint32_t mark_fp8() {
+    const uint32_t par = (wpar >> slot) & 1u;
+    wpar ^= 1u << slot;
+    wpend |= 1u << slot;
+    return par;
+  }
+  __device__ uint32_t last_wpar() const { return ((wpar >> slot) & 1u) ^ 1u; }
+
+  // Hands the FP8 stage in ring slot `s` (full-barrier parity `par`) to the converters;
+  // s = -1 tells them that no more stages follow.
+  __device__ bool push_conv(int s, uint32_t par) {
+    if (!wait_bar(&sm.cq_empty[cq_pos], cq_phase ^ 1u)) return false;
+    if (lane == 0) {
+      sm.cq_slot[cq_pos] = (int16_t)s;
+      sm.cq_par[cq_pos] = (uint8_t)par;
+      mbar_arrive(&sm.cq_full[cq_pos]);
+    }
+    __syncwarp();
+    if (++cq_pos == kCq) {
+      cq_pos = 0;
+      cq_phase ^= 1u;
+    }
+    return true;
+  }
 
   __device__ int grab() {
     int v = 0;
@@ -1812,7 +1877,8 @@ struct Producer {
 
   // After the last stage: the stop header and the drain of every bulk copy still in
   // flight.
-  __device__ void finish() {
+  __device__ void finish(bool fp8 = false) {
+    if (fp8) push_conv(-1, 0u);  // the converters stop (bounded: they also stop on abort)
     if (wait_slot()) {
       pend_mask &= ~(1u << slot);
       if (lane == 0) {
@@ -1828,6 +1894,16 @@ struct Producer {
         if (!((pend_mask >> s) & 1u)) continue;
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(&sm.full[s], (pend_parity >> s) & 1u)) {
+          if (globaltimer_ns() - t0 > 50000000ull) {
+            record_abort(p, MOE_ERR_TIMEOUT);
+            break;
+          }
+        }
+      }
+      for (int s = 0; s < nst; ++s) {  // FP8 codes and scales
+        if (!((wpend >> s) & 1u)) continue;
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&sm.wfull[s], ((wpar >> s) & 1u) ^ 1u)) {
           if (globaltimer_ns() - t0 > 50000000ull) {
             record_abort(p, MOE_ERR_TIMEOUT);
             break;
@@ -1995,8 +2071,12 @@ struct TcSeg {
   int arow;  // first activation row
   int dep;   // 0: normalised rows, 1: shared h, 2: the expert's h
   int pair;
+  int fp8;   // 1: the weight tiles are E4M3 codes (expert units of an FP8 layer)
+  const float* sc0;  // FP8: scales of tile 0 / tile 1 (K block 0 of the tile's rows)
+  const float* sc1;
 };
 
+template <bool kFp8>
 __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, const Sched& sc, const UnitDesc& d,
                                             TcSeg& x) {
   x.pair = d.pair;
@@ -2004,6 +2084,7 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
   x.N = sh.NA;
   x.ta = &p.tmaps[TM_T_AN];
   x.dep = 0;
+  x.fp8 = 0;
   switch (d.type) {
     case UT_ROUTER:
       x.tw0 = x.tw1 = &p.tmaps[TM_T_WR];
@@ -2021,10 +2102,16 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       // every token row is an MMA column; the epilogue keeps the expert's own rows
       int e = sc.slot_expert[sc.pair_slot[d.pair]];
       if (!IDX_OK(p, (unsigned)d.pair < (unsigned)kMaxSlots && (unsigned)e < (unsigned)p.E)) e = 0;
-      x.tw0 = &p.tmaps[TM_T_WG];
-      x.tw1 = &p.tmaps[TM_T_WU];
+      x.tw0 = &p.tmaps[kFp8 ? TM_Q_WG : TM_T_WG];
+      x.tw1 = &p.tmaps[kFp8 ? TM_Q_WU : TM_T_WU];
       x.y0 = x.y1 = e * p.I + d.tile * kTcRows;
       x.nbox = 2;
+      x.fp8 = kFp8;
+      if (kFp8) {  // gate and up blocks [e][tile][K block]
+        const size_t b = ((size_t)e * (p.I / kTcRows) + d.tile) * (p.H / kTcRows);
+        x.sc0 = p.sc_gate + b;
+        x.sc1 = p.sc_up + b;
+      }
       break;
     }
     case UT_DOWN_SHARED:
@@ -2041,7 +2128,12 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       if (!IDX_OK(p, (unsigned)i < (unsigned)kMaxE)) i = 0;
       int e = sc.slot_expert[i];
       if (!IDX_OK(p, (unsigned)e < (unsigned)p.E && (unsigned)sc.slot_base[i] < (unsigned)kMaxSlots)) e = 0;
-      x.tw0 = x.tw1 = &p.tmaps[TM_T_WD];
+      x.tw0 = x.tw1 = &p.tmaps[kFp8 ? TM_Q_WD : TM_T_WD];
+      x.fp8 = kFp8;
+      if (kFp8) {  // down blocks [e][row block 2 tile, 2 tile + 1][K block]
+        x.sc0 = p.sc_down + ((size_t)e * (p.H / kTcRows) + 2 * d.tile) * (p.I / kTcRows);
+        x.sc1 = x.sc0 + p.I / kTcRows;
+      }
       x.y0 = e * p.H + d.tile * 2 * kTcRows;
       x.y1 = x.y0 + kTcRows;
       x.nbox = d.tile * 2 * kTcRows + kTcRows < p.H ? 2 : 1;
@@ -2058,7 +2150,7 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
 // tiles and the activation operand (N rows, boxes of 16), all 128-byte swizzled.
 // last: the launch's last layer (then the stop header and the drain follow); false is
 // returned on abort (after the same stop header and drain).
-template <bool kTrace>
+template <bool kTrace, bool kFp8 = false>
 __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
   const Params& p = pr.p;
   Smem& sm = pr.sm;
@@ -2069,7 +2161,10 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
   // no-allocation path): the launch boundary orders them, no proxy fence is needed
   // (measured: one acquire fence per map cost ~4 us per step)
   if (lane == 0)
-    for (int t = TM_T_WR; t < TM_COUNT; ++t) prefetch_tensormap(&p.tmaps[t]);
+    for (int t = TM_T_WR; t < TM_COUNT; ++t) {
+      const bool qmap = t >= TM_Q_WG, bf16_expert = t == TM_T_WG || t == TM_T_WU || t == TM_T_WD;
+      if (kFp8 ? !bf16_expert : !qmap) prefetch_tensormap(&p.tmaps[t]);  // the maps this layer has
+    }
   if (p.layer > 0) {  // the previous layer's record of completed experts
     for (int w = lane; w < kMaxSlots / 32; w += 32) sm.known_done[w] = 0u;
     __syncwarp();
@@ -2110,30 +2205,50 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
     }
     if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(blockIdx.x * 7919u + (uint32_t)u) % 3000u);
     TcSeg x;
-    make_seg_tc(p, sh, sm.sc, d, x);
+    make_seg_tc<kFp8>(p, sh, sm.sc, d, x);
+    const bool xf = kFp8 && x.fp8;  // an FP8 stage (compiled out of the bf16 kernel)
     c_setup += (unsigned long long)(tclock<kTrace>() - tu0);
-    const uint32_t tx = (uint32_t)(x.nbox * kTcTileBytes + x.N * kTcAtomK * 2);
-    const int info0 = x.nbox | ((x.N / kTcActRows) << 2);
+    // bytes of a stage: on full the activations and (bf16) the weight tiles; on wfull the
+    // codes and scales of an FP8 stage
+    const uint32_t tx = (uint32_t)((xf ? 0 : x.nbox * kTcTileBytes) + x.N * kTcAtomK * 2);
+    const uint32_t wtx = (uint32_t)(x.nbox * (kFp8TileBytes + 16));
+    const int info0 = x.nbox | ((x.N / kTcActRows) << 2) | (xf ? kTcInfoFp8 : 0);
     const int ka_end = d.kb0 + d.nkb;
     // one stage: header, barrier armed for weights + activations, the weight tiles
     auto issue_weights = [&](int ka) {
       uint8_t* dst = ring + pr.slot * sh.slot_bytes;
       uint64_t* fb = &sm.full[pr.slot];
+      uint64_t* wb = &sm.wfull[pr.slot];
       pr.mark_pending();
+      if (xf) pr.mark_fp8();
       if (lane == 0) {
         StageHeader h;
         h.kind = HK_STAGE;
         h.unit = hunit;
         h.info = info0 | (ka == d.kb0 ? kTcInfoFirst : 0) | (ka == ka_end - 1 ? kTcInfoLast : 0);
-        h.wrow = -1;
+        h.wrow = xf ? (int)((((uintptr_t)(x.sc0 + (ka >> 1)) >> 2) & 3u) |
+                               ((((uintptr_t)(x.sc1 + (ka >> 1)) >> 2) & 3u) << 2))
+                       : -1;
         sm.hdr[pr.slot] = h;
+        if (xf) mbar_arrive_expect_tx(wb, wtx);
         mbar_arrive_expect_tx(fb, tx);
         if (kTrace && first_tma) {
           trace_stamp<kTrace>(p, TR_FIRST_TMA);
           first_tma = false;
         }
-        tma_load_2d(dst, x.tw0, ka * kTcAtomK, x.y0, fb, pol);
-        if (x.nbox == 2) tma_load_2d(dst + kTcTileBytes, x.tw1, ka * kTcAtomK, x.y1, fb, pol);
+        if (xf) {  // codes, converted into tensor memory by the routing warps
+          tma_load_2d(dst, x.tw0, ka * kTcAtomK, x.y0, wb, pol);
+          if (x.nbox == 2) tma_load_2d(dst + kFp8TileBytes, x.tw1, ka * kTcAtomK, x.y1, wb, pol);
+          // each tile's scale (K block ka / 2) in the aligned 16-byte group that holds it
+          const auto group = [](const float* s) {
+            return reinterpret_cast<const float*>(reinterpret_cast<uintptr_t>(s) & ~(uintptr_t)15);
+          };
+          bulk_load(dst + kFp8ScaleOff, group(x.sc0 + (ka >> 1)), 16, wb);
+          if (x.nbox == 2) bulk_load(dst + kFp8ScaleOff + 16, group(x.sc1 + (ka >> 1)), 16, wb);
+        } else {
+          tma_load_2d(dst, x.tw0, ka * kTcAtomK, x.y0, fb, pol);
+          if (x.nbox == 2) tma_load_2d(dst + kTcTileBytes, x.tw1, ka * kTcAtomK, x.y1, fb, pol);
+        }
       }
     };
     // the activation operand of stage ka into ring slot s (only after its publication)
@@ -2164,6 +2279,7 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
         if (!ok) break;
         issue_weights(ka);
         __syncwarp();
+        if (xf && !pr.push_conv(pr.slot, pr.last_wpar())) ok = false;
         pr.advance();
         ++c_stages;
       }
@@ -2198,6 +2314,7 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
       issue_weights(ka);
       issue_act(ka, slot);
       __syncwarp();
+      if (xf && !pr.push_conv(pr.slot, pr.last_wpar())) ok = false;
       pr.advance();
       c_issue += (unsigned long long)(tclock<kTrace>() - ti0);
       ++c_stages;
@@ -2221,7 +2338,7 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
     trace_put<kTrace>(p, TR_PROD_SCHED_CYC, c_schedw);
     trace_put<kTrace>(p, TR_PROD_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tploop0));
   }
-  if (last || !ok) pr.finish();
+  if (last || !ok) pr.finish(kFp8);
   return ok;
 }
 
@@ -2361,6 +2478,122 @@ __device__ void epilogue_cc(const Params& p, Smem& sm, int lane) {
   }
 }
 
+// ---- tensor-core path: FP8 converters (the routing warps, once the schedule exists) --------------
+
+// Four E4M3 codes (byte i of w = code i) to two bf16 pairs (codes 0, 1 and 2, 3), each
+// value(code) x 2^-120 exactly, with integer operations only: a code's 7 magnitude bits
+// (exponent field e, mantissa m) become the low bits of the bf16's exponent field and the
+// top 3 of its mantissa, so the bf16 reads 2^(e-127) (1 + m/8) = value x 2^-120 for e >= 1
+// and 2^-126 (m/8) = value x 2^-120 (a bf16 subnormal) for e = 0. With v = [0, c1, 0, c0]
+// in 16-bit lanes, adding 15 x (v's sign bits 7 and 23) moves each sign 4 places up
+// (bit 7 + 15 x 2^7 = 2^11), and the shift by 4 puts the magnitudes at bits 4-10 of their
+// lanes and the signs at bits 15 and 31.
+__device__ __forceinline__ void e4m3x4_to_bf16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t v0 = __byte_perm(w, 0u, 0x4140), v1 = __byte_perm(w, 0u, 0x4342);
+  lo = (v0 + 15u * (v0 & 0x00800080u)) << 4;
+  hi = (v1 + 15u * (v1 & 0x00800080u)) << 4;
+}
+
+// bf16 pair (s x 2^120, s x 2^120) of a power-of-two fp32 scale s in [2^-117, 2^7]: times
+// a converted code it gives the weight value(code) x s exactly (a bf16 normal, >= 2^-126).
+__device__ __forceinline__ uint32_t scale_bf16x2(float s) {
+  // exact: a power of two has no mantissa bits; the exponent field grows by 120
+  const uint32_t b = (__float_as_uint(s) >> 16) + (120u << 7);
+  return (b << 16) | b;
+}
+
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// The routing warps turn every FP8 stage (handed over by the producer through the
+// converter queue) into the MMA's A operand in tensor memory: warp w (of 8) converts
+// tile w / 4 of the stage, lane l the tile row 32 q + l of its lane quadrant q, each
+// code times the scale of its 128 x 128 block, and stores the row's 64 bf16 values as
+// 32 columns of its lane. The codes sit 64-byte swizzled (chunk c of row r at chunk
+// c ^ ((r / 2) mod 4) of the row), so the 8 lanes of a shared-memory phase read 8
+// distinct 16-byte chunks while the whole warp reads one logical chunk. A stages
+// rotate in stage order; one is rewritten only after the MMAs that read it completed.
+// The warps need nothing from one another: each waits for the stage itself (bounded)
+// and signals its part converted to the MMA warp.
+template <bool kTrace>
+__device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, int mw, int lane, bool ok) {
+  if (!ok) return;
+  unsigned long long c_wait = 0, c_work = 0;
+  struct Flush {  // the warp's cycle counts into the trace (warp 0) on every way out
+    const Params& p;
+    int mw, lane;
+    unsigned long long &w, &k;
+    __device__ ~Flush() {
+      if (kTrace && mw == 0 && lane == 0) {
+        trace_put<kTrace>(p, TR_CONV_WAIT_CYC, w);
+        trace_put<kTrace>(p, TR_CONV_WORK_CYC, k);
+      }
+    }
+  } flush{p, mw, lane, c_wait, c_work};
+  const Shape& sh = sm.sh;
+  const int quad = (mw + 1) & 3;     // lane quadrant of this warp (warp id mod 4)
+  const int j = mw >> 2;             // weight tile
+  const int r = quad * 32 + lane;    // tile row = tensor-memory lane
+  const uint32_t tq = sm.tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(kFp8ACol0 + j * (kFp8AStageCols / 2));
+  const int swz = (r >> 1) & 3;
+  int q = 0, as = 0;
+  uint32_t qph = 0u, asph = 0u;
+  for (;;) {
+    const long long t0 = tclock<kTrace>();
+    if (!warp_wait(&sm.cq_full[q], qph, p, lane, 64)) return;
+    const int slot = sm.cq_slot[q];
+    const uint32_t par = sm.cq_par[q];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.cq_empty[q]);  // the entry is read
+    if (++q == kCq) {
+      q = 0;
+      qph ^= 1u;
+    }
+    if (slot < 0) return;
+    if (!IDX_OK(p, slot < sh.nst)) return;
+    if (!warp_wait(&sm.wfull[slot], par, p, lane, 64)) return;
+    if (!warp_wait(&astage_empty(sm)[as], asph ^ 1u, p, lane, 64)) return;  // the A stage is free
+    const long long t1 = tclock<kTrace>();
+    c_wait += (unsigned long long)(t1 - t0);
+    const StageHeader hd = sm.hdr[slot];
+    if (j < (hd.info & 3)) {
+      tc_fence_after();
+      const uint8_t* sbase = ring + slot * sh.slot_bytes;
+      const uint32_t sc = scale_bf16x2(
+          reinterpret_cast<const float*>(sbase + kFp8ScaleOff + 16 * j)[(hd.wrow >> (2 * j)) & 3]);
+      const uint8_t* row = sbase + j * kFp8TileBytes + r * kTcAtomK;
+      uint4 v[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(row + ((c ^ swz) << 4));
+      const uint32_t col = (uint32_t)(as * kFp8AStageCols);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+        uint32_t o[8];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          e4m3x4_to_bf16x2x2(w[t], o[2 * t], o[2 * t + 1]);
+          o[2 * t] = mul_bf16x2(o[2 * t], sc);
+          o[2 * t + 1] = mul_bf16x2(o[2 * t + 1], sc);
+        }
+        tmem_st8(tq + col + (uint32_t)(8 * c), o);  // K elements 16 c .. 16 c + 15
+      }
+      tmem_st_wait();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.conv_bar[slot]);
+    if (++as == kFp8AStages) {
+      as = 0;
+      asph ^= 1u;
+    }
+    c_work += (unsigned long long)(tclock<kTrace>() - t1);
+  }
+}
+
 // ---- tensor-core path: MMA warp --------------------------------------------------------------------
 
 // One elected lane issues, per stage, 4 K-steps of 16 for each weight tile into the
@@ -2368,7 +2601,7 @@ __device__ void epilogue_cc(const Params& p, Smem& sm, int lane) {
 // (the slot is free once those MMAs have read it). At a unit's last stage the buffer
 // is handed to the epilogue warps: one commit arrive (the MMAs are complete) plus one
 // plain arrive that publishes the unit id.
-template <bool kTrace>
+template <bool kTrace, bool kFp8 = false>
 __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
   const uint32_t tmem = sm.tmem_base;
   int slot = 0;
@@ -2376,7 +2609,9 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
   int abuf = 0;
   uint32_t aphase = 0;
   bool issued = false;
-  unsigned long long c_full = 0, c_acc = 0, c_st = 0, c_issue = 0;
+  uint32_t cpar = 0u;  // per slot: parity of its next FP8 conversion
+  int as = 0;          // FP8: tensor-memory A stage of the next FP8 stage
+  unsigned long long c_full = 0, c_acc = 0, c_st = 0, c_issue = 0, c_conv = 0;
   const long long tloop0 = tclock<kTrace>();
   for (;;) {
     {
@@ -2391,6 +2626,13 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
       break;
     }
     const int info = hd.info;
+    if (kFp8 && (info & kTcInfoFp8)) {  // the activations landed; wait for the bf16 weight tiles
+      const long long t0 = tclock<kTrace>();
+      const bool got = warp_wait(&sm.conv_bar[slot], (cpar >> slot) & 1u, p, lane, 64);
+      c_conv += (unsigned long long)(tclock<kTrace>() - t0);
+      if (!got) break;
+      cpar ^= 1u << slot;
+    }
     const bool first = (info & kTcInfoFirst) != 0;
     const bool last = (info & kTcInfoLast) != 0;
     if (first) {
@@ -2409,11 +2651,24 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
       const int nbox = info & 3;
       const uint32_t idesc = idesc_bf16_m128((uint32_t)((info >> 2) & 7) * kTcActRows);
       const uint32_t t0 = tmem + (uint32_t)(abuf * kTcAccCols);
+      if (kFp8 && (info & kTcInfoFp8)) {  // A from the tensor-memory stage the converters filled
+        const uint32_t a0 = tmem + (uint32_t)(kFp8ACol0 + as * kFp8AStageCols);
 #pragma unroll
-      for (int ks = 0; ks < kTcAtomK / 16; ++ks) {
-        const uint32_t accum = (first && ks == 0) ? 0u : 1u;
-        tc_mma_bf16(t0, dw0 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
-        if (nbox == 2) tc_mma_bf16(t0 + 64u, dw1 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
+        for (int ks = 0; ks < kTcAtomK / 16; ++ks) {
+          const uint32_t accum = (first && ks == 0) ? 0u : 1u;
+          tc_mma_bf16_ta(t0, a0 + (uint32_t)(8 * ks), da + (uint64_t)(2 * ks), idesc, accum);
+          if (nbox == 2)
+            tc_mma_bf16_ta(t0 + 64u, a0 + (uint32_t)(kFp8AStageCols / 2 + 8 * ks), da + (uint64_t)(2 * ks), idesc,
+                           accum);
+        }
+        tc_commit(&astage_empty(sm)[as]);
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < kTcAtomK / 16; ++ks) {
+          const uint32_t accum = (first && ks == 0) ? 0u : 1u;
+          tc_mma_bf16(t0, dw0 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
+          if (nbox == 2) tc_mma_bf16(t0 + 64u, dw1 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
+        }
       }
       tc_commit(&sm.empty[slot]);
       if (last) {
@@ -2426,8 +2681,9 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
     __syncwarp();
     c_issue += (unsigned long long)(tclock<kTrace>() - ti0);
     ++c_st;
+    if (kFp8 && (info & kTcInfoFp8) && ++as == kFp8AStages) as = 0;
     if (last) {
-      if (++abuf == kTcAccBufs) {
+      if (++abuf == (kFp8 ? kFp8AccBufs : kTcAccBufs)) {
         abuf = 0;
         aphase ^= 1u;
       }
@@ -2440,6 +2696,7 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
   if (lane == 0 && kTrace) {
     trace_put<kTrace>(p, TR_MAC_LOOP_CYC, (unsigned long long)(tclock<kTrace>() - tloop0));
     trace_put<kTrace>(p, TR_MAC_WAIT_FULL_CYC, c_full);
+    trace_put<kTrace>(p, TR_MMA_WAIT_CONV_CYC, c_conv);
     trace_put<kTrace>(p, TR_MAC_WAIT_RB_CYC, c_acc);
     trace_put<kTrace>(p, TR_MAC_COMPUTE_CYC, c_issue);
     trace_put<kTrace>(p, TR_MAC_STAGES, c_st);
@@ -2569,7 +2826,7 @@ __device__ void combine_rows_tc(const Params& p, const Smem& sm, int t, const in
 
 // F: the layers of a fused launch (a unit's header names its layer), or nullptr when
 // the launch runs the one layer p0.
-template <bool kTrace>
+template <bool kTrace, bool kFp8 = false>
 __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, const FusedParams* F = nullptr) {
   const Shape& sh = sm.sh;
   const int quad = warp_id & 3;
@@ -2702,7 +2959,7 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.acc_empty[abuf]);
-    if (++abuf == kTcAccBufs) {
+    if (++abuf == (kFp8 ? kFp8AccBufs : kTcAccBufs)) {
       abuf = 0;
       aphase ^= 1u;
     }
@@ -2769,7 +3026,7 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
 
 // ---- the kernel ----------------------------------------------------------------------------------
 
-template <bool kTrace, bool kTC>
+template <bool kTrace, bool kTC, bool kFp8 = false>
 __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
     moe_decode_layer_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -2792,6 +3049,15 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       }
       mbar_init(&sm.mma_bar, 1);
       mbar_init(&sm.epi_bar, kTcEpiWarps);
+      for (int s = 0; s < kTcStagesMax; ++s) {
+        mbar_init(&sm.conv_bar[s], kMacWarps);
+        mbar_init(&sm.wfull[s], 1);
+      }
+      for (int a = 0; a < kFp8AStages; ++a) mbar_init(&astage_empty(sm)[a], 1);
+      for (int q = 0; q < kCq; ++q) {
+        mbar_init(&sm.cq_full[q], 1);
+        mbar_init(&sm.cq_empty[q], kMacWarps);  // every converter warp reads every entry
+      }
       make_shape_tc(p, sm.sh);
     } else {
       for (int b = 0; b < kRB; ++b) {
@@ -2824,7 +3090,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
 
   if (warp_id == 0) {
     Producer pr(p, sm, lane, sm.sh.nst);
-    if constexpr (kTC) producer_tc<kTrace>(pr, ring);
+    if constexpr (kTC) producer_tc<kTrace, kFp8>(pr, ring);
     else producer_cc<kTrace>(pr, ring);
   } else if (warp_id <= kMacWarps) {
     if constexpr (kTC) {
@@ -2850,15 +3116,16 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       if (ok) ok = p.B == 1 ? build_schedule_b1<kTrace>(p, sm, mw, lane, mphase, tag)
                             : build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, false);
       if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
+      if constexpr (kFp8) convert_fp8_stages<kTrace>(p, sm, ring, mw, lane, ok);
     } else {
       mac_warps_cc<kTrace>(p, sm, ring, warp_id - 1, lane);
     }
   } else if constexpr (!kTC) {
     epilogue_cc<kTrace>(p, sm, lane);
   } else if (warp_id == kTcMmaWarp) {
-    mma_warp<kTrace>(p, sm, ring, lane);
+    mma_warp<kTrace, kFp8>(p, sm, ring, lane);
   } else {
-    epilogue_tc<kTrace>(p, sm, warp_id, lane);
+    epilogue_tc<kTrace, kFp8>(p, sm, warp_id, lane);
   }
 
   if constexpr (kTC) tc_fence_before();
@@ -3032,6 +3299,10 @@ size_t tc_smem_bytes() { return kTcRingBytes + sizeof(Smem) + 1024; }
 int tc_threads_per_cta() { return kTcThreads; }
 const void* tc_kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false, true>); }
 const void* tc_kernel_fn_trace() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true, true>); }
+const void* tc_fp8_kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false, true, true>); }
+const void* tc_fp8_kernel_fn_trace() {
+  return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true, true, true>);
+}
 const void* fused_kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_fused_kernel<false>); }
 const void* fused_kernel_fn_trace() { return reinterpret_cast<const void*>(&moe_decode_fused_kernel<true>); }
 

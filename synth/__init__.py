@@ -97,6 +97,10 @@ def _host_lib():
         lib.ms_e4m3_encode_host.restype = None
         lib.ms_block_exps_host.argtypes = [u64, u64, u64, u64, ctypes.c_int, vp]
         lib.ms_block_exps_host.restype = None
+        lib.ms_fill_e4m3_cover_host.argtypes = [u64, u64, u64, u64, u64, u64, ctypes.c_uint32, vp]
+        lib.ms_fill_e4m3_cover_host.restype = None
+        lib.ms_block_exps_cover_host.argtypes = [u64, u64, ctypes.c_uint32, ctypes.c_int, vp]
+        lib.ms_block_exps_cover_host.restype = None
         _host = lib
     return _host
 
@@ -112,6 +116,8 @@ def _cuda_lib():
         lib.ms_fill_device.restype = ctypes.c_int
         lib.ms_fill_e4m3_device.argtypes = [u64, u64, u64, u64, vp, vp]
         lib.ms_fill_e4m3_device.restype = ctypes.c_int
+        lib.ms_fill_e4m3_cover_device.argtypes = [u64, u64, u64, u64, u64, u64, ctypes.c_uint32, vp, vp]
+        lib.ms_fill_e4m3_cover_device.restype = ctypes.c_int
         _cuda = lib
     return _cuda
 
@@ -190,6 +196,37 @@ def fill_e4m3_device(ptr: int, seed: int, tid: int, start: int, n: int, stream: 
         raise RuntimeError(f"ms_fill_e4m3_device failed with cudaError {rc}")
 
 
+# ---- coverage codes: every block's codes share one exponent field, cycling over all 16 ----
+def cover_phase(seed: int) -> int:
+    return int(seed) % 16
+
+
+def cover_t(fan_in: int) -> int:
+    """Coverage blocks' weights lie in [2^(t-3), 2^(t+1)): t = round(log2(1/sqrt(fan_in))) - 1."""
+    return int(np.round(np.log2(1.0 / np.sqrt(float(fan_in))))) - 1
+
+
+def fill_e4m3_cover_host(seed: int, tid: int, start: int, n: int, rows: int, cols: int) -> np.ndarray:
+    """Coverage codes (uint8) of elements start .. start + n - 1 of a stack [E][rows][cols]."""
+    out = np.empty(int(n), dtype=np.uint8)
+    _host_lib().ms_fill_e4m3_cover_host(seed, tid, start, n, rows, cols, cover_phase(seed), _ptr(out))
+    return out
+
+
+def block_exps_cover_host(seed: int, start: int, n: int, fan_in: int) -> np.ndarray:
+    out = np.empty(int(n), dtype=np.int32)
+    _host_lib().ms_block_exps_cover_host(start, n, cover_phase(seed), cover_t(fan_in), _ptr(out))
+    return out
+
+
+def fill_e4m3_cover_device(ptr: int, seed: int, tid: int, start: int, n: int, rows: int, cols: int,
+                           stream: int = 0) -> None:
+    rc = _cuda_lib().ms_fill_e4m3_cover_device(seed, tid, start, n, rows, cols, cover_phase(seed),
+                                               ctypes.c_void_p(ptr), ctypes.c_void_p(stream))
+    if rc != 0:
+        raise RuntimeError(f"ms_fill_e4m3_cover_device failed with cudaError {rc}")
+
+
 def fill_device(ptr: int, seed: int, tid: int, start: int, n: int, sigma: float, mean: float = 0.0,
                 stream: int = 0) -> None:
     rc = _cuda_lib().ms_fill_device(seed, tid, start, n, np.float32(sigma), np.float32(mean),
@@ -235,6 +272,9 @@ class Workload:
     nseq: int = 0
     rows_per_seq: int = 0
     gamma_sigma: float = 0.1
+    # "bf16" | "fp8" (E4M3 codes with 128 x 128 block scales) | "fp8_cover" (FP8 with the
+    # coverage codes: each block one exponent field, all 16 across the blocks)
+    experts: str = "bf16"
     notes: str = field(default="", compare=False)
 
     # ---- hidden states --------------------------------------------------
@@ -328,6 +368,10 @@ class Workload:
         return out
 
     # ---- FP8 expert weights (E4M3 codes, one power-of-two scale per 128 x 128 block) ----
+    @property
+    def is_fp8(self) -> bool:
+        return self.experts in ("fp8", "fp8_cover")
+
     def fp8_matrices(self):
         """(name, code kind, scale kind, rows, cols, fan_in) of each expert matrix."""
         H, I = self.H, self.I
@@ -341,7 +385,10 @@ class Workload:
         experts = range(self.E) if experts is None else experts
         out = np.empty((len(experts), rb, cb), dtype=np.float32)
         for i, e in enumerate(experts):
-            ex = block_exps_host(self.seed, tensor_id(layer, sk), int(e) * rb * cb, rb * cb, fp8_s0(fan_in))
+            if self.experts == "fp8_cover":
+                ex = block_exps_cover_host(self.seed, int(e) * rb * cb, rb * cb, fan_in)
+            else:
+                ex = block_exps_host(self.seed, tensor_id(layer, sk), int(e) * rb * cb, rb * cb, fp8_s0(fan_in))
             out[i] = np.ldexp(np.float32(1.0), ex).astype(np.float32).reshape(rb, cb)
         return out
 
@@ -350,7 +397,10 @@ class Workload:
         [rows/128, cols/128])} of expert e."""
         out = {}
         for name, qk, _, rows, cols, _ in self.fp8_matrices():
-            codes = fill_e4m3_host(self.seed, tensor_id(layer, qk), e * rows * cols, rows * cols)
+            if self.experts == "fp8_cover":
+                codes = fill_e4m3_cover_host(self.seed, tensor_id(layer, qk), e * rows * cols, rows * cols, rows, cols)
+            else:
+                codes = fill_e4m3_host(self.seed, tensor_id(layer, qk), e * rows * cols, rows * cols)
             out[name] = (codes.reshape(rows, cols), self.fp8_scales_host(layer, name, [e])[0])
         return out
 
@@ -374,12 +424,29 @@ class Workload:
         out["ws_down"] = out["ws_down"].view(H, Is)
         for name, qk, _, rows, cols, _ in self.fp8_matrices():
             q = torch.empty((E, rows, cols), dtype=torch.uint8, device=device)
-            fill_e4m3_device(q.data_ptr(), self.seed, tensor_id(layer, qk), 0, E * rows * cols, stream)
+            if self.experts == "fp8_cover":
+                fill_e4m3_cover_device(q.data_ptr(), self.seed, tensor_id(layer, qk), 0, E * rows * cols, rows, cols,
+                                       stream)
+            else:
+                fill_e4m3_device(q.data_ptr(), self.seed, tensor_id(layer, qk), 0, E * rows * cols, stream)
             out[f"w_{name}_q"] = q
             out[f"w_{name}_scale"] = torch.from_numpy(self.fp8_scales_host(layer, name)).to(device)
         bias = self.bias_host(layer)
         out["router_bias"] = None if bias is None else torch.from_numpy(bias).to(device)
         return out
+
+    def expert_bytes(self) -> int:
+        """Bytes of one expert's weights as stored (codes and block scales when FP8)."""
+        H, I = self.H, self.I
+        if self.is_fp8:
+            return 3 * I * H + 3 * (I // FP8_BLOCK) * (H // FP8_BLOCK) * 4
+        return 3 * I * H * 2
+
+    def device_layer_any(self, layer: int, device="cuda", stream: int = 0) -> dict:
+        """device_layer, or device_layer_fp8 for a workload with FP8 experts."""
+        if self.is_fp8:
+            return self.device_layer_fp8(layer, device=device, stream=stream)
+        return self.device_layer(layer, device=device, stream=stream)
 
     def weight_bytes_per_layer(self) -> int:
         return 2 * sum(s[2] for s in self.device_specs(0))
@@ -393,4 +460,10 @@ WORKLOADS = {
                 router="zipf"),
     4: Workload("verify_4x8_h7168_e896_k16_2layer", B=32, H=7168, E=896, k=16, I=1024, Is=2048,
                 seed=4, layers=2, rows="correlated", nseq=4, rows_per_seq=8),
+}
+
+# The same layers with FP8 expert weights (batch 1 and batch 8).
+FP8_WORKLOADS = {
+    1: Workload("b1_h7168_e896_k16_fp8", B=1, H=7168, E=896, k=16, I=1024, Is=2048, seed=1, experts="fp8"),
+    2: Workload("b8_h7168_e896_k16_fp8", B=8, H=7168, E=896, k=16, I=1024, Is=2048, seed=2, experts="fp8"),
 }

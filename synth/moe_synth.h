@@ -170,4 +170,29 @@ MS_FN int ms_block_exp(uint64_t key, uint64_t b, int s0) {
   return s0 + (int)(ms_word(key, b) % 3ULL) - 1;
 }
 
+/*
+ * Coverage codes (a test input that gives every E4M3 value full weight). In block b of
+ * an expert matrix stack [E][rows][cols] (b counted expert-major, then 128-row block,
+ * then 128-column block) every code has the exponent field f(b) = (b + phase) mod 16;
+ * sign and 3 mantissa bits are drawn per element (the NaN codes 0x7F / 0xFF become
+ * 0x7E / 0xFE). Block b's scale exponent is t + 7 - max(f(b), 1), so every block's
+ * weights lie in [2^(t-3), 2^(t+1)) whatever its binade, subnormal blocks included.
+ */
+MS_FN uint32_t ms_cover_field(uint64_t b, uint32_t phase) { return (uint32_t)((b + phase) % 16u); }
+
+MS_FN uint8_t ms_code_e4m3_cover(uint64_t key, uint64_t i, uint64_t rows, uint64_t cols, uint32_t phase) {
+  const uint64_t per = rows * cols, e = i / per, r = (i % per) / cols, c = i % cols;
+  const uint64_t b = (e * (rows / 128u) + r / 128u) * (cols / 128u) + c / 128u;
+  const uint32_t f = ms_cover_field(b, phase);
+  const uint64_t w = ms_word(key, i);
+  uint32_t m = (uint32_t)(w & 7u);
+  if (f == 15u && m == 7u) m = 6u;
+  return (uint8_t)((((uint32_t)(w >> 3) & 1u) << 7) | (f << 3) | m);
+}
+
+MS_FN int ms_block_exp_cover(uint64_t b, uint32_t phase, int t) {
+  const int f = (int)ms_cover_field(b, phase);
+  return t + 7 - (f > 1 ? f : 1);
+}
+
 #endif /* MOE_SYNTH_H */

@@ -29,9 +29,36 @@ __global__ void fill_e4m3_kernel(uint64_t key, uint64_t start, uint64_t n, uint8
     out[i] = ms_code_e4m3(key, start + i);
 }
 
+__global__ void fill_e4m3_cover_kernel(uint64_t key, uint64_t start, uint64_t n, uint64_t rows, uint64_t cols,
+                                       uint32_t phase, uint8_t* __restrict__ out) {
+  const uint64_t stride = (uint64_t)gridDim.x * blockDim.x;
+  for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    out[i] = ms_code_e4m3_cover(key, start + i, rows, cols, phase);
+}
+
 }  // namespace
 
 extern "C" {
+
+// Fills out[0..n) (device memory) with the coverage codes ms_code_e4m3_cover of elements
+// start .. start + n - 1 of an expert stack [E][rows][cols]. Asynchronous on `stream`;
+// returns a cudaError_t value (0 on success).
+int ms_fill_e4m3_cover_device(uint64_t seed, uint64_t tensor_id, uint64_t start, uint64_t n, uint64_t rows,
+                              uint64_t cols, uint32_t phase, void* out, void* stream) {
+  if (n == 0) return 0;
+  if (out == nullptr || rows == 0 || cols == 0) return (int)cudaErrorInvalidValue;
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return (int)e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return (int)e;
+  uint64_t blocks = (n + 255) / 256;
+  const uint64_t cap = (uint64_t)sms * 16;
+  if (blocks > cap) blocks = cap;
+  fill_e4m3_cover_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(ms_key(seed, tensor_id), start, n,
+                                                                             rows, cols, phase, (uint8_t*)out);
+  return (int)cudaGetLastError();
+}
 
 // Fills out[0..n) (device memory) with the E4M3 codes ms_code_e4m3(key(seed, tid), start + i).
 // Asynchronous on `stream`; returns a cudaError_t value (0 on success).

@@ -93,3 +93,17 @@ void ms_block_exps_host(uint64_t seed, uint64_t tensor_id, uint64_t start, uint6
   const uint64_t key = ms_key(seed, tensor_id);
   for (uint64_t i = 0; i < n; ++i) out[i] = ms_block_exp(key, start + i, s0);
 }
+
+/* Coverage codes of elements start .. start + n - 1 of an expert stack [E][rows][cols]. */
+void ms_fill_e4m3_cover_host(uint64_t seed, uint64_t tensor_id, uint64_t start, uint64_t n, uint64_t rows,
+                             uint64_t cols, uint32_t phase, uint8_t* out) {
+  const uint64_t key = ms_key(seed, tensor_id);
+  int64_t i;
+#pragma omp parallel for schedule(static)
+  for (i = 0; i < (int64_t)n; ++i) out[i] = ms_code_e4m3_cover(key, start + (uint64_t)i, rows, cols, phase);
+}
+
+/* Scale exponents of coverage blocks start .. start + n - 1. */
+void ms_block_exps_cover_host(uint64_t start, uint64_t n, uint32_t phase, int t, int32_t* out) {
+  for (uint64_t i = 0; i < n; ++i) out[i] = ms_block_exp_cover(start + i, phase, t);
+}

@@ -38,14 +38,15 @@ def bf16_ulp(v):
     return 2.0 ** (e - 7)
 
 
-def make_handle(wl, layers, device=0, max_batch=None, top_k_max=None, tc_min_batch=None, checked=False):
+def make_handle(wl, layers, device=0, max_batch=None, top_k_max=None, tc_min_batch=None, checked=False,
+                fp8=False):
     """A handle for the workload; tc_min_batch (if given) sets the batch-shape switch:
     1 sends every step to the tensor-core kernel, 0 every step to the CUDA-core one.
-    checked: the bounds-checked build of the library."""
+    checked: the bounds-checked build of the library; fp8: layers with FP8 experts."""
     import moe_decode_persistent_b200 as mdp
 
     h = mdp.MoeDecode(wl.H, wl.E, top_k_max or wl.k, wl.I, wl.Is, max_batch or wl.B, layers,
-                      eps=wl.eps, device=device, checked=checked)
+                      eps=wl.eps, device=device, checked=checked, fp8=fp8)
     if tc_min_batch is not None:
         h.set_tc_min_batch(tc_min_batch)
     return h
@@ -88,7 +89,7 @@ def oracle_rows(wl, x_bits, rows, n_layers=1, k=None):
     return res
 
 
-def oracle_rows_selected(wl, x_bits, rows, gpu_layers, k=None):
+def oracle_rows_selected(wl, x_bits, rows, gpu_layers, k=None, fp8=False):
     """The oracle chain of rows `rows` with every layer's selection taken from the GPU
     (gpu_layers[l]["idx"]), the weights from the oracle's own fp64 logits over that
     set, and each layer fed by the oracle's own previous output. Where the GPU's fp32
@@ -101,7 +102,7 @@ def oracle_rows_selected(wl, x_bits, rows, gpu_layers, k=None):
     x = x_bits[rows]
     for layer in range(len(gpu_layers)):
         sel = np.asarray(gpu_layers[layer]["idx"])[rows]
-        r = oracle.workload_layer(w, layer, x, selection=sel)
+        r = oracle.workload_layer(w, layer, x, selection=sel, fp8=fp8)
         res.append(r)
         x = r["y"]
     return res
@@ -128,12 +129,12 @@ def routing_oracle(wl, x_bits, rows, layers, gpu_inputs, k=None):
     return res
 
 
-def gpu_layer_outputs(wl, device_layers, x_bits, tc_min_batch=None, k=None):
+def gpu_layer_outputs(wl, device_layers, x_bits, tc_min_batch=None, k=None, fp8=False):
     """The GPU's output of each layer but the last, from handles over layer prefixes
     (a step is deterministic, so these equal the intermediates of the full stack)."""
     outs = []
     for n in range(1, wl.layers):
-        h = make_handle(wl, device_layers[:n], tc_min_batch=tc_min_batch)
+        h = make_handle(wl, device_layers[:n], tc_min_batch=tc_min_batch, fp8=fp8)
         o = run_gpu(h, wl, x_bits, k=k, n_layers=n)
         assert o["status"] == 0
         outs.append(o["y"])
@@ -212,13 +213,13 @@ def check_y(y_gpu_rows, orc_layers, tag=""):
     return float(d.max())
 
 
-def check_all(wl, out, x, rows, route, tag, k=None):
+def check_all(wl, out, x, rows, route, tag, k=None, fp8=False):
     """Every check of one step on rows `rows`: per layer the routing checks against
     `route` (router-only oracle on the layer's actual input), the unique-expert count,
     the chained selections' validity, and the output of every row against the oracle
     chain on the GPU's own selections. Returns (max |dy|, near-tie rows)."""
     k = k or wl.k
-    orc = oracle_rows_selected(wl, x, rows, out["layers"], k=k)
+    orc = oracle_rows_selected(wl, x, rows, out["layers"], k=k, fp8=fp8)
     ties = set(chained_flips(out["layers"], orc, rows, k, tag=tag))
     for l in range(len(out["layers"])):
         ties |= {rows.index(b) for b in check_layer(out["layers"][l], route[l], rows, k, tag=f"{tag} layer {l}")}

@@ -130,3 +130,37 @@ def test_fp8_block_scales_are_powers_of_two_around_the_weight_spread():
     s0 = synth.fp8_s0(wl.H)
     assert set(np.unique(e).astype(int)) <= {s0 - 1, s0, s0 + 1}
     assert len(np.unique(e)) == 3
+
+
+def test_fp8_cover_codes_give_every_block_one_binade_and_every_code_full_weight():
+    """Coverage codes: within a 128 x 128 block every code has the exponent field
+    (b + phase) mod 16, all 16 fields appear across the blocks, no NaN code is drawn, and
+    with the block scales every nonzero weight lies in [2^(t-3), 2^(t+1)) -- subnormal
+    blocks included -- so a wrong decode of any code changes the layer visibly."""
+    import torch
+
+    wl = synth.Workload("cover", B=1, H=512, E=4, k=2, I=256, Is=128, seed=7, experts="fp8_cover")
+    assert wl.is_fp8
+    t = synth.cover_t(wl.H)
+    fields = set()
+    for e in range(wl.E):
+        codes, scales = wl.expert_fp8_host(0, e)["gate"]
+        rb, cb = wl.I // 128, wl.H // 128
+        assert codes.shape == (wl.I, wl.H) and scales.shape == (rb, cb)
+        assert not np.any((codes & 0x7F) == 0x7F)
+        for r in range(rb):
+            for c in range(cb):
+                blk = codes[128 * r:128 * r + 128, 128 * c:128 * c + 128]
+                f = (blk >> 3) & 15
+                b = (e * rb + r) * cb + c
+                want = (b + synth.cover_phase(wl.seed)) % 16
+                assert np.all(f == want)
+                fields.add(int(want))
+                assert scales[r, c] == np.float32(2.0 ** (t + 7 - max(want, 1)))
+                # all mantissas (field 15: 0..6, mantissa 7 there being NaN) and both signs
+                assert len(np.unique(blk & 7)) == (7 if want == 15 else 8) and len(np.unique(blk >> 7)) == 2
+        w = torch.from_numpy(codes).view(torch.float8_e4m3fn).float().numpy()
+        w = w * np.kron(scales, np.ones((128, 128), dtype=np.float32))
+        a = np.abs(w[w != 0])
+        assert a.min() >= 2.0 ** (t - 3) and a.max() < 2.0 ** (t + 1)
+    assert fields == set(range(16))
