@@ -113,10 +113,7 @@ typedef struct {
  * sign) in [2^-117, 2^7], the range in which the kernel's in-register decode is exact;
  * moe_decode_create_fp8 reads the scales once and refuses any other value with
  * MOE_ERR_INVALID_ARG. Router and shared expert stay bf16. All
- * pointers 16-byte aligned (router_bias 4-byte aligned). The kernel reads the scale
- * arrays in whole aligned 16-byte groups, so each scale allocation must stay readable
- * up to the next 16-byte boundary past its last element (any cudaMalloc or torch
- * allocation is).
+ * pointers 16-byte aligned (router_bias and the scales 4-byte aligned).
  * (A more aggressive quantisation format is named on page "Kimi K3推理吞吐提升1.68倍",
  * intro, only as what the reported gain did not need; the format here is this
  * library's reading.) */
@@ -160,7 +157,7 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
  * MMA operand in shared memory by the CTA's routing warps once the routing is done.
  * Copies the scale arrays to the host once to check them (synchronous on `device`):
  * MOE_ERR_INVALID_ARG for a scale outside the range above or a scale pointer that is
- * not 16-byte aligned, MOE_ERR_CUDA if the copy fails. */
+ * not 4-byte aligned, MOE_ERR_CUDA if the copy fails. */
 int moe_decode_create_fp8(const moe_decode_config* cfg, const moe_decode_layer_weights_fp8* layers, int device,
                           moe_decode_handle** out);
 

@@ -102,17 +102,17 @@ static int encode_2d(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint
 
 // FP8 expert codes: boxes of 128 rows x 64 one-byte codes, no swizzle (the routing warps
 // read them and write the swizzled bf16 operand).
-// E4M3 codes [rows][cols], box 64 columns x 128 rows (64 bytes a row), 64-byte swizzled:
-// 16-byte chunk c of box row r lands at chunk c ^ ((r / 2) mod 4) of the row, so the
+// E4M3 codes [rows][cols], box 128 columns (one K block) x 128 rows, 128-byte swizzled:
+// 16-byte chunk c of box row r lands at chunk c ^ (r mod 8) of the row, so the
 // converters, one row per lane, read distinct banks.
 static int encode_fp8(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
   if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return MOE_ERR_INVALID_ARG;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols};
-  cuuint32_t box[2] = {(cuuint32_t)moe::kTcAtomK, (cuuint32_t)moe::kTcRows};
+  cuuint32_t box[2] = {(cuuint32_t)(2 * moe::kTcAtomK), (cuuint32_t)moe::kTcRows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -467,7 +467,7 @@ int moe_decode_create_fp8(const moe_decode_config* cfg, const moe_decode_layer_w
     const moe_decode_layer_weights_fp8& f = layers[l];
     if (!f.w_gate_scale || !f.w_up_scale || !f.w_down_scale ||
         ((reinterpret_cast<uintptr_t>(f.w_gate_scale) | reinterpret_cast<uintptr_t>(f.w_up_scale) |
-          reinterpret_cast<uintptr_t>(f.w_down_scale)) & 15u))
+          reinterpret_cast<uintptr_t>(f.w_down_scale)) & 3u))
       return MOE_ERR_INVALID_ARG;
     w[l] = moe_decode_layer_weights{f.gamma, f.w_router, f.router_bias, f.w_gate, f.w_up, f.w_down,
                                     f.ws_gate, f.ws_up, f.ws_down};

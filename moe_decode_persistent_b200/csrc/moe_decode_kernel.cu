@@ -95,22 +95,26 @@ constexpr int kTcRingBytes = 180 * 1024;
 // queues delay the routing's loads), so batches of at most 4 rows keep 4 stages.
 constexpr int kTcStagesMax = 5;
 __host__ __device__ constexpr int tc_slot_bytes(int na) { return 2 * kTcTileBytes + ((na * kTcAtomK * 2 + 1023) / 1024) * 1024; }
-__host__ __device__ constexpr int tc_stages(int na, int batch) {
-  return batch <= 4 ? 4
-       : kTcRingBytes / tc_slot_bytes(na) < kTcStagesMax ? kTcRingBytes / tc_slot_bytes(na) : kTcStagesMax;
+// A layer with FP8 experts: an FP8 stage holds one 128-column K block, so its slot takes
+// the activations of two K atoms (the second at +na x 128 bytes).
+__host__ __device__ constexpr int tc_slot_bytes_fp8(int na) { return 2 * kTcTileBytes + 2 * na * kTcAtomK * 2; }
+__host__ __device__ constexpr int tc_stages_of(int slot_bytes, int batch) {
+  return batch <= 4 ? 4 : kTcRingBytes / slot_bytes < kTcStagesMax ? kTcRingBytes / slot_bytes : kTcStagesMax;
 }
+__host__ __device__ constexpr int tc_stages(int na, int batch) { return tc_stages_of(tc_slot_bytes(na), batch); }
 static_assert(tc_stages(16, 1) == 4 && tc_stages(16, 8) == 5 && tc_stages(32, 32) == 5 && tc_stages(64, 64) == 4,
               "ring depths");
 constexpr int kTcAccBufs = 4;       // accumulator buffers in tensor memory
 constexpr int kTcAccCols = 128;     // columns per buffer: tile 0 at +0, tile 1 at +64
 constexpr int kTmemCols = kTcAccBufs * kTcAccCols;  // 512 (a power of two >= 32)
 // A layer with FP8 experts keeps 2 accumulator buffers (columns 0-255) and uses columns
-// 256-511 as 4 stages of the MMA's A operand: the converted bf16 weight tiles of an FP8
-// stage (tile j at +32 j; row m in lane m, K elements 2c and 2c + 1 in column c).
+// 256-511 as 2 stages of the MMA's A operand: the converted bf16 weight tiles of an FP8
+// stage (128 K columns; tile j at +64 j; row m in lane m, K elements 2c and 2c + 1 in
+// column c).
 constexpr int kFp8AccBufs = 2;
-constexpr int kFp8AStages = 4;
+constexpr int kFp8AStages = 2;
 constexpr int kFp8ACol0 = kFp8AccBufs * kTcAccCols;
-constexpr int kFp8AStageCols = 2 * kTcAtomK / 2;
+constexpr int kFp8AStageCols = 2 * kTcAtomK;
 static_assert(kFp8ACol0 + kFp8AStages * kFp8AStageCols <= kTmemCols, "FP8 tensor-memory plan");
 
 static_assert(kTcSlotBytes % 1024 == 0 && kTcTileBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
@@ -133,16 +137,18 @@ constexpr int kInfoKpair = 1 << 2, kInfoSegEnd = 1 << 6, kInfoUnitEnd = 1 << 7, 
 // Tensor-core stages: bits 0-1 weight tiles, 2-4 activation boxes of 16 rows (N / 16),
 // 5 first stage of the unit (overwrite the accumulator), 6 last stage of the unit.
 constexpr int kTcInfoFirst = 1 << 5, kTcInfoLast = 1 << 6;
-// Tensor-core stage whose weight tiles arrive as E4M3 codes (8 KB per tile at the start
-// of the slot, tile 1 at +8 KB; 64 bytes a row, 64-byte swizzled) and are converted by
-// the routing warps into an A stage in tensor memory, which the MMA reads instead of
-// shared memory. With the codes, each tile's block scale lands in the slot at +16 KB
-// (tile j at +16 j: the aligned 16-byte group of the scale array that holds it), both
-// counted on Smem::wfull of the slot (the activations stay on full); the header's wrow
-// holds the scale's position in its group, tile 0 in bits 0-1, tile 1 in bits 2-3.
-constexpr int kTcInfoFp8 = 1 << 7;
-constexpr int kFp8TileBytes = kTcRows * kTcAtomK;  // 8 KB: 128 rows x 64 codes
-constexpr int kFp8ScaleOff = 2 * kFp8TileBytes;    // the scale groups of an FP8 stage in its slot
+// Tensor-core stage whose weight tiles arrive as E4M3 codes: one 128-column K block (two
+// K atoms) per stage, 16 KB per tile at the start of the slot (tile 1 at +16 KB; 128
+// bytes a row, 128-byte swizzled), converted by the routing warps into an A stage in
+// tensor memory, which the MMA reads instead of shared memory. The activations of the
+// two atoms follow at +32 KB and +32 KB + NA x 128. The codes are counted on
+// Smem::wfull of the slot (the activations stay on full). The converters load the
+// tiles' block scales themselves: the header's wrow holds tile 0's scale index (gate or
+// down array; tile 1 of a gate/up stage: the same index of the up array, of a down
+// stage: I / 128 further), and info bit 8 marks a down stage.
+constexpr int kTcInfoFp8 = 1 << 7, kTcInfoFp8Down = 1 << 8;
+constexpr int kFp8TileBytes = kTcRows * 2 * kTcAtomK;  // 16 KB: 128 rows x 128 codes
+__device__ __forceinline__ int fp8_act1_off(int na) { return 2 * kTcTileBytes + na * kTcAtomK * 2; }
 constexpr int kCq = 8;                            // entries of the converter queue
 
 // Layout constants of one step (identical in every CTA).
@@ -157,6 +163,7 @@ struct Shape {
   int spp;  // stages per (expert, row group) pair of a down unit
   int NA;   // tensor-core path: token columns of n- and hs-based tiles (B rounded up to 16)
   int nst, slot_bytes;  // ring stages and slot size
+  int kblk;             // 1: FP8 experts (expert gate/up K splits at 128-column K blocks)
   int pre;  // units queued before the routing schedule (no unit before it needs the schedule)
   int router_target, hs_target, pair_target;  // tiles that publish logits / h_s / one pair's h
 };
@@ -499,8 +506,9 @@ __device__ void make_shape_tc(const Params& p, Shape& s) {
   s.k = p.k;
   s.GB = 1;
   s.NA = (p.B + kTcActRows - 1) / kTcActRows * kTcActRows;
-  s.slot_bytes = tc_slot_bytes(s.NA);
-  s.nst = tc_stages(s.NA, p.B);
+  s.kblk = p.fp8 ? 1 : 0;
+  s.slot_bytes = p.fp8 ? tc_slot_bytes_fp8(s.NA) : tc_slot_bytes(s.NA);
+  s.nst = tc_stages_of(s.slot_bytes, p.B);
   s.boxH = s.boxI = s.boxIs = kTcAtomK;
   s.nkbH = p.H / kTcAtomK;
   s.nkbI = p.I / kTcAtomK;
@@ -633,7 +641,13 @@ __device__ UnitDesc decode_unit_tc(const Shape& sh, const Sched& sc, int u) {
     d.tile = w / es;
     d.nsplit = es;
     d.ticket = sh.RT + sh.ST + lo * sh.IT + d.tile;
-    split_range(sh.nkbH, es, d.split, d.kb0, d.nkb);
+    if (sh.kblk) {  // FP8: whole 128-column K blocks
+      split_range(sh.nkbH / 2, es, d.split, d.kb0, d.nkb);
+      d.kb0 *= 2;
+      d.nkb *= 2;
+    } else {
+      split_range(sh.nkbH, es, d.split, d.kb0, d.nkb);
+    }
   } else {
     const int v = u - sh.pre - sc.NE;
     d.type = UT_DOWN_EXPERT;
@@ -1355,7 +1369,7 @@ __device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, u
       int r = 0;
 #pragma unroll 4
       for (int sl = 0; sl < 32; ++sl) r += __shfl_sync(0xffffffffu, e, sl) < e ? 1 : 0;
-      const int es = tc_expert_splits(1, sh.nkbH);
+      const int es = tc_expert_splits(1, sh.kblk ? sh.nkbH / 2 : sh.nkbH);
       if (lane < k && !IDX_OK(p, (unsigned)e < (unsigned)p.E && (unsigned)r < (unsigned)kMaxSlots)) {
         e = 0;  // reported; the step is abandoned
         r = lane;
@@ -1524,7 +1538,7 @@ __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw
       const int pr = p0 + lane;
       int units = 0;
       if (pr < U) {
-        const int es = tc_expert_splits(sc.slot_cnt[sc.pair_slot[pr]], sh.nkbH);
+        const int es = tc_expert_splits(sc.slot_cnt[sc.pair_slot[pr]], sh.kblk ? sh.nkbH / 2 : sh.nkbH);
         sc.pair_es[pr] = (uint8_t)es;
         sc.pair_group[pr] = 0;
         units = sh.IT * es;
@@ -2072,8 +2086,8 @@ struct TcSeg {
   int dep;   // 0: normalised rows, 1: shared h, 2: the expert's h
   int pair;
   int fp8;   // 1: the weight tiles are E4M3 codes (expert units of an FP8 layer)
-  const float* sc0;  // FP8: scales of tile 0 / tile 1 (K block 0 of the tile's rows)
-  const float* sc1;
+  int sc0;    // FP8: index of tile 0's scale at K block 0 (gate or down array)
+  int sdown;  // FP8: a down unit
 };
 
 template <bool kFp8>
@@ -2108,9 +2122,8 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       x.nbox = 2;
       x.fp8 = kFp8;
       if (kFp8) {  // gate and up blocks [e][tile][K block]
-        const size_t b = ((size_t)e * (p.I / kTcRows) + d.tile) * (p.H / kTcRows);
-        x.sc0 = p.sc_gate + b;
-        x.sc1 = p.sc_up + b;
+        x.sc0 = (e * (p.I / kTcRows) + d.tile) * (p.H / kTcRows);
+        x.sdown = 0;
       }
       break;
     }
@@ -2131,8 +2144,8 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       x.tw0 = x.tw1 = &p.tmaps[kFp8 ? TM_Q_WD : TM_T_WD];
       x.fp8 = kFp8;
       if (kFp8) {  // down blocks [e][row block 2 tile, 2 tile + 1][K block]
-        x.sc0 = p.sc_down + ((size_t)e * (p.H / kTcRows) + 2 * d.tile) * (p.I / kTcRows);
-        x.sc1 = x.sc0 + p.I / kTcRows;
+        x.sc0 = (e * (p.H / kTcRows) + 2 * d.tile) * (p.I / kTcRows);
+        x.sdown = 1;
       }
       x.y0 = e * p.H + d.tile * 2 * kTcRows;
       x.y1 = x.y0 + kTcRows;
@@ -2210,9 +2223,10 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
     c_setup += (unsigned long long)(tclock<kTrace>() - tu0);
     // bytes of a stage: on full the activations and (bf16) the weight tiles; on wfull the
     // codes and scales of an FP8 stage
-    const uint32_t tx = (uint32_t)((xf ? 0 : x.nbox * kTcTileBytes) + x.N * kTcAtomK * 2);
-    const uint32_t wtx = (uint32_t)(x.nbox * (kFp8TileBytes + 16));
-    const int info0 = x.nbox | ((x.N / kTcActRows) << 2) | (xf ? kTcInfoFp8 : 0);
+    const int kstep = xf ? 2 : 1;  // K atoms per stage
+    const uint32_t tx = (uint32_t)((xf ? 0 : x.nbox * kTcTileBytes) + kstep * x.N * kTcAtomK * 2);
+    const uint32_t wtx = (uint32_t)(x.nbox * kFp8TileBytes);
+    const int info0 = x.nbox | ((x.N / kTcActRows) << 2) | (xf ? kTcInfoFp8 | (x.sdown ? kTcInfoFp8Down : 0) : 0);
     const int ka_end = d.kb0 + d.nkb;
     // one stage: header, barrier armed for weights + activations, the weight tiles
     auto issue_weights = [&](int ka) {
@@ -2225,10 +2239,8 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
         StageHeader h;
         h.kind = HK_STAGE;
         h.unit = hunit;
-        h.info = info0 | (ka == d.kb0 ? kTcInfoFirst : 0) | (ka == ka_end - 1 ? kTcInfoLast : 0);
-        h.wrow = xf ? (int)((((uintptr_t)(x.sc0 + (ka >> 1)) >> 2) & 3u) |
-                               ((((uintptr_t)(x.sc1 + (ka >> 1)) >> 2) & 3u) << 2))
-                       : -1;
+        h.info = info0 | (ka == d.kb0 ? kTcInfoFirst : 0) | (ka + kstep >= ka_end ? kTcInfoLast : 0);
+        h.wrow = xf ? x.sc0 + (ka >> 1) : -1;
         sm.hdr[pr.slot] = h;
         if (xf) mbar_arrive_expect_tx(wb, wtx);
         mbar_arrive_expect_tx(fb, tx);
@@ -2236,15 +2248,9 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
           trace_stamp<kTrace>(p, TR_FIRST_TMA);
           first_tma = false;
         }
-        if (xf) {  // codes, converted into tensor memory by the routing warps
+        if (xf) {  // codes of K block ka / 2, converted into tensor memory by the routing warps
           tma_load_2d(dst, x.tw0, ka * kTcAtomK, x.y0, wb, pol);
           if (x.nbox == 2) tma_load_2d(dst + kFp8TileBytes, x.tw1, ka * kTcAtomK, x.y1, wb, pol);
-          // each tile's scale (K block ka / 2) in the aligned 16-byte group that holds it
-          const auto group = [](const float* s) {
-            return reinterpret_cast<const float*>(reinterpret_cast<uintptr_t>(s) & ~(uintptr_t)15);
-          };
-          bulk_load(dst + kFp8ScaleOff, group(x.sc0 + (ka >> 1)), 16, wb);
-          if (x.nbox == 2) bulk_load(dst + kFp8ScaleOff + 16, group(x.sc1 + (ka >> 1)), 16, wb);
         } else {
           tma_load_2d(dst, x.tw0, ka * kTcAtomK, x.y0, fb, pol);
           if (x.nbox == 2) tma_load_2d(dst + kTcTileBytes, x.tw1, ka * kTcAtomK, x.y1, fb, pol);
@@ -2256,8 +2262,10 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
       if (lane == 0) {
         uint8_t* act = ring + slot * sh.slot_bytes + 2 * kTcTileBytes;
         uint64_t* fb = &sm.full[slot];
-        for (int q = 0; q < x.N / kTcActRows; ++q)
-          tma_load_2d_plain(act + q * kTcActRows * kTcAtomK * 2, x.ta, ka * kTcAtomK, x.arow + q * kTcActRows, fb);
+        for (int a = 0; a < kstep; ++a)  // an FP8 stage: two atoms, the second at +NA x 128 bytes
+          for (int q = 0; q < x.N / kTcActRows; ++q)
+            tma_load_2d_plain(act + a * sh.NA * kTcAtomK * 2 + q * kTcActRows * kTcAtomK * 2, x.ta,
+                              (ka + a) * kTcAtomK, x.arow + q * kTcActRows, fb);
       }
     };
     bool dep_known = x.dep == 0 ? n_ok
@@ -2269,10 +2277,10 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
       // weights stream while the input is awaited -- a ring's worth for h, one stage
       // for the normalised rows (at the start of the step the HBM queue must stay short
       // for the loads of x that the normalisation waits on)
-      const int depth = x.dep == 0 ? 1 : pr.nst;
+      const int depth = (x.dep == 0 ? 1 : pr.nst) * kstep;  // in K atoms
       const int pre_end = ka_end < d.kb0 + depth ? ka_end : d.kb0 + depth;
       const int slot0 = pr.slot;
-      for (; ka < pre_end && ok; ++ka) {
+      for (; ka < pre_end && ok; ka += kstep) {
         const long long t0 = tclock<kTrace>();
         ok = pr.wait_slot();
         c_slot += (unsigned long long)(tclock<kTrace>() - t0);
@@ -2283,7 +2291,7 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
         pr.advance();
         ++c_stages;
       }
-      const int narmed = ka - d.kb0;
+      const int narmed = (ka - d.kb0) / kstep;  // stages
       bool dep_ok = ok;
       const long long td0 = tclock<kTrace>();
       if (ok) {
@@ -2298,11 +2306,11 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
       }
       c_dep += (unsigned long long)(tclock<kTrace>() - td0);
       // every armed barrier gets its activation bytes, also after a failed wait
-      for (int i = 0; i < narmed; ++i) issue_act(d.kb0 + i, (slot0 + i) % pr.nst);
+      for (int i = 0; i < narmed; ++i) issue_act(d.kb0 + i * kstep, (slot0 + i) % pr.nst);
       __syncwarp();
       if (!dep_ok) ok = false;
     }
-    for (; ka < ka_end && ok; ++ka) {
+    for (; ka < ka_end && ok; ka += kstep) {
       {
         const long long t0 = tclock<kTrace>();
         ok = pr.wait_slot();
@@ -2510,14 +2518,14 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
 
 // The routing warps turn every FP8 stage (handed over by the producer through the
 // converter queue) into the MMA's A operand in tensor memory: warp w (of 8) converts
-// tile w / 4 of the stage, lane l the tile row 32 q + l of its lane quadrant q, each
-// code times the scale of its 128 x 128 block, and stores the row's 64 bf16 values as
-// 32 columns of its lane. The codes sit 64-byte swizzled (chunk c of row r at chunk
-// c ^ ((r / 2) mod 4) of the row), so the 8 lanes of a shared-memory phase read 8
-// distinct 16-byte chunks while the whole warp reads one logical chunk. A stages
-// rotate in stage order; one is rewritten only after the MMAs that read it completed.
-// The warps need nothing from one another: each waits for the stage itself (bounded)
-// and signals its part converted to the MMA warp.
+// tile w / 4 of the stage, lane l the tile row 32 q + l of its lane quadrant q (its 128
+// codes, each times the scale of the tile's 128 x 128 block), and stores the row's 128
+// bf16 values as 64 columns of its lane. The codes sit 128-byte swizzled (chunk c of row
+// r at chunk c ^ (r mod 8)), so the 8 lanes of a shared-memory phase read 8 distinct
+// 16-byte chunks while the whole warp reads one logical chunk. A stages rotate in stage
+// order; one is rewritten only after the MMAs that read it completed. The warps need
+// nothing from one another: each waits for the stage itself (bounded) and signals its
+// part converted to the MMA warp.
 template <bool kTrace>
 __device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, int mw, int lane, bool ok) {
   if (!ok) return;
@@ -2538,7 +2546,7 @@ __device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, int
   const int j = mw >> 2;             // weight tile
   const int r = quad * 32 + lane;    // tile row = tensor-memory lane
   const uint32_t tq = sm.tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(kFp8ACol0 + j * (kFp8AStageCols / 2));
-  const int swz = (r >> 1) & 3;
+  const int swz = r & 7;
   int q = 0, as = 0;
   uint32_t qph = 0u, asph = 0u;
   for (;;) {
@@ -2554,32 +2562,43 @@ __device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, int
     }
     if (slot < 0) return;
     if (!IDX_OK(p, slot < sh.nst)) return;
+    // the header was written before the queue entry: the tile's scale loads while the
+    // codes are still in flight
+    const StageHeader hd = sm.hdr[slot];
+    const bool conv = j < (hd.info & 3);
+    float sv = 0.0f;
+    if (conv) {
+      const bool down = (hd.info & kTcInfoFp8Down) != 0;
+      const float* sa = down ? p.sc_down : (j ? p.sc_up : p.sc_gate);
+      sv = __ldg(sa + hd.wrow + (down && j ? p.I / kTcRows : 0));
+    }
     if (!warp_wait(&sm.wfull[slot], par, p, lane, 64)) return;
     if (!warp_wait(&astage_empty(sm)[as], asph ^ 1u, p, lane, 64)) return;  // the A stage is free
     const long long t1 = tclock<kTrace>();
     c_wait += (unsigned long long)(t1 - t0);
-    const StageHeader hd = sm.hdr[slot];
-    if (j < (hd.info & 3)) {
+    if (conv) {
       tc_fence_after();
       const uint8_t* sbase = ring + slot * sh.slot_bytes;
-      const uint32_t sc = scale_bf16x2(
-          reinterpret_cast<const float*>(sbase + kFp8ScaleOff + 16 * j)[(hd.wrow >> (2 * j)) & 3]);
-      const uint8_t* row = sbase + j * kFp8TileBytes + r * kTcAtomK;
-      uint4 v[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(row + ((c ^ swz) << 4));
+      const uint32_t sc = scale_bf16x2(sv);
+      const uint8_t* row = sbase + j * kFp8TileBytes + r * (2 * kTcAtomK);
       const uint32_t col = (uint32_t)(as * kFp8AStageCols);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-        uint32_t o[8];
+      for (int h = 0; h < 2; ++h) {  // codes 64 h .. 64 h + 63
+        uint4 v[4];
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          e4m3x4_to_bf16x2x2(w[t], o[2 * t], o[2 * t + 1]);
-          o[2 * t] = mul_bf16x2(o[2 * t], sc);
-          o[2 * t + 1] = mul_bf16x2(o[2 * t + 1], sc);
+        for (int c = 0; c < 4; ++c) v[c] = *reinterpret_cast<const uint4*>(row + (((4 * h + c) ^ swz) << 4));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t w[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+          uint32_t o[8];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            e4m3x4_to_bf16x2x2(w[t], o[2 * t], o[2 * t + 1]);
+            o[2 * t] = mul_bf16x2(o[2 * t], sc);
+            o[2 * t + 1] = mul_bf16x2(o[2 * t + 1], sc);
+          }
+          tmem_st8(tq + col + (uint32_t)(8 * (4 * h + c)), o);  // K elements 16 (4h + c) .. + 15
         }
-        tmem_st8(tq + col + (uint32_t)(8 * c), o);  // K elements 16 c .. 16 c + 15
       }
       tmem_st_wait();
     }
@@ -2652,14 +2671,15 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
       const uint32_t idesc = idesc_bf16_m128((uint32_t)((info >> 2) & 7) * kTcActRows);
       const uint32_t t0 = tmem + (uint32_t)(abuf * kTcAccCols);
       if (kFp8 && (info & kTcInfoFp8)) {  // A from the tensor-memory stage the converters filled
+        // one 128-column K block: 8 K steps, the activations of the second atom at +NA x 128
         const uint32_t a0 = tmem + (uint32_t)(kFp8ACol0 + as * kFp8AStageCols);
+        const uint64_t da1 = sw128_desc(sbase + (uint32_t)fp8_act1_off(sm.sh.NA));
 #pragma unroll
-        for (int ks = 0; ks < kTcAtomK / 16; ++ks) {
+        for (int ks = 0; ks < 2 * kTcAtomK / 16; ++ks) {
           const uint32_t accum = (first && ks == 0) ? 0u : 1u;
-          tc_mma_bf16_ta(t0, a0 + (uint32_t)(8 * ks), da + (uint64_t)(2 * ks), idesc, accum);
-          if (nbox == 2)
-            tc_mma_bf16_ta(t0 + 64u, a0 + (uint32_t)(kFp8AStageCols / 2 + 8 * ks), da + (uint64_t)(2 * ks), idesc,
-                           accum);
+          const uint64_t db = (ks < 4 ? da : da1) + (uint64_t)(2 * (ks & 3));
+          tc_mma_bf16_ta(t0, a0 + (uint32_t)(8 * ks), db, idesc, accum);
+          if (nbox == 2) tc_mma_bf16_ta(t0 + 64u, a0 + (uint32_t)(kFp8AStageCols / 2 + 8 * ks), db, idesc, accum);
         }
         tc_commit(&astage_empty(sm)[as]);
       } else {
