@@ -28,11 +28,16 @@ enum TensorMapSlot {
   TM_T_AN = 14,   // normalised rows n  [max_batch][H]
   TM_T_AHS = 15,  // shared SwiGLU rows [max_batch][Is]
   TM_T_AHE = 16,  // expert SwiGLU rows [slots][I]
-  // FP8 expert weights (E4M3 codes, one byte each): boxes of 128 rows x 64 codes, no swizzle
+  // FP8 expert weights (E4M3 codes, one byte each): boxes of 128 rows x 128 codes (one
+  // K block), 128-byte swizzled
   TM_Q_WG = 17,   // W_gate codes [E*I][H]
   TM_Q_WU = 18,   // W_up codes   [E*I][H]
   TM_Q_WD = 19,   // W_down codes [E*H][I]
-  TM_COUNT = 20
+  // FP8 layers: the activations of two K atoms in one box {64 columns, 16 rows, 2 atoms}
+  // (3-D view: column within the atom, row, atom), 128-byte swizzled
+  TM_Q_AN = 20,   // normalised rows n  [max_batch][H]
+  TM_Q_AHE = 21,  // expert SwiGLU rows [slots][I]
+  TM_COUNT = 22
 };
 
 // Counters of one layer step (reset by the last CTA of every launch, except the epoch).

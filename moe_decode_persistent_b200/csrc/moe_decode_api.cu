@@ -117,6 +117,21 @@ static int encode_fp8(EncodeTiledFn enc, CUtensorMap* map, const void* base, uin
   return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Activation rows [rows][cols] (bf16) as a 3-D view {64 columns, rows, cols / 64 atoms} with
+// box {64, 16, 2}: the 16 rows of two consecutive K atoms in one copy, laid out as two
+// 16-row, 128-byte-swizzled boxes one after the other.
+static int encode_act_pair(EncodeTiledFn enc, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols) {
+  if ((reinterpret_cast<uintptr_t>(base) & 15u) != 0) return MOE_ERR_INVALID_ARG;
+  cuuint64_t dims[3] = {(cuuint64_t)moe::kTcAtomK, rows, cols / moe::kTcAtomK};
+  cuuint64_t strides[2] = {cols * 2, (cuuint64_t)moe::kTcAtomK * 2};
+  cuuint32_t box[3] = {(cuuint32_t)moe::kTcAtomK, (cuuint32_t)moe::kTcActRows, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
 // Every FP8 block scale must be a power of two in [2^-117, 2^7] (either sign): the
 // kernel turns a code into the bf16 value(code) x 2^-120 (exact; a bf16 subnormal for
 // the E4M3 subnormals) and multiplies by scale x 2^120 (a bf16 normal for these scales),
@@ -426,6 +441,10 @@ static int create_impl(const moe_decode_config* cfg, const moe_decode_layer_weig
       rc |= encode_tc(enc, &m[moe::TM_T_AN], h->n, (uint64_t)actRows, (uint64_t)H, AR);
       rc |= encode_tc(enc, &m[moe::TM_T_AHS], h->hs, (uint64_t)actRows, (uint64_t)Is, AR);
       rc |= encode_tc(enc, &m[moe::TM_T_AHE], h->he, (uint64_t)moe::kMaxSlots, (uint64_t)I, AR);
+      if (fp8) {
+        rc |= encode_act_pair(enc, &m[moe::TM_Q_AN], h->n, (uint64_t)actRows, (uint64_t)H);
+        rc |= encode_act_pair(enc, &m[moe::TM_Q_AHE], h->he, (uint64_t)moe::kMaxSlots, (uint64_t)I);
+      }
     }
     if (rc != MOE_OK) {
       cudaFree(h->ws);

@@ -2086,6 +2086,7 @@ struct TcSeg {
   int dep;   // 0: normalised rows, 1: shared h, 2: the expert's h
   int pair;
   int fp8;   // 1: the weight tiles are E4M3 codes (expert units of an FP8 layer)
+  const CUtensorMap* ta2;  // FP8: the activations of two K atoms in one box (16-row tiles)
   int sc0;    // FP8: index of tile 0's scale at K block 0 (gate or down array)
   int sdown;  // FP8: a down unit
 };
@@ -2122,6 +2123,7 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       x.nbox = 2;
       x.fp8 = kFp8;
       if (kFp8) {  // gate and up blocks [e][tile][K block]
+        x.ta2 = &p.tmaps[TM_Q_AN];
         x.sc0 = (e * (p.I / kTcRows) + d.tile) * (p.H / kTcRows);
         x.sdown = 0;
       }
@@ -2144,6 +2146,7 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       x.tw0 = x.tw1 = &p.tmaps[kFp8 ? TM_Q_WD : TM_T_WD];
       x.fp8 = kFp8;
       if (kFp8) {  // down blocks [e][row block 2 tile, 2 tile + 1][K block]
+        x.ta2 = &p.tmaps[TM_Q_AHE];
         x.sc0 = (e * (p.H / kTcRows) + 2 * d.tile) * (p.I / kTcRows);
         x.sdown = 1;
       }
@@ -2175,7 +2178,7 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
   // (measured: one acquire fence per map cost ~4 us per step)
   if (lane == 0)
     for (int t = TM_T_WR; t < TM_COUNT; ++t) {
-      const bool qmap = t >= TM_Q_WG, bf16_expert = t == TM_T_WG || t == TM_T_WU || t == TM_T_WD;
+      const bool qmap = t >= TM_Q_WG, bf16_expert = t == TM_T_WG || t == TM_T_WU || t == TM_T_WD;  // (Q: FP8)
       if (kFp8 ? !bf16_expert : !qmap) prefetch_tensormap(&p.tmaps[t]);  // the maps this layer has
     }
   if (p.layer > 0) {  // the previous layer's record of completed experts
@@ -2262,6 +2265,11 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
       if (lane == 0) {
         uint8_t* act = ring + slot * sh.slot_bytes + 2 * kTcTileBytes;
         uint64_t* fb = &sm.full[slot];
+        if (xf && x.N == kTcActRows && sh.NA == kTcActRows) {
+          // an FP8 stage of 16 token rows: both atoms in one copy (the second at +16 x 128 bytes)
+          tma_load_3d_plain(act, x.ta2, 0, x.arow, ka, fb);
+          return;
+        }
         for (int a = 0; a < kstep; ++a)  // an FP8 stage: two atoms, the second at +NA x 128 bytes
           for (int q = 0; q < x.N / kTcActRows; ++q)
             tma_load_2d_plain(act + a * sh.NA * kTcAtomK * 2 + q * kTcActRows * kTcAtomK * 2, x.ta,
