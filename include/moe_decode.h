@@ -161,6 +161,38 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
 int moe_decode_create_fp8(const moe_decode_config* cfg, const moe_decode_layer_weights_fp8* layers, int device,
                           moe_decode_handle** out);
 
+/* Expert parallelism (one layer): a handle for the experts expert_begin <= e <
+ * expert_end of a layer whose routed experts are split over several GPUs, router and
+ * shared expert replicated on each (the pages spread the expert work over the GPUs and
+ * fold the cross-GPU exchange into the computation: page post.smzdm.com/p/a6zppe4g,
+ * section "改了什么：每层 23 个 kernel 砍到 13 个", items "把通信缝进计算" and "MoE
+ * 去重"). layers[0] holds the full router (E rows) and shared expert, but w_gate,
+ * w_up and w_down hold only this range's experts: [expert_end - expert_begin][I][H]
+ * and [..][H][I], local expert i being expert expert_begin + i. cfg->n_layers must
+ * be 1 and every dimension a multiple of 128 (the tensor-core kernel; otherwise
+ * MOE_ERR_UNSUPPORTED_SHAPE). Steps of the handle go through
+ * moe_decode_step_partial. */
+int moe_decode_create_ep(const moe_decode_config* cfg, const moe_decode_layer_weights* layers, int device,
+                         int expert_begin, int expert_end, moe_decode_handle** out);
+
+/* The partial output of a one-layer step over the handle's experts:
+ * y_partial[b] = sum over row b's top-k choices j whose expert the handle covers of
+ * w_j E_j(n_b), plus x_b + s_b (the residual and the shared expert) when
+ * add_residual_shared is nonzero -- exactly one rank sets it. Every row is written.
+ * y_partial: device fp32 [batch][H], 16-byte aligned, owned by the caller. The sum of
+ * the ranks' partials (an all-reduce) rounded by moe_decode_partial_to_bf16 is the
+ * layer's output. Routing (logits, top-k, softmax) is computed in full on every rank.
+ * Arguments as moe_decode_step; MOE_ERR_INVALID_ARG for a handle of several layers, an
+ * FP8 handle, or one whose shapes the tensor-core kernel cannot run. A whole-layer
+ * handle (moe_decode_create) gives the whole layer's output in fp32. */
+int moe_decode_step_partial(moe_decode_handle* h, const void* x_in, float* y_partial, int batch, int top_k,
+                            int add_residual_shared, void* stream, const moe_decode_debug* dbg);
+
+/* y_out[i] = bf16(y_partial[i]) (round to nearest even) for i < n, on `device`,
+ * asynchronous on `stream`: the output of an expert-parallel step after the
+ * all-reduce. Device pointers; y_out 2-byte aligned. */
+int moe_decode_partial_to_bf16(const float* y_partial, void* y_out, long long n, int device, void* stream);
+
 /* One decode step over all layers. x_in: device bf16 [batch][H]; y_out: device
  * bf16 [batch][H] (may not alias x_in). 1 <= batch <= max_batch, 1 <= top_k <=
  * top_k_max. stream: a cudaStream_t (NULL = legacy default stream). dbg: NULL or

@@ -154,6 +154,13 @@ def _load(path):
         L.moe_decode_step_noalloc.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerWeights),
                                               vp, vp, i, i, vp, vp]
         L.moe_decode_step_noalloc.restype = i
+        L.moe_decode_create_ep.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LayerWeights), i, i, i,
+                                           ctypes.POINTER(vp)]
+        L.moe_decode_create_ep.restype = i
+        L.moe_decode_step_partial.argtypes = [vp, vp, vp, i, i, i, vp, vp]
+        L.moe_decode_step_partial.restype = i
+        L.moe_decode_partial_to_bf16.argtypes = [vp, vp, ctypes.c_longlong, i, vp]
+        L.moe_decode_partial_to_bf16.restype = i
         L.moe_decode_strerror.argtypes = [i]
         L.moe_decode_strerror.restype = ctypes.c_char_p
     return L
@@ -161,6 +168,17 @@ def _load(path):
 
 def strerror(code: int) -> str:
     return lib().moe_decode_strerror(int(code)).decode()
+
+
+def partial_to_bf16(part, out, device: int = 0, stream=None) -> None:
+    """out <- bf16(part) elementwise (device fp32 -> device bf16, same element count),
+    asynchronous on `stream`: the output of an expert-parallel step once the ranks'
+    partials are summed."""
+    n = int(part.numel())
+    if int(out.numel()) != n or str(part.dtype) != "torch.float32":
+        raise ValueError("partial_to_bf16: fp32 input and an output of the same element count")
+    _check(lib().moe_decode_partial_to_bf16(_ptr(part), _ptr(out), n, int(device), _stream_handle(stream)),
+           "moe_decode_partial_to_bf16")
 
 
 class MoeDecodeError(RuntimeError):
@@ -243,10 +261,13 @@ class MoeDecode:
     The caller keeps those tensors alive for the handle's lifetime. checked: run the
     bounds-checked build (libmoe_decode_checked.so), which reports a schedule-derived
     index outside its buffer as MOE_ERR_BOUNDS instead of accessing it.
+    expert_range: (e0, e1) for one rank of an expert-parallel layer
+    (moe_decode_create_ep): one layer whose w_gate / w_up / w_down hold only experts
+    e0 .. e1 - 1; its steps go through step_partial.
     """
 
     def __init__(self, hidden, n_experts, top_k_max, inter, shared_inter, max_batch, layers,
-                 eps=1e-6, device=0, checked=False, fp8=False):
+                 eps=1e-6, device=0, checked=False, fp8=False, expert_range=None):
         self._lib = lib(checked)  # checked: the bounds-checked test build of the library
         self.cfg = Config(hidden, n_experts, top_k_max, inter, shared_inter, max_batch,
                           len(layers), eps)
@@ -262,8 +283,13 @@ class MoeDecode:
             arr = (LayerWeights * len(layers))()
             for i, w in enumerate(layers):
                 arr[i] = LayerWeights(*(_ptr(w.get(name)) for name, _ in LayerWeights._fields_))
-            _check(self._lib.moe_decode_create(ctypes.byref(self.cfg), arr, int(device), ctypes.byref(h)),
-                   "moe_decode_create")
+            if expert_range is not None:
+                e0, e1 = (int(v) for v in expert_range)
+                _check(self._lib.moe_decode_create_ep(ctypes.byref(self.cfg), arr, int(device), e0, e1,
+                                                      ctypes.byref(h)), "moe_decode_create_ep")
+            else:
+                _check(self._lib.moe_decode_create(ctypes.byref(self.cfg), arr, int(device), ctypes.byref(h)),
+                       "moe_decode_create")
         self.handle = h
         self.n_layers = len(layers)
 
@@ -274,6 +300,19 @@ class MoeDecode:
         dbg = self._debug(debug)
         _check(self._lib.moe_decode_step(self.handle, _ptr(x), _ptr(y), int(batch), int(top_k),
                                      _stream_handle(stream), dbg), "moe_decode_step")
+
+    def step_partial(self, x, y_part, batch, top_k, residual_shared=True, stream=None, debug=None) -> None:
+        """y_part <- the fp32 partial output of a one-layer step over the handle's experts
+        (x + shared expert included when residual_shared); x device bf16 and y_part device
+        fp32, both [batch, hidden]."""
+        _check_rows(x, "x", batch, self.cfg.hidden, "cuda", "moe_decode_step_partial")
+        if str(y_part.dtype) != "torch.float32" or tuple(y_part.shape) != (batch, self.cfg.hidden) or \
+                not y_part.is_contiguous() or y_part.device.type != "cuda":
+            raise ValueError("moe_decode_step_partial: y_part must be a contiguous CUDA fp32 [batch, hidden] tensor")
+        dbg = self._debug(debug)
+        _check(self._lib.moe_decode_step_partial(self.handle, _ptr(x), _ptr(y_part), int(batch), int(top_k),
+                                                 1 if residual_shared else 0, _stream_handle(stream), dbg),
+               "moe_decode_step_partial")
 
     def step_host(self, x_host, y_host, batch, top_k, stream=None, debug=None) -> None:
         """Same step on host buffers (pinned torch CPU tensors or host pointers)."""

@@ -111,6 +111,13 @@ struct Params {
   // activations
   const uint16_t* x;  // bf16 [B][H]
   uint16_t* y;        // bf16 [B][H]
+  // expert parallelism (tensor-core path): the step schedules only the selected experts e
+  // with ep_e0 <= e < ep_e1, whose weights sit at index e - ep_wbase of the expert arrays;
+  // with y_part set, row b's output is the fp32 partial sum_{local j} w_j E_j(n_b), plus
+  // x_b + s_b when ep_rs, written to y_part instead of y. A whole-layer step: 0, E, 0,
+  // nullptr, 1.
+  int ep_e0, ep_e1, ep_wbase, ep_rs;
+  float* y_part;      // fp32 [B][H] or nullptr
   // this layer's parameters
   const CUtensorMap* tmaps;  // TM_COUNT maps in global memory
   const uint16_t* gamma;     // bf16 [H]

@@ -19,6 +19,9 @@ int tc_threads_per_cta();
 const void* tc_kernel_fn();
 const void* tc_kernel_fn_trace();
 const void* tc_fp8_kernel_fn();
+const void* tc_ep_kernel_fn();
+const void* tc_ep_kernel_fn_trace();
+int launch_partial_to_bf16(const float* in, uint16_t* out, long long n, int sms, cudaStream_t stream);
 const void* tc_fp8_kernel_fn_trace();
 const void* fused_kernel_fn();
 const void* fused_kernel_fn_trace();
@@ -61,6 +64,8 @@ struct moe_decode_handle {
   uint16_t* x_stage;     // [max_batch][H] host-step staging
   uint16_t* y_stage;
   unsigned max_units, max_tiles;
+  int ep_e0, ep_e1;  // the experts this handle's steps cover (0, E unless created for a range);
+                     // its expert arrays hold experts ep_e0 .. ep_e1 - 1
   int tc_capable;    // every dimension a multiple of 128: the tensor-core kernel can run
   int tc_min_batch;  // batches of at least this many rows take the tensor-core path
   unsigned flags;
@@ -198,11 +203,15 @@ const char* moe_decode_strerror(int code) {
 
 // Both create entry points: layers (bf16 experts), or fp8 (FP8 experts; layers then
 // holds the same layers with the expert pointers set to the codes, for the checks).
+// e0, e1: the experts the handle covers and its expert arrays hold (0, E: all).
 static int create_impl(const moe_decode_config* cfg, const moe_decode_layer_weights* layers,
-                       const moe_decode_layer_weights_fp8* fp8, int device, moe_decode_handle** out) {
+                       const moe_decode_layer_weights_fp8* fp8, int device, moe_decode_handle** out,
+                       int e0 = 0, int e1 = -1) {
   if (!cfg || !layers || !out) return MOE_ERR_INVALID_ARG;
   *out = nullptr;
   const moe_decode_config c = *cfg;
+  if (e1 < 0) e1 = c.n_experts;
+  if (e0 < 0 || e0 >= e1 || e1 > c.n_experts) return MOE_ERR_INVALID_ARG;
   if (c.n_layers < 1 || c.n_layers > 8 || c.max_batch < 1 || c.max_batch > 64 || c.top_k_max < 1 ||
       c.top_k_max > 32 || c.top_k_max > c.n_experts || !(c.eps >= 0.0f))
     return MOE_ERR_INVALID_ARG;
@@ -252,6 +261,10 @@ static int create_impl(const moe_decode_config* cfg, const moe_decode_layer_weig
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::tc_kernel_fn_trace(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::tc_ep_kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(moe::tc_ep_kernel_fn_trace(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
+    if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::tc_fp8_kernel_fn(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(moe::tc_fp8_kernel_fn_trace(), cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsm);
@@ -282,6 +295,8 @@ static int create_impl(const moe_decode_config* cfg, const moe_decode_layer_weig
   h->num_sms = sms;
   h->wait_ns = 2000ull * 1000000ull;
   h->tc_capable = tc_ok;
+  h->ep_e0 = e0;
+  h->ep_e1 = e1;
   h->tc_min_batch = kDefaultTcMinBatch;
   h->layers = (moe_decode_layer_weights*)malloc(sizeof(moe_decode_layer_weights) * c.n_layers);
   memcpy(h->layers, layers, sizeof(moe_decode_layer_weights) * c.n_layers);
@@ -291,6 +306,7 @@ static int create_impl(const moe_decode_config* cfg, const moe_decode_layer_weig
   }
 
   const int H = c.hidden, E = c.n_experts, I = c.inter, Is = c.shared_inter, L = c.n_layers;
+  const int Ew = e1 - e0;  // experts held by the expert arrays
   // host tensor maps
   CUtensorMap* maps = (CUtensorMap*)aligned_alloc(64, sizeof(CUtensorMap) * moe::TM_COUNT * L);
   if (!maps) {
@@ -306,9 +322,9 @@ static int create_impl(const moe_decode_config* cfg, const moe_decode_layer_weig
     CUtensorMap* m = maps + l * moe::TM_COUNT;
     rc |= encode_2d(enc, &m[moe::TM_WR], w.w_router, (uint64_t)E, (uint64_t)H);
     if (!fp8) {  // (an FP8 handle never takes the CUDA-core path)
-      rc |= encode_2d(enc, &m[moe::TM_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H);
-      rc |= encode_2d(enc, &m[moe::TM_WU], w.w_up, (uint64_t)E * I, (uint64_t)H);
-      rc |= encode_2d(enc, &m[moe::TM_WD], w.w_down, (uint64_t)E * H, (uint64_t)I);
+      rc |= encode_2d(enc, &m[moe::TM_WG], w.w_gate, (uint64_t)Ew * I, (uint64_t)H);
+      rc |= encode_2d(enc, &m[moe::TM_WU], w.w_up, (uint64_t)Ew * I, (uint64_t)H);
+      rc |= encode_2d(enc, &m[moe::TM_WD], w.w_down, (uint64_t)Ew * H, (uint64_t)I);
     }
     rc |= encode_2d(enc, &m[moe::TM_WSG], w.ws_gate, (uint64_t)Is, (uint64_t)H);
     rc |= encode_2d(enc, &m[moe::TM_WSU], w.ws_up, (uint64_t)Is, (uint64_t)H);
@@ -317,13 +333,13 @@ static int create_impl(const moe_decode_config* cfg, const moe_decode_layer_weig
       const uint32_t R = (uint32_t)moe::kTcRows;
       rc |= encode_tc(enc, &m[moe::TM_T_WR], w.w_router, (uint64_t)E, (uint64_t)H, R);
       if (fp8) {
-        rc |= encode_fp8(enc, &m[moe::TM_Q_WG], fp8[l].w_gate, (uint64_t)E * I, (uint64_t)H);
-        rc |= encode_fp8(enc, &m[moe::TM_Q_WU], fp8[l].w_up, (uint64_t)E * I, (uint64_t)H);
-        rc |= encode_fp8(enc, &m[moe::TM_Q_WD], fp8[l].w_down, (uint64_t)E * H, (uint64_t)I);
+        rc |= encode_fp8(enc, &m[moe::TM_Q_WG], fp8[l].w_gate, (uint64_t)Ew * I, (uint64_t)H);
+        rc |= encode_fp8(enc, &m[moe::TM_Q_WU], fp8[l].w_up, (uint64_t)Ew * I, (uint64_t)H);
+        rc |= encode_fp8(enc, &m[moe::TM_Q_WD], fp8[l].w_down, (uint64_t)Ew * H, (uint64_t)I);
       } else {
-        rc |= encode_tc(enc, &m[moe::TM_T_WG], w.w_gate, (uint64_t)E * I, (uint64_t)H, R);
-        rc |= encode_tc(enc, &m[moe::TM_T_WU], w.w_up, (uint64_t)E * I, (uint64_t)H, R);
-        rc |= encode_tc(enc, &m[moe::TM_T_WD], w.w_down, (uint64_t)E * H, (uint64_t)I, R);
+        rc |= encode_tc(enc, &m[moe::TM_T_WG], w.w_gate, (uint64_t)Ew * I, (uint64_t)H, R);
+        rc |= encode_tc(enc, &m[moe::TM_T_WU], w.w_up, (uint64_t)Ew * I, (uint64_t)H, R);
+        rc |= encode_tc(enc, &m[moe::TM_T_WD], w.w_down, (uint64_t)Ew * H, (uint64_t)I, R);
       }
       rc |= encode_tc(enc, &m[moe::TM_T_WSG], w.ws_gate, (uint64_t)Is, (uint64_t)H, R);
       rc |= encode_tc(enc, &m[moe::TM_T_WSU], w.ws_up, (uint64_t)Is, (uint64_t)H, R);
@@ -478,6 +494,25 @@ int moe_decode_create(const moe_decode_config* cfg, const moe_decode_layer_weigh
   return create_impl(cfg, layers, nullptr, device, out);
 }
 
+int moe_decode_create_ep(const moe_decode_config* cfg, const moe_decode_layer_weights* layers, int device,
+                         int expert_begin, int expert_end, moe_decode_handle** out) {
+  if (!cfg || !out || cfg->n_layers != 1) return MOE_ERR_INVALID_ARG;
+  if (expert_begin < 0 || expert_begin >= expert_end || expert_end > cfg->n_experts) return MOE_ERR_INVALID_ARG;
+  const moe_decode_config c = *cfg;
+  if (c.hidden % moe::kTcRows || c.inter % moe::kTcRows || c.shared_inter % moe::kTcRows ||
+      c.n_experts % moe::kTcRows || c.max_batch > moe::kTcMaxN)
+    return MOE_ERR_UNSUPPORTED_SHAPE;  // the tensor-core kernel only
+  const int rc = create_impl(cfg, layers, nullptr, device, out, expert_begin, expert_end);
+  if (rc != MOE_OK) return rc;
+  if (!(*out)->tc_capable) {
+    moe_decode_destroy(*out);
+    *out = nullptr;
+    return MOE_ERR_UNSUPPORTED_SHAPE;
+  }
+  (*out)->tc_min_batch = 1;
+  return MOE_OK;
+}
+
 int moe_decode_create_fp8(const moe_decode_config* cfg, const moe_decode_layer_weights_fp8* layers, int device,
                           moe_decode_handle** out) {
   if (!cfg || !layers || !out || cfg->n_layers < 1 || cfg->n_layers > 8) return MOE_ERR_INVALID_ARG;
@@ -496,6 +531,7 @@ int moe_decode_create_fp8(const moe_decode_config* cfg, const moe_decode_layer_w
 
 static bool use_tc(const moe_decode_handle* h, int batch) {
   if (h->layers_fp8) return true;  // FP8 experts: the tensor-core kernel only
+  if (h->ep_e0 != 0 || h->ep_e1 != h->cfg.n_experts) return true;  // an expert range: tensor cores only
   return h->tc_capable && h->tc_min_batch > 0 && batch >= h->tc_min_batch;
 }
 
@@ -507,8 +543,11 @@ static bool fused_step(const moe_decode_handle* h, int batch) {
   return use_tc(h, batch) && h->cfg.n_layers > 1 && !h->layers_fp8;
 }
 
+// y_part (nullable): the fp32 partial output of a one-layer step over the handle's
+// experts (with x + s only when add_rs); y_out is then unused.
 static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, int batch, int top_k,
-                         cudaStream_t stream, const moe_decode_debug* dbg) {
+                         cudaStream_t stream, const moe_decode_debug* dbg, float* y_part = nullptr,
+                         int add_rs = 1) {
   const moe_decode_config& c = h->cfg;
   const int L = c.n_layers;
   const bool tc = use_tc(h, batch);
@@ -528,6 +567,11 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     p.eps = c.eps;
     p.x = l == 0 ? (const uint16_t*)x_in : h->layer_io + (size_t)(l - 1) * c.max_batch * c.hidden;
     p.y = l == L - 1 ? (uint16_t*)y_out : h->layer_io + (size_t)l * c.max_batch * c.hidden;
+    p.ep_e0 = h->ep_e0;
+    p.ep_e1 = h->ep_e1;
+    p.ep_wbase = h->ep_e0;
+    p.ep_rs = add_rs;
+    p.y_part = y_part;
     const moe_decode_layer_weights& w = h->layers[l];
     p.tmaps = h->d_tmaps + l * moe::TM_COUNT;
     p.gamma = (const uint16_t*)w.gamma;
@@ -582,8 +626,10 @@ static int launch_layers(moe_decode_handle* h, const void* x_in, void* y_out, in
     p.trace = h->trace ? h->trace + (size_t)l * h->num_sms * moe::kTraceSlots : nullptr;
     if (fused) continue;
     void* args[] = {&p};
+    const bool ep = y_part != nullptr || h->ep_e0 != 0 || h->ep_e1 != c.n_experts;
     const void* fn = !tc             ? (h->trace ? moe::kernel_fn_trace() : moe::kernel_fn())
                      : h->layers_fp8 ? (h->trace ? moe::tc_fp8_kernel_fn_trace() : moe::tc_fp8_kernel_fn())
+                     : ep            ? (h->trace ? moe::tc_ep_kernel_fn_trace() : moe::tc_ep_kernel_fn())
                                      : (h->trace ? moe::tc_kernel_fn_trace() : moe::tc_kernel_fn());
     const int threads = tc ? moe::tc_threads_per_cta() : moe::threads_per_cta();
     const size_t smem = tc ? moe::tc_smem_bytes() : moe::smem_bytes();
@@ -618,6 +664,29 @@ int moe_decode_step(moe_decode_handle* h, const void* x_in, void* y_out, int bat
     return MOE_ERR_INVALID_ARG;
   if (cudaSetDevice(h->device) != cudaSuccess) return MOE_ERR_CUDA;
   return launch_layers(h, x_in, y_out, batch, top_k, (cudaStream_t)stream, dbg);
+}
+
+int moe_decode_step_partial(moe_decode_handle* h, const void* x_in, float* y_partial, int batch, int top_k,
+                            int add_residual_shared, void* stream, const moe_decode_debug* dbg) {
+  int rc = check_step_args(h, x_in, y_partial, batch, top_k);
+  if (rc != MOE_OK) return rc;
+  // one bf16 layer on the tensor-core kernel (FP8 handles have no partial step)
+  if (h->cfg.n_layers != 1 || !h->tc_capable || h->layers_fp8) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(x_in) & 15u) || (reinterpret_cast<uintptr_t>(y_partial) & 15u))
+    return MOE_ERR_INVALID_ARG;
+  if (cudaSetDevice(h->device) != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_layers(h, x_in, nullptr, batch, top_k, (cudaStream_t)stream, dbg, y_partial,
+                       add_residual_shared ? 1 : 0);
+}
+
+int moe_decode_partial_to_bf16(const float* y_partial, void* y_out, long long n, int device, void* stream) {
+  if (!y_partial || !y_out || n < 0) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (cudaSetDevice(device) != cudaSuccess) return MOE_ERR_CUDA;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess) return MOE_ERR_CUDA;
+  return moe::launch_partial_to_bf16(y_partial, (uint16_t*)y_out, n, sms, (cudaStream_t)stream) == 0 ? MOE_OK
+                                                                                                    : MOE_ERR_CUDA;
 }
 
 int moe_decode_step_host(moe_decode_handle* h, const void* x_host, void* y_host, int batch,

@@ -6,8 +6,9 @@
 // 1.68倍", section "为什么解码阶段适合Megakernel"; page post.smzdm.com/p/a6zppe4g,
 // section "改了什么：每层 23 个 kernel 砍到 13 个": 23 -> 13 kernels per layer).
 //
-// Instances of moe_decode_layer_kernel<trace, tc, fp8> implement the step; the host
-// picks one per step (the batch-shape switch; fp8 for a handle with FP8 experts):
+// Instances of moe_decode_layer_kernel<trace, tc, fp8, ep> implement the step; the host
+// picks one per step (the batch-shape switch; fp8 for a handle with FP8 experts; ep for
+// a handle over a range of the experts, whose step yields its fp32 part of the output):
 //
 // Tensor-core kernel (tc = true, 14 warps)
 //   warp 0      producer: takes units of work from a global queue and streams, per
@@ -1354,7 +1355,7 @@ __device__ bool route_rows_tc(const Params& p, Smem& sm, int mw, int lane, uint3
 // row each, so the unique experts are the choices in ascending id (each one's slot is
 // its rank among them) and the hottest-first order is that same order. One warp
 // builds it (the general builder's result, without its masks, scans and rendezvous).
-template <bool kTrace>
+template <bool kTrace, bool kEp = false>
 __device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase, uint32_t tag) {
   const Shape& sh = sm.sh;
   Sched& sc = sm.sc;
@@ -1366,17 +1367,24 @@ __device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, u
     if (lane == 0) sm.bcast = ok ? 1 : 0;
     if (ok) {
       if (lane == 0) trace_clk<kTrace>(p, TR_TOPK_SYNCED);
+      // this step's experts (all, unless the step covers an expert range): rank r among them
+      const bool local = lane < k && (!kEp || (e >= p.ep_e0 && e < p.ep_e1));
+      const int el = local ? e : 0x7fffffff;
       int r = 0;
 #pragma unroll 4
-      for (int sl = 0; sl < 32; ++sl) r += __shfl_sync(0xffffffffu, e, sl) < e ? 1 : 0;
+      for (int sl = 0; sl < 32; ++sl) r += __shfl_sync(0xffffffffu, el, sl) < el ? 1 : 0;
+      const int kl = __popc(__ballot_sync(0xffffffffu, local));
       const int es = tc_expert_splits(1, sh.kblk ? sh.nkbH / 2 : sh.nkbH);
-      if (lane < k && !IDX_OK(p, (unsigned)e < (unsigned)p.E && (unsigned)r < (unsigned)kMaxSlots)) {
+      if (local && !IDX_OK(p, (unsigned)e < (unsigned)p.E && (unsigned)r < (unsigned)kMaxSlots)) {
         e = 0;  // reported; the step is abandoned
         r = lane;
       }
       if (lane < k) {
         sm.u.t.topk_idx[lane] = e;
         sm.u.t.topk_w[lane] = w;
+        if (!local) sc.slot_of[lane] = (int16_t)-1;  // another rank's expert: no slot row here
+      }
+      if (local) {
         sc.slot_expert[r] = (int16_t)e;
         sc.slot_cnt[r] = 1;
         sc.slot_base[r] = (int16_t)r;
@@ -1390,29 +1398,29 @@ __device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, u
         sc.slot_of[lane] = (int16_t)r;
       }
       if (lane == 0) {
-        sc.U = k;
-        sc.S = k;
-        sc.P = k;
-        sc.slot_base[k] = (int16_t)k;
-        sc.pair_ubase[k] = k * sh.IT * es;
-        sc.NE = k * sh.IT * es;
-        sc.down_splits = 1 + k;
-        sc.ND = sh.DT * k;
+        sc.U = kl;
+        sc.S = kl;
+        sc.P = kl;
+        sc.slot_base[kl] = (int16_t)kl;
+        sc.pair_ubase[kl] = kl * sh.IT * es;
+        sc.NE = kl * sh.IT * es;
+        sc.down_splits = 1 + kl;
+        sc.ND = sh.DT * kl;
         sc.total = sh.pre + sc.NE + sc.ND;
-        const unsigned tiles = (unsigned)(sh.RT + sh.ST + k * sh.IT + sh.DT);
+        const unsigned tiles = (unsigned)(sh.RT + sh.ST + kl * sh.IT + sh.DT);
         sm.bcast2 = ((unsigned)sc.total <= p.max_units && tiles <= p.max_tiles) ? 1 : 0;
         if (!sm.bcast2) record_abort(p, MOE_ERR_UNSUPPORTED_SHAPE);
       }
       __syncwarp();
 #ifdef MOE_BOUNDS_CHECK
-      if (lane == 0 && (p.flags & kFlagBadSlot)) sc.slot_of[0] = (int16_t)k;  // the first row past the schedule
+      if (lane == 0 && (p.flags & kFlagBadSlot)) sc.slot_of[0] = (int16_t)kl;  // the first row past the schedule
       __syncwarp();
 #endif
       if (blockIdx.x == 0 && lane < k) {
         if (p.dbg_idx) p.dbg_idx[lane] = e;
         if (p.dbg_w) p.dbg_w[lane] = w;
       }
-      if (blockIdx.x == 0 && lane == 0 && p.dbg_nuniq) *p.dbg_nuniq = k;
+      if (blockIdx.x == 0 && lane == 0 && p.dbg_nuniq) *p.dbg_nuniq = kl;
     }
   }
   const bool ok = mac_sync(sm, mphase, p, lane) && sm.bcast && sm.bcast2;
@@ -1425,7 +1433,7 @@ __device__ bool build_schedule_b1(const Params& p, Smem& sm, int mw, int lane, u
 // 13 * 128) with no global effects, made by CTAs that own no row while they wait for
 // the published choices, so that the real pass runs with its instructions cached
 // (one out-of-line copy of the code serves both passes).
-template <bool kTrace>
+template <bool kTrace, bool kEp = false>
 __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw, int lane, uint32_t& mphase,
                                                bool dry) {
   const Shape& sh = sm.sh;
@@ -1451,7 +1459,7 @@ __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw
     const float w = dry ? 1.0f : __uint_as_float((uint32_t)ch.y);
     sm.u.t.topk_idx[t] = e;
     sm.u.t.topk_w[t] = w;
-    atomicOr(&sm.u.t.mask[e], 1ull << (t / k));
+    if (!kEp || (e >= p.ep_e0 && e < p.ep_e1)) atomicOr(&sm.u.t.mask[e], 1ull << (t / k));  // this step's experts
   }
   if (!mac_sync(sm, mphase, p, lane)) return false;
   if (mtid == 0 && !dry) trace_clk<kTrace>(p, TR_TOPK_DONE);
@@ -1574,6 +1582,10 @@ __device__ __noinline__ bool build_schedule_tc(const Params& p, Smem& sm, int mw
   for (int t = mtid; t < B * k; t += kMacThreads) {
     const int b = t / k;
     const int e = sm.u.t.topk_idx[t];
+    if (kEp && (e < p.ep_e0 || e >= p.ep_e1)) {  // another rank's expert: no slot row here
+      sc.slot_of[t] = (int16_t)-1;
+      continue;
+    }
     const unsigned long long m = sm.u.t.mask[e];
     const int r = sc.slot_base[sc.eslot[e]] + __popcll(m & ((1ull << b) - 1ull));
     if (!IDX_OK(p, (unsigned)r < (unsigned)kMaxSlots)) continue;
@@ -2091,7 +2103,7 @@ struct TcSeg {
   int sdown;  // FP8: a down unit
 };
 
-template <bool kFp8>
+template <bool kFp8, bool kEp = false>
 __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, const Sched& sc, const UnitDesc& d,
                                             TcSeg& x) {
   x.pair = d.pair;
@@ -2115,8 +2127,9 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       break;
     case UT_EXPERT: {
       // every token row is an MMA column; the epilogue keeps the expert's own rows
-      int e = sc.slot_expert[sc.pair_slot[d.pair]];
-      if (!IDX_OK(p, (unsigned)d.pair < (unsigned)kMaxSlots && (unsigned)e < (unsigned)p.E)) e = 0;
+      // e: the expert's index in this layer's expert arrays (they start at expert ep_wbase)
+      int e = sc.slot_expert[sc.pair_slot[d.pair]] - (kEp ? p.ep_wbase : 0);
+      if (!IDX_OK(p, (unsigned)d.pair < (unsigned)kMaxSlots && (unsigned)e < (unsigned)(p.ep_e1 - (kEp ? p.ep_wbase : 0)))) e = 0;
       x.tw0 = &p.tmaps[kFp8 ? TM_Q_WG : TM_T_WG];
       x.tw1 = &p.tmaps[kFp8 ? TM_Q_WU : TM_T_WU];
       x.y0 = x.y1 = e * p.I + d.tile * kTcRows;
@@ -2141,8 +2154,10 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
       // the expert's slot rows of h are contiguous: they are the MMA columns
       int i = sc.pair_slot[d.pair];
       if (!IDX_OK(p, (unsigned)i < (unsigned)kMaxE)) i = 0;
-      int e = sc.slot_expert[i];
-      if (!IDX_OK(p, (unsigned)e < (unsigned)p.E && (unsigned)sc.slot_base[i] < (unsigned)kMaxSlots)) e = 0;
+      int e = sc.slot_expert[i] - (kEp ? p.ep_wbase : 0);  // index in this layer's expert arrays
+      if (!IDX_OK(p, (unsigned)e < (unsigned)(p.ep_e1 - (kEp ? p.ep_wbase : 0)) &&
+                         (unsigned)sc.slot_base[i] < (unsigned)kMaxSlots))
+        e = 0;
       x.tw0 = x.tw1 = &p.tmaps[kFp8 ? TM_Q_WD : TM_T_WD];
       x.fp8 = kFp8;
       if (kFp8) {  // down blocks [e][row block 2 tile, 2 tile + 1][K block]
@@ -2166,7 +2181,7 @@ __device__ __forceinline__ void make_seg_tc(const Params& p, const Shape& sh, co
 // tiles and the activation operand (N rows, boxes of 16), all 128-byte swizzled.
 // last: the launch's last layer (then the stop header and the drain follow); false is
 // returned on abort (after the same stop header and drain).
-template <bool kTrace, bool kFp8 = false>
+template <bool kTrace, bool kFp8 = false, bool kEp = false>
 __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
   const Params& p = pr.p;
   Smem& sm = pr.sm;
@@ -2221,7 +2236,7 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
     }
     if ((p.flags & kFlagJitter) && lane == 0) __nanosleep(hash32(blockIdx.x * 7919u + (uint32_t)u) % 3000u);
     TcSeg x;
-    make_seg_tc<kFp8>(p, sh, sm.sc, d, x);
+    make_seg_tc<kFp8, kEp>(p, sh, sm.sc, d, x);
     const bool xf = kFp8 && x.fp8;  // an FP8 stage (compiled out of the bf16 kernel)
     c_setup += (unsigned long long)(tclock<kTrace>() - tu0);
     // bytes of a stage: on full the activations and (bf16) the weight tiles; on wfull the
@@ -2811,7 +2826,10 @@ __device__ void fixup_tc(const Params& p, const Smem& sm, const UnitDesc& d, int
 // the shared one: y = bf16(x + s + sum_j w_j d_j), the shared part first, then the
 // row's choices in top-k order. Down partial rows: the shared expert's token row b at
 // b, expert slot row r at B + r. 64 threads cover a row's 256 features four at a
-// time (128-bit loads), two rows per pass.
+// time (128-bit loads), two rows per pass. A step over an expert range (y_part set)
+// sums the row's choices among its experts (slot_of >= 0) and writes the fp32 partial,
+// with x + s only when ep_rs.
+template <bool kEp>
 __device__ void combine_rows_tc(const Params& p, const Smem& sm, int t, const int16_t* rows, int n, int et) {
   const Shape& sh = sm.sh;
   const Sched& sc = sm.sc;
@@ -2823,19 +2841,20 @@ __device__ void combine_rows_tc(const Params& p, const Smem& sm, int t, const in
     const int16_t* so = &sc.slot_of[b * sh.k];
 #ifdef MOE_BOUNDS_CHECK
     bool bad = false;
-    for (int j = 0; j < sh.k; ++j) bad = bad || (unsigned)so[j] >= (unsigned)sc.S;
+    for (int j = 0; j < sh.k; ++j) bad = bad || ((!kEp || so[j] >= 0) && (unsigned)so[j] >= (unsigned)sc.S);
     if (!IDX_OK(p, !bad)) continue;
 #endif
-    float4 acc = __ldcg(reinterpret_cast<const float4*>(p.dpart + (size_t)b * p.H + h));
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (!kEp || p.ep_rs) acc = __ldcg(reinterpret_cast<const float4*>(p.dpart + (size_t)b * p.H + h));
     for (int j0 = 0; j0 < sh.k; j0 += 8) {
       float4 v[8];
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj)
-        if (j0 + jj < sh.k)
+        if (j0 + jj < sh.k && (!kEp || so[j0 + jj] >= 0))
           v[jj] = __ldcg(reinterpret_cast<const float4*>(p.dpart + (size_t)(sh.B + so[j0 + jj]) * p.H + h));
 #pragma unroll
       for (int jj = 0; jj < 8; ++jj) {
-        if (j0 + jj < sh.k) {
+        if (j0 + jj < sh.k && (!kEp || so[j0 + jj] >= 0)) {
           const float w = sc.w_of[so[j0 + jj]];
           acc.x = fmaf(w, v[jj].x, acc.x);
           acc.y = fmaf(w, v[jj].y, acc.y);
@@ -2843,6 +2862,17 @@ __device__ void combine_rows_tc(const Params& p, const Smem& sm, int t, const in
           acc.w = fmaf(w, v[jj].w, acc.w);
         }
       }
+    }
+    if (kEp && p.y_part) {  // the fp32 partial of a step over an expert range
+      if (p.ep_rs) {
+        const uint2 xv = __ldcg(reinterpret_cast<const uint2*>(p.x + (size_t)b * p.H + h));
+        acc.x += bf2f(xv.x & 0xFFFFu);
+        acc.y += bf2f(xv.x >> 16);
+        acc.z += bf2f(xv.y & 0xFFFFu);
+        acc.w += bf2f(xv.y >> 16);
+      }
+      *reinterpret_cast<float4*>(p.y_part + (size_t)b * p.H + h) = acc;
+      continue;
     }
     const uint2 xv = __ldcg(reinterpret_cast<const uint2*>(p.x + (size_t)b * p.H + h));
     uint2 yv;
@@ -2852,9 +2882,15 @@ __device__ void combine_rows_tc(const Params& p, const Smem& sm, int t, const in
   }
 }
 
+// The bf16 output of an expert-parallel step once the ranks' fp32 partials are summed.
+__global__ void partial_to_bf16_kernel(const float* __restrict__ in, uint16_t* __restrict__ out, long long n) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) out[i] = f2bf(in[i]);
+}
+
 // F: the layers of a fused launch (a unit's header names its layer), or nullptr when
 // the launch runs the one layer p0.
-template <bool kTrace, bool kFp8 = false>
+template <bool kTrace, bool kFp8 = false, bool kEp = false>
 __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, const FusedParams* F = nullptr) {
   const Shape& sh = sm.sh;
   const int quad = warp_id & 3;
@@ -2997,15 +3033,28 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
       __threadfence();
       if (!epi_sync(sm, ephase, p, lane)) break;
       const bool shared = d.type == UT_DOWN_SHARED;
+      const bool ranged = kEp && (p.ep_e0 > 0 || p.ep_e1 < p.E);  // a step over an expert range
+      if (ranged && shared && sched_layer < layer) {
+        // its rows' contribution counts come from the schedule, which a shared-expert
+        // tile can precede (this CTA's router units, queued earlier, are done)
+        if (!warp_wait(&sm.sched_bar, (uint32_t)(layer & 1), p, lane)) break;
+        sched_layer = layer;
+      }
       const int i = shared ? 0 : sc.pair_slot[d.pair];
       const int cnt = shared ? sh.B : sc.slot_cnt[i];
       if (et < cnt &&
           IDX_OK(p, shared || ((unsigned)(sc.slot_base[i] + et) < (unsigned)kMaxSlots &&
                                sc.row_of[sc.slot_base[i] + et] < sh.B))) {
         const int b = shared ? et : sc.row_of[sc.slot_base[i] + et];
+        // the row's contributions: the shared expert and its choices among this step's experts
+        int kloc = sh.k;
+        if (ranged) {
+          kloc = 0;
+          for (int j = 0; j < sh.k; ++j) kloc += sc.slot_of[b * sh.k + j] >= 0 ? 1 : 0;
+        }
         uint32_t* tix = &p.row_tix[d.tile * sh.B + b];
         const uint32_t old = atom_add_acq_rel(tix, 1u);
-        if (old == (uint32_t)sh.k) {
+        if (old == (uint32_t)kloc) {
           st_relaxed_gpu(tix, 0u);
           const int slot = atomicAdd(&sm.ncomb, 1);
           if (IDX_OK(p, slot < kTcMaxN)) sm.comb_rows[slot] = (int16_t)b;
@@ -3019,7 +3068,7 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
           if (!warp_wait(&sm.sched_bar, (uint32_t)(layer & 1), p, lane)) break;
           sched_layer = layer;
         }
-        combine_rows_tc(p, sm, d.tile, sm.comb_rows, ncomb, et);
+        combine_rows_tc<kEp>(p, sm, d.tile, sm.comb_rows, ncomb, et);
         if (p.rows_out) __threadfence();  // the rows' outputs, then their completion counts
         if (!epi_sync(sm, ephase, p, lane)) break;
         if (p.rows_out && et < ncomb) red_release_add(&p.rows_out[sm.comb_rows[et]], 1u);
@@ -3054,7 +3103,7 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
 
 // ---- the kernel ----------------------------------------------------------------------------------
 
-template <bool kTrace, bool kTC, bool kFp8 = false>
+template <bool kTrace, bool kTC, bool kFp8 = false, bool kEp = false>
 __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
     moe_decode_layer_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -3118,7 +3167,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
 
   if (warp_id == 0) {
     Producer pr(p, sm, lane, sm.sh.nst);
-    if constexpr (kTC) producer_tc<kTrace, kFp8>(pr, ring);
+    if constexpr (kTC) producer_tc<kTrace, kFp8, kEp>(pr, ring);
     else producer_cc<kTrace>(pr, ring);
   } else if (warp_id <= kMacWarps) {
     if constexpr (kTC) {
@@ -3139,10 +3188,10 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
           if (lane == 0) sm.bcast = r;
         }
         ok = mac_sync(sm, mphase, p, lane) && sm.bcast;
-        if (ok) ok = build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, true);
+        if (ok) ok = build_schedule_tc<kTrace, kEp>(p, sm, mw, lane, mphase, true);
       }
-      if (ok) ok = p.B == 1 ? build_schedule_b1<kTrace>(p, sm, mw, lane, mphase, tag)
-                            : build_schedule_tc<kTrace>(p, sm, mw, lane, mphase, false);
+      if (ok) ok = p.B == 1 ? build_schedule_b1<kTrace, kEp>(p, sm, mw, lane, mphase, tag)
+                            : build_schedule_tc<kTrace, kEp>(p, sm, mw, lane, mphase, false);
       if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
       if constexpr (kFp8) convert_fp8_stages<kTrace>(p, sm, ring, mw, lane, ok);
     } else {
@@ -3153,7 +3202,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
   } else if (warp_id == kTcMmaWarp) {
     mma_warp<kTrace, kFp8>(p, sm, ring, lane);
   } else {
-    epilogue_tc<kTrace, kFp8>(p, sm, warp_id, lane);
+    epilogue_tc<kTrace, kFp8, kEp>(p, sm, warp_id, lane);
   }
 
   if constexpr (kTC) tc_fence_before();
@@ -3327,6 +3376,17 @@ size_t tc_smem_bytes() { return kTcRingBytes + sizeof(Smem) + 1024; }
 int tc_threads_per_cta() { return kTcThreads; }
 const void* tc_kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false, true>); }
 const void* tc_kernel_fn_trace() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true, true>); }
+int launch_partial_to_bf16(const float* in, uint16_t* out, long long n, int sms, cudaStream_t stream) {
+  long long blocks = (n + 255) / 256;
+  if (blocks > 4LL * sms) blocks = 4LL * sms;
+  if (blocks < 1) blocks = 1;
+  partial_to_bf16_kernel<<<(unsigned)blocks, 256, 0, stream>>>(in, out, n);
+  return (int)cudaGetLastError();
+}
+const void* tc_ep_kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false, true, false, true>); }
+const void* tc_ep_kernel_fn_trace() {
+  return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true, true, false, true>);
+}
 const void* tc_fp8_kernel_fn() { return reinterpret_cast<const void*>(&moe_decode_layer_kernel<false, true, true>); }
 const void* tc_fp8_kernel_fn_trace() {
   return reinterpret_cast<const void*>(&moe_decode_layer_kernel<true, true, true>);

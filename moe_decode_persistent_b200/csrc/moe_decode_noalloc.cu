@@ -215,6 +215,9 @@ extern "C" int moe_decode_step_noalloc(const moe_decode_config* cfg, const moe_d
     uint16_t* io = reinterpret_cast<uint16_t*>(base + kOffIo);
     p.x = l == 0 ? (const uint16_t*)x_in : io;
     p.y = l == L - 1 ? (uint16_t*)y_out : io;
+    p.ep_e0 = 0;  // every expert, whole-layer output
+    p.ep_e1 = E;
+    p.ep_rs = 1;
     const moe_decode_layer_weights& w = layers[l];
     p.tmaps = d_maps + l * kNaMapsPerLayer;
     p.gamma = (const uint16_t*)w.gamma;

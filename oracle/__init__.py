@@ -81,6 +81,9 @@ def _load(path):
         lib.oracle_layer_selected.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Weights), i, vp,
                                               vp, vp, vp, vp, vp, vp]
         lib.oracle_layer_selected.restype = i
+        lib.oracle_layer_partial.argtypes = [ctypes.POINTER(_Dims), ctypes.POINTER(_Weights), i, vp, vp, i, i, i,
+                                             vp]
+        lib.oracle_layer_partial.restype = i
         lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
         lib.oracle_e4m3_to_double.restype = d
         lib.oracle_dequant_e4m3.argtypes = [i, i, vp, vp, vp]
@@ -218,6 +221,46 @@ def layer(dims: dict, weights: dict, x_bits: np.ndarray, selection=None) -> dict
     if selection is not None:
         sel = _c(selection, np.int32).reshape(B, k)
     keep = []  # keep arrays alive across the call
+    d, w = _structs(dims, weights, keep)
+    logits = np.empty((B, E), dtype=np.float64)
+    idx = np.empty((B, k), dtype=np.int32)
+    wts = np.empty((B, k), dtype=np.float64)
+    y_pre = np.empty((B, H), dtype=np.float64)
+    y = np.empty((B, H), dtype=np.uint16)
+    if sel is None:
+        rc = _L().oracle_layer(ctypes.byref(d), ctypes.byref(w), B, _p(x), _p(logits), _p(idx),
+                               _p(wts), _p(y_pre), _p(y))
+    else:
+        rc = _L().oracle_layer_selected(ctypes.byref(d), ctypes.byref(w), B, _p(x), _p(sel), _p(logits),
+                                        _p(idx), _p(wts), _p(y_pre), _p(y))
+    if rc != OK:
+        raise RuntimeError(f"oracle_layer failed: {rc}")
+    return {"logits": logits, "idx": idx, "w": wts, "y_pre": y_pre, "y": y}
+
+
+def layer_partial(dims: dict, weights: dict, x_bits: np.ndarray, e0: int, e1: int, with_rs: bool,
+                  selection=None) -> np.ndarray:
+    """The part of the layer's output (fp64 [B, H], unrounded) that experts e0 <= e < e1
+    contribute, plus x + s when with_rs (oracle_layer_partial). Summed over a partition
+    of the experts with with_rs set for one part, it is layer(...)["y_pre"]. weights as
+    for layer; only the experts in the range need be present. selection: as for layer."""
+    H, k = dims["H"], dims["k"]
+    x = _c(x_bits, np.uint16).reshape(-1, H)
+    B = x.shape[0]
+    sel = None if selection is None else _c(selection, np.int32).reshape(B, k)
+    keep = []
+    d, w = _structs(dims, weights, keep)
+    out = np.empty((B, H), dtype=np.float64)
+    rc = _L().oracle_layer_partial(ctypes.byref(d), ctypes.byref(w), B, _p(x), None if sel is None else _p(sel),
+                                   int(e0), int(e1), 1 if with_rs else 0, _p(out))
+    if rc != OK:
+        raise RuntimeError(f"oracle_layer_partial failed: {rc}")
+    return out
+
+
+def _structs(dims: dict, weights: dict, keep: list):
+    """The C structs of dims and weights (arrays kept alive in keep)."""
+    E = dims["E"]
 
     def arr(a, dt):
         a2 = _c(a, dt)
@@ -241,21 +284,9 @@ def layer(dims: dict, weights: dict, x_bits: np.ndarray, selection=None) -> dict
         ws_gate=arr(weights["ws_gate"], np.uint16).ctypes.data,
         ws_up=arr(weights["ws_up"], np.uint16).ctypes.data,
         ws_down=arr(weights["ws_down"], np.uint16).ctypes.data)
-    d = _Dims(H=H, E=E, k=k, I=dims["I"], Is=dims["Is"], eps=float(dims["eps"]))
-    logits = np.empty((B, E), dtype=np.float64)
-    idx = np.empty((B, k), dtype=np.int32)
-    wts = np.empty((B, k), dtype=np.float64)
-    y_pre = np.empty((B, H), dtype=np.float64)
-    y = np.empty((B, H), dtype=np.uint16)
-    if sel is None:
-        rc = _L().oracle_layer(ctypes.byref(d), ctypes.byref(w), B, _p(x), _p(logits), _p(idx),
-                               _p(wts), _p(y_pre), _p(y))
-    else:
-        rc = _L().oracle_layer_selected(ctypes.byref(d), ctypes.byref(w), B, _p(x), _p(sel), _p(logits),
-                                        _p(idx), _p(wts), _p(y_pre), _p(y))
-    if rc != OK:
-        raise RuntimeError(f"oracle_layer failed: {rc}")
-    return {"logits": logits, "idx": idx, "w": wts, "y_pre": y_pre, "y": y}
+    keep.append((gp, up, dp))
+    d = _Dims(H=dims["H"], E=E, k=dims["k"], I=dims["I"], Is=dims["Is"], eps=float(dims["eps"]))
+    return d, w
 
 
 def workload_layer(wl, layer_index: int, x_bits: np.ndarray, shared=None, w_router=None,

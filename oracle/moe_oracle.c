@@ -208,18 +208,21 @@ int oracle_dequant_e4m3(int rows, int cols, const uint8_t* codes, const float* s
 
 /* The output of one row once its selection and weights are known:
  * y = bf16(x + s + sum_j w[j] E_{S_j}(n)), the shared expert first, then the
- * selected experts in the order given. Scratch: s, ex, acc (H each). */
+ * selected experts in the order given. Restricted to the experts e0 <= e < e1 and,
+ * with_rs == 0, without x + s, it is the part of the row those experts contribute
+ * (a part of an expert-parallel layer). Scratch: s, ex, acc (H each). */
 static int combine_row(const oracle_dims* d, const oracle_weights* w, const uint16_t* xb,
-                       const double* n, const int32_t* ib, const double* wb, double* s, double* ex,
-                       double* acc, double* y_pre, uint16_t* y) {
+                       const double* n, const int32_t* ib, const double* wb, int e0, int e1, int with_rs,
+                       double* s, double* ex, double* acc, double* y_pre, uint16_t* y) {
   const int H = d->H, k = d->k, I = d->I, Is = d->Is;
-  oracle_swiglu(H, Is, n, w->ws_gate, w->ws_up, w->ws_down, s);
+  if (with_rs) oracle_swiglu(H, Is, n, w->ws_gate, w->ws_up, w->ws_down, s);
   for (int h = 0; h < H; ++h) {
     const double res = MUT(ORACLE_MUT_RESIDUAL_N) ? n[h] : bf(xb[h]);
-    acc[h] = res + (MUT(ORACLE_MUT_NO_SHARED) ? 0.0 : s[h]);
+    acc[h] = with_rs ? res + (MUT(ORACLE_MUT_NO_SHARED) ? 0.0 : s[h]) : 0.0;
   }
   for (int j = 0; j < k; ++j) {
     const int e = ib[j];
+    if (e < e0 || e >= e1) continue;
     if (!w->w_gate[e] || !w->w_up[e] || !w->w_down[e]) return ORACLE_EMISSING;
     oracle_swiglu(H, I, n, w->w_gate[e], w->w_up[e], w->w_down[e], ex);
     for (int h = 0; h < H; ++h) acc[h] += wb[j] * ex[h];
@@ -235,8 +238,8 @@ static int combine_row(const oracle_dims* d, const oracle_weights* w, const uint
  * of its logits. Otherwise sel [B][k] gives each row's selection (k distinct
  * experts); the weights are then the softmax of the row's own logits over it. */
 static int layer_rows(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
-                      const int32_t* sel, double* logits, int32_t* topk_idx, double* topk_w,
-                      double* y_pre, uint16_t* y) {
+                      const int32_t* sel, int e0, int e1, int with_rs, double* logits, int32_t* topk_idx,
+                      double* topk_w, double* y_pre, uint16_t* y) {
   const int H = d->H, E = d->E, k = d->k, I = d->I, Is = d->Is;
   if (B < 0 || H < 1 || E < 1 || k < 1 || k > E || I < 1 || Is < 1) return ORACLE_EINVAL;
   if (sel) {
@@ -271,7 +274,7 @@ static int layer_rows(const oracle_dims* d, const oracle_weights* w, int B, cons
       break;
     }
     oracle_softmax_selected(k, lb, ib, wb);
-    rc = combine_row(d, w, xb, n, ib, wb, s, ex, acc, y_pre ? y_pre + (size_t)b * H : NULL,
+    rc = combine_row(d, w, xb, n, ib, wb, e0, e1, with_rs, s, ex, acc, y_pre ? y_pre + (size_t)b * H : NULL,
                      y ? y + (size_t)b * H : NULL);
   }
   free(n);
@@ -283,12 +286,25 @@ static int layer_rows(const oracle_dims* d, const oracle_weights* w, int B, cons
 
 int oracle_layer(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
                  double* logits, int32_t* topk_idx, double* topk_w, double* y_pre, uint16_t* y) {
-  return layer_rows(d, w, B, x, NULL, logits, topk_idx, topk_w, y_pre, y);
+  return layer_rows(d, w, B, x, NULL, 0, d->E, 1, logits, topk_idx, topk_w, y_pre, y);
 }
 
 int oracle_layer_selected(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
                           const int32_t* sel, double* logits, int32_t* topk_idx, double* topk_w,
                           double* y_pre, uint16_t* y) {
   if (!sel) return ORACLE_EINVAL;
-  return layer_rows(d, w, B, x, sel, logits, topk_idx, topk_w, y_pre, y);
+  return layer_rows(d, w, B, x, sel, 0, d->E, 1, logits, topk_idx, topk_w, y_pre, y);
+}
+
+int oracle_layer_partial(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
+                         const int32_t* sel, int e0, int e1, int with_rs, double* y_part) {
+  if (!d || B < 0 || e0 < 0 || e1 < e0 || e1 > d->E || !y_part) return ORACLE_EINVAL;
+  double* logits = (double*)malloc(sizeof(double) * (size_t)(B > 0 ? B : 1) * (size_t)d->E);
+  int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)(B > 0 ? B : 1) * (size_t)d->k);
+  double* wts = (double*)malloc(sizeof(double) * (size_t)(B > 0 ? B : 1) * (size_t)d->k);
+  const int rc = layer_rows(d, w, B, x, sel, e0, e1, with_rs, logits, idx, wts, y_part, NULL);
+  free(logits);
+  free(idx);
+  free(wts);
+  return rc;
 }

@@ -82,4 +82,14 @@ int oracle_layer_selected(const oracle_dims* d, const oracle_weights* w, int B, 
                           const int32_t* sel, double* logits, int32_t* topk_idx, double* topk_w,
                           double* y_pre, uint16_t* y);
 
+/* The part of the layer's output (fp64, before the final rounding) that the experts
+ * e0 <= e < e1 contribute: y_part [B][H] = sum over each row's top-k choices j with
+ * e0 <= S_j < e1 of w_j E_{S_j}(n), plus x + s when with_rs -- the split of the layer
+ * over GPUs that each own a range of the experts (page post.smzdm.com/p/a6zppe4g,
+ * section "改了什么：每层 23 个 kernel 砍到 13 个", item "把通信缝进计算"). Only the
+ * experts in the range need weights. sel: NULL (each row's own top-k) or [B][k] given
+ * selections as for oracle_layer_selected. */
+int oracle_layer_partial(const oracle_dims* d, const oracle_weights* w, int B, const uint16_t* x,
+                         const int32_t* sel, int e0, int e1, int with_rs, double* y_part);
+
 #endif

@@ -293,9 +293,11 @@ def closed_form_layer(seed, force=None):
     ws = softmax(lg[sel])
     s = swiglu_closed_form(n, spg, sdg, spu, sdu, spd, sdd)
     y = xf + s
+    terms = []
     for j, e in enumerate(sel):
-        y = y + ws[j] * swiglu_closed_form(n, *maps[e])
-    return dims, W, x, dict(logits=lg, idx=np.array(sel), w=ws, y_pre=y)
+        terms.append(ws[j] * swiglu_closed_form(n, *maps[e]))
+        y = y + terms[-1]
+    return dims, W, x, dict(logits=lg, idx=np.array(sel), w=ws, y_pre=y, xs=xf + s, terms=terms)
 
 
 @pytest.mark.parametrize("seed", range(8))
@@ -349,6 +351,42 @@ def test_layer_with_given_selection_is_order_free_and_rejects_bad_sets():
     bad[1, 0] = TINY.E                             # out of range
     with pytest.raises(RuntimeError):
         oracle.layer(dims, W, x, selection=bad)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_layer_partial_closed_form(seed):
+    """The part of the layer an expert range contributes: x + s when with_rs, plus the
+    weighted outputs of the row's choices inside [e0, e1) -- against the closed form, with
+    range ends placed on a selected expert (inclusive start, exclusive end)."""
+    dims, W, x, want = closed_form_layer(seed)
+    E, sel = dims["E"], [int(e) for e in want["idx"]]
+    a = sel[0]
+    cases = [(0, E, True), (0, E, False), (0, a, True), (a, E, False), (a, a + 1, False), (a, a, True),
+             (0, 0, False)]
+    for e0, e1, rs in cases:
+        got = oracle.layer_partial(dims, W, x, e0, e1, rs)[0]
+        ref = want["xs"].copy() if rs else np.zeros(dims["H"])
+        for j, e in enumerate(sel):
+            if e0 <= e < e1:
+                ref = ref + want["terms"][j]
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12, err_msg=f"{(e0, e1, rs)}")
+
+
+def test_layer_partials_over_a_partition_sum_to_the_layer():
+    """Summed over a partition of the experts (residual and shared expert in one part),
+    the parts are the layer's unrounded output; the whole range with them is that output
+    bit for bit. Only each part's experts are given to it."""
+    dims, W = tiny_random_layer(TINY)
+    x = TINY.x_host()
+    full = oracle.layer(dims, W, x)["y_pre"]
+    whole = oracle.layer_partial(dims, W, x, 0, TINY.E, True)
+    assert np.array_equal(whole, full)
+    for cuts in ([0, 5, 16], [0, 1, 2, 9, 16], [0, 16]):
+        total = np.zeros_like(full)
+        for r, (e0, e1) in enumerate(zip(cuts[:-1], cuts[1:])):
+            Wr = dict(W, experts={e: W["experts"][e] for e in range(e0, e1)})
+            total += oracle.layer_partial(dims, Wr, x, e0, e1, r == 1 % (len(cuts) - 1))
+        np.testing.assert_allclose(total, full, rtol=1e-12, atol=1e-12)
 
 
 def test_layer_missing_expert_is_an_error():
