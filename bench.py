@@ -74,6 +74,9 @@ def parse_args(argv=None):
     ap.add_argument("--profile-small-b64", action="store_true",
                     help="batch 64 with the Zipf router, 128 experts of intermediate 512 (~2.9 GB of "
                          "weights): the small hot-expert case for full ncu captures of the tensor-core kernel")
+    ap.add_argument("--profile-small-fp8", action="store_true",
+                    help="batch 1, 128 FP8 experts of intermediate 512 (~1.5 GB of weights): the small case "
+                         "for full ncu captures of the FP8 tensor-core kernel")
     return ap.parse_args(argv)
 
 
@@ -615,6 +618,9 @@ def main(argv=None):
     if args.profile_small_b64:
         wl = synth.Workload("b64_h7168_e128_i512_k16_zipf_profile", B=64, H=7168, E=128, k=16, I=512, Is=1024,
                             seed=3, router="zipf")
+    if args.profile_small_fp8:
+        wl = synth.Workload("b1_h7168_e128_i512_k16_fp8_profile", B=1, H=7168, E=128, k=16, I=512, Is=1024,
+                            seed=1, experts="fp8")
     if args.impl == "reference":
         run_reference(args, wl)
     else:
