@@ -99,8 +99,12 @@ __host__ __device__ constexpr int tc_slot_bytes(int na) { return 2 * kTcTileByte
 // A layer with FP8 experts: an FP8 stage holds one 128-column K block, so its slot takes
 // the activations of two K atoms (the second at +na x 128 bytes).
 __host__ __device__ constexpr int tc_slot_bytes_fp8(int na) { return 2 * kTcTileBytes + 2 * na * kTcAtomK * 2; }
+__host__ __device__ constexpr int tc_stages_in(int ring_bytes, int slot_bytes, int batch) {
+  return batch <= 4 && ring_bytes / slot_bytes >= 4 ? 4
+       : ring_bytes / slot_bytes < kTcStagesMax ? ring_bytes / slot_bytes : kTcStagesMax;
+}
 __host__ __device__ constexpr int tc_stages_of(int slot_bytes, int batch) {
-  return batch <= 4 ? 4 : kTcRingBytes / slot_bytes < kTcStagesMax ? kTcRingBytes / slot_bytes : kTcStagesMax;
+  return tc_stages_in(kTcRingBytes, slot_bytes, batch);
 }
 __host__ __device__ constexpr int tc_stages(int na, int batch) { return tc_stages_of(tc_slot_bytes(na), batch); }
 static_assert(tc_stages(16, 1) == 4 && tc_stages(16, 8) == 5 && tc_stages(32, 32) == 5 && tc_stages(64, 64) == 4,
@@ -116,13 +120,19 @@ constexpr int kFp8AccBufs = 2;
 constexpr int kFp8AStages = 2;
 constexpr int kFp8ACol0 = kFp8AccBufs * kTcAccCols;
 constexpr int kFp8AStageCols = 2 * kTcAtomK;
+// The activations of each A stage (two K atoms of na rows, as they lay in the slot) sit in
+// front of an FP8 layer's ring, so a slot is free once its codes are converted.
+__host__ __device__ constexpr int fp8_act_stage_bytes(int na) { return 2 * na * kTcAtomK * 2; }
+__host__ __device__ constexpr int fp8_actbuf_bytes(int na) { return kFp8AStages * fp8_act_stage_bytes(na); }
 static_assert(kFp8ACol0 + kFp8AStages * kFp8AStageCols <= kTmemCols, "FP8 tensor-memory plan");
 
 static_assert(kTcSlotBytes % 1024 == 0 && kTcTileBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kCcRingBytes % 1024 == 0 && kTcRingBytes % 1024 == 0, "ring keeps the state block aligned");
 
 enum UnitType { UT_ROUTER = 0, UT_SHARED = 1, UT_EXPERT = 2, UT_DOWN_SHARED = 3, UT_DOWN_EXPERT = 4 };
-enum HeaderKind { HK_STAGE = 0, HK_SCHED = 1, HK_END = 2 };
+// HK_SWITCH (FP8 layers): the CTA's FP8 stages begin; the MMA warp takes them from the
+// tensor-memory A stages from now on, and the ring slots are released by the converters.
+enum HeaderKind { HK_STAGE = 0, HK_SCHED = 1, HK_END = 2, HK_SWITCH = 3 };
 
 // Written by the producer for every ring slot; everything a MAC warp needs for the
 // stage, so the MAC warps never decode units.
@@ -149,7 +159,6 @@ constexpr int kTcInfoFirst = 1 << 5, kTcInfoLast = 1 << 6;
 // stage: I / 128 further), and info bit 8 marks a down stage.
 constexpr int kTcInfoFp8 = 1 << 7, kTcInfoFp8Down = 1 << 8;
 constexpr int kFp8TileBytes = kTcRows * 2 * kTcAtomK;  // 16 KB: 128 rows x 128 codes
-__device__ __forceinline__ int fp8_act1_off(int na) { return 2 * kTcTileBytes + na * kTcAtomK * 2; }
 constexpr int kCq = 8;                            // entries of the converter queue
 
 // Layout constants of one step (identical in every CTA).
@@ -205,8 +214,11 @@ struct Smem {
   uint64_t cq_full[kCq];           // converter queue: FP8 stages issued (producer -> routing warps)
   uint64_t cq_empty[kCq];
   uint64_t wfull[kTcStagesMax];    // FP8 stage: codes and scales of the slot landed
+  uint64_t cdone[kTcStagesMax];    // FP8 stage: the converters are done with the slot (codes, activations)
   int16_t cq_slot[kCq];            // ring slot of the queued stage (-1: no more stages)
   uint8_t cq_par[kCq];             // the slot's wfull parity for that stage
+  uint8_t cq_fpar[kCq];            // the slot's full parity (its activations) for that stage
+  StageHeader ahdr[kFp8AStages];   // FP8: the header of the stage in each tensor-memory A stage
   StageHeader hdr[kMaxRingStages];
   int rb_unit[kRB];         // unit id of the buffer, or -1 (stop)
   int acc_unit[kTcAccBufs]; // unit id of the accumulator buffer, or -1 (stop)
@@ -509,7 +521,8 @@ __device__ void make_shape_tc(const Params& p, Shape& s) {
   s.NA = (p.B + kTcActRows - 1) / kTcActRows * kTcActRows;
   s.kblk = p.fp8 ? 1 : 0;
   s.slot_bytes = p.fp8 ? tc_slot_bytes_fp8(s.NA) : tc_slot_bytes(s.NA);
-  s.nst = tc_stages_of(s.slot_bytes, p.B);
+  s.nst = p.fp8 ? tc_stages_in(kTcRingBytes - fp8_actbuf_bytes(s.NA), s.slot_bytes, p.B)
+                : tc_stages_of(s.slot_bytes, p.B);
   s.boxH = s.boxI = s.boxIs = kTcAtomK;
   s.nkbH = p.H / kTcAtomK;
   s.nkbI = p.I / kTcAtomK;
@@ -1809,27 +1822,31 @@ struct Producer {
   int cq_pos;        // converter queue: next entry and its phase
   uint32_t cq_phase;
   uint32_t wpar, wpend;  // FP8: per slot the parity of its next wfull phase; slots used
+  uint32_t fp8prev, cdpar;  // FP8: slots whose last stage was FP8 (released on cdone); cdone parities
+  bool switched;            // FP8: HK_SWITCH issued (the MMA warp reads the A stages)
 
   __device__ Producer(const Params& p_, Smem& sm_, int lane_, int nst_)
       : p(p_), sm(sm_), lane(lane_), nst(nst_), slot(0), phase(0u), pend_mask(0u), pend_parity(0u), cq_pos(0),
-        cq_phase(0u), wpar(0u), wpend(0u) {}
+        cq_phase(0u), wpar(0u), wpend(0u), fp8prev(0u), cdpar(0u), switched(false) {}
 
   // An FP8 stage in the current slot: the parity of the wfull phase its codes complete.
   __device__ uint32_t mark_fp8() {
     const uint32_t par = (wpar >> slot) & 1u;
     wpar ^= 1u << slot;
     wpend |= 1u << slot;
+    fp8prev |= 1u << slot;
     return par;
   }
   __device__ uint32_t last_wpar() const { return ((wpar >> slot) & 1u) ^ 1u; }
 
-  // Hands the FP8 stage in ring slot `s` (full-barrier parity `par`) to the converters;
-  // s = -1 tells them that no more stages follow.
-  __device__ bool push_conv(int s, uint32_t par) {
+  // Hands the FP8 stage in ring slot `s` (wfull parity `par`, full parity `fpar`) to the
+  // converters; s = -1 tells them that no more stages follow.
+  __device__ bool push_conv(int s, uint32_t par, uint32_t fpar = 0u) {
     if (!wait_bar(&sm.cq_empty[cq_pos], cq_phase ^ 1u)) return false;
     if (lane == 0) {
       sm.cq_slot[cq_pos] = (int16_t)s;
       sm.cq_par[cq_pos] = (uint8_t)par;
+      sm.cq_fpar[cq_pos] = (uint8_t)fpar;
       mbar_arrive(&sm.cq_full[cq_pos]);
     }
     __syncwarp();
@@ -1862,10 +1879,31 @@ struct Producer {
     __syncwarp();
     return r != 0;
   }
-  // Waits for a free slot; the slot's previous stage has then been consumed.
+  // Waits for a free slot; the slot's previous stage has then been consumed (an FP8
+  // stage's by the converters, any other by the MMAs).
   __device__ bool wait_slot() {
-    const bool ok = wait_bar(&sm.empty[slot], phase ^ 1u);
-    return ok;
+    if ((fp8prev >> slot) & 1u) {
+      const uint32_t par = (cdpar >> slot) & 1u;
+      cdpar ^= 1u << slot;
+      fp8prev &= ~(1u << slot);
+      return wait_bar(&sm.cdone[slot], par);
+    }
+    return wait_bar(&sm.empty[slot], phase ^ 1u);
+  }
+  // FP8: the MMA warp is told, through the ring, that the A stages carry the rest.
+  __device__ bool emit_switch() {
+    if (!wait_slot()) return false;
+    // the slot's previous stage has been consumed, so its copies have landed; this use
+    // completes a full phase of its own (the drain must not wait for the earlier one)
+    pend_mask &= ~(1u << slot);
+    if (lane == 0) {
+      sm.hdr[slot].kind = HK_SWITCH;
+      mbar_arrive(&sm.full[slot]);
+    }
+    __syncwarp();
+    advance();
+    switched = true;
+    return true;
   }
   __device__ bool wait_dep(const uint32_t* c, uint32_t target) {
     int r = 1;
@@ -1904,8 +1942,10 @@ struct Producer {
   // After the last stage: the stop header and the drain of every bulk copy still in
   // flight.
   __device__ void finish(bool fp8 = false) {
-    if (fp8) push_conv(-1, 0u);  // the converters stop (bounded: they also stop on abort)
-    if (wait_slot()) {
+    // the converters stop (bounded: they also stop on abort); after HK_SWITCH they pass
+    // the end on to the MMA warp, otherwise it comes through the ring
+    if (fp8) push_conv(-1, 0u);
+    if (!switched && wait_slot()) {
       pend_mask &= ~(1u << slot);
       if (lane == 0) {
         sm.hdr[slot].kind = HK_END;
@@ -2238,6 +2278,10 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
     TcSeg x;
     make_seg_tc<kFp8, kEp>(p, sh, sm.sc, d, x);
     const bool xf = kFp8 && x.fp8;  // an FP8 stage (compiled out of the bf16 kernel)
+    if (xf && !pr.switched && !pr.emit_switch()) {
+      ok = false;
+      break;
+    }
     c_setup += (unsigned long long)(tclock<kTrace>() - tu0);
     // bytes of a stage: on full the activations and (bf16) the weight tiles; on wfull the
     // codes and scales of an FP8 stage
@@ -2310,7 +2354,7 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
         if (!ok) break;
         issue_weights(ka);
         __syncwarp();
-        if (xf && !pr.push_conv(pr.slot, pr.last_wpar())) ok = false;
+        if (xf && !pr.push_conv(pr.slot, pr.last_wpar(), pr.phase)) ok = false;
         pr.advance();
         ++c_stages;
       }
@@ -2345,7 +2389,7 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
       issue_weights(ka);
       issue_act(ka, slot);
       __syncwarp();
-      if (xf && !pr.push_conv(pr.slot, pr.last_wpar())) ok = false;
+      if (xf && !pr.push_conv(pr.slot, pr.last_wpar(), pr.phase)) ok = false;
       pr.advance();
       c_issue += (unsigned long long)(tclock<kTrace>() - ti0);
       ++c_stages;
@@ -2546,11 +2590,15 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
 // bf16 values as 64 columns of its lane. The codes sit 128-byte swizzled (chunk c of row
 // r at chunk c ^ (r mod 8)), so the 8 lanes of a shared-memory phase read 8 distinct
 // 16-byte chunks while the whole warp reads one logical chunk. A stages rotate in stage
-// order; one is rewritten only after the MMAs that read it completed. The warps need
-// nothing from one another: each waits for the stage itself (bounded) and signals its
-// part converted to the MMA warp.
+// order; one is rewritten only after the MMAs that read it completed. With its A stage a
+// stage's activations (two K atoms) are copied in front of the ring and its header into
+// Smem::ahdr, so the slot is released (cdone) once converted, before the MMAs run. The
+// warps need nothing from one another: each waits for the stage itself (bounded) and
+// signals its part done on the slot's cdone and the A stage's conv_bar; the end of the
+// stages reaches the MMA warp the same way (an HK_END header in the next A stage).
 template <bool kTrace>
-__device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, int mw, int lane, bool ok) {
+__device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, uint8_t* actring, int mw, int lane,
+                                   bool ok) {
   if (!ok) return;
   unsigned long long c_wait = 0, c_work = 0;
   struct Flush {  // the warp's cycle counts into the trace (warp 0) on every way out
@@ -2576,14 +2624,20 @@ __device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, int
     const long long t0 = tclock<kTrace>();
     if (!warp_wait(&sm.cq_full[q], qph, p, lane, 64)) return;
     const int slot = sm.cq_slot[q];
-    const uint32_t par = sm.cq_par[q];
+    const uint32_t par = sm.cq_par[q], fpar = sm.cq_fpar[q];
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.cq_empty[q]);  // the entry is read
     if (++q == kCq) {
       q = 0;
       qph ^= 1u;
     }
-    if (slot < 0) return;
+    if (slot < 0) {  // the end, in the next A stage once the MMAs left it
+      if (!warp_wait(&astage_empty(sm)[as], asph ^ 1u, p, lane, 64)) return;
+      if (mw == 0 && lane == 0) sm.ahdr[as].kind = HK_END;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.conv_bar[as]);
+      return;
+    }
     if (!IDX_OK(p, slot < sh.nst)) return;
     // the header was written before the queue entry: the tile's scale loads while the
     // codes are still in flight
@@ -2596,9 +2650,21 @@ __device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, int
       sv = __ldg(sa + hd.wrow + (down && j ? p.I / kTcRows : 0));
     }
     if (!warp_wait(&sm.wfull[slot], par, p, lane, 64)) return;
+    if (!warp_wait(&sm.full[slot], fpar, p, lane, 64)) return;                // its activations
     if (!warp_wait(&astage_empty(sm)[as], asph ^ 1u, p, lane, 64)) return;  // the A stage is free
     const long long t1 = tclock<kTrace>();
     c_wait += (unsigned long long)(t1 - t0);
+    {  // the activations of both atoms (n rows each, the second at +NA x 128 bytes), as laid out
+      const int n = ((hd.info >> 2) & 7) * kTcActRows;
+      const uint8_t* src = ring + slot * sh.slot_bytes + 2 * kTcTileBytes;
+      uint8_t* dst = actring + as * fp8_act_stage_bytes(sh.NA);
+      const int chunks = n * (kTcAtomK * 2 / 16);  // 16-byte chunks per atom
+      for (int i = mw * 32 + lane; i < 2 * chunks; i += kMacThreads) {
+        const int a = i >= chunks ? 1 : 0, c = i - a * chunks;
+        const int off = a * sh.NA * kTcAtomK * 2 + c * 16;
+        *reinterpret_cast<uint4*>(dst + off) = *reinterpret_cast<const uint4*>(src + off);
+      }
+    }
     if (conv) {
       tc_fence_after();
       const uint8_t* sbase = ring + slot * sh.slot_bytes;
@@ -2625,9 +2691,14 @@ __device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, int
       }
       tmem_st_wait();
     }
+    if (mw == 0 && lane == 0) sm.ahdr[as] = hd;
+    fence_proxy_async_shared();  // the copied activations, then the tensor cores' reads
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.conv_bar[slot]);
+    if (lane == 0) {
+      mbar_arrive(&sm.cdone[slot]);  // the slot is free
+      mbar_arrive(&sm.conv_bar[as]);
+    }
     if (++as == kFp8AStages) {
       as = 0;
       asph ^= 1u;
@@ -2644,37 +2715,48 @@ __device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, int
 // is handed to the epilogue warps: one commit arrive (the MMAs are complete) plus one
 // plain arrive that publishes the unit id.
 template <bool kTrace, bool kFp8 = false>
-__device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
+__device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane, uint8_t* aring = nullptr) {
   const uint32_t tmem = sm.tmem_base;
   int slot = 0;
   uint32_t phase = 0;
   int abuf = 0;
   uint32_t aphase = 0;
   bool issued = false;
-  uint32_t cpar = 0u;  // per slot: parity of its next FP8 conversion
-  int as = 0;          // FP8: tensor-memory A stage of the next FP8 stage
+  bool amode = false;  // FP8: the stages come from the tensor-memory A stages (after HK_SWITCH)
+  int as = 0;          // FP8: the next A stage and its conv_bar parity
+  uint32_t asph = 0u;
   unsigned long long c_full = 0, c_acc = 0, c_st = 0, c_issue = 0, c_conv = 0;
   const long long tloop0 = tclock<kTrace>();
   for (;;) {
-    {
+    StageHeader hd;
+    if (!amode) {
       const long long t0 = tclock<kTrace>();
       const bool got = warp_wait(&sm.full[slot], phase, p, lane);
       c_full += (unsigned long long)(tclock<kTrace>() - t0);
       if (!got) break;
+      hd = sm.hdr[slot];
+      if (kFp8 && hd.kind == HK_SWITCH) {  // the slot carries no tiles; the A stages follow
+        if (lane == 0) mbar_arrive(&sm.empty[slot]);
+        __syncwarp();
+        if (++slot == sm.sh.nst) {
+          slot = 0;
+          phase ^= 1u;
+        }
+        amode = true;
+        continue;
+      }
+    } else {  // the converters filled A stage `as` (weights in tensor memory, activations beside)
+      const long long t0 = tclock<kTrace>();
+      const bool got = warp_wait(&sm.conv_bar[as], asph, p, lane, 64);
+      c_conv += (unsigned long long)(tclock<kTrace>() - t0);
+      if (!got) break;
+      hd = sm.ahdr[as];
     }
-    const StageHeader hd = sm.hdr[slot];
     if (hd.kind == HK_END) {
       if (lane == 0) trace_stamp<kTrace>(p, TR_MAC_END);
       break;
     }
     const int info = hd.info;
-    if (kFp8 && (info & kTcInfoFp8)) {  // the activations landed; wait for the bf16 weight tiles
-      const long long t0 = tclock<kTrace>();
-      const bool got = warp_wait(&sm.conv_bar[slot], (cpar >> slot) & 1u, p, lane, 64);
-      c_conv += (unsigned long long)(tclock<kTrace>() - t0);
-      if (!got) break;
-      cpar ^= 1u << slot;
-    }
     const bool first = (info & kTcInfoFirst) != 0;
     const bool last = (info & kTcInfoLast) != 0;
     if (first) {
@@ -2686,17 +2768,16 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
     tc_fence_after();
     const long long ti0 = tclock<kTrace>();
     if (lane == 0) {
-      const uint32_t sbase = smem_u32(ring + slot * sm.sh.slot_bytes);
-      const uint64_t dw0 = sw128_desc(sbase);
-      const uint64_t dw1 = sw128_desc(sbase + kTcTileBytes);
-      const uint64_t da = sw128_desc(sbase + 2 * kTcTileBytes);
       const int nbox = info & 3;
       const uint32_t idesc = idesc_bf16_m128((uint32_t)((info >> 2) & 7) * kTcActRows);
       const uint32_t t0 = tmem + (uint32_t)(abuf * kTcAccCols);
-      if (kFp8 && (info & kTcInfoFp8)) {  // A from the tensor-memory stage the converters filled
-        // one 128-column K block: 8 K steps, the activations of the second atom at +NA x 128
+      if (kFp8 && amode) {
+        // one 128-column K block: 8 K steps of A from tensor memory; the activations of the
+        // two atoms beside the A stage, the second at +NA x 128 bytes
         const uint32_t a0 = tmem + (uint32_t)(kFp8ACol0 + as * kFp8AStageCols);
-        const uint64_t da1 = sw128_desc(sbase + (uint32_t)fp8_act1_off(sm.sh.NA));
+        const uint32_t abase = smem_u32(aring + as * fp8_act_stage_bytes(sm.sh.NA));
+        const uint64_t da = sw128_desc(abase);
+        const uint64_t da1 = sw128_desc(abase + (uint32_t)(sm.sh.NA * kTcAtomK * 2));
 #pragma unroll
         for (int ks = 0; ks < 2 * kTcAtomK / 16; ++ks) {
           const uint32_t accum = (first && ks == 0) ? 0u : 1u;
@@ -2706,14 +2787,18 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
         }
         tc_commit(&astage_empty(sm)[as]);
       } else {
+        const uint32_t sbase = smem_u32(ring + slot * sm.sh.slot_bytes);
+        const uint64_t dw0 = sw128_desc(sbase);
+        const uint64_t dw1 = sw128_desc(sbase + kTcTileBytes);
+        const uint64_t da = sw128_desc(sbase + 2 * kTcTileBytes);
 #pragma unroll
         for (int ks = 0; ks < kTcAtomK / 16; ++ks) {
           const uint32_t accum = (first && ks == 0) ? 0u : 1u;
           tc_mma_bf16(t0, dw0 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
           if (nbox == 2) tc_mma_bf16(t0 + 64u, dw1 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
         }
+        tc_commit(&sm.empty[slot]);
       }
-      tc_commit(&sm.empty[slot]);
       if (last) {
         sm.acc_unit[abuf] = hd.unit;
         tc_commit(&sm.acc_full[abuf]);
@@ -2724,14 +2809,18 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane) {
     __syncwarp();
     c_issue += (unsigned long long)(tclock<kTrace>() - ti0);
     ++c_st;
-    if (kFp8 && (info & kTcInfoFp8) && ++as == kFp8AStages) as = 0;
     if (last) {
       if (++abuf == (kFp8 ? kFp8AccBufs : kTcAccBufs)) {
         abuf = 0;
         aphase ^= 1u;
       }
     }
-    if (++slot == sm.sh.nst) {
+    if (kFp8 && amode) {
+      if (++as == kFp8AStages) {
+        as = 0;
+        asph ^= 1u;
+      }
+    } else if (++slot == sm.sh.nst) {
       slot = 0;
       phase ^= 1u;
     }
@@ -3129,6 +3218,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       for (int s = 0; s < kTcStagesMax; ++s) {
         mbar_init(&sm.conv_bar[s], kMacWarps);
         mbar_init(&sm.wfull[s], 1);
+        mbar_init(&sm.cdone[s], kMacWarps);
       }
       for (int a = 0; a < kFp8AStages; ++a) mbar_init(&astage_empty(sm)[a], 1);
       for (int q = 0; q < kCq; ++q) {
@@ -3164,6 +3254,8 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
   __syncthreads();
   if constexpr (kTC) tc_fence_after();
   if (tid == 0) trace_stamp<kTrace>(p, TR_ROLES);
+  uint8_t* const aring = ring;                            // FP8: the A stages' activations
+  if constexpr (kFp8) ring += fp8_actbuf_bytes(sm.sh.NA);  // FP8: the slots follow them
 
   if (warp_id == 0) {
     Producer pr(p, sm, lane, sm.sh.nst);
@@ -3193,14 +3285,14 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
       if (ok) ok = p.B == 1 ? build_schedule_b1<kTrace, kEp>(p, sm, mw, lane, mphase, tag)
                             : build_schedule_tc<kTrace, kEp>(p, sm, mw, lane, mphase, false);
       if (mw == 0 && lane == 0 && ok) mbar_arrive(&sm.sched_bar);
-      if constexpr (kFp8) convert_fp8_stages<kTrace>(p, sm, ring, mw, lane, ok);
+      if constexpr (kFp8) convert_fp8_stages<kTrace>(p, sm, ring, aring, mw, lane, ok);
     } else {
       mac_warps_cc<kTrace>(p, sm, ring, warp_id - 1, lane);
     }
   } else if constexpr (!kTC) {
     epilogue_cc<kTrace>(p, sm, lane);
   } else if (warp_id == kTcMmaWarp) {
-    mma_warp<kTrace, kFp8>(p, sm, ring, lane);
+    mma_warp<kTrace, kFp8>(p, sm, ring, lane, aring);
   } else {
     epilogue_tc<kTrace, kFp8, kEp>(p, sm, warp_id, lane);
   }
