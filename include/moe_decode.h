@@ -297,7 +297,6 @@ int moe_decode_step_path(const moe_decode_handle* h, int batch);
  *    (no host buffer is read after the call returns).
  *  - The first call on a device (the current device) sets up that device: it
  *    looks up the scratch array's device address and the kernel's attributes.
- *    Make that first call before any stream capture.
  *  - All calls share the one array and each call clears its counters before it
  *    runs: calls that overlap on the GPU (other streams, other threads) race and
  *    must be serialised by the caller.
