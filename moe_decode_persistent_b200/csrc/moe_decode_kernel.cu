@@ -112,19 +112,23 @@ static_assert(tc_stages(16, 1) == 4 && tc_stages(16, 8) == 5 && tc_stages(32, 32
 constexpr int kTcAccBufs = 4;       // accumulator buffers in tensor memory
 constexpr int kTcAccCols = 128;     // columns per buffer: tile 0 at +0, tile 1 at +64
 constexpr int kTmemCols = kTcAccBufs * kTcAccCols;  // 512 (a power of two >= 32)
-// A layer with FP8 experts keeps 2 accumulator buffers (columns 0-255) and uses columns
-// 256-511 as 2 stages of the MMA's A operand: the converted bf16 weight tiles of an FP8
-// stage (128 K columns; tile j at +64 j; row m in lane m, K elements 2c and 2c + 1 in
-// column c).
+// A layer with FP8 experts keeps 2 accumulator buffers and uses the rest of tensor memory
+// as stages of the MMA's A operand: the converted bf16 weight tiles of an FP8 stage (128
+// K columns, 128 TMEM columns; tile j at +64 j; row m in lane m, K elements 2c and 2c + 1
+// in column c). With at most 32 token columns an accumulator buffer needs only 64 columns
+// (tile 1 at +32): 2 x 64 + 3 A stages; with more, 2 x 128 + 2 A stages.
 constexpr int kFp8AccBufs = 2;
-constexpr int kFp8AStages = 2;
-constexpr int kFp8ACol0 = kFp8AccBufs * kTcAccCols;
+constexpr int kFp8AStagesMax = 3;
 constexpr int kFp8AStageCols = 2 * kTcAtomK;
+__host__ __device__ constexpr int fp8_acc_cols(int na) { return na <= 32 ? kTcAccCols / 2 : kTcAccCols; }
+__host__ __device__ constexpr int fp8_astages(int na) { return na <= 32 ? 3 : 2; }
+static_assert(kFp8AccBufs * kTcAccCols / 2 + 3 * kFp8AStageCols <= kTmemCols &&
+                  kFp8AccBufs * kTcAccCols + 2 * kFp8AStageCols <= kTmemCols,
+              "FP8 tensor-memory plans");
 // The activations of each A stage (two K atoms of na rows, as they lay in the slot) sit in
 // front of an FP8 layer's ring, so a slot is free once its codes are converted.
 __host__ __device__ constexpr int fp8_act_stage_bytes(int na) { return 2 * na * kTcAtomK * 2; }
-__host__ __device__ constexpr int fp8_actbuf_bytes(int na) { return kFp8AStages * fp8_act_stage_bytes(na); }
-static_assert(kFp8ACol0 + kFp8AStages * kFp8AStageCols <= kTmemCols, "FP8 tensor-memory plan");
+__host__ __device__ constexpr int fp8_actbuf_bytes(int na) { return fp8_astages(na) * fp8_act_stage_bytes(na); }
 
 static_assert(kTcSlotBytes % 1024 == 0 && kTcTileBytes % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(kCcRingBytes % 1024 == 0 && kTcRingBytes % 1024 == 0, "ring keeps the state block aligned");
@@ -174,6 +178,7 @@ struct Shape {
   int NA;   // tensor-core path: token columns of n- and hs-based tiles (B rounded up to 16)
   int nst, slot_bytes;  // ring stages and slot size
   int kblk;             // 1: FP8 experts (expert gate/up K splits at 128-column K blocks)
+  int acc_cols, nas;    // FP8: TMEM columns per accumulator buffer; tensor-memory A stages
   int pre;  // units queued before the routing schedule (no unit before it needs the schedule)
   int router_target, hs_target, pair_target;  // tiles that publish logits / h_s / one pair's h
 };
@@ -218,7 +223,7 @@ struct Smem {
   int16_t cq_slot[kCq];            // ring slot of the queued stage (-1: no more stages)
   uint8_t cq_par[kCq];             // the slot's wfull parity for that stage
   uint8_t cq_fpar[kCq];            // the slot's full parity (its activations) for that stage
-  StageHeader ahdr[kFp8AStages];   // FP8: the header of the stage in each tensor-memory A stage
+  StageHeader ahdr[kFp8AStagesMax];  // FP8: the header of the stage in each tensor-memory A stage
   StageHeader hdr[kMaxRingStages];
   int rb_unit[kRB];         // unit id of the buffer, or -1 (stop)
   int acc_unit[kTcAccBufs]; // unit id of the accumulator buffer, or -1 (stop)
@@ -253,7 +258,7 @@ static_assert(kCcRingBytes + sizeof(Smem) + 1024 <= 227 * 1024, "shared memory b
 // The CUDA-core path's result-buffer barriers (rb_full) serve a tensor-core launch with
 // FP8 experts as its A-stage barriers: the MMAs that read a tensor-memory A stage
 // completed (the two paths never run in one launch).
-static_assert(kFp8AStages <= kRB, "A-stage barriers");
+static_assert(kFp8AStagesMax <= kRB, "A-stage barriers");
 __device__ __forceinline__ uint64_t* astage_empty(Smem& sm) { return sm.rb_full; }
 static_assert(kTcRingBytes + sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget of one CTA");
 static_assert(offsetof(Smem, rb) % 16 == 0 && offsetof(Smem, fin) % 16 == 0, "float4 views of rb / fin");
@@ -520,6 +525,8 @@ __device__ void make_shape_tc(const Params& p, Shape& s) {
   s.GB = 1;
   s.NA = (p.B + kTcActRows - 1) / kTcActRows * kTcActRows;
   s.kblk = p.fp8 ? 1 : 0;
+  s.acc_cols = p.fp8 ? fp8_acc_cols(s.NA) : kTcAccCols;
+  s.nas = fp8_astages(s.NA);
   s.slot_bytes = p.fp8 ? tc_slot_bytes_fp8(s.NA) : tc_slot_bytes(s.NA);
   s.nst = p.fp8 ? tc_stages_in(kTcRingBytes - fp8_actbuf_bytes(s.NA), s.slot_bytes, p.B)
                 : tc_stages_of(s.slot_bytes, p.B);
@@ -2616,7 +2623,8 @@ __device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, uin
   const int quad = (mw + 1) & 3;     // lane quadrant of this warp (warp id mod 4)
   const int j = mw >> 2;             // weight tile
   const int r = quad * 32 + lane;    // tile row = tensor-memory lane
-  const uint32_t tq = sm.tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(kFp8ACol0 + j * (kFp8AStageCols / 2));
+  const uint32_t tq = sm.tmem_base + ((uint32_t)(quad * 32) << 16) +
+                      (uint32_t)(kFp8AccBufs * sh.acc_cols + j * (kFp8AStageCols / 2));
   const int swz = r & 7;
   int q = 0, as = 0;
   uint32_t qph = 0u, asph = 0u;
@@ -2699,7 +2707,7 @@ __device__ void convert_fp8_stages(const Params& p, Smem& sm, uint8_t* ring, uin
       mbar_arrive(&sm.cdone[slot]);  // the slot is free
       mbar_arrive(&sm.conv_bar[as]);
     }
-    if (++as == kFp8AStages) {
+    if (++as == sh.nas) {
       as = 0;
       asph ^= 1u;
     }
@@ -2770,11 +2778,12 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane, uin
     if (lane == 0) {
       const int nbox = info & 3;
       const uint32_t idesc = idesc_bf16_m128((uint32_t)((info >> 2) & 7) * kTcActRows);
-      const uint32_t t0 = tmem + (uint32_t)(abuf * kTcAccCols);
+      const uint32_t acols = kFp8 ? (uint32_t)sm.sh.acc_cols : (uint32_t)kTcAccCols;
+      const uint32_t t0 = tmem + abuf * acols;
       if (kFp8 && amode) {
         // one 128-column K block: 8 K steps of A from tensor memory; the activations of the
         // two atoms beside the A stage, the second at +NA x 128 bytes
-        const uint32_t a0 = tmem + (uint32_t)(kFp8ACol0 + as * kFp8AStageCols);
+        const uint32_t a0 = tmem + kFp8AccBufs * acols + (uint32_t)(as * kFp8AStageCols);
         const uint32_t abase = smem_u32(aring + as * fp8_act_stage_bytes(sm.sh.NA));
         const uint64_t da = sw128_desc(abase);
         const uint64_t da1 = sw128_desc(abase + (uint32_t)(sm.sh.NA * kTcAtomK * 2));
@@ -2783,7 +2792,7 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane, uin
           const uint32_t accum = (first && ks == 0) ? 0u : 1u;
           const uint64_t db = (ks < 4 ? da : da1) + (uint64_t)(2 * (ks & 3));
           tc_mma_bf16_ta(t0, a0 + (uint32_t)(8 * ks), db, idesc, accum);
-          if (nbox == 2) tc_mma_bf16_ta(t0 + 64u, a0 + (uint32_t)(kFp8AStageCols / 2 + 8 * ks), db, idesc, accum);
+          if (nbox == 2) tc_mma_bf16_ta(t0 + acols / 2, a0 + (uint32_t)(kFp8AStageCols / 2 + 8 * ks), db, idesc, accum);
         }
         tc_commit(&astage_empty(sm)[as]);
       } else {
@@ -2795,7 +2804,7 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane, uin
         for (int ks = 0; ks < kTcAtomK / 16; ++ks) {
           const uint32_t accum = (first && ks == 0) ? 0u : 1u;
           tc_mma_bf16(t0, dw0 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
-          if (nbox == 2) tc_mma_bf16(t0 + 64u, dw1 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
+          if (nbox == 2) tc_mma_bf16(t0 + acols / 2, dw1 + (uint64_t)(2 * ks), da + (uint64_t)(2 * ks), idesc, accum);
         }
         tc_commit(&sm.empty[slot]);
       }
@@ -2816,7 +2825,7 @@ __device__ void mma_warp(const Params& p, Smem& sm, uint8_t* ring, int lane, uin
       }
     }
     if (kFp8 && amode) {
-      if (++as == kFp8AStages) {
+      if (++as == sm.sh.nas) {
         as = 0;
         asph ^= 1u;
       }
@@ -2872,9 +2881,11 @@ __device__ __forceinline__ bool epi_sync(Smem& sm, uint32_t& phase, const Params
 
 // Loads accumulator columns [j0, j0 + 16) of both tiles of the buffer (lane quadrant of
 // the calling warp). `two` is warp-uniform.
-__device__ __forceinline__ void tmem_cols16(uint32_t ta, int j0, bool two, uint32_t (&v0)[16], uint32_t (&v1)[16]) {
+// Columns j0 .. j0 + 15 of tile 0 (v0) and, if two, of tile 1 (v1, `half` columns on).
+__device__ __forceinline__ void tmem_cols16(uint32_t ta, int j0, bool two, uint32_t (&v0)[16], uint32_t (&v1)[16],
+                                            uint32_t half = kTcAccCols / 2) {
   tmem_ld16(ta + (uint32_t)j0, v0);
-  if (two) tmem_ld16(ta + 64u + (uint32_t)j0, v1);
+  if (two) tmem_ld16(ta + half + (uint32_t)j0, v1);
   tmem_ld_wait();
   tmem_regs_after_wait(v0);
   if (two) tmem_regs_after_wait(v1);
@@ -3006,7 +3017,8 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
     const long long tb0 = tclock<kTrace>();
     const Sched& sc = sm.sc;
     const UnitDesc d = decode_unit_tc(sh, sc, u);
-    const uint32_t ta = tq + (uint32_t)(abuf * kTcAccCols);
+    const uint32_t acols = kFp8 ? (uint32_t)sh.acc_cols : (uint32_t)kTcAccCols;  // tile 1 at +acols / 2
+    const uint32_t ta = tq + abuf * acols;
     const bool direct = d.nsplit == 1 && (d.type == UT_SHARED || d.type == UT_EXPERT);
     uint32_t v0[16], v1[16];
     switch (d.type) {
@@ -3016,7 +3028,7 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
         // this split's partial logits; the row owners sum the splits
         float* dst = p.rpart + (size_t)d.split * sh.B * p.E;
         for (int j0 = 0; j0 < sh.B; j0 += 16) {
-          tmem_cols16(ta, j0, two, v0, v1);
+          tmem_cols16(ta, j0, two, v0, v1, acols / 2);
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int b = j0 + jj;
@@ -3030,7 +3042,7 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
       }
       case UT_SHARED: {
         for (int j0 = 0; j0 < sh.B; j0 += 16) {
-          tmem_cols16(ta, j0, true, v0, v1);
+          tmem_cols16(ta, j0, true, v0, v1, acols / 2);
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int b = j0 + jj;
@@ -3061,7 +3073,7 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
             uint32_t col = (uint32_t)sc.row_of[r0 + j];
             if (!IDX_OK(p, col < (uint32_t)sh.NA)) col = 0;
             tmem_ld1(ta + col, v0[jj]);
-            tmem_ld1(ta + 64u + col, v1[jj]);
+            tmem_ld1(ta + acols / 2 + col, v1[jj]);
           }
           tmem_ld_wait();
           tmem_regs_after_wait(v0);
@@ -3094,7 +3106,7 @@ __device__ void epilogue_tc(const Params& p0, Smem& sm, int warp_id, int lane, c
         const int h0 = d.tile * 2 * kTcRows + row, h1 = h0 + kTcRows;
         const bool two = d.tile * 2 * kTcRows + kTcRows < p.H;
         for (int j0 = 0; j0 < cnt; j0 += 16) {
-          tmem_cols16(ta, j0, two, v0, v1);
+          tmem_cols16(ta, j0, two, v0, v1, acols / 2);
 #pragma unroll
           for (int jj = 0; jj < 16; ++jj) {
             const int j = j0 + jj;
@@ -3220,7 +3232,7 @@ __global__ void __launch_bounds__(kTC ? kTcThreads : kThreads, 1)
         mbar_init(&sm.wfull[s], 1);
         mbar_init(&sm.cdone[s], kMacWarps);
       }
-      for (int a = 0; a < kFp8AStages; ++a) mbar_init(&astage_empty(sm)[a], 1);
+      for (int a = 0; a < kFp8AStagesMax; ++a) mbar_init(&astage_empty(sm)[a], 1);
       for (int q = 0; q < kCq; ++q) {
         mbar_init(&sm.cq_full[q], 1);
         mbar_init(&sm.cq_empty[q], kMacWarps);  // every converter warp reads every entry
