@@ -91,23 +91,23 @@ constexpr int kTcSlotBytes = 2 * kTcTileBytes + kTcActBytes;       // 40 KB: a s
 constexpr int kTcRingBytes = 180 * 1024;
 // The slot holds the two weight tiles and N x 128 bytes of activations (N = the step's
 // token columns, rounded up to 16): the ring fits 5 stages up to 32 columns, 4 above.
-// Measured: the fifth stage speeds the streaming-dominated steps (batch 8: 864 -> 854
-// us) and slows the routing-dominated ones (batch 1: 170 -> 172.5 us, the deeper HBM
-// queues delay the routing's loads), so batches of at most 4 rows keep 4 stages.
+// A fifth stage speeds streaming but, before the routing schedule exists, its deeper HBM
+// queue delays the routing's own loads: a step of at most 4 rows keeps at most 4 stages
+// in flight until the schedule is built (Producer::wait_slot_pre; measured: batch 1
+// 156.0 -> 154.9 us, batch 4 451.5 -> 442.4 us against 4 stages throughout).
 constexpr int kTcStagesMax = 5;
 __host__ __device__ constexpr int tc_slot_bytes(int na) { return 2 * kTcTileBytes + ((na * kTcAtomK * 2 + 1023) / 1024) * 1024; }
 // A layer with FP8 experts: an FP8 stage holds one 128-column K block, so its slot takes
 // the activations of two K atoms (the second at +na x 128 bytes).
 __host__ __device__ constexpr int tc_slot_bytes_fp8(int na) { return 2 * kTcTileBytes + 2 * na * kTcAtomK * 2; }
 __host__ __device__ constexpr int tc_stages_in(int ring_bytes, int slot_bytes, int batch) {
-  return batch <= 4 && ring_bytes / slot_bytes >= 4 ? 4
-       : ring_bytes / slot_bytes < kTcStagesMax ? ring_bytes / slot_bytes : kTcStagesMax;
+  return ring_bytes / slot_bytes < kTcStagesMax ? ring_bytes / slot_bytes : kTcStagesMax;
 }
 __host__ __device__ constexpr int tc_stages_of(int slot_bytes, int batch) {
   return tc_stages_in(kTcRingBytes, slot_bytes, batch);
 }
 __host__ __device__ constexpr int tc_stages(int na, int batch) { return tc_stages_of(tc_slot_bytes(na), batch); }
-static_assert(tc_stages(16, 1) == 4 && tc_stages(16, 8) == 5 && tc_stages(32, 32) == 5 && tc_stages(64, 64) == 4,
+static_assert(tc_stages(16, 1) == 5 && tc_stages(16, 8) == 5 && tc_stages(32, 32) == 5 && tc_stages(64, 64) == 4,
               "ring depths");
 constexpr int kTcAccBufs = 4;       // accumulator buffers in tensor memory
 constexpr int kTcAccCols = 128;     // columns per buffer: tile 0 at +0, tile 1 at +64
@@ -1888,6 +1888,13 @@ struct Producer {
   }
   // Waits for a free slot; the slot's previous stage has then been consumed (an FP8
   // stage's by the converters, any other by the MMAs).
+  // Before the schedule of a step of at most 4 rows, at most nst - 1 stages in flight: the
+  // next slot's previous stage must be consumed too.
+  __device__ bool wait_slot_pre() {
+    if (p.B > 4 || nst < 5) return true;
+    const int s1 = slot + 1 == nst ? 0 : slot + 1;
+    return wait_bar(&sm.empty[s1], s1 == 0 ? phase : phase ^ 1u);
+  }
   __device__ bool wait_slot() {
     if ((fp8prev >> slot) & 1u) {
       const uint32_t par = (cdpar >> slot) & 1u;
@@ -2351,12 +2358,15 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
       // weights stream while the input is awaited -- a ring's worth for h, one stage
       // for the normalised rows (at the start of the step the HBM queue must stay short
       // for the loads of x that the normalisation waits on)
-      const int depth = (x.dep == 0 ? 1 : pr.nst) * kstep;  // in K atoms
+      // before the schedule of a small step at most nst - 1 stages are in flight, also
+      // while arming (arming all nst would wait on the first armed stage, which has no
+      // activations yet)
+      const int depth = (x.dep == 0 ? 1 : (!sched_ready && p.B <= 4 && pr.nst >= 5 ? pr.nst - 1 : pr.nst)) * kstep;
       const int pre_end = ka_end < d.kb0 + depth ? ka_end : d.kb0 + depth;
       const int slot0 = pr.slot;
       for (; ka < pre_end && ok; ka += kstep) {
         const long long t0 = tclock<kTrace>();
-        ok = pr.wait_slot();
+        ok = (sched_ready || pr.wait_slot_pre()) && pr.wait_slot();
         c_slot += (unsigned long long)(tclock<kTrace>() - t0);
         if (!ok) break;
         issue_weights(ka);
@@ -2387,7 +2397,7 @@ __device__ bool producer_tc(Producer& pr, uint8_t* ring, bool last = true) {
     for (; ka < ka_end && ok; ka += kstep) {
       {
         const long long t0 = tclock<kTrace>();
-        ok = pr.wait_slot();
+        ok = (sched_ready || pr.wait_slot_pre()) && pr.wait_slot();
         c_slot += (unsigned long long)(tclock<kTrace>() - t0);
       }
       if (!ok) break;
