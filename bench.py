@@ -212,6 +212,13 @@ class ClockSampler:
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+        # nvidia-smi's own start-up (its first driver queries) stays out of the timed
+        # region: wait, at most 5 s, for its first sample
+        t0 = time.perf_counter()
+        while self.proc is not None and time.perf_counter() - t0 < 5.0:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.02)
         time.sleep(0.25)
 
     def stop(self):
@@ -362,11 +369,20 @@ def aggregate(local_bytes, local_ms, world):
     return float(b.item()), float(t.item())
 
 
-def step_stats(step_ms):
+TIMING = ("value: one CUDA-event pair around the K back-to-back timed steps; us_per_step_p10/median/"
+          "p90/max: a second pass of K steps with an event pair around every step (an event between two "
+          "launches delays the second, so these run a few us above the back-to-back mean)")
+
+
+def step_stats(step_ms, total_ms=None):
+    """us_per_step: the back-to-back mean (total_ms / K) when given, else the per-step mean;
+    the quantiles and the slowest step: the per-step times."""
     a = np.asarray(step_ms, dtype=np.float64) * 1e3  # µs
-    return {"us_per_step": round(float(a.mean()), 2), "us_per_step_p10": round(float(np.percentile(a, 10)), 2),
+    mean = total_ms * 1e3 / len(a) if total_ms is not None else float(a.mean())
+    return {"us_per_step": round(mean, 2), "us_per_step_p10": round(float(np.percentile(a, 10)), 2),
             "us_per_step_median": round(float(np.median(a)), 2),
-            "us_per_step_p90": round(float(np.percentile(a, 90)), 2)}
+            "us_per_step_p90": round(float(np.percentile(a, 90)), 2),
+            "us_per_step_max": round(float(a.max()), 2), "slowest_step": int(a.argmax())}
 
 
 L2_PROTOCOL = ("no flush: every step streams more weight bytes than the 126 MB L2, and single-layer "
@@ -407,31 +423,42 @@ class ConfigRun:
         self.y = torch.empty((wl.B, wl.H), dtype=torch.bfloat16, device=self.dev)
         self.flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=self.dev)
 
-    def steps(self, K, W, stream, barrier, host=None, launch_log=None, flush=False):
+    def steps(self, K, W, stream, barrier, host=None, launch_log=None, flush=False, per_step=False):
         """W untimed warm-up steps immediately followed (no idle gap, so the clocks stay
-        up) by K timed steps; step i runs weight set i mod (number of sets); CUDA events
-        on `stream` bracket every step. flush: a 256 MB write before every step (the
-        secondary, flushed figure). host = (x_host, y_host): the host-buffer entry point
-        instead. Returns per-step ms and the unique-expert count of every timed step and
-        layer."""
+        up) by K timed steps; step i runs weight set i mod (number of sets). One CUDA-event
+        pair on `stream` brackets the K back-to-back steps (launches follow one another as
+        in a decode loop); per_step: a pair around every step instead (an event recorded
+        between two launches delays the second by a few µs, so these per-step times run a
+        little above the back-to-back mean). flush: a 256 MB write before every step (the
+        secondary, flushed figure; per-step events, so the writes stay out of the timing).
+        host = (x_host, y_host): the host-buffer entry point instead. Returns the per-step
+        ms (per_step) or the K steps' total ms as one value, and the unique-expert count of
+        every timed step and layer."""
+        assert per_step or not flush
         import torch
 
         wl = self.wl
         nu = torch.zeros((W + K, wl.layers), dtype=torch.int32, device=self.dev)
         dbg = lambda i: [dict(n_unique=nu[i, l:l + 1]) for l in range(wl.layers)]
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K if per_step else 1)]
+
+        # every step's handle, input view and debug record, made before any step runs (the
+        # harness's own bookkeeping stays out of the timed steps' host time)
+        src = self.pool if host is None else host[0]
+        plan = [(self.sets[i % len(self.sets)][1], src[i % POOL], dbg(i)) for i in range(W + K)]
 
         def one(i, timed):
-            h = self.sets[i % len(self.sets)][1]
+            h, x, d = plan[i]
             if flush:
                 self.flush.zero_()
-            if timed:
+            if timed and per_step:
                 ev[i - W][0].record(stream)
             if host is None:
-                h.step(self.pool[i % POOL], self.y, wl.B, wl.k, stream=stream, debug=dbg(i))
+                h.step(x, self.y, wl.B, wl.k, stream=stream, debug=d)
             else:
-                h.step_host(host[0][i % POOL], host[1], wl.B, wl.k, stream=stream, debug=dbg(i))
-            if timed:
+                h.step_host(x, host[1], wl.B, wl.k, stream=stream, debug=d)
+            if timed and per_step:
                 ev[i - W][1].record(stream)
 
         for i in range(W):
@@ -441,8 +468,12 @@ class ConfigRun:
         barrier()
         torch.cuda.synchronize()
         wall0 = time.perf_counter()
+        if not per_step:
+            ev[0][0].record(stream)
         for i in range(W, W + K):
             one(i, True)
+        if not per_step:
+            ev[0][1].record(stream)
         torch.cuda.synchronize()
         barrier()
         self.wall = time.perf_counter() - wall0
@@ -509,17 +540,18 @@ def run_ours(args, wl):
     run = ConfigRun(wl, local, args.tc_min_batch)
     sampler = ClockSampler(local)
     sampler.start()
-    step_ms, U = run.steps(K, W, stream, barrier, launch_log=launch_log)
+    tot_ms, U = run.steps(K, W, stream, barrier, launch_log=launch_log)
     wall = run.wall
+    step_ms, _ = run.steps(K, W, stream, barrier, per_step=True)
     clocks = sampler.stop()
     bytes_steps = [step_bytes(wl, list(U[i])) for i in range(K)]
-    local_ms = float(sum(step_ms))
+    local_ms = float(sum(tot_ms))
     tot_bytes, max_ms = aggregate(sum(bytes_steps), local_ms, world)
     value = tot_bytes / (max_ms * 1e-3) / 1e9
     achieved = sum(bytes_steps) / (local_ms * 1e-3) / 1e9  # this rank's launching stream
     # secondary figure: the same steps with a 256 MB write between steps (which also
     # evicts the kernel's instructions and leaves L2 full of dirty lines to write back)
-    f_ms, fU = run.steps(K, W, stream, barrier, flush=True)
+    f_ms, fU = run.steps(K, W, stream, barrier, flush=True, per_step=True)
     f_bytes, f_max = aggregate(sum(step_bytes(wl, list(fU[i])) for i in range(K)), float(sum(f_ms)), world)
     l2_flushed = {"value": round(f_bytes / (f_max * 1e-3) / 1e9, 2), "unit": "GB/s", **step_stats(f_ms),
                   "l2": "flushed between timed steps (256 MB write)"}
@@ -542,7 +574,8 @@ def run_ours(args, wl):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic: seeded counter-hash weights ~N(0,1/sqrt(fan_in)) and inputs, no trained weights",
         "config": dict(workload_config(wl, L2_PROTOCOL), kernel_path=run.kernel_path),
-        **step_stats(step_ms),
+        **step_stats(step_ms, local_ms),
+        "timing": TIMING,
         "l2_flushed": l2_flushed,
         "tokens_per_s": round(world * wl.B * K / (max_ms * 1e-3), 1),
         "unique_experts_mean": float(U.mean()),
@@ -566,17 +599,18 @@ def run_ours(args, wl):
         r = ConfigRun(cw, local, args.tc_min_batch)
         smp = ClockSampler(local)
         smp.start()
-        c_ms, cU = r.steps(K, W, stream, barrier, launch_log=launch_log)
+        c_tot, cU = r.steps(K, W, stream, barrier, launch_log=launch_log)
+        c_ms, _ = r.steps(K, W, stream, barrier, per_step=True)
         c_clocks = smp.stop()
         c_bytes = [step_bytes(cw, list(cU[i])) for i in range(K)]
-        c_local = float(sum(c_ms))
+        c_local = float(sum(c_tot))
         c_tot, c_max = aggregate(sum(c_bytes), c_local, world)
         c_ach = sum(c_bytes) / (c_local * 1e-3) / 1e9
         per_config[cw.name] = {
             "config": workload_config(cw, L2_PROTOCOL) | {"kernel_path": r.kernel_path},
             "dtype": "fp8 (e4m3) experts, bf16 activations" if cw.is_fp8 else "bf16",
             "value": round(c_tot / (c_max * 1e-3) / 1e9, 2), "unit": "GB/s",
-            **step_stats(c_ms),
+            **step_stats(c_ms, c_local),
             "tokens_per_s": round(world * cw.B * K / (c_max * 1e-3), 1),
             "unique_experts_mean": float(cU.mean()), "bytes_per_step_mean": float(np.mean(c_bytes)),
             "roofline": roofline_entry(cw, c_ach, peak, peak_kind),
