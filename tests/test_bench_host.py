@@ -1,5 +1,5 @@
 """Host-side arithmetic of bench.py on CPU: the algorithmic bytes behind every GB/s
-and roofline figure, and the rule that ncu traffic counters apply only to the kernel
+and roofline figure, the step statistics, and the rule that ncu traffic counters apply only to the kernel
 sources they were taken on."""
 import json
 
@@ -88,3 +88,12 @@ def test_ingest_traffic_matches_each_captured_launch_to_its_own_step(tmp_path, m
     t = bench.ingest_traffic(str(tmp_path / "b.csv"), str(tmp_path / "log2.json"), v.name, "ncu -s 1 -c 1 x")
     assert t["launches"][0]["step"] == 1
     assert t["launches"][0]["algorithmic_bytes"] == bench.step_bytes(v, [80, 81])
+
+
+def test_step_stats_mean_is_the_back_to_back_figure_and_quantiles_the_per_step_times():
+    per_step_ms = [0.170, 0.150, 0.152, 0.151, 0.153]
+    s = bench.step_stats(per_step_ms, total_ms=0.745)  # 5 back-to-back steps: 149 us each
+    assert s["us_per_step"] == 149.0
+    assert s["us_per_step_median"] == 152.0
+    assert s["us_per_step_max"] == 170.0 and s["slowest_step"] == 0
+    assert bench.step_stats(per_step_ms)["us_per_step"] == 155.2  # no total: the per-step mean
